@@ -1,0 +1,369 @@
+#!/usr/bin/env python
+"""Benchmark of the In-Place TTT MLP layer forward (libipttt) on B200.
+
+One step = one full layer forward (all stages: metadata, masked conv, gate/up
+GEMM, target GEMM, Gram/clip pass, chunk scan with apply and update) over one
+batch of the workload, inputs resident in HBM.  With --gpus N under torchrun,
+every rank runs its own replica on its own batch (weak scaling, no collective on
+the data path); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle instead (rank 0 only), on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from chunk_wise_weight_gate_b200 import ipttt as ip  # noqa: E402
+from chunk_wise_weight_gate_b200 import synth  # noqa: E402
+
+METRIC = "In-Place TTT MLP layer tokens/s and TFLOP/s (% of bf16 peak) at Qwen3-4B shape"
+DEFAULT_WORKLOAD = "qwen3_4b_128k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+WEIGHTS = ("Wgate", "Wup", "Wdown0", "conv_w", "Wtarget")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons, power = [], [], set(), []
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def layer_flops(w: synth.Workload) -> int:
+    """Credited flops of one step (all layers): 10 d F + 2 d^2 + 10 d per token."""
+    return ip.flops_per_token(w.d, w.F) * w.B * w.T * w.layers
+
+
+def phase_flops(w: synth.Workload) -> dict:
+    """Algorithmic flops per call of each phase (per layer)."""
+    B, T, d, F, C = w.B, w.T, w.d, w.F, w.C
+    k = (T + C - 1) // C
+    ct = C // 128
+    return {
+        "prep": 10 * B * T * d,
+        "gate_up": 4 * B * T * d * F,
+        "target": 2 * B * T * d * d,
+        "gram": 2 * B * k * (ct * (ct + 1) // 2) * 128 * 128 * (d + F),
+        "scan": 6 * B * T * d * F,
+    }
+
+
+def oracle_sample(w: synth.Workload, inp: dict, chunks: int) -> tuple[float, int]:
+    """Runs the fp64 oracle on the first `chunks` chunks of row 0; returns (seconds, tokens)."""
+    from oracle import ipttt_oracle as orc
+    n = min(w.T, chunks * w.C)
+    a = {k: inp[k][:1, :n].double().numpy() for k in ("H", "X0")}
+    wts = {k: inp[k].double().numpy() for k in WEIGHTS}
+    ds = inp["doc_starts"].numpy()
+    ds = ds[(ds // w.T == 0) & (ds % w.T < n)]
+    t0 = time.perf_counter()
+    orc.layer_forward(a["H"], a["X0"], wts["Wgate"], wts["Wup"], wts["Wdown0"], wts["conv_w"], wts["Wtarget"], w.C,
+                      ds, w.eta, w.clip)
+    return time.perf_counter() - t0, n
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def config_dict(w: synth.Workload, n: int) -> dict:
+    return {"workload": w.name, "batch": w.B, "seq_len": w.T, "chunk": w.C, "d_model": w.d, "d_ff": w.F,
+            "layers": w.layers, "eta": w.eta, "clip": w.clip, "docs": w.docs,
+            "global_batch": w.B * n, "parallelism": f"replicas{n}" if n > 1 else "single",
+            "l2": "inputs larger than L2 (H and X0 are B*T*d bf16; Z is B*T*F bf16)"}
+
+
+def run_reference(args, w: synth.Workload):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    inp = synth.make_inputs(w.replace(B=1), seed=0)
+    chunks = max(1, args.cpu_sample_chunks)
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, chunks)
+    secs, toks = 0.0, 0
+    for _ in range(args.steps):
+        s, n = oracle_sample(w, inp, chunks)
+        secs += s
+        toks += n
+    value = toks / secs
+    sample = f"first {chunks} chunk(s) ({toks // args.steps} tokens) of row 0 per step, fp64 numpy oracle"
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * secs / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": config_dict(w, 1),
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def run_ours(args, w: synth.Workload):
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+        pg = dist
+
+    layers = []
+    for layer in range(w.layers):
+        inp = synth.make_inputs(w, seed=rank, layer=layer, with_activations=(layer == 0))
+        layers.append(inp)
+    host = {k: layers[0][k] for k in ("H", "X0")}
+    dev_in = {k: v.to(dev) for k, v in host.items()}
+    dev_w = [{k: l[k].to(dev) for k in WEIGHTS} for l in layers]
+    docs = layers[0]["doc_starts"]
+    cfg = ip.LayerConfig(B=w.B, T=w.T, d=w.d, F=w.F, C=w.C, eta=w.eta, clip=w.clip, dtype=w.dtype)
+    ws = ip.alloc_workspace(cfg, dev)
+    O = torch.empty(w.B, w.T, w.d, dtype=cfg.torch_dtype, device=dev)
+    Hbuf = [torch.empty_like(dev_in["H"]) for _ in range(2)] if w.layers > 1 else None
+    docs_dev = docs.to(dev)
+    stream = torch.cuda.current_stream()
+
+    def step(H, X0, out):
+        if w.layers == 1:
+            ip.forward(cfg, H, X0, *(dev_w[0][k] for k in WEIGHTS), docs_dev, O=out, workspace=ws)
+            return
+        cur = H
+        for l in range(w.layers):
+            nxt = Hbuf[l % 2] if l + 1 < w.layers else out
+            ip.forward(cfg, cur, X0, *(dev_w[l][k] for k in WEIGHTS), docs_dev, O=nxt, workspace=ws,
+                       residual=True)
+            cur = nxt
+
+    for _ in range(args.warmup):
+        step(dev_in["H"], dev_in["X0"], O)
+    torch.cuda.synchronize()
+    if ip.get_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    gpu_id = str(local)
+    try:
+        gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
+        if not gpu_id.startswith("GPU-"):
+            gpu_id = "GPU-" + gpu_id
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    ip.profile_read()
+    ip.profile_enable(True)
+    launches0 = ip.kernel_launches()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(dev_in["H"], dev_in["X0"], O)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if pg:
+        pg.barrier()
+    ip.profile_enable(False)
+    launches = ip.kernel_launches() - launches0
+    phases = ip.profile_read()
+    ms = e0.elapsed_time(e1) / args.steps
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    status = ip.get_status()
+
+    tokens = w.B * w.T * w.layers
+    value = world * tokens / (ms / 1000.0)
+    flops = layer_flops(w)
+    tflops = world * flops / (ms / 1000.0) / 1e12
+    peaks, peak_src = load_peaks()
+
+    # roofline of the dominant kernel (the phase with the largest share of device time)
+    pf = phase_flops(w)
+    dom = max(phases, key=lambda k: phases[k][0])
+    dom_ms, dom_launches = phases[dom]
+    if dom in ("prep",):
+        algo_bytes = w.B * w.T * w.d * 2 * 2 * w.layers * args.steps
+        achieved = algo_bytes / (dom_ms / 1000.0) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None}
+    else:
+        total = pf[dom] * w.layers * args.steps
+        achieved = total / (dom_ms / 1000.0) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "launches": dom_launches,
+                "avg_launch_ms": dom_ms / max(1, dom_launches),
+                "peak_note": f"sustained bf16 ({peak_src}); burst {peaks['bf16_tflops']}"}
+    phase_report = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
+                    for k, v in phases.items()}
+
+    # end to end through the public API: pinned host inputs in, result read back, every step
+    e2e = None
+    if not args.no_e2e:
+        hp = {k: v.pin_memory() for k, v in host.items()}
+        o_host = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        step(dev_in["H"], dev_in["X0"], O)
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            dev_in["H"].copy_(hp["H"], non_blocking=True)
+            dev_in["X0"].copy_(hp["X0"], non_blocking=True)
+            step(dev_in["H"], dev_in["X0"], O)
+            o_host.copy_(O, non_blocking=True)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ems = a0.elapsed_time(a1) / args.steps
+        if pg:
+            t = torch.tensor([ems], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        e2e = {"value": world * tokens / (ems / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": o_host.numel() * o_host.element_size(), "ms_per_step": ems}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, n = oracle_sample(w, layers[0], args.cpu_sample_chunks)
+        cpu = {"value": n / secs, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"first {args.cpu_sample_chunks} chunk(s) ({n} tokens) of row 0, one layer, "
+                         f"fp64 numpy oracle, {secs:.1f} s"}
+
+    if rank == 0:
+        out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w, world),
+               "tflops": tflops, "frac_of_peak": tflops / world / peaks.get("bf16_tflops_sustained", 1.0),
+               "frac_of_burst_peak": tflops / world / peaks["bf16_tflops"], "peak_source": peak_src,
+               "roofline": roof, "phases": phase_report, "clocks": clocks, "e2e": e2e,
+               "gpu_launches": launches, "cpu_baseline": cpu, "device_status": status}
+        print(json.dumps(out), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--chunk", type=int, default=None, help="override the chunk size C")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-chunks", type=int, default=2)
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    w = synth.WORKLOADS[args.workload]
+    if args.chunk:
+        w = w.replace(C=args.chunk)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,595 @@
+// C ABI of libipttt (declared in include/ipttt.h): argument checks, workspace
+// carve-up, and the order of kernel launches for one In-Place TTT MLP layer.
+//
+// Launch order (bf16 path), all on the caller's stream:
+//   metadata -> masked conv U -> Z = SiLU(H Wg^T)*(H Wu^T) -> V = U Wt (last-segment
+//   rows) -> Gram partials -> alpha -> for each chunk i: one scan launch holding the
+//   apply tiles of chunk i (reads S_i) and the delta tiles (S_i -> S_{i+1}).
+// The chunk order follows lijianxiong.blog notes "In-Place Test-Time Training",
+// 方法 (apply with the current fast weight, then update) and iplexlaw.co.kr review
+// §3 (a chunk's output always comes from the pre-update state).
+#include <cuda_runtime.h>
+#include <math.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "aux_kernels.h"
+#include "common.cuh"
+#include "tc_kernels.h"
+
+namespace ipttt {
+
+__device__ int g_status_word = 0;
+
+ipttt_status cuda_status(cudaError_t e) { return e == cudaSuccess ? IPTTT_OK : IPTTT_ERR_CUDA; }
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  int* status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+ipttt_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return IPTTT_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    if (cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return IPTTT_ERR_CUDA;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess) return IPTTT_ERR_CUDA;
+    di.status = static_cast<int*>(addr);
+    di.ready = true;
+  }
+  *out = &di;
+  return IPTTT_OK;
+}
+
+// ---------------------------------------------------------------- profiling
+constexpr int kPhases = 5;
+enum Phase { PH_PREP = 0, PH_GATEUP = 1, PH_TARGET = 2, PH_GRAM = 3, PH_SCAN = 4 };
+
+std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_profile_on{0};
+
+struct Profiler {
+  std::mutex mu;
+  std::vector<cudaEvent_t> pool;
+  struct Pending {
+    cudaEvent_t a, b;
+    int phase;
+    uint64_t launches;
+  };
+  std::vector<Pending> pending;
+  double ms[kPhases] = {0};
+  uint64_t launches[kPhases] = {0};
+
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+};
+Profiler g_prof;
+
+// Brackets one phase of a call: records an event now and one when finished.
+struct PhaseScope {
+  cudaStream_t st;
+  int phase;
+  uint64_t start_count;
+  cudaEvent_t a = nullptr;
+  PhaseScope(cudaStream_t s, int ph) : st(s), phase(ph), start_count(g_launches.load()) {
+    if (g_profile_on.load()) {
+      std::lock_guard<std::mutex> lk(g_prof.mu);
+      a = g_prof.get();
+      if (a) cudaEventRecord(a, st);
+    }
+  }
+  ~PhaseScope() {
+    if (!a) return;
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    cudaEvent_t b = g_prof.get();
+    if (!b) return;
+    cudaEventRecord(b, st);
+    g_prof.pending.push_back({a, b, phase, g_launches.load() - start_count});
+  }
+};
+
+inline void counted(int n) { g_launches.fetch_add((uint64_t)n); }
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+struct Layout {
+  size_t flags, meta, alpha, partials, Z, U, V, S, snap, raw, dpart, total;
+};
+
+bool is_bf16(const ipttt_params& p) { return p.dtype == IPTTT_BF16; }
+
+Shape shape_of(const ipttt_params& p) {
+  Shape s;
+  s.B = p.B;
+  s.T = p.T;
+  s.d = p.d;
+  s.F = p.F;
+  s.C = p.C;
+  s.k = (p.T + p.C - 1) / p.C;
+  return s;
+}
+
+Layout layout_of(const ipttt_params& p) {
+  const Shape s = shape_of(p);
+  const size_t B = s.B, T = s.T, d = s.d, F = s.F, k = s.k;
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  L.flags = take(B * T);
+  L.meta = take(B * k * sizeof(ChunkMeta));
+  L.alpha = take(B * k * sizeof(float));
+  if (is_bf16(p)) {
+    const size_t ct = s.C / 128;
+    L.partials = take(B * k * (ct * (ct + 1) / 2) * sizeof(float));
+    L.Z = take(B * T * F * 2);
+    L.U = take(B * T * d * 2);
+    L.V = take(B * T * d * 2);
+    L.S = take(B * d * F * 4);
+    L.snap = take(2 * B * d * F * 2);
+    L.raw = L.dpart = 0;
+  } else {
+    L.partials = 0;
+    L.Z = take(B * T * F * 4);
+    L.U = take(B * T * d * 4);
+    L.V = take(B * T * d * 4);
+    L.S = take(B * d * F * 4);
+    L.raw = take(B * d * F * 4);
+    L.dpart = take(B * 64 * sizeof(double));
+    L.snap = 0;
+  }
+  L.total = off;
+  return L;
+}
+
+ipttt_status check_params(const ipttt_params* p) {
+  if (!p) return IPTTT_ERR_ARG;
+  if (p->dtype != IPTTT_F32 && p->dtype != IPTTT_BF16) return IPTTT_ERR_DTYPE;
+  if (p->B <= 0 || p->T <= 0 || p->d <= 0 || p->F <= 0 || p->C <= 0) return IPTTT_ERR_ARG;
+  if (!isfinite(p->eta) || isnan(p->clip_thresh)) return IPTTT_ERR_ARG;
+  if ((p->flags & ~IPTTT_FLAG_RESIDUAL) != 0) return IPTTT_ERR_ARG;
+  const long long BT = (long long)p->B * p->T;
+  if (BT > (1ll << 30) || (long long)p->d * p->F > (1ll << 31) || (long long)p->d * p->d > (1ll << 31) ||
+      BT * (long long)p->F > (1ll << 40))
+    return IPTTT_ERR_SHAPE;
+  if (p->dtype == IPTTT_BF16) {
+    if (p->d % 128 != 0 || p->F % 256 != 0 || p->C % 128 != 0 || p->C > 4096) return IPTTT_ERR_UNSUPPORTED;
+  }
+  return IPTTT_OK;
+}
+
+struct Tensors {
+  const void *H, *X0, *Wg, *Wu, *W0, *cw, *Wt;
+  const void *Zin, *Vin;  // ipttt_core
+  const int32_t* doc;
+  int n_doc;
+  void* O;
+  float *D, *Sfinal, *alpha;
+  void *Zout, *Vout;
+};
+
+struct StreamState {
+  float* S;
+  long long* pos;
+  int32_t* cont;
+};
+
+size_t state_bytes(const ipttt_params& p) {
+  const size_t B = p.B;
+  return align256(B * p.d * (size_t)p.F * 4) + align256(B * 8) + align256(B * 4);
+}
+
+StreamState state_of(const ipttt_params& p, void* state) {
+  uint8_t* base = static_cast<uint8_t*>(state);
+  StreamState s;
+  const size_t sbytes = align256((size_t)p.B * p.d * (size_t)p.F * 4);
+  s.S = reinterpret_cast<float*>(base);
+  s.pos = reinterpret_cast<long long*>(base + sbytes);
+  s.cont = reinterpret_cast<int32_t*>(base + sbytes + align256((size_t)p.B * 8));
+  return s;
+}
+
+#define IP_CHECK(expr)                                  \
+  do {                                                  \
+    cudaError_t e_ = (expr);                            \
+    if (e_ != cudaSuccess) return IPTTT_ERR_CUDA;       \
+  } while (0)
+
+ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, const Layout& L, StreamState* ss,
+                      DeviceInfo* di, cudaStream_t st) {
+  using namespace tck;
+  const Shape s = shape_of(p);
+  uint8_t* flags = ws + L.flags;
+  ChunkMeta* meta = reinterpret_cast<ChunkMeta*>(ws + L.meta);
+  float* alpha = reinterpret_cast<float*>(ws + L.alpha);
+  float* partials = reinterpret_cast<float*>(ws + L.partials);
+  void* Z = t.Zin ? const_cast<void*>(t.Zin) : static_cast<void*>(ws + L.Z);
+  void* U = ws + L.U;
+  void* V = ws + L.V;
+  float* S = ss ? ss->S : reinterpret_cast<float*>(ws + L.S);
+  void* snap = ws + L.snap;
+  const float tau = (p.clip_thresh > 0.0f && isfinite(p.clip_thresh)) ? p.clip_thresh : 0.0f;
+
+  {
+    PhaseScope ph(st, PH_PREP);
+    IP_CHECK(aux::build_meta(flags, meta, s, t.doc, t.n_doc, ss ? ss->cont : nullptr, di->status, st));
+    counted(3);
+    if (!t.Zin) {
+      IP_CHECK(aux::conv_target(IPTTT_BF16, t.X0, t.cw, flags, U, s, st));
+    } else {
+      IP_CHECK(aux::mask_last_segment(IPTTT_BF16, t.Vin, V, meta, s, st));
+    }
+    counted(1);
+  }
+
+  TcParams tp;
+  memset(&tp, 0, sizeof(tp));
+  tp.B = s.B;
+  tp.T = s.T;
+  tp.d = s.d;
+  tp.F = s.F;
+  tp.C = s.C;
+  tp.k = s.k;
+  tp.ct = s.C / 128;
+  tp.npairs = tp.ct * (tp.ct + 1) / 2;
+  tp.eta = p.eta;
+  tp.meta = meta;
+  tp.alpha = alpha;
+  tp.status = di->status;
+
+  if (!t.Zin) {
+    PhaseScope ph(st, PH_GATEUP);
+    TcParams g = tp;
+    g.kind = kind_gateup();
+    if (!make_map_bf16(&g.map[0], t.H, s.d, s.T, s.B, 64, 128) ||
+        !make_map_bf16(&g.map[1], t.Wg, s.d, s.F, 1, 64, 128) ||
+        !make_map_bf16(&g.map[2], t.Wu, s.d, s.F, 1, 64, 128))
+      return IPTTT_ERR_CUDA;
+    g.out0 = Z;
+    g.n_tiles = s.B * ((s.T + 127) / 128) * (s.F / 128);
+    IP_CHECK(launch_tc(FAM_ZV, g, di->num_sms, st));
+    counted(1);
+  }
+  if (!t.Zin) {
+    PhaseScope ph(st, PH_TARGET);
+    TcParams v = tp;
+    v.kind = kind_vhat();
+    if (!make_map_bf16(&v.map[0], U, s.d, s.T, s.B, 64, 128) ||
+        !make_map_bf16(&v.map[1], t.Wt, s.d, s.d, 1, 64, 64))
+      return IPTTT_ERR_CUDA;
+    v.out0 = V;
+    v.n_tiles = s.B * ((s.T + 127) / 128) * (s.d / 128);
+    IP_CHECK(launch_tc(FAM_ZV, v, di->num_sms, st));
+    counted(1);
+  }
+  if (t.Zout) IP_CHECK(cudaMemcpyAsync(t.Zout, Z, (size_t)s.B * s.T * s.F * 2, cudaMemcpyDeviceToDevice, st));
+  if (t.Vout) IP_CHECK(cudaMemcpyAsync(t.Vout, V, (size_t)s.B * s.T * s.d * 2, cudaMemcpyDeviceToDevice, st));
+
+  {
+    PhaseScope ph(st, PH_GRAM);
+    TcParams g = tp;
+    if (!make_map_bf16(&g.map[0], Z, s.F, s.T, s.B, 64, 128) ||
+        !make_map_bf16(&g.map[1], V, s.d, s.T, s.B, 64, 128))
+      return IPTTT_ERR_CUDA;
+    g.partials = partials;
+    g.n_tiles = s.B * s.k * tp.npairs;
+    IP_CHECK(launch_tc(FAM_GRAM, g, di->num_sms, st));
+    IP_CHECK(aux::alpha_from_partials(partials, alpha, s.B * s.k, tp.npairs, p.eta, tau, st));
+    counted(2);
+  }
+  if (t.alpha) IP_CHECK(cudaMemcpyAsync(t.alpha, alpha, (size_t)s.B * s.k * 4, cudaMemcpyDeviceToDevice, st));
+
+  PhaseScope scan_phase(st, PH_SCAN);
+  // A streaming piece that continues a row starts from the carried state S.
+  if (ss) {
+    IP_CHECK(aux::state_snapshot(S, snap, s, st));
+    counted(1);
+  }
+
+  TcParams sc = tp;
+  if (!make_map_bf16(&sc.map[0], Z, s.F, s.T, s.B, 64, 128) ||
+      !make_map_bf16(&sc.map[1], t.W0, s.F, s.d, 1, 64, 128) ||
+      !make_map_bf16(&sc.map[2], snap, s.F, s.d, 2 * s.B, 64, 128) ||
+      !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, 64) ||
+      !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, 64) ||
+      !make_map_bf16(&sc.map[5], snap, s.F, s.d, 2 * s.B, 64, 32))
+    return IPTTT_ERR_CUDA;
+  sc.out0 = t.O;
+  sc.out1 = t.D;
+  sc.resid = (p.flags & IPTTT_FLAG_RESIDUAL) ? t.H : nullptr;
+  sc.S = S;
+  const bool need_final = t.Sfinal != nullptr || ss != nullptr;
+  for (int i = 0; i < s.k; ++i) {
+    const bool last = i + 1 == s.k;
+    sc.chunk = i;
+    sc.snap_in = i & 1;
+    sc.snap_out = (i + 1) & 1;
+    sc.write_snap = last ? 0 : 1;
+    sc.n_apply = s.B * sc.ct * (s.d / 128);
+    const int n_delta = (!last || need_final) ? s.B * (s.d / 128) * (s.F / 256) : 0;
+    sc.n_tiles = sc.n_apply + n_delta;
+    IP_CHECK(launch_tc(FAM_SCAN, sc, di->num_sms, st));
+    counted(1);
+  }
+  if (t.Sfinal) {
+    IP_CHECK(aux::state_export(true, S, t.Sfinal, s, st));
+    counted(1);
+  }
+  if (ss) {
+    IP_CHECK(aux::stream_advance(ss->pos, ss->cont, s.B, s.T, st));
+    counted(1);
+  }
+  return IPTTT_OK;
+}
+
+ipttt_status run_f32(const ipttt_params& p, const Tensors& t, uint8_t* ws, const Layout& L, StreamState* ss,
+                     DeviceInfo* di, cudaStream_t st) {
+  using namespace aux;
+  const Shape s = shape_of(p);
+  uint8_t* flags = ws + L.flags;
+  ChunkMeta* meta = reinterpret_cast<ChunkMeta*>(ws + L.meta);
+  float* alpha = reinterpret_cast<float*>(ws + L.alpha);
+  const float* Z = t.Zin ? static_cast<const float*>(t.Zin) : reinterpret_cast<float*>(ws + L.Z);
+  float* U = reinterpret_cast<float*>(ws + L.U);
+  float* V = reinterpret_cast<float*>(ws + L.V);
+  float* S = ss ? ss->S : reinterpret_cast<float*>(ws + L.S);
+  float* raw = reinterpret_cast<float*>(ws + L.raw);
+  double* dpart = reinterpret_cast<double*>(ws + L.dpart);
+  const float tau = (p.clip_thresh > 0.0f && isfinite(p.clip_thresh)) ? p.clip_thresh : 0.0f;
+  const long long T = s.T, d = s.d, F = s.F;
+
+  IP_CHECK(build_meta(flags, meta, s, t.doc, t.n_doc, ss ? ss->cont : nullptr, di->status, st));
+  counted(3 + (t.Zin ? 1 : 3) + 5 * s.k + (ss ? 1 : 0) + (t.Sfinal ? 1 : 0));
+  if (!t.Zin) {
+    IP_CHECK(conv_target(IPTTT_F32, t.X0, t.cw, flags, U, s, st));
+    SimtArgs a{};
+    a.M = s.T; a.N = s.F; a.K = s.d;
+    a.A = static_cast<const float*>(t.H); a.sam = d; a.sak = 1; a.sab = T * d;
+    a.B0 = static_cast<const float*>(t.Wg); a.s0n = d; a.s0k = 1; a.s0b = 0;
+    a.B1 = static_cast<const float*>(t.Wu); a.s1n = d; a.s1k = 1; a.s1b = 0;
+    a.mode = SM_Z;
+    a.out = const_cast<float*>(Z); a.som = F; a.son = 1; a.sob = T * F;
+    IP_CHECK(simt_gemm(a, s.B, st));
+
+    SimtArgs v{};
+    v.M = s.T; v.N = s.d; v.K = s.d;
+    v.A = U; v.sam = d; v.sak = 1; v.sab = T * d;
+    v.B0 = static_cast<const float*>(t.Wt); v.s0n = 1; v.s0k = d; v.s0b = 0;
+    v.mode = SM_V;
+    v.out = V; v.som = d; v.son = 1; v.sob = T * d;
+    v.meta = meta; v.k = s.k; v.C = s.C; v.row0 = 0;
+    IP_CHECK(simt_gemm(v, s.B, st));
+  } else {
+    IP_CHECK(mask_last_segment(IPTTT_F32, t.Vin, V, meta, s, st));
+  }
+  if (t.Zout) IP_CHECK(cudaMemcpyAsync(t.Zout, Z, (size_t)s.B * T * F * 4, cudaMemcpyDeviceToDevice, st));
+  if (t.Vout) IP_CHECK(cudaMemcpyAsync(t.Vout, V, (size_t)s.B * T * d * 4, cudaMemcpyDeviceToDevice, st));
+
+  for (int i = 0; i < s.k; ++i) {
+    const long long t0 = (long long)i * s.C;
+    const int rows = (int)std::min<long long>(s.C, T - t0);
+    SimtArgs a{};
+    a.M = rows; a.N = s.d; a.K = s.F;
+    a.A = Z + t0 * F; a.sam = F; a.sak = 1; a.sab = T * F;
+    a.B0 = static_cast<const float*>(t.W0); a.s0n = F; a.s0k = 1; a.s0b = 0;
+    a.B1 = S; a.s1n = F; a.s1k = 1; a.s1b = d * F;
+    a.mode = SM_APPLY;
+    a.out = static_cast<float*>(t.O) + t0 * d; a.som = d; a.son = 1; a.sob = T * d;
+    a.out2 = t.D ? t.D + t0 * d : nullptr;
+    a.resid = (p.flags & IPTTT_FLAG_RESIDUAL) ? static_cast<const float*>(t.H) + t0 * d : nullptr;
+    a.meta = meta; a.k = s.k; a.C = s.C; a.chunk = i; a.row0 = (int)t0;
+    IP_CHECK(simt_gemm(a, s.B, st));
+
+    SimtArgs r{};
+    r.M = s.d; r.N = s.F; r.K = rows;
+    r.A = V + t0 * d; r.sam = 1; r.sak = d; r.sab = T * d;
+    r.B0 = Z + t0 * F; r.s0n = 1; r.s0k = F; r.s0b = T * F;
+    r.mode = SM_RAW;
+    r.out = raw; r.som = F; r.son = 1; r.sob = d * F;
+    IP_CHECK(simt_gemm(r, s.B, st));
+    IP_CHECK(simt_update_state(S, raw, dpart, alpha, meta, s, i, p.eta, tau, st));
+  }
+  if (t.alpha) IP_CHECK(cudaMemcpyAsync(t.alpha, alpha, (size_t)s.B * s.k * 4, cudaMemcpyDeviceToDevice, st));
+  if (t.Sfinal) IP_CHECK(state_export(false, S, t.Sfinal, s, st));
+  if (ss) IP_CHECK(stream_advance(ss->pos, ss->cont, s.B, s.T, st));
+  return IPTTT_OK;
+}
+
+ipttt_status check_tensor(const void* ptr) {
+  if (!ptr) return IPTTT_ERR_ARG;
+  if (!aligned(ptr, 16)) return IPTTT_ERR_ALIGN;
+  return IPTTT_OK;
+}
+
+ipttt_status run(const ipttt_params* pp, const Tensors& t, void* workspace, size_t ws_bytes, void* state,
+                 void* stream) {
+  ipttt_status rc = check_params(pp);
+  if (rc != IPTTT_OK) return rc;
+  const ipttt_params& p = *pp;
+  const bool core = t.Zin != nullptr;
+  if (core && (p.flags & IPTTT_FLAG_RESIDUAL)) return IPTTT_ERR_ARG;
+  if ((p.flags & IPTTT_FLAG_RESIDUAL) && t.O == t.H) return IPTTT_ERR_ARG;
+  const void* must[] = {core ? t.Zin : t.H, core ? t.Vin : t.X0, core ? t.W0 : t.Wg, core ? t.W0 : t.Wu, t.W0,
+                        core ? t.W0 : t.cw, core ? t.W0 : t.Wt, t.O};
+  for (const void* q : must)
+    if ((rc = check_tensor(q)) != IPTTT_OK) return rc;
+  const void* optional[] = {t.D, t.Sfinal, t.alpha, t.Zout, t.Vout};
+  for (const void* q : optional)
+    if (q && !aligned(q, 16)) return IPTTT_ERR_ALIGN;
+  if (t.n_doc < 0 || (t.n_doc > 0 && !t.doc)) return IPTTT_ERR_ARG;
+  if (t.doc && !aligned(t.doc, 4)) return IPTTT_ERR_ALIGN;
+  const Layout L = layout_of(p);
+  if (!workspace || ws_bytes < L.total) return IPTTT_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return IPTTT_ERR_ALIGN;
+  if (state && !aligned(state, 256)) return IPTTT_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((rc = device_info(&di)) != IPTTT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  StreamState ss;
+  StreamState* ssp = nullptr;
+  if (state) {
+    ss = state_of(p, state);
+    ssp = &ss;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  rc = is_bf16(p) ? run_bf16(p, t, ws, L, ssp, di, st) : run_f32(p, t, ws, L, ssp, di, st);
+  if (rc == IPTTT_OK && cudaPeekAtLastError() != cudaSuccess) rc = IPTTT_ERR_CUDA;
+  return rc;
+}
+
+}  // namespace
+}  // namespace ipttt
+
+using namespace ipttt;
+
+extern "C" {
+
+size_t ipttt_workspace_size(const ipttt_params* p) {
+  if (check_params(p) != IPTTT_OK) return 0;
+  return layout_of(*p).total;
+}
+
+ipttt_status ipttt_forward(const ipttt_params* p, const void* H, const void* X0, const void* Wgate, const void* Wup,
+                           const void* Wdown0, const void* conv_w, const void* Wtarget, const int32_t* doc_starts,
+                           int32_t n_doc_starts, void* O, void* workspace, size_t workspace_bytes, void* stream) {
+  Tensors t{H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, nullptr, nullptr, doc_starts, n_doc_starts, O,
+            nullptr, nullptr, nullptr, nullptr, nullptr};
+  return run(p, t, workspace, workspace_bytes, nullptr, stream);
+}
+
+ipttt_status ipttt_forward_ex(const ipttt_params* p, const void* H, const void* X0, const void* Wgate,
+                              const void* Wup, const void* Wdown0, const void* conv_w, const void* Wtarget,
+                              const int32_t* doc_starts, int32_t n_doc_starts, void* O, float* D_opt,
+                              float* S_final_opt, float* alpha_opt, void* Z_opt, void* V_opt, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  Tensors t{H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, nullptr, nullptr, doc_starts, n_doc_starts, O,
+            D_opt, S_final_opt, alpha_opt, Z_opt, V_opt};
+  return run(p, t, workspace, workspace_bytes, nullptr, stream);
+}
+
+ipttt_status ipttt_core(const ipttt_params* p, const void* Z, const void* V, const void* Wdown0,
+                        const int32_t* doc_starts, int32_t n_doc_starts, void* O, float* D_opt, float* S_final_opt,
+                        float* alpha_opt, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Z || !V) return IPTTT_ERR_ARG;
+  Tensors t{nullptr, nullptr, nullptr, nullptr, Wdown0, nullptr, nullptr, Z, V, doc_starts, n_doc_starts, O,
+            D_opt, S_final_opt, alpha_opt, nullptr, nullptr};
+  return run(p, t, workspace, workspace_bytes, nullptr, stream);
+}
+
+size_t ipttt_stream_state_size(const ipttt_params* p) {
+  if (check_params(p) != IPTTT_OK) return 0;
+  return state_bytes(*p);
+}
+
+ipttt_status ipttt_stream_reset(const ipttt_params* p, void* state, void* stream) {
+  ipttt_status rc = check_params(p);
+  if (rc != IPTTT_OK) return rc;
+  if (!state) return IPTTT_ERR_ARG;
+  if (!aligned(state, 256)) return IPTTT_ERR_ALIGN;
+  return cuda_status(cudaMemsetAsync(state, 0, state_bytes(*p), static_cast<cudaStream_t>(stream)));
+}
+
+ipttt_status ipttt_stream_forward(const ipttt_params* p, void* state, const void* H, const void* X0,
+                                  const void* Wgate, const void* Wup, const void* Wdown0, const void* conv_w,
+                                  const void* Wtarget, const int32_t* doc_starts, int32_t n_doc_starts, void* O,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (!state) return IPTTT_ERR_ARG;
+  Tensors t{H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, nullptr, nullptr, doc_starts, n_doc_starts, O,
+            nullptr, nullptr, nullptr, nullptr, nullptr};
+  return run(p, t, workspace, workspace_bytes, state, stream);
+}
+
+ipttt_status ipttt_stream_export(const ipttt_params* p, const void* state, float* S_out, void* stream) {
+  ipttt_status rc = check_params(p);
+  if (rc != IPTTT_OK) return rc;
+  if (!state || !S_out) return IPTTT_ERR_ARG;
+  if (!aligned(state, 256) || !aligned(S_out, 16)) return IPTTT_ERR_ALIGN;
+  const StreamState ss = state_of(*p, const_cast<void*>(state));
+  return cuda_status(aux::state_export(is_bf16(*p), ss.S, S_out, shape_of(*p), static_cast<cudaStream_t>(stream)));
+}
+
+ipttt_status ipttt_get_status(void* stream) {
+  DeviceInfo* di = nullptr;
+  ipttt_status rc = device_info(&di);
+  if (rc != IPTTT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return IPTTT_ERR_CUDA;
+  if (cudaMemcpyAsync(&v, di->status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return IPTTT_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyAsync(di->status, &zero, sizeof(int), cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return IPTTT_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return IPTTT_ERR_CUDA;
+  return static_cast<ipttt_status>(v);
+}
+
+const char* ipttt_strerror(ipttt_status s) {
+  switch (s) {
+    case IPTTT_OK: return "ok";
+    case IPTTT_ERR_ARG: return "invalid argument";
+    case IPTTT_ERR_SHAPE: return "inconsistent or oversized shape";
+    case IPTTT_ERR_ALIGN: return "misaligned pointer";
+    case IPTTT_ERR_DTYPE: return "unknown dtype";
+    case IPTTT_ERR_UNSUPPORTED: return "shape not supported by the bf16 tensor-core path";
+    case IPTTT_ERR_CUDA: return "CUDA error";
+    case IPTTT_ERR_TIMEOUT: return "a device-side bounded wait gave up";
+    case IPTTT_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+const char* ipttt_version(void) { return "0.1.0"; }
+
+void ipttt_profile_enable(int on) { g_profile_on.store(on ? 1 : 0); }
+
+int ipttt_profile_read(double* ms, uint64_t* launches, int n_phases) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  for (auto& pd : g_prof.pending) {
+    float e = 0.0f;
+    if (cudaEventSynchronize(pd.b) == cudaSuccess && cudaEventElapsedTime(&e, pd.a, pd.b) == cudaSuccess) {
+      g_prof.ms[pd.phase] += e;
+      g_prof.launches[pd.phase] += pd.launches;
+    }
+    g_prof.pool.push_back(pd.a);
+    g_prof.pool.push_back(pd.b);
+  }
+  g_prof.pending.clear();
+  const int n = n_phases < kPhases ? n_phases : kPhases;
+  for (int i = 0; i < n; ++i) {
+    if (ms) ms[i] = g_prof.ms[i];
+    if (launches) launches[i] = g_prof.launches[i];
+    g_prof.ms[i] = 0.0;
+    g_prof.launches[i] = 0;
+  }
+  return n < 0 ? 0 : n;
+}
+
+uint64_t ipttt_kernel_launches(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,366 @@
+// Non-tensor-core kernels of libipttt: document/chunk metadata, the masked
+// depthwise conv of the LM-aligned target, the clip factor, state layout
+// conversions, and the all-fp32 (SIMT) path.
+//
+// Sources: cloud.tencent.com "榨干MLP的剩余价值", 详细步骤 3 (depthwise conv of
+// kernel 5 over the token embeddings, no look past the chunk) and 4 (Frobenius
+// clip); iplexlaw.co.kr review of arXiv 2604.06169, §6 (chunk and document
+// boundaries, fast weight reset per document); lijianxiong.blog notes
+// "In-Place Test-Time Training", 方法 (gated MLP, apply/update, Hebbian rule).
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "aux_kernels.h"
+#include "common.cuh"
+
+namespace ipttt {
+namespace aux {
+
+constexpr int kTaps = 5;
+
+// ------------------------------------------------------------------ metadata
+__global__ void k_fill_u8(uint8_t* p, size_t n, uint8_t v) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    p[i] = v;
+}
+
+// flags[b*T + t] = 1 at every document start.  A row start is a start unless the
+// row continues a document from an earlier streaming piece (row_cont[b] != 0).
+__global__ void k_mark_starts(uint8_t* flags, int B, int T, const int32_t* ds, int n, const int32_t* row_cont,
+                              int* status) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const long long g = ds[i];
+    if (g < 0 || g >= (long long)B * T || (i > 0 && (long long)ds[i - 1] >= g))
+      set_status(status, IPTTT_ERR_ARG);
+    else
+      flags[g] = 1;
+  }
+  if (i < B && (row_cont == nullptr || row_cont[i] == 0)) flags[(size_t)i * T] = 1;
+}
+
+__global__ void k_chunk_meta(const uint8_t* flags, ChunkMeta* meta, int B, int T, int C, int k) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B * k) return;
+  const int b = i / k, c = i % k;
+  const int s = c * C, e = min(s + C, T);
+  const uint8_t* f = flags + (size_t)b * T;
+  int first_end = e, last_start = s, any = 0;
+  for (int t = s; t < e; ++t) {
+    if (f[t]) {
+      any = 1;
+      last_start = t;
+      if (t > s && first_end == e) first_end = t;
+    }
+  }
+  ChunkMeta m;
+  m.first_end = first_end;
+  m.last_start = last_start;
+  m.cont = f[s] ? 0 : 1;
+  m.has_start = any;
+  meta[i] = m;
+}
+
+cudaError_t build_meta(uint8_t* flags, ChunkMeta* meta, const Shape& s, const int32_t* doc_starts, int n_doc,
+                       const int32_t* row_cont, int* status, cudaStream_t st) {
+  const size_t n = (size_t)s.B * s.T;
+  k_fill_u8<<<(unsigned)std::min<size_t>((n + 255) / 256, 4096), 256, 0, st>>>(flags, n, 0);
+  const int nt = std::max(n_doc, s.B);
+  k_mark_starts<<<(nt + 255) / 256, 256, 0, st>>>(flags, s.B, s.T, doc_starts, n_doc, row_cont, status);
+  k_chunk_meta<<<(s.B * s.k + 127) / 128, 128, 0, st>>>(flags, meta, s.B, s.T, s.C, s.k);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ conv
+// U[b,t,c] = sum_o conv_w[c,o] X0[b,t+o,c]; tap o is dropped (and every later
+// one) once t+o reaches the chunk end or T, or a document starts at t+o.
+template <typename T, int VEC>
+__global__ void k_conv(const T* __restrict__ X0, const T* __restrict__ cw, const uint8_t* __restrict__ flags,
+                       T* __restrict__ U, int B, int Tn, int d, int C) {
+  const int groups = d / VEC;
+  const size_t total = (size_t)B * Tn * groups;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int g = (int)(idx % groups);
+    const size_t bt = idx / groups;
+    const int t = (int)(bt % Tn);
+    const int b = (int)(bt / Tn);
+    const int cend = min((t / C + 1) * C, Tn);
+    const uint8_t* f = flags + (size_t)b * Tn;
+    float acc[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
+#pragma unroll
+    for (int o = 0; o < kTaps; ++o) {
+      const int src = t + o;
+      if (src >= cend || (o > 0 && f[src])) break;
+      const T* x = X0 + ((size_t)b * Tn + src) * d + (size_t)g * VEC;
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] = fmaf(to_f<T>(cw[(size_t)(g * VEC + v) * kTaps + o]), to_f<T>(x[v]), acc[v]);
+    }
+    T* u = U + ((size_t)b * Tn + t) * d + (size_t)g * VEC;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) u[v] = from_f<T>(acc[v]);
+  }
+}
+
+cudaError_t conv_target(int dtype, const void* X0, const void* cw, const uint8_t* flags, void* U, const Shape& s,
+                        cudaStream_t st) {
+  const int blocks = 148 * 8;
+  if (dtype == IPTTT_BF16 && s.d % 8 == 0)
+    k_conv<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)X0, (const __nv_bfloat16*)cw, flags,
+                                                       (__nv_bfloat16*)U, s.B, s.T, s.d, s.C);
+  else if (dtype == IPTTT_BF16)
+    k_conv<__nv_bfloat16, 1><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)X0, (const __nv_bfloat16*)cw, flags,
+                                                       (__nv_bfloat16*)U, s.B, s.T, s.d, s.C);
+  else if (s.d % 4 == 0)
+    k_conv<float, 4><<<blocks, 256, 0, st>>>((const float*)X0, (const float*)cw, flags, (float*)U, s.B, s.T, s.d,
+                                             s.C);
+  else
+    k_conv<float, 1><<<blocks, 256, 0, st>>>((const float*)X0, (const float*)cw, flags, (float*)U, s.B, s.T, s.d,
+                                             s.C);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ clip factor
+__device__ __forceinline__ float clip_alpha(double sumsq, float eta, float tau) {
+  const float nrm = eta * (float)sqrt(fmax(sumsq, 0.0));
+  return (tau > 0.0f && isfinite(tau) && nrm > tau) ? tau / nrm : 1.0f;
+}
+
+// alpha[i] from the per-tile-pair Gram partials of ||V^T Z||_F^2, summed in a
+// fixed order.
+__global__ void k_alpha_from_partials(const float* partials, float* alpha, int n, int npairs, float eta,
+                                      float tau) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  double s = 0.0;
+  for (int q = 0; q < npairs; ++q) s += (double)partials[(size_t)i * npairs + q];
+  alpha[i] = clip_alpha(s, eta, tau);
+}
+
+cudaError_t alpha_from_partials(const float* partials, float* alpha, int n, int npairs, float eta, float tau,
+                                cudaStream_t st) {
+  k_alpha_from_partials<<<(n + 127) / 128, 128, 0, st>>>(partials, alpha, n, npairs, eta, tau);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ state layouts
+// The bf16 path keeps S [d][F] (fp32) as 128 x 256 tiles, tile (mt, nt) at
+// ((mt * F/256) + nt) * 32768, element (r, c) of a tile at ((c/4) * 128 + r) * 4 + c%4.
+__device__ __forceinline__ size_t blocked_index(int r, int c, int F) {
+  const size_t tile = (size_t)(r >> 7) * (F >> 8) + (c >> 8);
+  return tile * 32768 + ((size_t)((c & 255) >> 2) * 128 + (r & 127)) * 4 + (c & 3);
+}
+
+__global__ void k_blocked_to_rowmajor(const float* Sb, float* out, int B, int d, int F) {
+  const size_t total = (size_t)B * d * F;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int c = (int)(i % F);
+    const size_t br = i / F;
+    const int r = (int)(br % d);
+    const size_t b = br / d;
+    out[i] = Sb[b * d * F + blocked_index(r, c, F)];
+  }
+}
+
+__global__ void k_blocked_to_bf16(const float* Sb, __nv_bfloat16* out, int B, int d, int F) {
+  const size_t total = (size_t)B * d * F;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int c = (int)(i % F);
+    const size_t br = i / F;
+    const int r = (int)(br % d);
+    const size_t b = br / d;
+    out[i] = __float2bfloat16_rn(Sb[b * d * F + blocked_index(r, c, F)]);
+  }
+}
+
+cudaError_t state_export(bool blocked, const float* S, float* out, const Shape& s, cudaStream_t st) {
+  const size_t n = (size_t)s.B * s.d * s.F;
+  if (!blocked) return cudaMemcpyAsync(out, S, n * sizeof(float), cudaMemcpyDeviceToDevice, st);
+  k_blocked_to_rowmajor<<<148 * 8, 256, 0, st>>>(S, out, s.B, s.d, s.F);
+  return cudaGetLastError();
+}
+
+cudaError_t state_snapshot(const float* Sb, void* snap_bf16, const Shape& s, cudaStream_t st) {
+  k_blocked_to_bf16<<<148 * 8, 256, 0, st>>>(Sb, (__nv_bfloat16*)snap_bf16, s.B, s.d, s.F);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ fp32 SIMT path
+// C(m,n) = sum_k A(m,k) B(n,k) with arbitrary element strides, 64 x 64 tiles,
+// 16 x 16 threads of 4 x 4 outputs, and up to two B operands sharing A.
+constexpr int ST = 64, SK = 16;
+
+__global__ void __launch_bounds__(256) k_simt_gemm(SimtArgs a) {
+  __shared__ float As[SK][ST + 1];
+  __shared__ float Bs0[SK][ST + 1];
+  __shared__ float Bs1[SK][ST + 1];
+  const int b = blockIdx.z;
+  const int m0 = blockIdx.y * ST, n0 = blockIdx.x * ST;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  const float* A = a.A + b * a.sab;
+  const float* B0 = a.B0 + b * a.s0b;
+  const float* B1 = a.B1 ? a.B1 + b * a.s1b : nullptr;
+  float acc0[4][4] = {}, acc1[4][4] = {};
+  for (int k0 = 0; k0 < a.K; k0 += SK) {
+    for (int e = threadIdx.x; e < ST * SK; e += 256) {
+      const int mm = e / SK, kk = e % SK;
+      const int gm = m0 + mm, gk = k0 + kk;
+      As[kk][mm] = (gm < a.M && gk < a.K) ? A[gm * a.sam + gk * a.sak] : 0.0f;
+      const int gn = n0 + mm;
+      Bs0[kk][mm] = (gn < a.N && gk < a.K) ? B0[gn * a.s0n + gk * a.s0k] : 0.0f;
+      if (B1) Bs1[kk][mm] = (gn < a.N && gk < a.K) ? B1[gn * a.s1n + gk * a.s1k] : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < SK; ++kk) {
+      float av[4], bv0[4], bv1[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        av[i] = As[kk][ty * 4 + i];
+        bv0[i] = Bs0[kk][tx * 4 + i];
+        bv1[i] = B1 ? Bs1[kk][tx * 4 + i] : 0.0f;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          acc0[i][jj] = fmaf(av[i], bv0[jj], acc0[i][jj]);
+          acc1[i][jj] = fmaf(av[i], bv1[jj], acc1[i][jj]);
+        }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= a.M) continue;
+    const int t = a.row0 + m;  // token index for the token-row modes
+    bool keep_row = true;
+    if (a.mode == SM_V) {
+      const int c = t / a.C;
+      keep_row = t >= a.meta[(size_t)b * a.k + c].last_start;
+    } else if (a.mode == SM_APPLY) {
+      const ChunkMeta cm = a.meta[(size_t)b * a.k + a.chunk];
+      keep_row = cm.cont && t < cm.first_end;
+    }
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int n = n0 + tx * 4 + jj;
+      if (n >= a.N) continue;
+      float* o = a.out + b * a.sob + (long long)m * a.som + (long long)n * a.son;
+      switch (a.mode) {
+        case SM_Z: *o = silu_precise(acc0[i][jj]) * acc1[i][jj]; break;
+        case SM_V: *o = keep_row ? acc0[i][jj] : 0.0f; break;
+        case SM_RAW: *o = acc0[i][jj]; break;
+        case SM_APPLY: {
+          const float dv = keep_row ? acc1[i][jj] : 0.0f;
+          *o = acc0[i][jj] + dv +
+               (a.resid ? a.resid[b * a.sob + (long long)m * a.som + (long long)n * a.son] : 0.0f);
+          if (a.out2) a.out2[b * a.sob + (long long)m * a.som + (long long)n * a.son] = dv;
+        } break;
+      }
+    }
+  }
+}
+
+cudaError_t simt_gemm(const SimtArgs& a, int batches, cudaStream_t st) {
+  dim3 grid((a.N + ST - 1) / ST, (a.M + ST - 1) / ST, batches);
+  k_simt_gemm<<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+// Sum of squares of each row-b slice [n] of x, as per-block partials [B][nblk].
+__global__ void k_sumsq_partials(const float* x, size_t n, double* part, int nblk) {
+  __shared__ double sh[256];
+  const int b = blockIdx.y;
+  const float* xb = x + b * n;
+  double s = 0.0;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)nblk * blockDim.x)
+    s += (double)xb[i] * (double)xb[i];
+  sh[threadIdx.x] = s;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) sh[threadIdx.x] += sh[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) part[(size_t)b * nblk + blockIdx.x] = sh[0];
+}
+
+__global__ void k_alpha_direct(const double* part, int nblk, float* alpha, int B, int k, int chunk, float eta,
+                               float tau) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  double s = 0.0;
+  for (int q = 0; q < nblk; ++q) s += part[(size_t)b * nblk + q];
+  alpha[(size_t)b * k + chunk] = clip_alpha(s, eta, tau);
+}
+
+// S = (chunk holds a document start ? 0 : S) + alpha * eta * raw, per row b.
+__global__ void k_state_update(float* S, const float* raw, size_t n, const float* alpha, const ChunkMeta* meta,
+                               int k, int chunk, float eta) {
+  const int b = blockIdx.y;
+  const float ae = alpha[(size_t)b * k + chunk] * eta;
+  const bool keep = !meta[(size_t)b * k + chunk].has_start;
+  float* Sb = S + b * n;
+  const float* rb = raw + b * n;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    Sb[i] = fmaf(ae, rb[i], keep ? Sb[i] : 0.0f);
+}
+
+cudaError_t simt_update_state(float* S, const float* raw, double* part, float* alpha, const ChunkMeta* meta,
+                              const Shape& s, int chunk, float eta, float tau, cudaStream_t st) {
+  const size_t n = (size_t)s.d * s.F;
+  const int nblk = 64;
+  k_sumsq_partials<<<dim3(nblk, s.B), 256, 0, st>>>(raw, n, part, nblk);
+  k_alpha_direct<<<(s.B + 63) / 64, 64, 0, st>>>(part, nblk, alpha, s.B, s.k, chunk, eta, tau);
+  k_state_update<<<dim3(256, s.B), 256, 0, st>>>(S, raw, n, alpha, meta, s.k, chunk, eta);
+  return cudaGetLastError();
+}
+
+}  // namespace aux
+}  // namespace ipttt
+
+namespace ipttt {
+namespace aux {
+
+// out[b,t,:] = in[b,t,:] on rows inside their chunk's last document segment, 0 elsewhere.
+template <typename T>
+__global__ void k_mask_last_segment(const T* in, T* out, const ChunkMeta* meta, int B, int Tn, int d, int C, int k) {
+  const size_t total = (size_t)B * Tn * d;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t bt = i / d;
+    const int t = (int)(bt % Tn);
+    const int b = (int)(bt / Tn);
+    const bool keep = t >= meta[(size_t)b * k + t / C].last_start;
+    out[i] = keep ? in[i] : from_f<T>(0.0f);
+  }
+}
+
+cudaError_t mask_last_segment(int dtype, const void* in, void* out, const ChunkMeta* meta, const Shape& s,
+                              cudaStream_t st) {
+  if (dtype == IPTTT_BF16)
+    k_mask_last_segment<__nv_bfloat16><<<148 * 8, 256, 0, st>>>((const __nv_bfloat16*)in, (__nv_bfloat16*)out, meta,
+                                                                 s.B, s.T, s.d, s.C, s.k);
+  else
+    k_mask_last_segment<float><<<148 * 8, 256, 0, st>>>((const float*)in, (float*)out, meta, s.B, s.T, s.d, s.C, s.k);
+  return cudaGetLastError();
+}
+
+// Streaming bookkeeping: every row has now consumed `T` more tokens.
+__global__ void k_stream_advance(long long* pos, int32_t* cont, int B, int T) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) {
+    pos[b] += T;
+    cont[b] = 1;
+  }
+}
+
+cudaError_t stream_advance(long long* pos, int32_t* cont, int B, int T, cudaStream_t st) {
+  k_stream_advance<<<(B + 127) / 128, 128, 0, st>>>(pos, cont, B, T);
+  return cudaGetLastError();
+}
+
+}  // namespace aux
+}  // namespace ipttt

@@ -1,0 +1,57 @@
+// Internal interface of the non-tensor-core kernels (aux_kernels.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace ipttt {
+namespace aux {
+
+cudaError_t build_meta(uint8_t* flags, ChunkMeta* meta, const Shape& s, const int32_t* doc_starts, int n_doc,
+                       const int32_t* row_cont, int* status, cudaStream_t st);
+cudaError_t conv_target(int dtype, const void* X0, const void* cw, const uint8_t* flags, void* U, const Shape& s,
+                        cudaStream_t st);
+cudaError_t alpha_from_partials(const float* partials, float* alpha, int n, int npairs, float eta, float tau,
+                                cudaStream_t st);
+cudaError_t state_export(bool blocked, const float* S, float* out, const Shape& s, cudaStream_t st);
+cudaError_t state_snapshot(const float* Sb, void* snap_bf16, const Shape& s, cudaStream_t st);
+
+enum SimtMode { SM_Z = 0, SM_V = 1, SM_RAW = 2, SM_APPLY = 3 };
+
+// Strided fp32 GEMM for the all-fp32 path: out(m,n) = epilogue(sum_k A(m,k) B0(n,k),
+// sum_k A(m,k) B1(n,k)), one batch row b per blockIdx.z.
+struct SimtArgs {
+  int M, N, K;
+  const float* A;
+  long long sam, sak, sab;
+  const float* B0;
+  long long s0n, s0k, s0b;
+  const float* B1;  // may be null
+  long long s1n, s1k, s1b;
+  int mode;
+  float* out;
+  long long som, son, sob;
+  float* out2;      // SM_APPLY: optional D
+  const float* resid;  // SM_APPLY: optional residual added to out (same strides as out)
+  const ChunkMeta* meta;
+  int k, C, chunk;
+  int row0;         // token index of m = 0 (SM_V, SM_APPLY)
+};
+
+cudaError_t simt_gemm(const SimtArgs& a, int batches, cudaStream_t st);
+cudaError_t simt_update_state(float* S, const float* raw, double* part, float* alpha, const ChunkMeta* meta,
+                              const Shape& s, int chunk, float eta, float tau, cudaStream_t st);
+
+}  // namespace aux
+}  // namespace ipttt
+
+namespace ipttt {
+namespace aux {
+cudaError_t mask_last_segment(int dtype, const void* in, void* out, const ChunkMeta* meta, const Shape& s,
+                              cudaStream_t st);
+cudaError_t stream_advance(long long* pos, int32_t* cont, int B, int T, cudaStream_t st);
+}  // namespace aux
+}  // namespace ipttt

@@ -1,0 +1,617 @@
+// Tensor-core (tcgen05) kernels of the bf16 path of the In-Place TTT MLP layer.
+//
+// One persistent, warp-specialised kernel template serves every contraction of
+// the layer.  Per CTA (one per SM): warp 0 issues TMA loads into a ring of
+// shared-memory stages, warp 1 allocates TMEM and one thread of it issues
+// tcgen05.mma into a double-buffered fp32 accumulator (2 x 256 TMEM columns),
+// and 8 epilogue warps drain finished accumulators with tcgen05.ld.  Tiles are
+// handed out statically: tile = blockIdx.x + j * gridDim.x, and every role
+// decodes the same tile index into the same Job.
+//
+// Families (template parameter FAM):
+//   FAM_ZV   gate/up GEMM with the SiLU-product epilogue, Z = SiLU(H Wg^T) * (H Wu^T)
+//            [notes "In-Place Test-Time Training", 方法 › 原地自适应], and the
+//            target GEMM V = U Wtarget with rows outside each chunk's last document
+//            segment zeroed [notes, 对齐语言模型的目标函数].
+//   FAM_GRAM per-chunk Gram pass: ||V_L^T Z_L||_F^2 = sum_{s,t}(V V^T)_{st}(Z Z^T)_{st},
+//            written as deterministic partial sums per 128x128 tile pair; the clip
+//            factor follows [cloud.tencent.com "榨干MLP的剩余价值", 详细步骤 4].
+//   FAM_SCAN one chunk i of the scan: "apply" tiles O_i = Z_i W0^T + M_i (Z_i S_i^T)
+//            (both products side by side in one N=256 accumulator, S_i read from a
+//            bf16 snapshot) and "delta" tiles S_{i+1} = keep_i S_i + alpha_i eta
+//            V_i^T Z_i on the fp32 state [notes, 步骤一/步骤二 and 工程实现; iplexlaw.co.kr
+//            review §3 apply-before-update, §6 exclusive scan and document reset].
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "tc.cuh"
+#include "tc_kernels.h"
+
+namespace ipttt {
+namespace tck {
+
+using namespace ipttt::tc;
+
+constexpr int BM = 128;                 // accumulator rows (TMEM lanes)
+constexpr int BK = 64;                  // K elements per stage (one 128-byte swizzle row)
+constexpr int A_BYTES = BM * BK * 2;    // 16 KB
+constexpr int B_BYTES = 256 * BK * 2;   // 32 KB (up to N = 256)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int NTHREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int ACC_COLS = 256;           // per accumulator buffer
+constexpr int SNAP_STAGE_BYTES = 32 * 128;  // one 32-row x 64-col bf16 box
+
+enum Kind { K_GATEUP = 0, K_VHAT = 1, K_GRAM = 2, K_APPLY = 3, K_DELTA = 4 };
+
+template <int FAM> struct Cfg;
+template <> struct Cfg<FAM_ZV> { static constexpr int STAGES = 4; static constexpr int EPI_BYTES = 0; };
+template <> struct Cfg<FAM_GRAM> { static constexpr int STAGES = 4; static constexpr int EPI_BYTES = 0; };
+template <> struct Cfg<FAM_SCAN> {
+  static constexpr int STAGES = 3;
+  static constexpr int EPI_BYTES = NUM_EPI_WARPS * 2 * SNAP_STAGE_BYTES;  // 64 KB
+};
+
+template <int FAM>
+constexpr int smem_bytes() {
+  return 1024 /*alignment slack*/ + Cfg<FAM>::STAGES * STAGE_BYTES + Cfg<FAM>::EPI_BYTES + 256 /*barriers*/;
+}
+
+struct Job {
+  int kind;
+  int b;
+  int m0, n0;     // tile origin: rows / columns of the accumulator in the operand index spaces
+  int t0;         // first token of the tile's chunk (GRAM, SCAN)
+  int chunk;
+  int pair;       // GRAM: tile pair index
+  int nseg;
+  int kb0[2], kb1[2];
+  int acc_col[2];
+  int n_mma;
+  int nsrc;       // APPLY: 1 = W0 only, 2 = W0 and the state snapshot
+  uint32_t tx;    // bytes per stage
+  bool a_mn, b_mn;
+};
+
+__device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------------ decoding
+__device__ __forceinline__ void decode_zv(const TcParams& p, int tile, Job& j) {
+  const int tiles_m = cdiv(p.T, BM);
+  const int N = p.kind == K_GATEUP ? p.F : p.d;
+  const int tiles_n = N / 128;
+  const int M_all = p.B * tiles_m;
+  constexpr int G = 16;  // m-tiles per raster group
+  const int per_group = G * tiles_n;
+  const int g = tile / per_group, r = tile % per_group;
+  const int m_first = g * G;
+  const int gm = min(G, M_all - m_first);
+  const int mm = m_first + r % gm;
+  const int nt = r / gm;
+  j.kind = p.kind;
+  j.b = mm / tiles_m;
+  j.m0 = (mm % tiles_m) * BM;
+  j.n0 = nt * 128;
+  j.t0 = 0;
+  j.chunk = 0;
+  j.pair = 0;
+  j.nseg = 1;
+  j.kb0[0] = 0;
+  j.kb1[0] = p.d / BK;
+  j.acc_col[0] = 0;
+  j.nsrc = 1;
+  if (p.kind == K_GATEUP) {
+    j.n_mma = 256;
+    j.tx = A_BYTES + 2 * 128 * BK * 2;
+    j.a_mn = false;
+    j.b_mn = false;
+  } else {
+    j.n_mma = 128;
+    j.tx = A_BYTES + 128 * BK * 2;
+    j.a_mn = false;
+    j.b_mn = true;
+  }
+}
+
+__device__ __forceinline__ void decode_gram(const TcParams& p, int tile, Job& j) {
+  const int per_row = p.k * p.npairs;
+  j.kind = K_GRAM;
+  j.b = tile / per_row;
+  const int r = tile % per_row;
+  j.chunk = r / p.npairs;
+  j.pair = r % p.npairs;
+  int ti = 0, rem = j.pair;
+  while (rem >= p.ct - ti) { rem -= p.ct - ti; ++ti; }
+  j.m0 = ti * BM;
+  j.n0 = (ti + rem) * BM;
+  j.t0 = j.chunk * p.C;
+  j.nseg = 2;
+  j.kb0[0] = 0; j.kb1[0] = p.F / BK; j.acc_col[0] = 0;     // Z Z^T
+  j.kb0[1] = 0; j.kb1[1] = p.d / BK; j.acc_col[1] = 128;   // V V^T
+  j.n_mma = 128;
+  j.nsrc = 1;
+  j.tx = A_BYTES + 128 * BK * 2;
+  j.a_mn = false;
+  j.b_mn = false;
+}
+
+__device__ __forceinline__ void decode_scan(const TcParams& p, int tile, Job& j) {
+  j.chunk = p.chunk;
+  j.t0 = p.chunk * p.C;
+  j.pair = 0;
+  j.nseg = 1;
+  j.acc_col[0] = 0;
+  const ChunkMeta* mrow;
+  if (tile < p.n_apply) {
+    const int tiles_n = p.d / 128;
+    const int per_row = p.ct * tiles_n;
+    j.kind = K_APPLY;
+    j.b = tile / per_row;
+    const int r = tile % per_row;
+    j.m0 = (r / tiles_n) * BM;      // row offset inside the chunk
+    j.n0 = (r % tiles_n) * 128;     // output column (d index)
+    mrow = p.meta + (size_t)j.b * p.k + p.chunk;
+    j.nsrc = mrow->cont ? 2 : 1;
+    j.kb0[0] = 0;
+    j.kb1[0] = p.F / BK;
+    j.n_mma = 128 * j.nsrc;
+    j.tx = A_BYTES + j.nsrc * 128 * BK * 2;
+    j.a_mn = false;
+    j.b_mn = false;
+  } else {
+    const int t = tile - p.n_apply;
+    const int tiles_n = p.F / 256;
+    const int per_row = (p.d / 128) * tiles_n;
+    j.kind = K_DELTA;
+    j.b = t / per_row;
+    const int r = t % per_row;
+    j.m0 = (r / tiles_n) * 128;     // d index
+    j.n0 = (r % tiles_n) * 256;     // F index
+    mrow = p.meta + (size_t)j.b * p.k + p.chunk;
+    const int rows = min(p.C, p.T - j.t0);
+    j.kb0[0] = (mrow->last_start - j.t0) / BK;
+    j.kb1[0] = cdiv(rows, BK);
+    j.n_mma = 256;
+    j.nsrc = 1;
+    j.tx = A_BYTES + B_BYTES;
+    j.a_mn = true;
+    j.b_mn = true;
+  }
+}
+
+template <int FAM>
+__device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
+  if constexpr (FAM == FAM_ZV) decode_zv(p, tile, j);
+  else if constexpr (FAM == FAM_GRAM) decode_gram(p, tile, j);
+  else decode_scan(p, tile, j);
+}
+
+// ------------------------------------------------------------------ producer
+template <int FAM>
+__device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int seg, int kb, uint8_t* sa,
+                                            uint8_t* sb, uint64_t* bar) {
+  const int kx = kb * BK;
+  if constexpr (FAM == FAM_ZV) {
+    if (j.kind == K_GATEUP) {
+      tma_load_3d(sa, &p.map[0], bar, kx, j.m0, j.b);              // H rows
+      tma_load_3d(sb, &p.map[1], bar, kx, j.n0, 0);                   // Wgate rows
+      tma_load_3d(sb + 128 * BK * 2, &p.map[2], bar, kx, j.n0, 0);    // Wup rows
+    } else {
+      tma_load_3d(sa, &p.map[0], bar, kx, j.m0, j.b);              // U rows
+      tma_load_3d(sb, &p.map[1], bar, j.n0, kx, 0);                   // Wtarget[k][n], n contiguous
+      tma_load_3d(sb + 64 * BK * 2, &p.map[1], bar, j.n0 + 64, kx, 0);
+    }
+  } else if constexpr (FAM == FAM_GRAM) {
+    const CUtensorMap* m = seg == 0 ? &p.map[0] : &p.map[1];       // Z or V
+    tma_load_3d(sa, m, bar, kx, j.t0 + j.m0, j.b);
+    tma_load_3d(sb, m, bar, kx, j.t0 + j.n0, j.b);
+  } else {
+    if (j.kind == K_APPLY) {
+      tma_load_3d(sa, &p.map[0], bar, kx, j.t0 + j.m0, j.b);      // Z rows of the chunk
+      tma_load_3d(sb, &p.map[1], bar, kx, j.n0, 0);                   // Wdown0 rows
+      if (j.nsrc == 2)
+        tma_load_3d(sb + 128 * BK * 2, &p.map[2], bar, kx, j.n0, p.snap_in * p.B + j.b);  // S_i rows
+    } else {
+      const int ty = j.t0 + kx;                                    // token rows = K
+      tma_load_3d(sa, &p.map[3], bar, j.m0, ty, j.b);              // V[t][d], d contiguous
+      tma_load_3d(sa + 64 * BK * 2, &p.map[3], bar, j.m0 + 64, ty, j.b);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        tma_load_3d(sb + q * 64 * BK * 2, &p.map[4], bar, j.n0 + 64 * q, ty, j.b);  // Z[t][f]
+    }
+  }
+}
+
+// ------------------------------------------------------------------ epilogues
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float* v) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+    d4[q] = w;
+  }
+}
+
+// Named barrier among the epilogue warps only.
+__device__ __forceinline__ void epi_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(NUM_EPI_WARPS * 32) : "memory");
+}
+
+template <int FAM>
+__device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, uint32_t tacc, int half, int row,
+                                              int lane, int ew, float* red, uint8_t* snap_stage,
+                                              int& snap_uses) {
+  uint32_t r0[32], r1[32];
+  float v[32];
+  if constexpr (FAM == FAM_ZV) {
+    const int t = j.m0 + row;
+    const bool valid = t < p.T;
+    if (j.kind == K_GATEUP) {
+      __nv_bfloat16* zrow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.F + j.n0;
+#pragma unroll 1
+      for (int c = half * 64; c < half * 64 + 64; c += 32) {
+        tmem_ld32(tacc + c, r0);
+        tmem_ld32(tacc + 128 + c, r1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = silu_fast(__uint_as_float(r0[i])) * __uint_as_float(r1[i]);
+        if (valid) st_bf16x32(zrow + c, v);
+      }
+    } else {
+      const int chunk = t / p.C;
+      const bool keep = valid && t >= p.meta[(size_t)j.b * p.k + min(chunk, p.k - 1)].last_start;
+      __nv_bfloat16* vrow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.d + j.n0;
+#pragma unroll 1
+      for (int c = half * 64; c < half * 64 + 64; c += 32) {
+        tmem_ld32(tacc + c, r0);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = keep ? __uint_as_float(r0[i]) : 0.0f;
+        if (valid) st_bf16x32(vrow + c, v);
+      }
+    }
+  } else if constexpr (FAM == FAM_GRAM) {
+    float s = 0.0f;
+#pragma unroll 1
+    for (int c = half * 64; c < half * 64 + 64; c += 32) {
+      tmem_ld32(tacc + c, r0);
+      tmem_ld32(tacc + 128 + c, r1);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s = fmaf(__uint_as_float(r0[i]), __uint_as_float(r1[i]), s);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) red[ew] = s;
+    epi_sync();
+    if (ew == 0 && lane == 0) {
+      float tot = 0.0f;
+      for (int w = 0; w < NUM_EPI_WARPS; ++w) tot += red[w];
+      const float wgt = j.m0 == j.n0 ? 1.0f : 2.0f;
+      p.partials[((size_t)j.b * p.k + j.chunk) * p.npairs + j.pair] = wgt * tot;
+    }
+    epi_sync();
+  } else {
+    if (j.kind == K_APPLY) {
+      const ChunkMeta m = p.meta[(size_t)j.b * p.k + j.chunk];
+      const int t = j.t0 + j.m0 + row;
+      const bool valid = t < p.T;
+      const bool carry = j.nsrc == 2 && m.cont && t < m.first_end;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.d + j.n0;
+      const __nv_bfloat16* hrow =
+          p.resid ? reinterpret_cast<const __nv_bfloat16*>(p.resid) + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
+      float* drow = p.out1 ? p.out1 + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
+#pragma unroll 1
+      for (int c = half * 64; c < half * 64 + 64; c += 32) {
+        tmem_ld32(tacc + c, r0);
+        if (j.nsrc == 2) tmem_ld32(tacc + 128 + c, r1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float dv = carry ? __uint_as_float(r1[i]) : 0.0f;
+          v[i] = __uint_as_float(r0[i]) + dv;
+          r1[i] = __float_as_uint(dv);
+        }
+        if (valid) {
+          if (hrow) {
+            const uint4* h4 = reinterpret_cast<const uint4*>(hrow + c);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 hv = h4[q];
+              const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hw[e]);
+                v[8 * q + 2 * e] += __low2float(h2);
+                v[8 * q + 2 * e + 1] += __high2float(h2);
+              }
+            }
+          }
+          st_bf16x32(orow + c, v);
+          if (drow) {
+            float4* d4 = reinterpret_cast<float4*>(drow + c);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              d4[q] = make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
+                                  __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3]));
+          }
+        }
+      }
+    } else {
+      // delta: fp32 state tile in the blocked layout [c/4][row][4] of 128 x 256.
+      const ChunkMeta m = p.meta[(size_t)j.b * p.k + j.chunk];
+      const bool keep = !m.has_start;
+      const float ae = p.alpha[(size_t)j.b * p.k + j.chunk] * p.eta;
+      float* Sb = p.S + (size_t)j.b * p.d * p.F + ((size_t)(j.m0 / 128) * (p.F / 256) + j.n0 / 256) * (128 * 256);
+#pragma unroll 1
+      for (int c = half * 128; c < half * 128 + 128; c += 64) {
+        float4 old[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const size_t idx = ((size_t)((c >> 2) + q) * 128 + row) * 4;
+          old[q] = keep ? *reinterpret_cast<const float4*>(Sb + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        tmem_ld32(tacc + c, r0);
+        tmem_ld32(tacc + c + 32, r1);
+        tmem_ld_wait();
+        uint32_t packed[32];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const uint32_t* src = q < 8 ? &r0[4 * q] : &r1[4 * (q - 8)];
+          float4 nv;
+          nv.x = fmaf(ae, __uint_as_float(src[0]), old[q].x);
+          nv.y = fmaf(ae, __uint_as_float(src[1]), old[q].y);
+          nv.z = fmaf(ae, __uint_as_float(src[2]), old[q].z);
+          nv.w = fmaf(ae, __uint_as_float(src[3]), old[q].w);
+          const size_t idx = ((size_t)((c >> 2) + q) * 128 + row) * 4;
+          *reinterpret_cast<float4*>(Sb + idx) = nv;
+          packed[2 * q] = pack_bf16(nv.x, nv.y);
+          packed[2 * q + 1] = pack_bf16(nv.z, nv.w);
+        }
+        if (p.write_snap) {
+          // Stage this warp's 32 rows x 64 columns (bf16, 128 B per row) in the
+          // 128-byte-swizzled layout of the TMA box, then store the box.
+          uint8_t* buf = snap_stage + (snap_uses & 1) * SNAP_STAGE_BYTES;
+          if (snap_uses >= 2) {
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            uint4 w = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+            *reinterpret_cast<uint4*>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) = w;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&p.map[5], buf, j.n0 + c, j.m0 + (row & ~31), p.snap_out * p.B + j.b);
+            bulk_commit();
+          }
+          ++snap_uses;
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+template <int FAM>
+__global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__ TcParams p) {
+  constexpr int STAGES = Cfg<FAM>::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  uint8_t* epi = smem + STAGES * STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi + Cfg<FAM>::EPI_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(tmem_slot + 2);  // [0] issued, [1] consumed
+  float* red = reinterpret_cast<float*>(tmem_slot + 4);              // NUM_EPI_WARPS floats
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], NUM_EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    counters[0] = counters[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    const int nmaps = FAM == FAM_SCAN ? 6 : (FAM == FAM_GRAM ? 2 : (p.kind == K_GATEUP ? 3 : 2));
+    for (int i = 0; i < nmaps; ++i) prefetch_tmap(&p.map[i]);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * ACC_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+        Job j;
+        decode<FAM>(p, tile, j);
+        for (int seg = 0; seg < j.nseg && ok; ++seg) {
+          for (int kb = j.kb0[seg]; kb < j.kb1[seg]; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) { ok = false; break; }
+            uint8_t* sa = stages + s * STAGE_BYTES;
+            mbar_arrive_expect_tx(&full[s], j.tx);
+            issue_loads<FAM>(p, j, seg, kb, sa, sa + A_BYTES, &full[s]);
+          }
+        }
+      }
+      if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
+      counters[0] = it;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++tcount) {
+        Job j;
+        decode<FAM>(p, tile, j);
+        const int buf = tcount & 1;
+        const uint32_t aph = (tcount >> 1) & 1;
+        if (!mbar_wait(&acc_empty[buf], aph ^ 1) || *abort_flag) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tacc = tmem_base + buf * ACC_COLS;
+        const uint32_t idesc = idesc_bf16(BM, j.n_mma, j.a_mn, j.b_mn);
+        for (int seg = 0; seg < j.nseg && ok; ++seg) {
+          for (int kb = j.kb0[seg]; kb < j.kb1[seg]; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!mbar_wait(&full[s], ph) || *abort_flag) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(stages + s * STAGE_BYTES);
+            const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+            for (int ks = 0; ks < BK / 16; ++ks) {
+              const uint64_t ad = j.a_mn ? sdesc_sw128(a_addr + ks * 2048, 64 * 128, 1024)
+                                         : sdesc_sw128(a_addr + ks * 32, 16, 1024);
+              const uint64_t bd = j.b_mn ? sdesc_sw128(b_addr + ks * 2048, 64 * 128, 1024)
+                                         : sdesc_sw128(b_addr + ks * 32, 16, 1024);
+              mma_bf16(tacc + j.acc_col[seg], ad, bd, idesc, (kb > j.kb0[seg] || ks > 0) ? 1u : 0u);
+            }
+            mma_commit(&empty[s]);
+          }
+        }
+        if (ok) mma_commit(&acc_full[buf]);
+      }
+      if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
+      counters[1] = it;
+      // Let every MMA issued by this thread finish before TMEM is released.
+      mma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+  } else {
+    const int ew = warp - 2;
+    const int quarter = warp & 3;      // TMEM lanes this warp may access
+    const int half = ew >> 2;          // which half of the columns this warp drains
+    const int row = quarter * 32 + lane;
+    uint8_t* snap_stage = epi + ew * 2 * SNAP_STAGE_BYTES;
+    int snap_uses = 0;
+    uint32_t tcount = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++tcount) {
+      Job j;
+      decode<FAM>(p, tile, j);
+      const int buf = tcount & 1;
+      const uint32_t aph = (tcount >> 1) & 1;
+      // Every epilogue warp leaves only through this wait, so all of them stop at
+      // the same tile and none is left waiting at the epilogue's named barrier.
+      if (!mbar_wait(&acc_full[buf], aph)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + buf * ACC_COLS + ((uint32_t)(quarter * 32) << 16);
+      epilogue_tile<FAM>(p, j, tacc, half, row, lane, ew, red, snap_stage, snap_uses);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+    if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    // Wait (bounded) for stage loads that were issued but never consumed, so no
+    // TMA write lands in shared memory after the block has exited.
+    for (uint32_t it = counters[1]; it < counters[0]; ++it)
+      mbar_wait(&full[it % STAGES], (it / STAGES) & 1);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * ACC_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// bf16 tensor [outer][rows][inner] (outer may be 1), box {box_inner, box_rows, 1},
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+                   uint32_t box_inner, uint32_t box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {inner, rows, outer};
+  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int FAM>
+static cudaError_t launch(const TcParams& p, int num_sms, cudaStream_t st) {
+  static bool attr_set[16] = {false};
+  const int dev_slot = 0;
+  (void)dev_slot;
+  constexpr int smem = smem_bytes<FAM>();
+  cudaError_t e = cudaFuncSetAttribute(tc_kernel<FAM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  (void)attr_set;
+  const int grid = std::max(1, std::min(p.n_tiles, num_sms));
+  tc_kernel<FAM><<<grid, NTHREADS, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st) {
+  if (p.n_tiles <= 0) return cudaSuccess;
+  switch (fam) {
+    case FAM_ZV: return launch<FAM_ZV>(p, num_sms, st);
+    case FAM_GRAM: return launch<FAM_GRAM>(p, num_sms, st);
+    default: return launch<FAM_SCAN>(p, num_sms, st);
+  }
+}
+
+int kind_gateup() { return K_GATEUP; }
+int kind_vhat() { return K_VHAT; }
+
+}  // namespace tck
+}  // namespace ipttt

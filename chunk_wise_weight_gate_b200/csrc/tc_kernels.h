@@ -1,0 +1,43 @@
+// Internal interface between the C-ABI layer and the tensor-core kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace ipttt {
+namespace tck {
+
+enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_SCAN = 2 };
+
+struct TcParams {
+  CUtensorMap map[6];
+  int kind;          // FAM_ZV: kind_gateup() or kind_vhat()
+  int B, T, d, F, C, k;
+  int ct;            // 128-row tiles per chunk (C / 128)
+  int npairs;        // GRAM: tile pairs per chunk, ct (ct + 1) / 2
+  int chunk;         // SCAN: chunk index
+  int n_apply;       // SCAN: apply tiles (all rows); delta tiles follow
+  int n_tiles;
+  int write_snap;    // SCAN: delta tiles store the bf16 snapshot of S_{i+1}
+  int snap_in, snap_out;  // SCAN: ring slots read by apply / written by delta
+  float eta;
+  const ChunkMeta* meta;  // [B][k]
+  const float* alpha;     // [B][k]
+  float* partials;        // GRAM output [B][k][npairs]
+  void* out0;             // Z (gate/up), V (target), O (scan)
+  float* out1;            // SCAN: optional fp32 D
+  const void* resid;      // SCAN: optional residual H added to O
+  float* S;               // SCAN: fp32 state, blocked 128 x 256 tiles
+  int* status;            // device status word
+};
+
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+                   uint32_t box_inner, uint32_t box_rows);
+cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st);
+int kind_gateup();
+int kind_vhat();
+
+}  // namespace tck
+}  // namespace ipttt

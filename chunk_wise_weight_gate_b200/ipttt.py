@@ -1,0 +1,302 @@
+"""Python binding of libipttt.so (the In-Place TTT MLP layer forward on B200).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch provides device memory and streams.  There is no fallback: if
+the shared library is missing, or a tensor is not on a CUDA device, the call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libipttt.so")
+
+F32, BF16 = 0, 1
+STATUS = {0: "IPTTT_OK", 1: "IPTTT_ERR_ARG", 2: "IPTTT_ERR_SHAPE", 3: "IPTTT_ERR_ALIGN", 4: "IPTTT_ERR_DTYPE",
+          5: "IPTTT_ERR_UNSUPPORTED", 6: "IPTTT_ERR_CUDA", 7: "IPTTT_ERR_TIMEOUT", 8: "IPTTT_ERR_WORKSPACE"}
+EXPORTS = ("ipttt_workspace_size", "ipttt_forward", "ipttt_forward_ex", "ipttt_core", "ipttt_stream_state_size",
+           "ipttt_stream_reset", "ipttt_stream_forward", "ipttt_stream_export", "ipttt_get_status",
+           "ipttt_strerror", "ipttt_version", "ipttt_profile_enable", "ipttt_profile_read",
+           "ipttt_kernel_launches")
+PHASES = ("prep", "gate_up", "target", "gram", "scan")
+DEBUG_OUTPUTS = ("D", "S_final", "alpha", "Z", "V")
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("d", ctypes.c_int32), ("F", ctypes.c_int32),
+                ("C", ctypes.c_int32), ("dtype", ctypes.c_int32), ("eta", ctypes.c_float),
+                ("clip_thresh", ctypes.c_float), ("flags", ctypes.c_int32)]
+
+
+FLAG_RESIDUAL = 1
+
+
+class IptttError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({strerror(code)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libipttt.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libipttt.so not built ({LIB_PATH}); run python -m chunk_wise_weight_gate_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P, vp, sz, i32 = ctypes.POINTER(Params), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
+        L.ipttt_workspace_size.argtypes = [P]
+        L.ipttt_workspace_size.restype = sz
+        L.ipttt_forward.argtypes = [P] + [vp] * 7 + [vp, i32, vp, vp, sz, vp]
+        L.ipttt_forward.restype = ctypes.c_int
+        L.ipttt_forward_ex.argtypes = [P] + [vp] * 7 + [vp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.ipttt_forward_ex.restype = ctypes.c_int
+        L.ipttt_core.argtypes = [P, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
+        L.ipttt_core.restype = ctypes.c_int
+        L.ipttt_stream_state_size.argtypes = [P]
+        L.ipttt_stream_state_size.restype = sz
+        L.ipttt_stream_reset.argtypes = [P, vp, vp]
+        L.ipttt_stream_reset.restype = ctypes.c_int
+        L.ipttt_stream_forward.argtypes = [P, vp] + [vp] * 7 + [vp, i32, vp, vp, sz, vp]
+        L.ipttt_stream_forward.restype = ctypes.c_int
+        L.ipttt_stream_export.argtypes = [P, vp, vp, vp]
+        L.ipttt_stream_export.restype = ctypes.c_int
+        L.ipttt_get_status.argtypes = [vp]
+        L.ipttt_get_status.restype = ctypes.c_int
+        L.ipttt_strerror.argtypes = [ctypes.c_int]
+        L.ipttt_strerror.restype = ctypes.c_char_p
+        L.ipttt_version.argtypes = []
+        L.ipttt_version.restype = ctypes.c_char_p
+        L.ipttt_profile_enable.argtypes = [ctypes.c_int]
+        L.ipttt_profile_enable.restype = None
+        L.ipttt_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64),
+                                         ctypes.c_int]
+        L.ipttt_profile_read.restype = ctypes.c_int
+        L.ipttt_kernel_launches.argtypes = []
+        L.ipttt_kernel_launches.restype = ctypes.c_uint64
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    try:
+        return lib().ipttt_strerror(code).decode()
+    except Exception:  # library missing while formatting an error
+        return "?"
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise IptttError(code, where)
+
+
+@dataclass
+class LayerConfig:
+    B: int
+    T: int
+    d: int
+    F: int
+    C: int
+    eta: float
+    clip: float = 0.0
+    dtype: str = "bf16"
+
+    def params(self, flags: int = 0) -> Params:
+        return Params(self.B, self.T, self.d, self.F, self.C, BF16 if self.dtype == "bf16" else F32,
+                      float(self.eta), float(self.clip), int(flags))
+
+    @property
+    def k(self) -> int:
+        return (self.T + self.C - 1) // self.C
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+
+def _ptr(t: torch.Tensor | None, dtype=None, name="tensor") -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _docs(doc_starts, device) -> tuple[int | None, int, torch.Tensor | None]:
+    if doc_starts is None:
+        return None, 0, None
+    ds = doc_starts if isinstance(doc_starts, torch.Tensor) else torch.as_tensor(doc_starts, dtype=torch.int32)
+    ds = ds.to(device=device, dtype=torch.int32).contiguous()
+    if ds.numel() == 0:
+        return None, 0, ds
+    return ds.data_ptr(), int(ds.numel()), ds
+
+
+def workspace_size(cfg: LayerConfig) -> int:
+    n = lib().ipttt_workspace_size(ctypes.byref(cfg.params()))
+    if n == 0:
+        raise ValueError(f"invalid layer configuration {cfg}")
+    return int(n)
+
+
+def alloc_workspace(cfg: LayerConfig, device="cuda") -> torch.Tensor:
+    return torch.empty(workspace_size(cfg), dtype=torch.uint8, device=device)
+
+
+def _shape_check(cfg: LayerConfig, **tensors):
+    want = {"H": (cfg.B, cfg.T, cfg.d), "X0": (cfg.B, cfg.T, cfg.d), "Wgate": (cfg.F, cfg.d),
+            "Wup": (cfg.F, cfg.d), "Wdown0": (cfg.d, cfg.F), "conv_w": (cfg.d, 5), "Wtarget": (cfg.d, cfg.d),
+            "Z": (cfg.B, cfg.T, cfg.F), "V": (cfg.B, cfg.T, cfg.d), "O": (cfg.B, cfg.T, cfg.d)}
+    for name, t in tensors.items():
+        if t is not None and tuple(t.shape) != want[name]:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {want[name]}")
+
+
+def forward(cfg: LayerConfig, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_starts=None, *, O=None,
+            workspace=None, stream=None, debug=False, residual=False):
+    """One layer forward.  Returns O, or with debug=True (or a subset of
+    DEBUG_OUTPUTS) a dict with O and the chosen internals D, S_final, alpha, Z, V,
+    produced by the same kernels as O.  residual=True writes H + output into O."""
+    dt = cfg.torch_dtype
+    _shape_check(cfg, H=H, X0=X0, Wgate=Wgate, Wup=Wup, Wdown0=Wdown0, conv_w=conv_w, Wtarget=Wtarget, O=O)
+    dev = H.device
+    if O is None:
+        O = torch.empty(cfg.B, cfg.T, cfg.d, dtype=dt, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(cfg, dev)
+    if residual and O.data_ptr() == H.data_ptr():
+        raise ValueError("O must not alias H when residual=True")
+    dp, nd, keep = _docs(doc_starts, dev)
+    p = cfg.params(FLAG_RESIDUAL if residual else 0)
+    args = [_ptr(H, dt, "H"), _ptr(X0, dt, "X0"), _ptr(Wgate, dt, "Wgate"), _ptr(Wup, dt, "Wup"),
+            _ptr(Wdown0, dt, "Wdown0"), _ptr(conv_w, dt, "conv_w"), _ptr(Wtarget, dt, "Wtarget"), dp, nd,
+            _ptr(O, dt, "O")]
+    if not debug:
+        _check(lib().ipttt_forward(ctypes.byref(p), *args, workspace.data_ptr(), workspace.numel(),
+                                   _stream(stream)), "ipttt_forward")
+        return O
+    want = set(DEBUG_OUTPUTS) if debug is True else set(debug)
+    shapes = {"D": ((cfg.B, cfg.T, cfg.d), torch.float32), "S_final": ((cfg.B, cfg.d, cfg.F), torch.float32),
+              "alpha": ((cfg.B, cfg.k), torch.float32), "Z": ((cfg.B, cfg.T, cfg.F), dt),
+              "V": ((cfg.B, cfg.T, cfg.d), dt)}
+    out = {"O": O}
+    for name in DEBUG_OUTPUTS:
+        out[name] = torch.empty(*shapes[name][0], dtype=shapes[name][1], device=dev) if name in want else None
+    ptrs = [out[n].data_ptr() if out[n] is not None else None for n in DEBUG_OUTPUTS]
+    _check(lib().ipttt_forward_ex(ctypes.byref(p), *args, *ptrs, workspace.data_ptr(), workspace.numel(),
+                                  _stream(stream)), "ipttt_forward_ex")
+    return out
+
+
+def core(cfg: LayerConfig, Z, V, Wdown0, doc_starts=None, *, workspace=None, stream=None):
+    """The chunk scan alone on given Z [B,T,F] and V [B,T,d]; returns O, D, S_final, alpha."""
+    dt = cfg.torch_dtype
+    _shape_check(cfg, Z=Z, V=V, Wdown0=Wdown0)
+    dev = Z.device
+    if workspace is None:
+        workspace = alloc_workspace(cfg, dev)
+    dp, nd, keep = _docs(doc_starts, dev)
+    out = {"O": torch.empty(cfg.B, cfg.T, cfg.d, dtype=dt, device=dev),
+           "D": torch.empty(cfg.B, cfg.T, cfg.d, dtype=torch.float32, device=dev),
+           "S_final": torch.empty(cfg.B, cfg.d, cfg.F, dtype=torch.float32, device=dev),
+           "alpha": torch.empty(cfg.B, cfg.k, dtype=torch.float32, device=dev)}
+    p = cfg.params()
+    _check(lib().ipttt_core(ctypes.byref(p), _ptr(Z, dt, "Z"), _ptr(V, dt, "V"), _ptr(Wdown0, dt, "Wdown0"), dp,
+                            nd, out["O"].data_ptr(), out["D"].data_ptr(), out["S_final"].data_ptr(),
+                            out["alpha"].data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "ipttt_core")
+    return out
+
+
+class StreamState:
+    """Caller-owned fast-weight state carried between pieces of long sequences."""
+
+    def __init__(self, cfg: LayerConfig, device="cuda", stream=None):
+        self.cfg = cfg
+        n = lib().ipttt_stream_state_size(ctypes.byref(cfg.params()))
+        if n == 0:
+            raise ValueError(f"invalid layer configuration {cfg}")
+        self.buf = torch.empty(int(n), dtype=torch.uint8, device=device)
+        self.reset(stream)
+
+    def reset(self, stream=None):
+        _check(lib().ipttt_stream_reset(ctypes.byref(self.cfg.params()), self.buf.data_ptr(), _stream(stream)),
+               "ipttt_stream_reset")
+
+    def forward(self, piece_cfg: LayerConfig, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_starts=None, *,
+                workspace=None, stream=None):
+        dt = piece_cfg.torch_dtype
+        _shape_check(piece_cfg, H=H, X0=X0)
+        dev = H.device
+        O = torch.empty(piece_cfg.B, piece_cfg.T, piece_cfg.d, dtype=dt, device=dev)
+        if workspace is None:
+            workspace = alloc_workspace(piece_cfg, dev)
+        dp, nd, keep = _docs(doc_starts, dev)
+        p = piece_cfg.params()
+        _check(lib().ipttt_stream_forward(ctypes.byref(p), self.buf.data_ptr(), _ptr(H, dt, "H"),
+                                          _ptr(X0, dt, "X0"), _ptr(Wgate, dt, "Wgate"), _ptr(Wup, dt, "Wup"),
+                                          _ptr(Wdown0, dt, "Wdown0"), _ptr(conv_w, dt, "conv_w"),
+                                          _ptr(Wtarget, dt, "Wtarget"), dp, nd, O.data_ptr(),
+                                          workspace.data_ptr(), workspace.numel(), _stream(stream)),
+               "ipttt_stream_forward")
+        return O
+
+    def export(self, stream=None) -> torch.Tensor:
+        S = torch.empty(self.cfg.B, self.cfg.d, self.cfg.F, dtype=torch.float32, device=self.buf.device)
+        _check(lib().ipttt_stream_export(ctypes.byref(self.cfg.params()), self.buf.data_ptr(), S.data_ptr(),
+                                         _stream(stream)), "ipttt_stream_export")
+        return S
+
+
+def get_status(stream=None) -> int:
+    """Waits for the stream and returns (and clears) the device status word."""
+    return int(lib().ipttt_get_status(_stream(stream)))
+
+
+def profile_enable(on: bool = True):
+    lib().ipttt_profile_enable(1 if on else 0)
+
+
+def profile_read() -> dict:
+    """Per phase: (milliseconds, kernel launches) accumulated since the last read."""
+    n = len(PHASES)
+    ms = (ctypes.c_double * n)()
+    ln = (ctypes.c_uint64 * n)()
+    lib().ipttt_profile_read(ms, ln, n)
+    return {PHASES[i]: (float(ms[i]), int(ln[i])) for i in range(n)}
+
+
+def kernel_launches() -> int:
+    return int(lib().ipttt_kernel_launches())
+
+
+def version() -> str:
+    return lib().ipttt_version().decode()
+
+
+def flops_per_token(d: int, F: int) -> int:
+    """Credited flops per token: gate/up 4dF, Z W0^T 2dF, Z S^T 2dF, delta 2dF,
+    target projection 2d^2, conv 10d (the Gram pass for the clip is not credited)."""
+    return 10 * d * F + 2 * d * d + 10 * d
+
+
+def chunks(T: int, C: int) -> int:
+    return math.ceil(T / C)

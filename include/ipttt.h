@@ -1,0 +1,183 @@
+/*
+ * ipttt.h -- C ABI of libipttt.so, the B200 (sm_100a) forward of one In-Place
+ * Test-Time-Training MLP layer: a gated MLP whose down projection is a fast
+ * weight updated chunk by chunk.
+ *
+ * What one call computes, for every row b of a batch of B sequences of T tokens
+ * (sources: lijianxiong.blog notes "In-Place Test-Time Training", section 方法:
+ * gated MLP, step 1 "apply", step 2 "update", the LM-aligned target and the
+ * Hebbian rule, and 工程实现 for the exclusive prefix sum; cloud.tencent.com
+ * "榨干MLP的剩余价值", 详细步骤 3 (depthwise conv, kernel 5, no look past the chunk)
+ * and 4 (Frobenius clip); iplexlaw.co.kr review of arXiv 2604.06169, section 3
+ * (apply before update) and section 6 (exclusive scan, document reset, clip)):
+ *
+ *   Z   = SiLU(H Wgate^T) * (H Wup^T)                              [T, F]
+ *   U[t,c] = sum_{o=0..4} conv_w[c,o] * X0[t+o,c]   (tap zero when t+o is past the
+ *            chunk end, past T, or in another document)
+ *   V   = U Wtarget                                                  [T, d]
+ *   chunks i = 0..k-1 of C tokens (the last may be short), k = ceil(T/C);
+ *   S_0 = 0;   O_[i] = Z_[i] Wdown0^T + M_i * (Z_[i] S_i^T)          (pre-update state)
+ *   dW_i = eta V_L^T Z_L over the rows L of the chunk's last document segment,
+ *          scaled by alpha_i = tau/||dW_i||_F when ||dW_i||_F > tau (clip on)
+ *   S_{i+1} = (chunk i holds a document start ? 0 : S_i) + alpha_i dW_i
+ * M_i selects the rows of chunk i that belong to a document begun before the
+ * chunk; rows of a document begun inside the chunk use Wdown0 alone.  A row start
+ * is always a document start.
+ *
+ * Conventions for every entry point:
+ *  - Tensors are DEVICE pointers owned by the caller, row-major and contiguous,
+ *    16-byte aligned.  H, X0, O: [B, T, d].  Wgate, Wup: [F, d].  Wdown0: [d, F].
+ *    conv_w: [d, 5] (tap o multiplies X0[t+o]).  Wtarget: [d, d], used as U Wtarget.
+ *    All float tensors share params->dtype; O has that dtype.
+ *  - doc_starts: DEVICE int32 array of n_doc_starts strictly increasing global
+ *    token offsets b*T + t (row starts are implicit and may be omitted).
+ *    Entries out of range or out of order make the call fail on the device
+ *    (status IPTTT_ERR_ARG, see ipttt_get_status) and leave O unspecified.
+ *  - The library allocates nothing.  Scratch memory is the caller's workspace
+ *    (size from ipttt_workspace_size), 256-byte aligned, not shared between
+ *    calls that may run concurrently.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Argument errors are returned synchronously and launch nothing.
+ *    Errors found on the device (invalid doc_starts, a bounded wait that gave up)
+ *    are recorded in a per-device status word read by ipttt_get_status.
+ *  - Results are deterministic run to run (no floating-point atomics).
+ *  - dtype IPTTT_F32 runs an all-fp32 path (SIMT FMA) for any shape.  dtype
+ *    IPTTT_BF16 runs the tensor-core path (tcgen05, fp32 accumulation, fp32 fast
+ *    weight state) and needs d % 128 == 0, F % 256 == 0, C % 128 == 0; other shapes
+ *    return IPTTT_ERR_UNSUPPORTED.
+ */
+#ifndef IPTTT_H_
+#define IPTTT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define IPTTT_API __attribute__((visibility("default")))
+#else
+#define IPTTT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  IPTTT_OK = 0,
+  IPTTT_ERR_ARG = 1,          /* null pointer, non-positive size, bad eta/clip, bad doc_starts */
+  IPTTT_ERR_SHAPE = 2,        /* sizes inconsistent or too large for 32-bit indexing */
+  IPTTT_ERR_ALIGN = 3,        /* a tensor pointer is not 16-byte aligned (workspace: 256) */
+  IPTTT_ERR_DTYPE = 4,        /* unknown dtype */
+  IPTTT_ERR_UNSUPPORTED = 5,  /* shape outside what the bf16 tensor-core path handles */
+  IPTTT_ERR_CUDA = 6,         /* a CUDA runtime call or a launch failed */
+  IPTTT_ERR_TIMEOUT = 7,      /* a device-side bounded wait gave up */
+  IPTTT_ERR_WORKSPACE = 8     /* workspace pointer null or smaller than required */
+} ipttt_status;
+
+typedef enum { IPTTT_F32 = 0, IPTTT_BF16 = 1 } ipttt_dtype;
+
+typedef struct {
+  int32_t B;          /* sequences in the batch                                  */
+  int32_t T;          /* tokens per sequence (for streaming: tokens in this piece) */
+  int32_t d;          /* d_model                                                  */
+  int32_t F;          /* d_ff                                                     */
+  int32_t C;          /* chunk size                                               */
+  int32_t dtype;      /* ipttt_dtype                                              */
+  float eta;          /* fast-weight learning rate                                */
+  float clip_thresh;  /* Frobenius-norm threshold tau; <= 0 or +inf: no clip      */
+  int32_t flags;      /* IPTTT_FLAG_* bits, 0 for none                            */
+} ipttt_params;
+
+/* O receives H + (layer output) instead of the layer output: the residual of a
+ * stack of TTT layers, H_{l+1} = H_l + O_l, added in fp32 before the one rounding
+ * to dtype.  O must not alias H. */
+#define IPTTT_FLAG_RESIDUAL 1
+
+/* Bytes of workspace that ipttt_forward / _ex / stream_forward need for *p.
+ * Returns 0 when *p is invalid.  Pure host function. */
+IPTTT_API size_t ipttt_workspace_size(const ipttt_params* p);
+
+/* One layer forward.  O: [B, T, d] output (device, dtype).  See the top of this
+ * file for the computation and the argument conventions. */
+IPTTT_API ipttt_status ipttt_forward(const ipttt_params* p,
+                           const void* H, const void* X0,
+                           const void* Wgate, const void* Wup, const void* Wdown0,
+                           const void* conv_w, const void* Wtarget,
+                           const int32_t* doc_starts, int32_t n_doc_starts,
+                           void* O, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* ipttt_forward plus optional fp32 views of the internals, each NULL to skip:
+ *   D_opt       [B, T, d]  the fast-weight term M_i * (Z_[i] S_i^T) of O
+ *   S_final_opt [B, d, F]  the fast-weight state after the last chunk
+ *   alpha_opt   [B, k]     the clip factor of every chunk (1 when not clipped)
+ *   Z_opt       [B, T, F]  the gated activation (dtype)
+ *   V_opt       [B, T, d]  the target V restricted to each chunk's last document
+ *                          segment (other rows 0) (dtype)
+ * The computation of O is the same code path as ipttt_forward. */
+IPTTT_API ipttt_status ipttt_forward_ex(const ipttt_params* p,
+                              const void* H, const void* X0,
+                              const void* Wgate, const void* Wup, const void* Wdown0,
+                              const void* conv_w, const void* Wtarget,
+                              const int32_t* doc_starts, int32_t n_doc_starts,
+                              void* O, float* D_opt, float* S_final_opt, float* alpha_opt,
+                              void* Z_opt, void* V_opt,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* The chunk scan alone, with Z [B, T, F] and V [B, T, d] given (dtype); rows of V
+ * outside a chunk's last document segment are ignored.  Same outputs as
+ * ipttt_forward_ex.  Used to test the scan on hand-built activations such as the
+ * induction-head setting of the notes' 理论分析 section. */
+IPTTT_API ipttt_status ipttt_core(const ipttt_params* p, const void* Z, const void* V,
+                        const void* Wdown0, const int32_t* doc_starts, int32_t n_doc_starts,
+                        void* O, float* D_opt, float* S_final_opt, float* alpha_opt,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Streaming.  A caller-owned state carries each row's fp32 fast weight and
+ * position between calls, so a long sequence can be fed in pieces; the result
+ * equals one call over the whole sequence.  params->T is the piece length and
+ * must be a multiple of C except for the final piece of a sequence (the conv
+ * look-ahead and the update both close at chunk ends).  doc_starts are offsets
+ * b*T + t within the piece; a piece start is a document start only when the row
+ * has consumed nothing yet or when doc_starts lists it.
+ * State layout (opaque, 256-byte aligned): fp32 S[B][d][F], then per-row int64
+ * position and int32 flags.  ipttt_stream_reset zeroes it (stream-ordered). */
+IPTTT_API size_t ipttt_stream_state_size(const ipttt_params* p);
+IPTTT_API ipttt_status ipttt_stream_reset(const ipttt_params* p, void* state, void* stream);
+IPTTT_API ipttt_status ipttt_stream_forward(const ipttt_params* p, void* state,
+                                  const void* H, const void* X0,
+                                  const void* Wgate, const void* Wup, const void* Wdown0,
+                                  const void* conv_w, const void* Wtarget,
+                                  const int32_t* doc_starts, int32_t n_doc_starts,
+                                  void* O, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+/* Copies the state's fp32 S [B, d, F] to S_out (device). */
+IPTTT_API ipttt_status ipttt_stream_export(const ipttt_params* p, const void* state, float* S_out,
+                                 void* stream);
+
+/* Waits for `stream`, then returns and clears the per-device status word that
+ * kernels set on device-side errors (IPTTT_OK if none). */
+IPTTT_API ipttt_status ipttt_get_status(void* stream);
+
+/* Static description of a status code. */
+IPTTT_API const char* ipttt_strerror(ipttt_status s);
+
+/* Diagnostics.  While profiling is on, every call records CUDA events on its own
+ * stream around each phase: 0 metadata + conv, 1 gate/up GEMM, 2 target GEMM,
+ * 3 Gram pass + clip factors, 4 chunk scan (apply + update launches).
+ * ipttt_profile_read waits for the recorded events and returns, per phase, the
+ * milliseconds and kernel launches accumulated since the previous read
+ * (n_phases <= 5); it returns the number of phases written.
+ * ipttt_kernel_launches counts every kernel this library has launched in the
+ * process. */
+IPTTT_API void ipttt_profile_enable(int on);
+IPTTT_API int ipttt_profile_read(double* ms, uint64_t* launches, int n_phases);
+IPTTT_API uint64_t ipttt_kernel_launches(void);
+
+/* Library version, "major.minor.patch". */
+IPTTT_API const char* ipttt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* IPTTT_H_ */

@@ -10,4 +10,7 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
-    config.addinivalue_line("markers", "slow: long-running CPU test")
+    config.addinivalue_line("markers", "slow: long-running test")
+    # The CUDA library is compiled in-tree (nvcc cross-compiles without a GPU).
+    from chunk_wise_weight_gate_b200 import build
+    build.build()

@@ -1,0 +1,185 @@
+"""GPU parity of libipttt against the fp64 oracle on the same seeded inputs.
+
+Tolerances: the all-fp32 path must match to max relative error 1e-5 on O; the
+bf16 tensor-core path (bf16 operands, fp32 accumulation and fp32 state) to 2e-2
+on O (max |err| / max |ref|).  Because the clip keeps the fast-weight term near
+1e-7 of O at the workload's settings, the bf16 cases also compare the term itself
+(D, normwise 2e-2 and max-relative 5e-2), the final state S (normwise 2e-2), the
+clip factors (relative 1e-2), and the intermediate Z and V (max-relative 2e-2).
+"""
+import numpy as np
+import pytest
+import torch
+
+from chunk_wise_weight_gate_b200 import ipttt as ip
+from chunk_wise_weight_gate_b200 import synth
+from oracle import ipttt_oracle as orc
+from tests.gpu_util import case, gpu, maxrel, normrel, oracle, to_np
+
+pytestmark = pytest.mark.gpu
+
+TOL_O_BF16 = 2e-2
+TOL_O_F32 = 1e-5
+
+
+def check_bf16(out, ref, clip):
+    o = maxrel(to_np(out["O"]), ref["O"])
+    assert o <= TOL_O_BF16, f"O max-rel {o}"
+    assert maxrel(to_np(out["Z"]), ref["Z"]) <= 2e-2
+    assert maxrel(to_np(out["V"]), ref["V"]) <= 2e-2
+    a = np.max(np.abs(to_np(out["alpha"]) / ref["alpha"] - 1.0))
+    assert a <= 1e-2, f"alpha rel {a}"
+    if np.any(ref["D"] != 0):
+        assert normrel(to_np(out["D"]), ref["D"]) <= 2e-2
+        assert maxrel(to_np(out["D"]), ref["D"]) <= 5e-2
+    else:
+        assert np.all(to_np(out["D"]) == 0)
+    assert normrel(to_np(out["S_final"]), ref["S_final"]) <= 2e-2
+    if clip > 0:
+        assert np.any(ref["alpha"] < 1)
+
+
+def test_fp32_tiny_config():
+    """The tiny all-fp32 workload exactly as specified (T=256, C=32, d=64, F=256)."""
+    w = synth.WORKLOADS["tiny_f32"]
+    inp = synth.make_inputs(w, seed=0)
+    cfg = ip.LayerConfig(B=w.B, T=w.T, d=w.d, F=w.F, C=w.C, eta=w.eta, clip=w.clip, dtype="f32")
+    out = gpu(cfg, inp)
+    ref = oracle(cfg, inp)
+    assert maxrel(to_np(out["O"]), ref["O"]) <= TOL_O_F32
+    assert normrel(to_np(out["S_final"]), ref["S_final"]) <= TOL_O_F32
+    assert maxrel(to_np(out["D"]), ref["D"]) <= 1e-4
+    # The fast-weight term is visible in O at this size: without it O would miss.
+    assert maxrel(ref["O"] - ref["D"], ref["O"]) > 100 * TOL_O_F32
+
+
+@pytest.mark.parametrize("C,T,docs,clip", [(12, 100, [13, 40, 41, 100 + 7, 100 + 70], 0.05),
+                                           (7, 64, [], 0.0), (64, 50, [20], 0.02)])
+def test_fp32_docs_ragged_clip(C, T, docs, clip):
+    cfg, inp = case(2, T, C, 24, 40, dtype="f32", eta=0.05, clip=clip, docs=docs, conv_std=0.3,
+                    wtarget="identity_noise")
+    out = gpu(cfg, inp)
+    ref = oracle(cfg, inp)
+    assert maxrel(to_np(out["O"]), ref["O"]) <= TOL_O_F32
+    assert normrel(to_np(out["S_final"]), ref["S_final"]) <= TOL_O_F32
+    assert np.max(np.abs(to_np(out["alpha"]) - ref["alpha"])) <= 1e-5
+
+
+BF16_CASES = {
+    "clip_single_doc": dict(B=1, T=512, C=128, d=256, F=512, eta=1e-3, clip=1e-5),
+    "clip_docs_ragged_multitile": dict(B=2, T=1000, C=256, d=384, F=768, eta=1e-3, clip=1e-5,
+                                       docs=[100, 300, 301, 1000 + 256, 1000 + 700]),
+    "noclip_stress": dict(B=1, T=1024, C=256, d=256, F=512, eta=1e-2, clip=0.0),
+    "noclip_docs_ragged": dict(B=2, T=777, C=128, d=256, F=512, eta=2e-2, clip=0.0,
+                               docs=[129, 500, 777 + 1, 777 + 384]),
+    "long_chunk": dict(B=1, T=2048, C=1024, d=256, F=512, eta=1e-3, clip=1e-5),
+}
+
+
+@pytest.mark.parametrize("name", list(BF16_CASES))
+def test_bf16_parity(name):
+    kw = dict(BF16_CASES[name])
+    cfg, inp = case(**kw)
+    out = gpu(cfg, inp)
+    ref = oracle(cfg, inp)
+    check_bf16(out, ref, cfg.clip)
+    if cfg.clip == 0:
+        # the fast-weight term is large here, so O itself checks the scan
+        assert maxrel(ref["O"] - ref["D"], ref["O"]) > 5 * TOL_O_BF16
+
+
+def test_bf16_eta_zero_is_plain_gated_mlp():
+    cfg, inp = case(1, 384, 128, 256, 512, eta=0.0, clip=1e-5)
+    out = gpu(cfg, inp)
+    ref = oracle(cfg, inp)
+    assert np.all(to_np(out["D"]) == 0) and np.all(to_np(out["S_final"]) == 0)
+    assert maxrel(to_np(out["O"]), ref["O"]) <= TOL_O_BF16
+
+
+def test_bf16_deterministic():
+    cfg, inp = case(2, 640, 128, 256, 512, docs=[200, 640 + 333])
+    a = gpu(cfg, inp)
+    b = gpu(cfg, inp)
+    for key in ("O", "D", "S_final", "alpha", "Z", "V"):
+        assert torch.equal(a[key], b[key]), key
+
+
+def test_bf16_causality_bitwise():
+    """Perturbing tokens from s on changes no output row before s (P: no look-ahead)."""
+    cfg, inp = case(1, 768, 128, 256, 512, eta=1e-3, clip=0.0)
+    base = gpu(cfg, inp, debug=False)
+    for s in (200, 383, 512):
+        pert = dict(inp)
+        pert["H"] = inp["H"].clone()
+        pert["X0"] = inp["X0"].clone()
+        pert["H"][:, s:] += 1.0
+        pert["X0"][:, s:] *= -1.0
+        o = gpu(cfg, pert, debug=False)
+        assert torch.equal(o[:, :s], base[:, :s])
+        assert not torch.equal(o[:, s:], base[:, s:])
+
+
+def test_bf16_streaming_equals_one_shot():
+    cfg, inp = case(2, 768, 128, 256, 512, eta=1e-3, clip=0.0, docs=[100, 300, 768 + 500])
+    one = gpu(cfg, inp)
+    dev = torch.device("cuda")
+    w = {k: inp[k].to(dev) for k in ("Wgate", "Wup", "Wdown0", "conv_w", "Wtarget")}
+    st = ip.StreamState(cfg)
+    outs = []
+    docs = inp["doc_starts"].numpy()
+    for a, b in ((0, 256), (256, 640), (640, 768)):
+        pc = ip.LayerConfig(B=2, T=b - a, d=cfg.d, F=cfg.F, C=cfg.C, eta=cfg.eta, clip=cfg.clip)
+        pd = [int((g // cfg.T) * (b - a) + (g % cfg.T - a)) for g in docs if a <= g % cfg.T < b]
+        H = inp["H"][:, a:b].contiguous().to(dev)
+        X0 = inp["X0"][:, a:b].contiguous().to(dev)
+        outs.append(st.forward(pc, H, X0, w["Wgate"], w["Wup"], w["Wdown0"], w["conv_w"], w["Wtarget"], pd))
+    torch.cuda.synchronize()
+    assert ip.get_status() == 0
+    assert torch.equal(torch.cat(outs, dim=1), one["O"])
+    assert torch.equal(st.export(), one["S_final"])
+
+
+def test_bf16_theorem1_induction_head():
+    """Induction-head setting of the notes' 理论分析: one-hot keys and values, the LM
+    target raises exactly the next-token logit by eta (Wdown0 = 0, no clip)."""
+    d, F, C, T = 128, 256, 128, 512
+    eta = 0.25
+    Z = torch.zeros(1, T, F)
+    V = torch.zeros(1, T, d)
+    t_star, n, v_star = 5, 300, 77
+    Z[0, t_star, 17] = 1.0
+    Z[0, n, 17] = 1.0
+    for t in range(T):
+        if t not in (t_star, n):
+            Z[0, t, t % 16] = 0.5
+            V[0, t, (t + 1) % d] = 1.0
+    V[0, t_star, v_star] = 1.0
+    cfg = ip.LayerConfig(B=1, T=T, d=d, F=F, C=C, eta=eta, clip=0.0)
+    dev = torch.device("cuda")
+    out = ip.core(cfg, Z.bfloat16().to(dev), V.bfloat16().to(dev), torch.zeros(d, F, dtype=torch.bfloat16,
+                                                                                   device=dev))
+    torch.cuda.synchronize()
+    row = out["O"][0, n].float().cpu()
+    expect = torch.zeros(d)
+    expect[v_star] = eta
+    assert torch.equal(row, expect)
+    ref = orc.core_forward(Z.double().numpy(), V.double().numpy(), np.zeros((d, F)), C, [], eta, 0.0)
+    assert maxrel(to_np(out["O"]), ref["O"]) <= TOL_O_BF16
+
+
+def test_bad_doc_starts_set_status():
+    cfg, inp = case(1, 256, 128, 256, 512, docs=[100, 50])
+    dev = torch.device("cuda")
+    t = {k: inp[k].to(dev) for k in ("H", "X0", "Wgate", "Wup", "Wdown0", "conv_w", "Wtarget")}
+    ip.forward(cfg, t["H"], t["X0"], t["Wgate"], t["Wup"], t["Wdown0"], t["conv_w"], t["Wtarget"],
+               inp["doc_starts"])
+    assert ip.get_status() == 1
+    assert ip.get_status() == 0
+
+
+def test_unsupported_shape_raises():
+    cfg, inp = case(1, 256, 96, 256, 512)
+    dev = torch.device("cuda")
+    t = {k: inp[k].to(dev) for k in ("H", "X0", "Wgate", "Wup", "Wdown0", "conv_w", "Wtarget")}
+    with pytest.raises(ValueError):
+        ip.forward(cfg, t["H"], t["X0"], t["Wgate"], t["Wup"], t["Wdown0"], t["conv_w"], t["Wtarget"])
