@@ -125,7 +125,8 @@ def phase_flops(w: synth.Workload) -> dict:
         "gate_up": 4 * B * T * d * F,
         "target": 2 * B * T * d * d,
         "gram": 2 * B * k * (ct * (ct + 1) // 2) * 128 * 128 * (d + F),
-        "scan": 6 * B * T * d * F,
+        "apply": 4 * B * T * d * F,
+        "update": 2 * B * T * d * F,
     }
 
 

@@ -12,6 +12,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -56,8 +57,8 @@ ipttt_status device_info(DeviceInfo** out) {
 }
 
 // ---------------------------------------------------------------- profiling
-constexpr int kPhases = 5;
-enum Phase { PH_PREP = 0, PH_GATEUP = 1, PH_TARGET = 2, PH_GRAM = 3, PH_SCAN = 4 };
+constexpr int kPhases = 6;
+enum Phase { PH_PREP = 0, PH_GATEUP = 1, PH_TARGET = 2, PH_GRAM = 3, PH_APPLY = 4, PH_UPDATE = 5 };
 
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_profile_on{0};
@@ -117,7 +118,21 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 
 struct Layout {
   size_t flags, meta, alpha, partials, Z, U, V, S, snap, raw, dpart, total;
+  int group;  // bf16 path: chunks whose apply tiles share one launch (= snapshot ring slots)
 };
+
+// Apply tiles of `group` consecutive chunks share one launch, so that one launch
+// holds about kApplyTilesPerLaunch tiles (several even waves over the SMs).
+constexpr int kApplyTilesPerLaunch = 1280;
+
+int apply_group(const ipttt_params& p) {
+  const int k = (p.T + p.C - 1) / p.C;
+  const long long per_chunk = (long long)p.B * (p.C / 128) * (p.d / 128);
+  long long g = (kApplyTilesPerLaunch + per_chunk - 1) / per_chunk;
+  if (g < 1) g = 1;
+  if (g > k) g = k;
+  return (int)g;
+}
 
 bool is_bf16(const ipttt_params& p) { return p.dtype == IPTTT_BF16; }
 
@@ -152,7 +167,8 @@ Layout layout_of(const ipttt_params& p) {
     L.U = take(B * T * d * 2);
     L.V = take(B * T * d * 2);
     L.S = take(B * d * F * 4);
-    L.snap = take(2 * B * d * F * 2);
+    L.group = apply_group(p);
+    L.snap = take((size_t)L.group * B * d * F * 2);
     L.raw = L.dpart = 0;
   } else {
     L.partials = 0;
@@ -179,7 +195,7 @@ ipttt_status check_params(const ipttt_params* p) {
       BT * (long long)p->F > (1ll << 40))
     return IPTTT_ERR_SHAPE;
   if (p->dtype == IPTTT_BF16) {
-    if (p->d % 128 != 0 || p->F % 256 != 0 || p->C % 128 != 0 || p->C > 4096) return IPTTT_ERR_UNSUPPORTED;
+    if (p->d % 128 != 0 || p->F % 128 != 0 || p->C % 128 != 0 || p->C > 4096) return IPTTT_ERR_UNSUPPORTED;
   }
   return IPTTT_OK;
 }
@@ -235,6 +251,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   float* S = ss ? ss->S : reinterpret_cast<float*>(ws + L.S);
   void* snap = ws + L.snap;
   const float tau = (p.clip_thresh > 0.0f && isfinite(p.clip_thresh)) ? p.clip_thresh : 0.0f;
+  ipttt_status rc_ = IPTTT_OK;
 
   {
     PhaseScope ph(st, PH_PREP);
@@ -305,37 +322,63 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   }
   if (t.alpha) IP_CHECK(cudaMemcpyAsync(t.alpha, alpha, (size_t)s.B * s.k * 4, cudaMemcpyDeviceToDevice, st));
 
-  PhaseScope scan_phase(st, PH_SCAN);
   // A streaming piece that continues a row starts from the carried state S.
   if (ss) {
+    PhaseScope ph(st, PH_UPDATE);
     IP_CHECK(aux::state_snapshot(S, snap, s, st));
     counted(1);
   }
 
+  // The scan.  S_i (bf16 snapshot) lives in ring slot i % G.  For each group of G
+  // chunks [a, b): state updates of chunks a .. b-2 (each writes S_{j+1}), then
+  // one launch with the apply tiles of chunks a .. b-1 (they read S_a .. S_{b-1}),
+  // then the update of chunk b-1 (writes S_b into the slot S_a has left).
+  const int G = L.group;
   TcParams sc = tp;
   if (!make_map_bf16(&sc.map[0], Z, s.F, s.T, s.B, 64, 128) ||
       !make_map_bf16(&sc.map[1], t.W0, s.F, s.d, 1, 64, 128) ||
-      !make_map_bf16(&sc.map[2], snap, s.F, s.d, 2 * s.B, 64, 128) ||
-      !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, 64) ||
-      !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, 64) ||
-      !make_map_bf16(&sc.map[5], snap, s.F, s.d, 2 * s.B, 64, 32))
+      !make_map_bf16(&sc.map[2], snap, s.F, s.d, (uint64_t)G * s.B, 64, 128) ||
+      !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, 128) ||
+      !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, 128) ||
+      !make_map_bf16(&sc.map[5], snap, s.F, s.d, (uint64_t)G * s.B, 64, 32))
     return IPTTT_ERR_CUDA;
   sc.out0 = t.O;
   sc.out1 = t.D;
   sc.resid = (p.flags & IPTTT_FLAG_RESIDUAL) ? t.H : nullptr;
   sc.S = S;
+  sc.nslots = G;
   const bool need_final = t.Sfinal != nullptr || ss != nullptr;
-  for (int i = 0; i < s.k; ++i) {
-    const bool last = i + 1 == s.k;
-    sc.chunk = i;
-    sc.snap_in = i & 1;
-    sc.snap_out = (i + 1) & 1;
-    sc.write_snap = last ? 0 : 1;
-    sc.n_apply = s.B * sc.ct * (s.d / 128);
-    const int n_delta = (!last || need_final) ? s.B * (s.d / 128) * (s.F / 256) : 0;
-    sc.n_tiles = sc.n_apply + n_delta;
-    IP_CHECK(launch_tc(FAM_SCAN, sc, di->num_sms, st));
+  const int delta_tiles = s.B * (s.d / 128) * (s.F / 128);
+  const int apply_tiles_per_chunk = s.B * sc.ct * (s.d / 128);
+  auto delta = [&](int j) -> ipttt_status {
+    PhaseScope ph(st, PH_UPDATE);
+    TcParams q = sc;
+    q.chunk = j;
+    q.write_snap = (j + 1 < s.k) ? 1 : 0;
+    q.apply_chunk0 = 0;
+    q.n_apply = 0;
+    q.n_tiles = delta_tiles;
+    IP_CHECK(launch_tc(FAM_DELTA, q, di->num_sms, st));
     counted(1);
+    return IPTTT_OK;
+  };
+  for (int a = 0; a < s.k; a += G) {
+    const int b = std::min(a + G, s.k);
+    for (int j = a; j + 1 < b; ++j)
+      if ((rc_ = delta(j)) != IPTTT_OK) return rc_;
+    {
+      PhaseScope ph(st, PH_APPLY);
+      TcParams q = sc;
+      q.chunk = 0;
+      q.write_snap = 0;
+      q.apply_chunk0 = a;
+      q.n_apply = (b - a) * apply_tiles_per_chunk;
+      q.n_tiles = q.n_apply;
+      IP_CHECK(launch_tc(FAM_APPLY, q, di->num_sms, st));
+      counted(1);
+    }
+    if (b < s.k || need_final)
+      if ((rc_ = delta(b - 1)) != IPTTT_OK) return rc_;
   }
   if (t.Sfinal) {
     IP_CHECK(aux::state_export(true, S, t.Sfinal, s, st));

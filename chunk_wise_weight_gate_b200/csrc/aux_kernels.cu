@@ -39,26 +39,41 @@ __global__ void k_mark_starts(uint8_t* flags, int B, int T, const int32_t* ds, i
   if (i < B && (row_cont == nullptr || row_cont[i] == 0)) flags[(size_t)i * T] = 1;
 }
 
+// One block per (row, chunk): the chunk's flags are scanned by all threads and
+// reduced to the first start after the chunk start, the last start, and "any".
 __global__ void k_chunk_meta(const uint8_t* flags, ChunkMeta* meta, int B, int T, int C, int k) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= B * k) return;
+  __shared__ int s_first, s_last, s_any;
+  const int i = blockIdx.x;
   const int b = i / k, c = i % k;
   const int s = c * C, e = min(s + C, T);
   const uint8_t* f = flags + (size_t)b * T;
-  int first_end = e, last_start = s, any = 0;
-  for (int t = s; t < e; ++t) {
+  if (threadIdx.x == 0) {
+    s_first = e;
+    s_last = -1;
+    s_any = 0;
+  }
+  __syncthreads();
+  int first = e, last = -1;
+  for (int t = s + threadIdx.x; t < e; t += blockDim.x) {
     if (f[t]) {
-      any = 1;
-      last_start = t;
-      if (t > s && first_end == e) first_end = t;
+      if (t > s) first = min(first, t);
+      last = max(last, t);
     }
   }
-  ChunkMeta m;
-  m.first_end = first_end;
-  m.last_start = last_start;
-  m.cont = f[s] ? 0 : 1;
-  m.has_start = any;
-  meta[i] = m;
+  if (first < e) atomicMin(&s_first, first);
+  if (last >= 0) {
+    atomicMax(&s_last, last);
+    s_any = 1;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    ChunkMeta m;
+    m.first_end = s_first;
+    m.last_start = s_last >= 0 ? s_last : s;
+    m.cont = f[s] ? 0 : 1;
+    m.has_start = s_any;
+    meta[i] = m;
+  }
 }
 
 cudaError_t build_meta(uint8_t* flags, ChunkMeta* meta, const Shape& s, const int32_t* doc_starts, int n_doc,
@@ -67,40 +82,116 @@ cudaError_t build_meta(uint8_t* flags, ChunkMeta* meta, const Shape& s, const in
   k_fill_u8<<<(unsigned)std::min<size_t>((n + 255) / 256, 4096), 256, 0, st>>>(flags, n, 0);
   const int nt = std::max(n_doc, s.B);
   k_mark_starts<<<(nt + 255) / 256, 256, 0, st>>>(flags, s.B, s.T, doc_starts, n_doc, row_cont, status);
-  k_chunk_meta<<<(s.B * s.k + 127) / 128, 128, 0, st>>>(flags, meta, s.B, s.T, s.C, s.k);
+  k_chunk_meta<<<s.B * s.k, 256, 0, st>>>(flags, meta, s.B, s.T, s.C, s.k);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ conv
 // U[b,t,c] = sum_o conv_w[c,o] X0[b,t+o,c]; tap o is dropped (and every later
 // one) once t+o reaches the chunk end or T, or a document starts at t+o.
+// A thread owns VEC channels of one row over RUN consecutive tokens: it keeps
+// its 5 x VEC taps and a 5-row window of X0 in registers, so every X0 element
+// is read about once and a warp's loads and stores cover contiguous bytes.
+constexpr int kConvRun = 64;
+
 template <typename T, int VEC>
-__global__ void k_conv(const T* __restrict__ X0, const T* __restrict__ cw, const uint8_t* __restrict__ flags,
-                       T* __restrict__ U, int B, int Tn, int d, int C) {
+__device__ __forceinline__ void load_vec(const T* p, float (&out)[VEC]) {
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) out[v] = to_f<T>(p[v]);
+}
+template <>
+__device__ __forceinline__ void load_vec<__nv_bfloat16, 8>(const __nv_bfloat16* p, float (&out)[8]) {
+  const uint4 q = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
+    out[2 * e] = __low2float(h);
+    out[2 * e + 1] = __high2float(h);
+  }
+}
+template <>
+__device__ __forceinline__ void load_vec<float, 4>(const float* p, float (&out)[4]) {
+  const float4 q = *reinterpret_cast<const float4*>(p);
+  out[0] = q.x; out[1] = q.y; out[2] = q.z; out[3] = q.w;
+}
+template <typename T, int VEC>
+__device__ __forceinline__ void store_vec(T* p, const float (&in)[VEC]) {
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) p[v] = from_f<T>(in[v]);
+}
+template <>
+__device__ __forceinline__ void store_vec<__nv_bfloat16, 8>(__nv_bfloat16* p, const float (&in)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(in[2 * e], in[2 * e + 1]);
+    w[e] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+template <>
+__device__ __forceinline__ void store_vec<float, 4>(float* p, const float (&in)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(in[0], in[1], in[2], in[3]);
+}
+
+template <typename T, int VEC>
+__global__ void __launch_bounds__(256) k_conv(const T* __restrict__ X0, const T* __restrict__ cw,
+                                              const uint8_t* __restrict__ flags, T* __restrict__ U, int B, int Tn,
+                                              int d, int C) {
   const int groups = d / VEC;
-  const size_t total = (size_t)B * Tn * groups;
+  const int runs = (Tn + kConvRun - 1) / kConvRun;
+  const size_t total = (size_t)B * runs * groups;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
        idx += (size_t)gridDim.x * blockDim.x) {
     const int g = (int)(idx % groups);
-    const size_t bt = idx / groups;
-    const int t = (int)(bt % Tn);
-    const int b = (int)(bt / Tn);
-    const int cend = min((t / C + 1) * C, Tn);
+    const size_t rr = idx / groups;
+    const int run = (int)(rr % runs);
+    const int b = (int)(rr / runs);
+    float w[kTaps][VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v)
+#pragma unroll
+      for (int o = 0; o < kTaps; ++o) w[o][v] = to_f<T>(cw[(size_t)(g * VEC + v) * kTaps + o]);
+    const int t_begin = run * kConvRun;
+    const int t_end = min(t_begin + kConvRun, Tn);
     const uint8_t* f = flags + (size_t)b * Tn;
-    float acc[VEC];
+    const T* xb = X0 + (size_t)b * Tn * d + (size_t)g * VEC;
+    T* ub = U + (size_t)b * Tn * d + (size_t)g * VEC;
+    float win[kTaps][VEC];
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
+    for (int o = 0; o < kTaps - 1; ++o) {
+      const int src = t_begin + o;
 #pragma unroll
-    for (int o = 0; o < kTaps; ++o) {
-      const int src = t + o;
-      if (src >= cend || (o > 0 && f[src])) break;
-      const T* x = X0 + ((size_t)b * Tn + src) * d + (size_t)g * VEC;
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) acc[v] = fmaf(to_f<T>(cw[(size_t)(g * VEC + v) * kTaps + o]), to_f<T>(x[v]), acc[v]);
+      for (int v = 0; v < VEC; ++v) win[o + 1][v] = 0.0f;
+      if (src < Tn) load_vec<T, VEC>(xb + (size_t)src * d, win[o + 1]);
     }
-    T* u = U + ((size_t)b * Tn + t) * d + (size_t)g * VEC;
+    for (int t = t_begin; t < t_end; ++t) {
+      // slide: win[o] holds X0[t + o]
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) u[v] = from_f<T>(acc[v]);
+      for (int o = 0; o < kTaps - 1; ++o)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) win[o][v] = win[o + 1][v];
+      const int nxt = t + kTaps - 1;
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) win[kTaps - 1][v] = 0.0f;
+      if (nxt < Tn) load_vec<T, VEC>(xb + (size_t)nxt * d, win[kTaps - 1]);
+      const int cend = min((t / C + 1) * C, Tn);
+      int ntaps = 1;
+#pragma unroll
+      for (int o = 1; o < kTaps; ++o)
+        if (ntaps == o && t + o < cend && !f[t + o]) ntaps = o + 1;
+      float acc[VEC];
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
+#pragma unroll
+      for (int o = 0; o < kTaps; ++o)
+        if (o < ntaps) {
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) acc[v] = fmaf(w[o][v], win[o][v], acc[v]);
+        }
+      store_vec<T, VEC>(ub + (size_t)t * d, acc);
+    }
   }
 }
 
@@ -146,11 +237,12 @@ cudaError_t alpha_from_partials(const float* partials, float* alpha, int n, int 
 }
 
 // ------------------------------------------------------------------ state layouts
-// The bf16 path keeps S [d][F] (fp32) as 128 x 256 tiles, tile (mt, nt) at
-// ((mt * F/256) + nt) * 32768, element (r, c) of a tile at ((c/4) * 128 + r) * 4 + c%4.
+// The bf16 path keeps S [d][F] (fp32) as 128 x 128 tiles, tile (mt, nt) at
+// ((mt * F/128) + nt) * 16384, element (r, c) of a tile at ((c/4) * 128 + r) * 4 + c%4,
+// so a tile is one contiguous 64 KB block laid out as the TMEM lanes read it.
 __device__ __forceinline__ size_t blocked_index(int r, int c, int F) {
-  const size_t tile = (size_t)(r >> 7) * (F >> 8) + (c >> 8);
-  return tile * 32768 + ((size_t)((c & 255) >> 2) * 128 + (r & 127)) * 4 + (c & 3);
+  const size_t tile = (size_t)(r >> 7) * (F >> 7) + (c >> 7);
+  return tile * 16384 + ((size_t)((c & 127) >> 2) * 128 + (r & 127)) * 4 + (c & 3);
 }
 
 __global__ void k_blocked_to_rowmajor(const float* Sb, float* out, int B, int d, int F) {

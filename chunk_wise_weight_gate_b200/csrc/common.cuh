@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/ipttt.h"
+#include "ipttt.h"
 
 namespace ipttt {
 

@@ -16,11 +16,15 @@
 //   FAM_GRAM per-chunk Gram pass: ||V_L^T Z_L||_F^2 = sum_{s,t}(V V^T)_{st}(Z Z^T)_{st},
 //            written as deterministic partial sums per 128x128 tile pair; the clip
 //            factor follows [cloud.tencent.com "榨干MLP的剩余价值", 详细步骤 4].
-//   FAM_SCAN one chunk i of the scan: "apply" tiles O_i = Z_i W0^T + M_i (Z_i S_i^T)
-//            (both products side by side in one N=256 accumulator, S_i read from a
-//            bf16 snapshot) and "delta" tiles S_{i+1} = keep_i S_i + alpha_i eta
-//            V_i^T Z_i on the fp32 state [notes, 步骤一/步骤二 and 工程实现; iplexlaw.co.kr
-//            review §3 apply-before-update, §6 exclusive scan and document reset].
+//   FAM_APPLY apply tiles of a group of chunks: O_i = Z_i W0^T + M_i (Z_i S_i^T), both
+//            products side by side in one N=256 accumulator, S_i read from a bf16
+//            snapshot [notes, 步骤一 and 工程实现; iplexlaw.co.kr review §3: a chunk's output
+//            comes from the pre-update state].
+//   FAM_DELTA the state update of one chunk: S_{i+1} = keep_i S_i + alpha_i eta V_i^T Z_i
+//            on 128 x 128 tiles of the fp32 state, which move between HBM and shared
+//            memory as contiguous 64 KB bulk copies, plus the bf16 snapshot of S_{i+1}
+//            [notes, 步骤二 and the Hebbian rule; iplexlaw.co.kr review §6 exclusive scan
+//            and document reset].
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -38,27 +42,39 @@ using namespace ipttt::tc;
 constexpr int BM = 128;                 // accumulator rows (TMEM lanes)
 constexpr int BK = 64;                  // K elements per stage (one 128-byte swizzle row)
 constexpr int A_BYTES = BM * BK * 2;    // 16 KB
-constexpr int B_BYTES = 256 * BK * 2;   // 32 KB (up to N = 256)
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int NTHREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr int ACC_COLS = 256;           // per accumulator buffer
-constexpr int SNAP_STAGE_BYTES = 32 * 128;  // one 32-row x 64-col bf16 box
+constexpr int SNAP_BOX_BYTES = 32 * 128;     // 32 rows x 64 bf16 columns (one warp's snapshot box)
 
 enum Kind { K_GATEUP = 0, K_VHAT = 1, K_GRAM = 2, K_APPLY = 3, K_DELTA = 4 };
 
+// Per family: pipeline stages, bytes per stage, K elements per stage (KB), offset
+// of the B operand inside a stage, and shared memory for the epilogue.
 template <int FAM> struct Cfg;
-template <> struct Cfg<FAM_ZV> { static constexpr int STAGES = 4; static constexpr int EPI_BYTES = 0; };
-template <> struct Cfg<FAM_GRAM> { static constexpr int STAGES = 4; static constexpr int EPI_BYTES = 0; };
-template <> struct Cfg<FAM_SCAN> {
-  static constexpr int STAGES = 3;
-  static constexpr int EPI_BYTES = NUM_EPI_WARPS * 2 * SNAP_STAGE_BYTES;  // 64 KB
+template <> struct Cfg<FAM_ZV> {
+  static constexpr int STAGES = 4, STAGE_BYTES = 48 * 1024, KB = 64, B_OFF = A_BYTES, EPI_BYTES = 0;
+};
+template <> struct Cfg<FAM_GRAM> {
+  static constexpr int STAGES = 6, STAGE_BYTES = 32 * 1024, KB = 64, B_OFF = A_BYTES, EPI_BYTES = 0;
+};
+template <> struct Cfg<FAM_APPLY> {
+  static constexpr int STAGES = 4, STAGE_BYTES = 48 * 1024, KB = 64, B_OFF = A_BYTES, EPI_BYTES = 0;
+};
+// The update contracts over tokens with MN-major operands; 128-token stages keep
+// every TMA box at 16 KB (128 rows of 128 bytes).
+template <> struct Cfg<FAM_DELTA> {
+  static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 128, B_OFF = 32 * 1024,
+                       EPI_BYTES = NUM_EPI_WARPS * SNAP_BOX_BYTES;
 };
 
 template <int FAM>
 constexpr int smem_bytes() {
-  return 1024 /*alignment slack*/ + Cfg<FAM>::STAGES * STAGE_BYTES + Cfg<FAM>::EPI_BYTES + 256 /*barriers*/;
+  return 1024 /*alignment slack*/ + Cfg<FAM>::STAGES * Cfg<FAM>::STAGE_BYTES + Cfg<FAM>::EPI_BYTES +
+         256 /*barriers*/;
 }
+static_assert(smem_bytes<FAM_DELTA>() <= 232448, "delta kernel exceeds shared memory");
+static_assert(smem_bytes<FAM_ZV>() <= 232448, "kernel exceeds shared memory");
 
 struct Job {
   int kind;
@@ -138,55 +154,59 @@ __device__ __forceinline__ void decode_gram(const TcParams& p, int tile, Job& j)
   j.b_mn = false;
 }
 
-__device__ __forceinline__ void decode_scan(const TcParams& p, int tile, Job& j) {
-  j.chunk = p.chunk;
-  j.t0 = p.chunk * p.C;
+__device__ __forceinline__ void decode_apply(const TcParams& p, int tile, Job& j) {
+  const int tiles_n = p.d / 128;
+  const int per_row = p.ct * tiles_n;
+  const int per_chunk = p.B * per_row;
+  j.kind = K_APPLY;
+  j.chunk = p.apply_chunk0 + tile / per_chunk;
+  j.t0 = j.chunk * p.C;
+  j.b = (tile % per_chunk) / per_row;
+  const int r = tile % per_row;
+  j.m0 = (r / tiles_n) * BM;      // row offset inside the chunk
+  j.n0 = (r % tiles_n) * 128;     // output column (d index)
   j.pair = 0;
   j.nseg = 1;
   j.acc_col[0] = 0;
-  const ChunkMeta* mrow;
-  if (tile < p.n_apply) {
-    const int tiles_n = p.d / 128;
-    const int per_row = p.ct * tiles_n;
-    j.kind = K_APPLY;
-    j.b = tile / per_row;
-    const int r = tile % per_row;
-    j.m0 = (r / tiles_n) * BM;      // row offset inside the chunk
-    j.n0 = (r % tiles_n) * 128;     // output column (d index)
-    mrow = p.meta + (size_t)j.b * p.k + p.chunk;
-    j.nsrc = mrow->cont ? 2 : 1;
-    j.kb0[0] = 0;
-    j.kb1[0] = p.F / BK;
-    j.n_mma = 128 * j.nsrc;
-    j.tx = A_BYTES + j.nsrc * 128 * BK * 2;
-    j.a_mn = false;
-    j.b_mn = false;
-  } else {
-    const int t = tile - p.n_apply;
-    const int tiles_n = p.F / 256;
-    const int per_row = (p.d / 128) * tiles_n;
-    j.kind = K_DELTA;
-    j.b = t / per_row;
-    const int r = t % per_row;
-    j.m0 = (r / tiles_n) * 128;     // d index
-    j.n0 = (r % tiles_n) * 256;     // F index
-    mrow = p.meta + (size_t)j.b * p.k + p.chunk;
-    const int rows = min(p.C, p.T - j.t0);
-    j.kb0[0] = (mrow->last_start - j.t0) / BK;
-    j.kb1[0] = cdiv(rows, BK);
-    j.n_mma = 256;
-    j.nsrc = 1;
-    j.tx = A_BYTES + B_BYTES;
-    j.a_mn = true;
-    j.b_mn = true;
-  }
+  j.nsrc = p.meta[(size_t)j.b * p.k + j.chunk].cont ? 2 : 1;
+  j.kb0[0] = 0;
+  j.kb1[0] = p.F / BK;
+  j.n_mma = 128 * j.nsrc;
+  j.tx = A_BYTES + j.nsrc * 128 * BK * 2;
+  j.a_mn = false;
+  j.b_mn = false;
+}
+
+__device__ __forceinline__ void decode_delta(const TcParams& p, int tile, Job& j) {
+  const int tiles_n = p.F / 128;
+  const int per_row = (p.d / 128) * tiles_n;
+  j.kind = K_DELTA;
+  j.chunk = p.chunk;
+  j.t0 = p.chunk * p.C;
+  j.b = tile / per_row;
+  const int r = tile % per_row;
+  j.m0 = (r / tiles_n) * 128;     // d index
+  j.n0 = (r % tiles_n) * 128;     // F index
+  j.pair = 0;
+  j.nseg = 1;
+  j.acc_col[0] = 0;
+  constexpr int KB = Cfg<FAM_DELTA>::KB;
+  const int rows = min(p.C, p.T - j.t0);
+  j.kb0[0] = (p.meta[(size_t)j.b * p.k + j.chunk].last_start - j.t0) / KB;
+  j.kb1[0] = cdiv(rows, KB);
+  j.n_mma = 128;
+  j.nsrc = 1;
+  j.tx = 4 * 64 * KB * 2;  // two 64-column boxes of V and two of Z, KB token rows each
+  j.a_mn = true;
+  j.b_mn = true;
 }
 
 template <int FAM>
 __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
   if constexpr (FAM == FAM_ZV) decode_zv(p, tile, j);
   else if constexpr (FAM == FAM_GRAM) decode_gram(p, tile, j);
-  else decode_scan(p, tile, j);
+  else if constexpr (FAM == FAM_APPLY) decode_apply(p, tile, j);
+  else decode_delta(p, tile, j);
 }
 
 // ------------------------------------------------------------------ producer
@@ -208,20 +228,18 @@ __device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int
     const CUtensorMap* m = seg == 0 ? &p.map[0] : &p.map[1];       // Z or V
     tma_load_3d(sa, m, bar, kx, j.t0 + j.m0, j.b);
     tma_load_3d(sb, m, bar, kx, j.t0 + j.n0, j.b);
+  } else if constexpr (FAM == FAM_APPLY) {
+    tma_load_3d(sa, &p.map[0], bar, kx, j.t0 + j.m0, j.b);        // Z rows of the chunk
+    tma_load_3d(sb, &p.map[1], bar, kx, j.n0, 0);                 // Wdown0 rows
+    if (j.nsrc == 2)
+      tma_load_3d(sb + 128 * BK * 2, &p.map[2], bar, kx, j.n0, (j.chunk % p.nslots) * p.B + j.b);  // S_i rows
   } else {
-    if (j.kind == K_APPLY) {
-      tma_load_3d(sa, &p.map[0], bar, kx, j.t0 + j.m0, j.b);      // Z rows of the chunk
-      tma_load_3d(sb, &p.map[1], bar, kx, j.n0, 0);                   // Wdown0 rows
-      if (j.nsrc == 2)
-        tma_load_3d(sb + 128 * BK * 2, &p.map[2], bar, kx, j.n0, p.snap_in * p.B + j.b);  // S_i rows
-    } else {
-      const int ty = j.t0 + kx;                                    // token rows = K
-      tma_load_3d(sa, &p.map[3], bar, j.m0, ty, j.b);              // V[t][d], d contiguous
-      tma_load_3d(sa + 64 * BK * 2, &p.map[3], bar, j.m0 + 64, ty, j.b);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        tma_load_3d(sb + q * 64 * BK * 2, &p.map[4], bar, j.n0 + 64 * q, ty, j.b);  // Z[t][f]
-    }
+    constexpr int KB = Cfg<FAM_DELTA>::KB;
+    const int ty = j.t0 + kb * KB;                                 // token rows = K
+    tma_load_3d(sa, &p.map[3], bar, j.m0, ty, j.b);                // V[t][d], d contiguous
+    tma_load_3d(sa + 64 * KB * 2, &p.map[3], bar, j.m0 + 64, ty, j.b);
+    tma_load_3d(sb, &p.map[4], bar, j.n0, ty, j.b);                // Z[t][f], f contiguous
+    tma_load_3d(sb + 64 * KB * 2, &p.map[4], bar, j.n0 + 64, ty, j.b);
   }
 }
 
@@ -246,13 +264,13 @@ __device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float* v) {
 
 // Named barrier among the epilogue warps only.
 __device__ __forceinline__ void epi_sync() {
+  __syncwarp();
   asm volatile("bar.sync 1, %0;" ::"n"(NUM_EPI_WARPS * 32) : "memory");
 }
 
 template <int FAM>
 __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, uint32_t tacc, int half, int row,
-                                              int lane, int ew, float* red, uint8_t* snap_stage,
-                                              int& snap_uses) {
+                                              int lane, int ew, float* red) {
   uint32_t r0[32], r1[32];
   float v[32];
   if constexpr (FAM == FAM_ZV) {
@@ -303,105 +321,105 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
       p.partials[((size_t)j.b * p.k + j.chunk) * p.npairs + j.pair] = wgt * tot;
     }
     epi_sync();
-  } else {
-    if (j.kind == K_APPLY) {
-      const ChunkMeta m = p.meta[(size_t)j.b * p.k + j.chunk];
-      const int t = j.t0 + j.m0 + row;
-      const bool valid = t < p.T;
-      const bool carry = j.nsrc == 2 && m.cont && t < m.first_end;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.d + j.n0;
-      const __nv_bfloat16* hrow =
-          p.resid ? reinterpret_cast<const __nv_bfloat16*>(p.resid) + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
-      float* drow = p.out1 ? p.out1 + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
+  } else if constexpr (FAM == FAM_APPLY) {
+    const ChunkMeta m = p.meta[(size_t)j.b * p.k + j.chunk];
+    const int t = j.t0 + j.m0 + row;
+    const bool valid = t < p.T;
+    const bool carry = j.nsrc == 2 && m.cont && t < m.first_end;
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.d + j.n0;
+    const __nv_bfloat16* hrow =
+        p.resid ? reinterpret_cast<const __nv_bfloat16*>(p.resid) + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
+    float* drow = p.out1 ? p.out1 + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
 #pragma unroll 1
-      for (int c = half * 64; c < half * 64 + 64; c += 32) {
-        tmem_ld32(tacc + c, r0);
-        if (j.nsrc == 2) tmem_ld32(tacc + 128 + c, r1);
-        tmem_ld_wait();
+    for (int c = half * 64; c < half * 64 + 64; c += 32) {
+      tmem_ld32(tacc + c, r0);
+      if (j.nsrc == 2) tmem_ld32(tacc + 128 + c, r1);
+      tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float dv = carry ? __uint_as_float(r1[i]) : 0.0f;
-          v[i] = __uint_as_float(r0[i]) + dv;
-          r1[i] = __float_as_uint(dv);
-        }
-        if (valid) {
-          if (hrow) {
-            const uint4* h4 = reinterpret_cast<const uint4*>(hrow + c);
+      for (int i = 0; i < 32; ++i) {
+        const float dv = carry ? __uint_as_float(r1[i]) : 0.0f;
+        v[i] = __uint_as_float(r0[i]) + dv;
+        r1[i] = __float_as_uint(dv);
+      }
+      if (valid) {
+        if (hrow) {
+          const uint4* h4 = reinterpret_cast<const uint4*>(hrow + c);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 hv = h4[q];
-              const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+          for (int q = 0; q < 4; ++q) {
+            const uint4 hv = h4[q];
+            const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hw[e]);
-                v[8 * q + 2 * e] += __low2float(h2);
-                v[8 * q + 2 * e + 1] += __high2float(h2);
-              }
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hw[e]);
+              v[8 * q + 2 * e] += __low2float(h2);
+              v[8 * q + 2 * e + 1] += __high2float(h2);
             }
           }
-          st_bf16x32(orow + c, v);
-          if (drow) {
-            float4* d4 = reinterpret_cast<float4*>(drow + c);
+        }
+        st_bf16x32(orow + c, v);
+        if (drow) {
+          float4* d4 = reinterpret_cast<float4*>(drow + c);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              d4[q] = make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
-                                  __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3]));
-          }
+          for (int q = 0; q < 8; ++q)
+            d4[q] = make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
+                                __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3]));
         }
       }
-    } else {
-      // delta: fp32 state tile in the blocked layout [c/4][row][4] of 128 x 256.
-      const ChunkMeta m = p.meta[(size_t)j.b * p.k + j.chunk];
-      const bool keep = !m.has_start;
-      const float ae = p.alpha[(size_t)j.b * p.k + j.chunk] * p.eta;
-      float* Sb = p.S + (size_t)j.b * p.d * p.F + ((size_t)(j.m0 / 128) * (p.F / 256) + j.n0 / 256) * (128 * 256);
-#pragma unroll 1
-      for (int c = half * 128; c < half * 128 + 128; c += 64) {
-        float4 old[16];
+    }
+  }
+}
+
+__device__ __forceinline__ float4* state_tile(const TcParams& p, const Job& j) {
+  return reinterpret_cast<float4*>(p.S + (size_t)j.b * p.d * p.F +
+                                   ((size_t)(j.m0 / 128) * (p.F / 128) + j.n0 / 128) * (128 * 128));
+}
+
+// This thread's 64 old state values of tile `tile` (row `row`, columns
+// 64*half..64*half+63), or zeros when the chunk resets the state.  In the blocked
+// layout a warp's 16-byte loads cover 512 contiguous bytes.
+__device__ __forceinline__ void delta_load_old(const TcParams& p, int tile, int half, int row, float4 (&old)[16]) {
+  Job j;
+  decode_delta(p, tile, j);
+  const bool keep = !p.meta[(size_t)j.b * p.k + j.chunk].has_start;
+  const float4* src = state_tile(p, j);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const size_t idx = ((size_t)((c >> 2) + q) * 128 + row) * 4;
-          old[q] = keep ? *reinterpret_cast<const float4*>(Sb + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        tmem_ld32(tacc + c, r0);
-        tmem_ld32(tacc + c + 32, r1);
-        tmem_ld_wait();
-        uint32_t packed[32];
+  for (int q = 0; q < 16; ++q)
+    old[q] = keep ? src[(16 * half + q) * 128 + row] : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// State update of one 128 x 128 tile (d rows m0.., F columns n0..):
+// S_new = old + alpha eta acc, where `old` already holds S_old (or zeros after a
+// document start).  The bf16 snapshot of this warp's 32 x 64 block is staged in
+// the 128-byte-swizzled layout of a TMA box and stored by lane 0.
+__device__ __forceinline__ void delta_epilogue_tile(const TcParams& p, const Job& j, uint32_t tacc, int half,
+                                                    int quarter, int lane, const float4 (&old)[16],
+                                                    uint8_t* box) {
+  const int row = quarter * 32 + lane;
+  const float ae = p.alpha[(size_t)j.b * p.k + j.chunk] * p.eta;
+  float4* dst = state_tile(p, j);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const uint32_t* src = q < 8 ? &r0[4 * q] : &r1[4 * (q - 8)];
-          float4 nv;
-          nv.x = fmaf(ae, __uint_as_float(src[0]), old[q].x);
-          nv.y = fmaf(ae, __uint_as_float(src[1]), old[q].y);
-          nv.z = fmaf(ae, __uint_as_float(src[2]), old[q].z);
-          nv.w = fmaf(ae, __uint_as_float(src[3]), old[q].w);
-          const size_t idx = ((size_t)((c >> 2) + q) * 128 + row) * 4;
-          *reinterpret_cast<float4*>(Sb + idx) = nv;
-          packed[2 * q] = pack_bf16(nv.x, nv.y);
-          packed[2 * q + 1] = pack_bf16(nv.z, nv.w);
-        }
-        if (p.write_snap) {
-          // Stage this warp's 32 rows x 64 columns (bf16, 128 B per row) in the
-          // 128-byte-swizzled layout of the TMA box, then store the box.
-          uint8_t* buf = snap_stage + (snap_uses & 1) * SNAP_STAGE_BYTES;
-          if (snap_uses >= 2) {
-            if (lane == 0) bulk_wait_read<1>();
-            __syncwarp();
-          }
+  for (int g = 0; g < 2; ++g) {
+    uint32_t r[32];
+    tmem_ld32(tacc + half * 64 + g * 32, r);
+    tmem_ld_wait();
+    uint32_t packed[16];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            uint4 w = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-            *reinterpret_cast<uint4*>(buf + lane * 128 + ((q ^ (lane & 7)) << 4)) = w;
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&p.map[5], buf, j.n0 + c, j.m0 + (row & ~31), p.snap_out * p.B + j.b);
-            bulk_commit();
-          }
-          ++snap_uses;
-        }
-      }
+    for (int q = 0; q < 8; ++q) {
+      const float4 o = old[8 * g + q];
+      float4 nv;
+      nv.x = fmaf(ae, __uint_as_float(r[4 * q + 0]), o.x);
+      nv.y = fmaf(ae, __uint_as_float(r[4 * q + 1]), o.y);
+      nv.z = fmaf(ae, __uint_as_float(r[4 * q + 2]), o.z);
+      nv.w = fmaf(ae, __uint_as_float(r[4 * q + 3]), o.w);
+      dst[(16 * half + 8 * g + q) * 128 + row] = nv;
+      packed[2 * q] = pack_bf16(nv.x, nv.y);
+      packed[2 * q + 1] = pack_bf16(nv.z, nv.w);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int chunk16 = g * 4 + e;  // 16-byte chunk of this row inside the 128-byte box row
+      *reinterpret_cast<uint4*>(box + lane * 128 + ((chunk16 ^ (lane & 7)) << 4)) =
+          make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
     }
   }
 }
@@ -410,10 +428,11 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
 template <int FAM>
 __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__ TcParams p) {
   constexpr int STAGES = Cfg<FAM>::STAGES;
+  constexpr int STAGE_BYTES = Cfg<FAM>::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* epi = smem + STAGES * STAGE_BYTES;
+  uint8_t* epi = smem + STAGES * STAGE_BYTES;    // FAM_DELTA: per-warp snapshot staging boxes
   uint64_t* bars = reinterpret_cast<uint64_t*>(epi + Cfg<FAM>::EPI_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
@@ -423,7 +442,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* counters = reinterpret_cast<uint32_t*>(tmem_slot + 2);  // [0] issued, [1] consumed
-  float* red = reinterpret_cast<float*>(tmem_slot + 4);              // NUM_EPI_WARPS floats
+  float* red = reinterpret_cast<float*>(tmem_slot + 5);              // NUM_EPI_WARPS floats
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -443,8 +462,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    const int nmaps = FAM == FAM_SCAN ? 6 : (FAM == FAM_GRAM ? 2 : (p.kind == K_GATEUP ? 3 : 2));
-    for (int i = 0; i < nmaps; ++i) prefetch_tmap(&p.map[i]);
+    const int first = FAM == FAM_DELTA ? 3 : 0;
+    const int nmaps = FAM == FAM_DELTA ? 3 : (FAM == FAM_APPLY ? 3 : (FAM == FAM_GRAM ? 2 : (p.kind == K_GATEUP ? 3 : 2)));
+    for (int i = 0; i < nmaps; ++i) prefetch_tmap(&p.map[first + i]);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 2 * ACC_COLS);
@@ -469,7 +489,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
             if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) { ok = false; break; }
             uint8_t* sa = stages + s * STAGE_BYTES;
             mbar_arrive_expect_tx(&full[s], j.tx);
-            issue_loads<FAM>(p, j, seg, kb, sa, sa + A_BYTES, &full[s]);
+            issue_loads<FAM>(p, j, seg, kb, sa, sa + Cfg<FAM>::B_OFF, &full[s]);
           }
         }
       }
@@ -496,12 +516,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
             if (!mbar_wait(&full[s], ph) || *abort_flag) { ok = false; break; }
             tc_fence_after();
             const uint32_t a_addr = smem_u32(stages + s * STAGE_BYTES);
-            const uint32_t b_addr = a_addr + A_BYTES;
+            const uint32_t b_addr = a_addr + Cfg<FAM>::B_OFF;
+            constexpr int KB = Cfg<FAM>::KB;
 #pragma unroll
-            for (int ks = 0; ks < BK / 16; ++ks) {
-              const uint64_t ad = j.a_mn ? sdesc_sw128(a_addr + ks * 2048, 64 * 128, 1024)
+            for (int ks = 0; ks < KB / 16; ++ks) {
+              // MN-major: 16 K rows of 128 B per step, MN blocks KB rows apart.
+              const uint64_t ad = j.a_mn ? sdesc_sw128(a_addr + ks * 2048, KB * 128, 1024)
                                          : sdesc_sw128(a_addr + ks * 32, 16, 1024);
-              const uint64_t bd = j.b_mn ? sdesc_sw128(b_addr + ks * 2048, 64 * 128, 1024)
+              const uint64_t bd = j.b_mn ? sdesc_sw128(b_addr + ks * 2048, KB * 128, 1024)
                                          : sdesc_sw128(b_addr + ks * 32, 16, 1024);
               mma_bf16(tacc + j.acc_col[seg], ad, bd, idesc, (kb > j.kb0[seg] || ks > 0) ? 1u : 0u);
             }
@@ -521,24 +543,51 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     const int quarter = warp & 3;      // TMEM lanes this warp may access
     const int half = ew >> 2;          // which half of the columns this warp drains
     const int row = quarter * 32 + lane;
-    uint8_t* snap_stage = epi + ew * 2 * SNAP_STAGE_BYTES;
-    int snap_uses = 0;
+    uint8_t* box = epi + ew * SNAP_BOX_BYTES;  // FAM_DELTA: this warp's snapshot staging box
     uint32_t tcount = 0;
     bool ok = true;
+    float4 old[16];
+    if constexpr (FAM == FAM_DELTA) {
+      if ((int)blockIdx.x < p.n_tiles) delta_load_old(p, blockIdx.x, half, row, old);
+    }
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++tcount) {
       Job j;
       decode<FAM>(p, tile, j);
       const int buf = tcount & 1;
       const uint32_t aph = (tcount >> 1) & 1;
-      // Every epilogue warp leaves only through this wait, so all of them stop at
-      // the same tile and none is left waiting at the epilogue's named barrier.
+      // Every epilogue warp leaves only through this wait (all of them wait on the
+      // same phases), so none is left behind at the epilogue's named barrier.
       if (!mbar_wait(&acc_full[buf], aph)) { ok = false; break; }
       tc_fence_after();
       const uint32_t tacc = tmem_base + buf * ACC_COLS + ((uint32_t)(quarter * 32) << 16);
-      epilogue_tile<FAM>(p, j, tacc, half, row, lane, ew, red, snap_stage, snap_uses);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if constexpr (FAM == FAM_DELTA) {
+        if (tcount >= 1 && p.write_snap) {
+          if (lane == 0) bulk_wait_read<0>();  // the previous tile's store has read the box
+          __syncwarp();
+        }
+        delta_epilogue_tile(p, j, tacc, half, quarter, lane, old, box);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        // Start loading the next tile's old state now; it lands while that tile's
+        // MMAs run.
+        const int next = tile + gridDim.x;
+        if (next < p.n_tiles) delta_load_old(p, next, half, row, old);
+        if (p.write_snap) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&p.map[5], box, j.n0 + 64 * half, j.m0 + 32 * quarter,
+                         ((j.chunk + 1) % p.nslots) * p.B + j.b);
+            bulk_commit();
+          }
+        }
+      } else {
+        epilogue_tile<FAM>(p, j, tacc, half, row, lane, ew, red);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      }
     }
     if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
     if (lane == 0) bulk_wait<0>();
@@ -546,8 +595,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
 
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {
-    // Wait (bounded) for stage loads that were issued but never consumed, so no
-    // TMA write lands in shared memory after the block has exited.
+    // Wait (bounded) for copies that were issued but never consumed, so no TMA
+    // write lands in shared memory after the block has exited.
     for (uint32_t it = counters[1]; it < counters[0]; ++it)
       mbar_wait(&full[it % STAGES], (it / STAGES) & 1);
   }
@@ -606,7 +655,8 @@ cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st) 
   switch (fam) {
     case FAM_ZV: return launch<FAM_ZV>(p, num_sms, st);
     case FAM_GRAM: return launch<FAM_GRAM>(p, num_sms, st);
-    default: return launch<FAM_SCAN>(p, num_sms, st);
+    case FAM_APPLY: return launch<FAM_APPLY>(p, num_sms, st);
+    default: return launch<FAM_DELTA>(p, num_sms, st);
   }
 }
 

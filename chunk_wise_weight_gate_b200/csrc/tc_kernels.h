@@ -9,7 +9,7 @@
 namespace ipttt {
 namespace tck {
 
-enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_SCAN = 2 };
+enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_DELTA = 3 };
 
 struct TcParams {
   CUtensorMap map[6];
@@ -17,11 +17,12 @@ struct TcParams {
   int B, T, d, F, C, k;
   int ct;            // 128-row tiles per chunk (C / 128)
   int npairs;        // GRAM: tile pairs per chunk, ct (ct + 1) / 2
-  int chunk;         // SCAN: chunk index
-  int n_apply;       // SCAN: apply tiles (all rows); delta tiles follow
+  int chunk;         // SCAN: chunk whose state update the delta tiles perform
+  int apply_chunk0;  // SCAN: first chunk of the apply tiles
+  int n_apply;       // SCAN: apply tiles (chunks apply_chunk0.., all rows); delta tiles follow
   int n_tiles;
-  int write_snap;    // SCAN: delta tiles store the bf16 snapshot of S_{i+1}
-  int snap_in, snap_out;  // SCAN: ring slots read by apply / written by delta
+  int write_snap;    // SCAN: delta tiles store the bf16 snapshot of S_{chunk+1}
+  int nslots;        // SCAN: snapshot ring slots; S_i lives in slot i % nslots
   float eta;
   const ChunkMeta* meta;  // [B][k]
   const float* alpha;     // [B][k]
@@ -29,7 +30,7 @@ struct TcParams {
   void* out0;             // Z (gate/up), V (target), O (scan)
   float* out1;            // SCAN: optional fp32 D
   const void* resid;      // SCAN: optional residual H added to O
-  float* S;               // SCAN: fp32 state, blocked 128 x 256 tiles
+  float* S;               // DELTA: fp32 state, blocked 128 x 128 tiles
   int* status;            // device status word
 };
 

@@ -24,7 +24,7 @@ EXPORTS = ("ipttt_workspace_size", "ipttt_forward", "ipttt_forward_ex", "ipttt_c
            "ipttt_stream_reset", "ipttt_stream_forward", "ipttt_stream_export", "ipttt_get_status",
            "ipttt_strerror", "ipttt_version", "ipttt_profile_enable", "ipttt_profile_read",
            "ipttt_kernel_launches")
-PHASES = ("prep", "gate_up", "target", "gram", "scan")
+PHASES = ("prep", "gate_up", "target", "gram", "apply", "update")
 DEBUG_OUTPUTS = ("D", "S_final", "alpha", "Z", "V")
 
 

@@ -43,7 +43,7 @@
  *  - Results are deterministic run to run (no floating-point atomics).
  *  - dtype IPTTT_F32 runs an all-fp32 path (SIMT FMA) for any shape.  dtype
  *    IPTTT_BF16 runs the tensor-core path (tcgen05, fp32 accumulation, fp32 fast
- *    weight state) and needs d % 128 == 0, F % 256 == 0, C % 128 == 0; other shapes
+ *    weight state) and needs d % 128 == 0, F % 128 == 0, C % 128 == 0; other shapes
  *    return IPTTT_ERR_UNSUPPORTED.
  */
 #ifndef IPTTT_H_
@@ -164,10 +164,10 @@ IPTTT_API const char* ipttt_strerror(ipttt_status s);
 
 /* Diagnostics.  While profiling is on, every call records CUDA events on its own
  * stream around each phase: 0 metadata + conv, 1 gate/up GEMM, 2 target GEMM,
- * 3 Gram pass + clip factors, 4 chunk scan (apply + update launches).
- * ipttt_profile_read waits for the recorded events and returns, per phase, the
- * milliseconds and kernel launches accumulated since the previous read
- * (n_phases <= 5); it returns the number of phases written.
+ * 3 Gram pass + clip factors, 4 apply launches of the chunk scan, 5 state-update
+ * launches of the chunk scan.  ipttt_profile_read waits for the recorded events
+ * and returns, per phase, the milliseconds and kernel launches accumulated since
+ * the previous read (n_phases <= 6); it returns the number of phases written.
  * ipttt_kernel_launches counts every kernel this library has launched in the
  * process. */
 IPTTT_API void ipttt_profile_enable(int on);
