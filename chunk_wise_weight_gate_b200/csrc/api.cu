@@ -125,9 +125,13 @@ struct Layout {
 // holds about kApplyTilesPerLaunch tiles (several even waves over the SMs).
 constexpr int kApplyTilesPerLaunch = 1280;
 
+// Token rows of an apply or Gram tile: 128, or 64 for chunks that are odd
+// multiples of 64 (the MMA still spans 128 rows; the upper 64 are not used).
+int tile_rows(const ipttt_params& p) { return p.C % 128 == 0 ? 128 : 64; }
+
 int apply_group(const ipttt_params& p) {
   const int k = (p.T + p.C - 1) / p.C;
-  const long long per_chunk = (long long)p.B * (p.C / 128) * (p.d / 128);
+  const long long per_chunk = (long long)p.B * (p.C / tile_rows(p)) * (p.d / 128);
   long long g = (kApplyTilesPerLaunch + per_chunk - 1) / per_chunk;
   if (g < 1) g = 1;
   if (g > k) g = k;
@@ -161,7 +165,7 @@ Layout layout_of(const ipttt_params& p) {
   L.meta = take(B * k * sizeof(ChunkMeta));
   L.alpha = take(B * k * sizeof(float));
   if (is_bf16(p)) {
-    const size_t ct = s.C / 128;
+    const size_t ct = s.C / tile_rows(p);
     L.partials = take(B * k * (ct * (ct + 1) / 2) * sizeof(float));
     L.Z = take(B * T * F * 2);
     L.U = take(B * T * d * 2);
@@ -195,7 +199,7 @@ ipttt_status check_params(const ipttt_params* p) {
       BT * (long long)p->F > (1ll << 40))
     return IPTTT_ERR_SHAPE;
   if (p->dtype == IPTTT_BF16) {
-    if (p->d % 128 != 0 || p->F % 128 != 0 || p->C % 128 != 0 || p->C > 4096) return IPTTT_ERR_UNSUPPORTED;
+    if (p->d % 128 != 0 || p->F % 128 != 0 || p->C % 64 != 0 || p->C > 4096) return IPTTT_ERR_UNSUPPORTED;
   }
   return IPTTT_OK;
 }
@@ -273,7 +277,8 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   tp.F = s.F;
   tp.C = s.C;
   tp.k = s.k;
-  tp.ct = s.C / 128;
+  tp.tr = tile_rows(p);
+  tp.ct = s.C / tp.tr;
   tp.npairs = tp.ct * (tp.ct + 1) / 2;
   tp.eta = p.eta;
   tp.meta = meta;
@@ -311,8 +316,8 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   {
     PhaseScope ph(st, PH_GRAM);
     TcParams g = tp;
-    if (!make_map_bf16(&g.map[0], Z, s.F, s.T, s.B, 64, 128) ||
-        !make_map_bf16(&g.map[1], V, s.d, s.T, s.B, 64, 128))
+    if (!make_map_bf16(&g.map[0], Z, s.F, s.T, s.B, 64, tp.tr) ||
+        !make_map_bf16(&g.map[1], V, s.d, s.T, s.B, 64, tp.tr))
       return IPTTT_ERR_CUDA;
     g.partials = partials;
     g.n_tiles = s.B * s.k * tp.npairs;
@@ -335,11 +340,13 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   // then the update of chunk b-1 (writes S_b into the slot S_a has left).
   const int G = L.group;
   TcParams sc = tp;
-  if (!make_map_bf16(&sc.map[0], Z, s.F, s.T, s.B, 64, 128) ||
+  const int delta_fam = s.C % 128 == 0 ? FAM_DELTA : FAM_DELTA64;
+  const int delta_kb = s.C % 128 == 0 ? 128 : 64;
+  if (!make_map_bf16(&sc.map[0], Z, s.F, s.T, s.B, 64, tp.tr) ||
       !make_map_bf16(&sc.map[1], t.W0, s.F, s.d, 1, 64, 128) ||
       !make_map_bf16(&sc.map[2], snap, s.F, s.d, (uint64_t)G * s.B, 64, 128) ||
-      !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, 128) ||
-      !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, 128) ||
+      !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, delta_kb) ||
+      !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, delta_kb) ||
       !make_map_bf16(&sc.map[5], snap, s.F, s.d, (uint64_t)G * s.B, 64, 32))
     return IPTTT_ERR_CUDA;
   sc.out0 = t.O;
@@ -358,7 +365,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     q.apply_chunk0 = 0;
     q.n_apply = 0;
     q.n_tiles = delta_tiles;
-    IP_CHECK(launch_tc(FAM_DELTA, q, di->num_sms, st));
+    IP_CHECK(launch_tc(delta_fam, q, di->num_sms, st));
     counted(1);
     return IPTTT_OK;
   };

@@ -21,10 +21,13 @@
 //            snapshot [notes, 步骤一 and 工程实现; iplexlaw.co.kr review §3: a chunk's output
 //            comes from the pre-update state].
 //   FAM_DELTA the state update of one chunk: S_{i+1} = keep_i S_i + alpha_i eta V_i^T Z_i
-//            on 128 x 128 tiles of the fp32 state, which move between HBM and shared
-//            memory as contiguous 64 KB bulk copies, plus the bf16 snapshot of S_{i+1}
+//            on 128 x 128 tiles of the fp32 state (kept in a blocked layout whose
+//            rows match the TMEM lanes, so every warp access is 512 contiguous bytes;
+//            the next tile's old state is loaded into registers while the current
+//            tile's MMAs run), plus the bf16 snapshot of S_{i+1} stored with TMA
 //            [notes, 步骤二 and the Hebbian rule; iplexlaw.co.kr review §6 exclusive scan
-//            and document reset].
+//            and document reset].  FAM_DELTA64 is the same with 64-token stages, for
+//            chunk sizes that are odd multiples of 64.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -62,11 +65,17 @@ template <> struct Cfg<FAM_APPLY> {
   static constexpr int STAGES = 4, STAGE_BYTES = 48 * 1024, KB = 64, B_OFF = A_BYTES, EPI_BYTES = 0;
 };
 // The update contracts over tokens with MN-major operands; 128-token stages keep
-// every TMA box at 16 KB (128 rows of 128 bytes).
+// every TMA box at 16 KB (128 rows of 128 bytes).  Chunks of 64 (mod 128) tokens
+// use 64-token stages.
 template <> struct Cfg<FAM_DELTA> {
   static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 128, B_OFF = 32 * 1024,
                        EPI_BYTES = NUM_EPI_WARPS * SNAP_BOX_BYTES;
 };
+template <> struct Cfg<FAM_DELTA64> {
+  static constexpr int STAGES = 5, STAGE_BYTES = 32 * 1024, KB = 64, B_OFF = 16 * 1024,
+                       EPI_BYTES = NUM_EPI_WARPS * SNAP_BOX_BYTES;
+};
+template <int FAM> constexpr bool is_delta() { return FAM == FAM_DELTA || FAM == FAM_DELTA64; }
 
 template <int FAM>
 constexpr int smem_bytes() {
@@ -74,6 +83,7 @@ constexpr int smem_bytes() {
          256 /*barriers*/;
 }
 static_assert(smem_bytes<FAM_DELTA>() <= 232448, "delta kernel exceeds shared memory");
+static_assert(smem_bytes<FAM_DELTA64>() <= 232448, "delta kernel exceeds shared memory");
 static_assert(smem_bytes<FAM_ZV>() <= 232448, "kernel exceeds shared memory");
 
 struct Job {
@@ -141,15 +151,15 @@ __device__ __forceinline__ void decode_gram(const TcParams& p, int tile, Job& j)
   j.pair = r % p.npairs;
   int ti = 0, rem = j.pair;
   while (rem >= p.ct - ti) { rem -= p.ct - ti; ++ti; }
-  j.m0 = ti * BM;
-  j.n0 = (ti + rem) * BM;
+  j.m0 = ti * p.tr;
+  j.n0 = (ti + rem) * p.tr;
   j.t0 = j.chunk * p.C;
   j.nseg = 2;
   j.kb0[0] = 0; j.kb1[0] = p.F / BK; j.acc_col[0] = 0;     // Z Z^T
   j.kb0[1] = 0; j.kb1[1] = p.d / BK; j.acc_col[1] = 128;   // V V^T
   j.n_mma = 128;
   j.nsrc = 1;
-  j.tx = A_BYTES + 128 * BK * 2;
+  j.tx = 2 * p.tr * BK * 2;
   j.a_mn = false;
   j.b_mn = false;
 }
@@ -163,7 +173,7 @@ __device__ __forceinline__ void decode_apply(const TcParams& p, int tile, Job& j
   j.t0 = j.chunk * p.C;
   j.b = (tile % per_chunk) / per_row;
   const int r = tile % per_row;
-  j.m0 = (r / tiles_n) * BM;      // row offset inside the chunk
+  j.m0 = (r / tiles_n) * p.tr;    // row offset inside the chunk
   j.n0 = (r % tiles_n) * 128;     // output column (d index)
   j.pair = 0;
   j.nseg = 1;
@@ -172,11 +182,12 @@ __device__ __forceinline__ void decode_apply(const TcParams& p, int tile, Job& j
   j.kb0[0] = 0;
   j.kb1[0] = p.F / BK;
   j.n_mma = 128 * j.nsrc;
-  j.tx = A_BYTES + j.nsrc * 128 * BK * 2;
+  j.tx = p.tr * BK * 2 + j.nsrc * 128 * BK * 2;
   j.a_mn = false;
   j.b_mn = false;
 }
 
+template <int KB>
 __device__ __forceinline__ void decode_delta(const TcParams& p, int tile, Job& j) {
   const int tiles_n = p.F / 128;
   const int per_row = (p.d / 128) * tiles_n;
@@ -190,7 +201,6 @@ __device__ __forceinline__ void decode_delta(const TcParams& p, int tile, Job& j
   j.pair = 0;
   j.nseg = 1;
   j.acc_col[0] = 0;
-  constexpr int KB = Cfg<FAM_DELTA>::KB;
   const int rows = min(p.C, p.T - j.t0);
   j.kb0[0] = (p.meta[(size_t)j.b * p.k + j.chunk].last_start - j.t0) / KB;
   j.kb1[0] = cdiv(rows, KB);
@@ -206,7 +216,7 @@ __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
   if constexpr (FAM == FAM_ZV) decode_zv(p, tile, j);
   else if constexpr (FAM == FAM_GRAM) decode_gram(p, tile, j);
   else if constexpr (FAM == FAM_APPLY) decode_apply(p, tile, j);
-  else decode_delta(p, tile, j);
+  else decode_delta<Cfg<FAM>::KB>(p, tile, j);
 }
 
 // ------------------------------------------------------------------ producer
@@ -234,7 +244,7 @@ __device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int
     if (j.nsrc == 2)
       tma_load_3d(sb + 128 * BK * 2, &p.map[2], bar, kx, j.n0, (j.chunk % p.nslots) * p.B + j.b);  // S_i rows
   } else {
-    constexpr int KB = Cfg<FAM_DELTA>::KB;
+    constexpr int KB = Cfg<FAM>::KB;
     const int ty = j.t0 + kb * KB;                                 // token rows = K
     tma_load_3d(sa, &p.map[3], bar, j.m0, ty, j.b);                // V[t][d], d contiguous
     tma_load_3d(sa + 64 * KB * 2, &p.map[3], bar, j.m0 + 64, ty, j.b);
@@ -301,14 +311,18 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
       }
     }
   } else if constexpr (FAM == FAM_GRAM) {
+    // Only rows and columns below tr hold Gram entries of this tile pair.
     float s = 0.0f;
 #pragma unroll 1
     for (int c = half * 64; c < half * 64 + 64; c += 32) {
+      if (c >= p.tr) break;  // warp-uniform
       tmem_ld32(tacc + c, r0);
       tmem_ld32(tacc + 128 + c, r1);
       tmem_ld_wait();
+      if (row < p.tr) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) s = fmaf(__uint_as_float(r0[i]), __uint_as_float(r1[i]), s);
+        for (int i = 0; i < 32; ++i) s = fmaf(__uint_as_float(r0[i]), __uint_as_float(r1[i]), s);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -324,7 +338,7 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
   } else if constexpr (FAM == FAM_APPLY) {
     const ChunkMeta m = p.meta[(size_t)j.b * p.k + j.chunk];
     const int t = j.t0 + j.m0 + row;
-    const bool valid = t < p.T;
+    const bool valid = row < p.tr && t < p.T;
     const bool carry = j.nsrc == 2 && m.cont && t < m.first_end;
     __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.d + j.n0;
     const __nv_bfloat16* hrow =
@@ -377,9 +391,10 @@ __device__ __forceinline__ float4* state_tile(const TcParams& p, const Job& j) {
 // This thread's 64 old state values of tile `tile` (row `row`, columns
 // 64*half..64*half+63), or zeros when the chunk resets the state.  In the blocked
 // layout a warp's 16-byte loads cover 512 contiguous bytes.
+template <int KB>
 __device__ __forceinline__ void delta_load_old(const TcParams& p, int tile, int half, int row, float4 (&old)[16]) {
   Job j;
-  decode_delta(p, tile, j);
+  decode_delta<KB>(p, tile, j);
   const bool keep = !p.meta[(size_t)j.b * p.k + j.chunk].has_start;
   const float4* src = state_tile(p, j);
 #pragma unroll
@@ -462,8 +477,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    const int first = FAM == FAM_DELTA ? 3 : 0;
-    const int nmaps = FAM == FAM_DELTA ? 3 : (FAM == FAM_APPLY ? 3 : (FAM == FAM_GRAM ? 2 : (p.kind == K_GATEUP ? 3 : 2)));
+    const int first = is_delta<FAM>() ? 3 : 0;
+    const int nmaps = is_delta<FAM>() ? 3 : (FAM == FAM_APPLY ? 3 : (FAM == FAM_GRAM ? 2 : (p.kind == K_GATEUP ? 3 : 2)));
     for (int i = 0; i < nmaps; ++i) prefetch_tmap(&p.map[first + i]);
   }
   if (warp == 1) {
@@ -547,8 +562,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     uint32_t tcount = 0;
     bool ok = true;
     float4 old[16];
-    if constexpr (FAM == FAM_DELTA) {
-      if ((int)blockIdx.x < p.n_tiles) delta_load_old(p, blockIdx.x, half, row, old);
+    if constexpr (is_delta<FAM>()) {
+      if ((int)blockIdx.x < p.n_tiles) delta_load_old<Cfg<FAM>::KB>(p, blockIdx.x, half, row, old);
     }
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++tcount) {
       Job j;
@@ -560,7 +575,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
       if (!mbar_wait(&acc_full[buf], aph)) { ok = false; break; }
       tc_fence_after();
       const uint32_t tacc = tmem_base + buf * ACC_COLS + ((uint32_t)(quarter * 32) << 16);
-      if constexpr (FAM == FAM_DELTA) {
+      if constexpr (is_delta<FAM>()) {
         if (tcount >= 1 && p.write_snap) {
           if (lane == 0) bulk_wait_read<0>();  // the previous tile's store has read the box
           __syncwarp();
@@ -572,7 +587,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
         // Start loading the next tile's old state now; it lands while that tile's
         // MMAs run.
         const int next = tile + gridDim.x;
-        if (next < p.n_tiles) delta_load_old(p, next, half, row, old);
+        if (next < p.n_tiles) delta_load_old<Cfg<FAM>::KB>(p, next, half, row, old);
         if (p.write_snap) {
           fence_proxy_async_smem();
           __syncwarp();
@@ -656,6 +671,7 @@ cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st) 
     case FAM_ZV: return launch<FAM_ZV>(p, num_sms, st);
     case FAM_GRAM: return launch<FAM_GRAM>(p, num_sms, st);
     case FAM_APPLY: return launch<FAM_APPLY>(p, num_sms, st);
+    case FAM_DELTA64: return launch<FAM_DELTA64>(p, num_sms, st);
     default: return launch<FAM_DELTA>(p, num_sms, st);
   }
 }

@@ -9,13 +9,14 @@
 namespace ipttt {
 namespace tck {
 
-enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_DELTA = 3 };
+enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_DELTA = 3, FAM_DELTA64 = 4 };
 
 struct TcParams {
   CUtensorMap map[6];
   int kind;          // FAM_ZV: kind_gateup() or kind_vhat()
   int B, T, d, F, C, k;
-  int ct;            // 128-row tiles per chunk (C / 128)
+  int tr;            // token rows per apply / Gram tile: 128, or 64 when C % 128 != 0
+  int ct;            // tiles per chunk (C / tr)
   int npairs;        // GRAM: tile pairs per chunk, ct (ct + 1) / 2
   int chunk;         // SCAN: chunk whose state update the delta tiles perform
   int apply_chunk0;  // SCAN: first chunk of the apply tiles

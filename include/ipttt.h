@@ -43,7 +43,7 @@
  *  - Results are deterministic run to run (no floating-point atomics).
  *  - dtype IPTTT_F32 runs an all-fp32 path (SIMT FMA) for any shape.  dtype
  *    IPTTT_BF16 runs the tensor-core path (tcgen05, fp32 accumulation, fp32 fast
- *    weight state) and needs d % 128 == 0, F % 128 == 0, C % 128 == 0; other shapes
+ *    weight state) and needs d % 128 == 0, F % 128 == 0, C % 64 == 0; other shapes
  *    return IPTTT_ERR_UNSUPPORTED.
  */
 #ifndef IPTTT_H_

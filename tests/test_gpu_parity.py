@@ -73,6 +73,9 @@ BF16_CASES = {
     "noclip_docs_ragged": dict(B=2, T=777, C=128, d=256, F=512, eta=2e-2, clip=0.0,
                                docs=[129, 500, 777 + 1, 777 + 384]),
     "long_chunk": dict(B=1, T=2048, C=1024, d=256, F=512, eta=1e-3, clip=1e-5),
+    "chunk64_docs_ragged": dict(B=2, T=700, C=64, d=256, F=384, eta=2e-2, clip=0.0,
+                                docs=[70, 200, 201, 700 + 64, 700 + 450]),
+    "chunk192_clip": dict(B=1, T=1000, C=192, d=128, F=256, eta=1e-3, clip=1e-5),
 }
 
 
