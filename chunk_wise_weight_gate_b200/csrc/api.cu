@@ -129,9 +129,13 @@ constexpr int kApplyTilesPerLaunch = 1280;
 // multiples of 64 (the MMA still spans 128 rows; the upper 64 are not used).
 int tile_rows(const ipttt_params& p) { return p.C % 128 == 0 ? 128 : 64; }
 
+// Token rows of an apply tile: 256 (two M=128 MMAs per B stage) when the chunk
+// allows it, else the Gram tile rows.
+int apply_rows(const ipttt_params& p) { return p.C % 256 == 0 ? 256 : tile_rows(p); }
+
 int apply_group(const ipttt_params& p) {
   const int k = (p.T + p.C - 1) / p.C;
-  const long long per_chunk = (long long)p.B * (p.C / tile_rows(p)) * (p.d / 128);
+  const long long per_chunk = (long long)p.B * (p.C / apply_rows(p)) * (p.d / 128);
   long long g = (kApplyTilesPerLaunch + per_chunk - 1) / per_chunk;
   if (g < 1) g = 1;
   if (g > k) g = k;
@@ -340,9 +344,11 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   // then the update of chunk b-1 (writes S_b into the slot S_a has left).
   const int G = L.group;
   TcParams sc = tp;
+  const int arows = apply_rows(p);
+  const int apply_fam = arows == 256 ? FAM_APPLY256 : FAM_APPLY;
   const int delta_fam = s.C % 128 == 0 ? FAM_DELTA : FAM_DELTA64;
   const int delta_kb = s.C % 128 == 0 ? 128 : 64;
-  if (!make_map_bf16(&sc.map[0], Z, s.F, s.T, s.B, 64, tp.tr) ||
+  if (!make_map_bf16(&sc.map[0], Z, s.F, s.T, s.B, 64, arows == 256 ? 128 : tp.tr) ||
       !make_map_bf16(&sc.map[1], t.W0, s.F, s.d, 1, 64, 128) ||
       !make_map_bf16(&sc.map[2], snap, s.F, s.d, (uint64_t)G * s.B, 64, 128) ||
       !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, delta_kb) ||
@@ -356,7 +362,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   sc.nslots = G;
   const bool need_final = t.Sfinal != nullptr || ss != nullptr;
   const int delta_tiles = s.B * (s.d / 128) * (s.F / 128);
-  const int apply_tiles_per_chunk = s.B * sc.ct * (s.d / 128);
+  const int apply_tiles_per_chunk = s.B * (s.C / arows) * (s.d / 128);
   auto delta = [&](int j) -> ipttt_status {
     PhaseScope ph(st, PH_UPDATE);
     TcParams q = sc;
@@ -381,7 +387,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
       q.apply_chunk0 = a;
       q.n_apply = (b - a) * apply_tiles_per_chunk;
       q.n_tiles = q.n_apply;
-      IP_CHECK(launch_tc(FAM_APPLY, q, di->num_sms, st));
+      IP_CHECK(launch_tc(apply_fam, q, di->num_sms, st));
       counted(1);
     }
     if (b < s.k || need_final)

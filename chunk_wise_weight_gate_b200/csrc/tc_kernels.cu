@@ -56,25 +56,33 @@ enum Kind { K_GATEUP = 0, K_VHAT = 1, K_GRAM = 2, K_APPLY = 3, K_DELTA = 4 };
 // of the B operand inside a stage, and shared memory for the epilogue.
 template <int FAM> struct Cfg;
 template <> struct Cfg<FAM_ZV> {
-  static constexpr int STAGES = 4, STAGE_BYTES = 48 * 1024, KB = 64, B_OFF = A_BYTES, EPI_BYTES = 0;
+  static constexpr int STAGES = 4, STAGE_BYTES = 48 * 1024, KB = 64, B_OFF = A_BYTES, EPI_BYTES = 0, NBUF = 2;
 };
 template <> struct Cfg<FAM_GRAM> {
-  static constexpr int STAGES = 6, STAGE_BYTES = 32 * 1024, KB = 64, B_OFF = A_BYTES, EPI_BYTES = 0;
+  static constexpr int STAGES = 6, STAGE_BYTES = 32 * 1024, KB = 64, B_OFF = A_BYTES, EPI_BYTES = 0, NBUF = 2;
 };
 template <> struct Cfg<FAM_APPLY> {
-  static constexpr int STAGES = 4, STAGE_BYTES = 48 * 1024, KB = 64, B_OFF = A_BYTES, EPI_BYTES = 0;
+  static constexpr int STAGES = 4, STAGE_BYTES = 48 * 1024, KB = 64, B_OFF = A_BYTES, EPI_BYTES = 0, NBUF = 2;
+};
+// 256 token rows per apply tile: two M=128 MMAs share every B stage, so a byte
+// fetched from L2 feeds twice the flops; the two accumulators fill all of TMEM
+// (no double buffering; the epilogue is short next to the K = d_ff mainloop).
+template <> struct Cfg<FAM_APPLY256> {
+  static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 64, B_OFF = 2 * A_BYTES, EPI_BYTES = 0,
+                       NBUF = 1;
 };
 // The update contracts over tokens with MN-major operands; 128-token stages keep
 // every TMA box at 16 KB (128 rows of 128 bytes).  Chunks of 64 (mod 128) tokens
 // use 64-token stages.
 template <> struct Cfg<FAM_DELTA> {
   static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 128, B_OFF = 32 * 1024,
-                       EPI_BYTES = NUM_EPI_WARPS * SNAP_BOX_BYTES;
+                       EPI_BYTES = NUM_EPI_WARPS * SNAP_BOX_BYTES, NBUF = 2;
 };
 template <> struct Cfg<FAM_DELTA64> {
   static constexpr int STAGES = 5, STAGE_BYTES = 32 * 1024, KB = 64, B_OFF = 16 * 1024,
-                       EPI_BYTES = NUM_EPI_WARPS * SNAP_BOX_BYTES;
+                       EPI_BYTES = NUM_EPI_WARPS * SNAP_BOX_BYTES, NBUF = 2;
 };
+template <int FAM> constexpr bool is_apply() { return FAM == FAM_APPLY || FAM == FAM_APPLY256; }
 template <int FAM> constexpr bool is_delta() { return FAM == FAM_DELTA || FAM == FAM_DELTA64; }
 
 template <int FAM>
@@ -100,6 +108,7 @@ struct Job {
   int nsrc;       // APPLY: 1 = W0 only, 2 = W0 and the state snapshot
   uint32_t tx;    // bytes per stage
   bool a_mn, b_mn;
+  int halves;     // M=128 MMAs per K step (2: A holds 256 rows, accumulators 256 columns apart)
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -164,16 +173,18 @@ __device__ __forceinline__ void decode_gram(const TcParams& p, int tile, Job& j)
   j.b_mn = false;
 }
 
+template <int ROWS>  // 0: p.tr rows per tile; 256: two 128-row halves
 __device__ __forceinline__ void decode_apply(const TcParams& p, int tile, Job& j) {
+  const int rows = ROWS ? ROWS : p.tr;
   const int tiles_n = p.d / 128;
-  const int per_row = p.ct * tiles_n;
+  const int per_row = (p.C / rows) * tiles_n;
   const int per_chunk = p.B * per_row;
   j.kind = K_APPLY;
   j.chunk = p.apply_chunk0 + tile / per_chunk;
   j.t0 = j.chunk * p.C;
   j.b = (tile % per_chunk) / per_row;
   const int r = tile % per_row;
-  j.m0 = (r / tiles_n) * p.tr;    // row offset inside the chunk
+  j.m0 = (r / tiles_n) * rows;    // row offset inside the chunk
   j.n0 = (r % tiles_n) * 128;     // output column (d index)
   j.pair = 0;
   j.nseg = 1;
@@ -182,7 +193,8 @@ __device__ __forceinline__ void decode_apply(const TcParams& p, int tile, Job& j
   j.kb0[0] = 0;
   j.kb1[0] = p.F / BK;
   j.n_mma = 128 * j.nsrc;
-  j.tx = p.tr * BK * 2 + j.nsrc * 128 * BK * 2;
+  j.tx = rows * BK * 2 + j.nsrc * 128 * BK * 2;
+  j.halves = ROWS == 256 ? 2 : 1;
   j.a_mn = false;
   j.b_mn = false;
 }
@@ -213,9 +225,11 @@ __device__ __forceinline__ void decode_delta(const TcParams& p, int tile, Job& j
 
 template <int FAM>
 __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
+  j.halves = 1;
   if constexpr (FAM == FAM_ZV) decode_zv(p, tile, j);
   else if constexpr (FAM == FAM_GRAM) decode_gram(p, tile, j);
-  else if constexpr (FAM == FAM_APPLY) decode_apply(p, tile, j);
+  else if constexpr (FAM == FAM_APPLY) decode_apply<0>(p, tile, j);
+  else if constexpr (FAM == FAM_APPLY256) decode_apply<256>(p, tile, j);
   else decode_delta<Cfg<FAM>::KB>(p, tile, j);
 }
 
@@ -238,8 +252,9 @@ __device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int
     const CUtensorMap* m = seg == 0 ? &p.map[0] : &p.map[1];       // Z or V
     tma_load_3d(sa, m, bar, kx, j.t0 + j.m0, j.b);
     tma_load_3d(sb, m, bar, kx, j.t0 + j.n0, j.b);
-  } else if constexpr (FAM == FAM_APPLY) {
+  } else if constexpr (is_apply<FAM>()) {
     tma_load_3d(sa, &p.map[0], bar, kx, j.t0 + j.m0, j.b);        // Z rows of the chunk
+    if (j.halves == 2) tma_load_3d(sa + A_BYTES, &p.map[0], bar, kx, j.t0 + j.m0 + 128, j.b);
     tma_load_3d(sb, &p.map[1], bar, kx, j.n0, 0);                 // Wdown0 rows
     if (j.nsrc == 2)
       tma_load_3d(sb + 128 * BK * 2, &p.map[2], bar, kx, j.n0, (j.chunk % p.nslots) * p.B + j.b);  // S_i rows
@@ -335,17 +350,24 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
       p.partials[((size_t)j.b * p.k + j.chunk) * p.npairs + j.pair] = wgt * tot;
     }
     epi_sync();
-  } else if constexpr (FAM == FAM_APPLY) {
+  } else if constexpr (is_apply<FAM>()) {
+    // FAM_APPLY: this warp drains columns [64 half, 64 half + 64) of a 128-row tile;
+    // FAM_APPLY256: all 128 columns of rows 128 half .. of a 256-row tile, whose
+    // accumulator sits 256 TMEM columns further for the upper half.
+    constexpr bool two = FAM == FAM_APPLY256;
+    const int row_in_tile = two ? half * 128 + row : row;
+    if (two) tacc += half * 256;
+    const int c_begin = two ? 0 : half * 64, c_end = two ? 128 : half * 64 + 64;
     const ChunkMeta m = p.meta[(size_t)j.b * p.k + j.chunk];
-    const int t = j.t0 + j.m0 + row;
-    const bool valid = row < p.tr && t < p.T;
+    const int t = j.t0 + j.m0 + row_in_tile;
+    const bool valid = (two || row < p.tr) && t < p.T;
     const bool carry = j.nsrc == 2 && m.cont && t < m.first_end;
     __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.d + j.n0;
     const __nv_bfloat16* hrow =
         p.resid ? reinterpret_cast<const __nv_bfloat16*>(p.resid) + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
     float* drow = p.out1 ? p.out1 + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
 #pragma unroll 1
-    for (int c = half * 64; c < half * 64 + 64; c += 32) {
+    for (int c = c_begin; c < c_end; c += 32) {
       tmem_ld32(tacc + c, r0);
       if (j.nsrc == 2) tmem_ld32(tacc + 128 + c, r1);
       tmem_ld_wait();
@@ -478,7 +500,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
   }
   if (warp == 0 && lane == 0) {
     const int first = is_delta<FAM>() ? 3 : 0;
-    const int nmaps = is_delta<FAM>() ? 3 : (FAM == FAM_APPLY ? 3 : (FAM == FAM_GRAM ? 2 : (p.kind == K_GATEUP ? 3 : 2)));
+    const int nmaps = is_delta<FAM>() ? 3 : (is_apply<FAM>() ? 3 : (FAM == FAM_GRAM ? 2 : (p.kind == K_GATEUP ? 3 : 2)));
     for (int i = 0; i < nmaps; ++i) prefetch_tmap(&p.map[first + i]);
   }
   if (warp == 1) {
@@ -518,8 +540,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
       for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++tcount) {
         Job j;
         decode<FAM>(p, tile, j);
-        const int buf = tcount & 1;
-        const uint32_t aph = (tcount >> 1) & 1;
+        const int buf = Cfg<FAM>::NBUF == 2 ? (tcount & 1) : 0;
+        const uint32_t aph = Cfg<FAM>::NBUF == 2 ? ((tcount >> 1) & 1) : (tcount & 1);
         if (!mbar_wait(&acc_empty[buf], aph ^ 1) || *abort_flag) { ok = false; break; }
         tc_fence_after();
         const uint32_t tacc = tmem_base + buf * ACC_COLS;
@@ -540,7 +562,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
                                          : sdesc_sw128(a_addr + ks * 32, 16, 1024);
               const uint64_t bd = j.b_mn ? sdesc_sw128(b_addr + ks * 2048, KB * 128, 1024)
                                          : sdesc_sw128(b_addr + ks * 32, 16, 1024);
-              mma_bf16(tacc + j.acc_col[seg], ad, bd, idesc, (kb > j.kb0[seg] || ks > 0) ? 1u : 0u);
+              const uint32_t acc_flag = (kb > j.kb0[seg] || ks > 0) ? 1u : 0u;
+              mma_bf16(tacc + j.acc_col[seg], ad, bd, idesc, acc_flag);
+              if (j.halves == 2)  // rows 128..255 of A (K-major, 16 KB further), next 256 columns
+                mma_bf16(tacc + 256 + j.acc_col[seg], sdesc_sw128(a_addr + A_BYTES + ks * 32, 16, 1024), bd,
+                         idesc, acc_flag);
             }
             mma_commit(&empty[s]);
           }
@@ -568,8 +594,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++tcount) {
       Job j;
       decode<FAM>(p, tile, j);
-      const int buf = tcount & 1;
-      const uint32_t aph = (tcount >> 1) & 1;
+      const int buf = Cfg<FAM>::NBUF == 2 ? (tcount & 1) : 0;
+      const uint32_t aph = Cfg<FAM>::NBUF == 2 ? ((tcount >> 1) & 1) : (tcount & 1);
       // Every epilogue warp leaves only through this wait (all of them wait on the
       // same phases), so none is left behind at the epilogue's named barrier.
       if (!mbar_wait(&acc_full[buf], aph)) { ok = false; break; }
@@ -672,6 +698,7 @@ cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st) 
     case FAM_GRAM: return launch<FAM_GRAM>(p, num_sms, st);
     case FAM_APPLY: return launch<FAM_APPLY>(p, num_sms, st);
     case FAM_DELTA64: return launch<FAM_DELTA64>(p, num_sms, st);
+    case FAM_APPLY256: return launch<FAM_APPLY256>(p, num_sms, st);
     default: return launch<FAM_DELTA>(p, num_sms, st);
   }
 }

@@ -9,7 +9,7 @@
 namespace ipttt {
 namespace tck {
 
-enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_DELTA = 3, FAM_DELTA64 = 4 };
+enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_DELTA = 3, FAM_DELTA64 = 4, FAM_APPLY256 = 5 };
 
 struct TcParams {
   CUtensorMap map[6];
