@@ -110,6 +110,15 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(x: float, pg, device) -> float:
+    """Max of x over all ranks of the default process group (identity when pg is None)."""
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
 def layer_flops(w: synth.Workload) -> int:
     """Credited flops of one step (all layers): 10 d F + 2 d^2 + 10 d per token."""
     return ip.flops_per_token(w.d, w.F) * w.B * w.T * w.layers
@@ -127,6 +136,7 @@ def phase_flops(w: synth.Workload) -> dict:
         "gram": 2 * B * k * (ct * (ct + 1) // 2) * 128 * 128 * (d + F),
         "apply": 4 * B * T * d * F,
         "update": 2 * B * T * d * F,
+        "scan": 6 * B * T * d * F,
     }
 
 
@@ -261,11 +271,7 @@ def run_ours(args, w: synth.Workload):
     ip.profile_enable(False)
     launches = ip.kernel_launches() - launches0
     phases = ip.profile_read()
-    ms = e0.elapsed_time(e1) / args.steps
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, pg, dev)
     status = ip.get_status()
 
     tokens = w.B * w.T * w.layers
@@ -313,11 +319,7 @@ def run_ours(args, w: synth.Workload):
             o_host.copy_(O, non_blocking=True)
         a1.record(stream)
         torch.cuda.synchronize()
-        ems = a0.elapsed_time(a1) / args.steps
-        if pg:
-            t = torch.tensor([ems], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(a0.elapsed_time(a1) / args.steps, pg, dev)
         h2d = sum(v.numel() * v.element_size() for v in host.values())
         e2e = {"value": world * tokens / (ems / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": o_host.numel() * o_host.element_size(), "ms_per_step": ems}

@@ -648,4 +648,14 @@ int ipttt_profile_read(double* ms, uint64_t* launches, int n_phases) {
 
 uint64_t ipttt_kernel_launches(void) { return g_launches.load(); }
 
+ipttt_status ipttt_selftest_wait_timeout(uint32_t limit_ns, void* stream) {
+  DeviceInfo* di = nullptr;
+  ipttt_status rc = device_info(&di);
+  if (rc != IPTTT_OK) return rc;
+  const uint64_t lim = limit_ns ? limit_ns : 2000000000ull;
+  rc = cuda_status(tck::launch_wait_timeout(di->status, lim, static_cast<cudaStream_t>(stream)));
+  if (rc == IPTTT_OK) counted(1);
+  return rc;
+}
+
 }  // extern "C"

@@ -648,6 +648,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
   }
 }
 
+// ------------------------------------------------------------------ failure-path self test
+// One thread waits, with the kernels' bounded wait, on an mbarrier phase that
+// nothing completes; when the limit passes it records a timeout in the status word.
+__global__ void k_wait_timeout(int* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait(&bar, 0, limit_ns)) set_status(status, IPTTT_ERR_TIMEOUT);
+  }
+}
+
+cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st) {
+  k_wait_timeout<<<1, 32, 0, st>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ host side
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;

@@ -38,6 +38,7 @@ struct TcParams {
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
                    uint32_t box_inner, uint32_t box_rows);
 cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st);
+cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st);
 int kind_gateup();
 int kind_vhat();
 

@@ -23,7 +23,7 @@ STATUS = {0: "IPTTT_OK", 1: "IPTTT_ERR_ARG", 2: "IPTTT_ERR_SHAPE", 3: "IPTTT_ERR
 EXPORTS = ("ipttt_workspace_size", "ipttt_forward", "ipttt_forward_ex", "ipttt_core", "ipttt_stream_state_size",
            "ipttt_stream_reset", "ipttt_stream_forward", "ipttt_stream_export", "ipttt_get_status",
            "ipttt_strerror", "ipttt_version", "ipttt_profile_enable", "ipttt_profile_read",
-           "ipttt_kernel_launches")
+           "ipttt_kernel_launches", "ipttt_selftest_wait_timeout")
 PHASES = ("prep", "gate_up", "target", "gram", "apply", "update")
 DEBUG_OUTPUTS = ("D", "S_final", "alpha", "Z", "V")
 
@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.ipttt_profile_read.restype = ctypes.c_int
         L.ipttt_kernel_launches.argtypes = []
         L.ipttt_kernel_launches.restype = ctypes.c_uint64
+        L.ipttt_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
+        L.ipttt_selftest_wait_timeout.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -282,6 +284,11 @@ def profile_read() -> dict:
     ln = (ctypes.c_uint64 * n)()
     lib().ipttt_profile_read(ms, ln, n)
     return {PHASES[i]: (float(ms[i]), int(ln[i])) for i in range(n)}
+
+
+def selftest_wait_timeout(limit_ns: int = 100_000_000, stream=None):
+    """Runs the bounded-wait failure path on the device (see include/ipttt.h)."""
+    _check(lib().ipttt_selftest_wait_timeout(int(limit_ns), _stream(stream)), "ipttt_selftest_wait_timeout")
 
 
 def kernel_launches() -> int:

@@ -174,6 +174,13 @@ IPTTT_API void ipttt_profile_enable(int on);
 IPTTT_API int ipttt_profile_read(double* ms, uint64_t* launches, int n_phases);
 IPTTT_API uint64_t ipttt_kernel_launches(void);
 
+/* Self-test of the device-side failure path: launches one block that waits, with
+ * the same bounded wait the kernels use, on a barrier phase that nothing ever
+ * completes.  After limit_ns nanoseconds (0: the kernels' own limit, 2 s) it gives
+ * up and records IPTTT_ERR_TIMEOUT in the status word (read it with
+ * ipttt_get_status); the context stays usable.  Meant for tests. */
+IPTTT_API ipttt_status ipttt_selftest_wait_timeout(uint32_t limit_ns, void* stream);
+
 /* Library version, "major.minor.patch". */
 IPTTT_API const char* ipttt_version(void);
 

@@ -186,3 +186,14 @@ def test_unsupported_shape_raises():
     t = {k: inp[k].to(dev) for k in ("H", "X0", "Wgate", "Wup", "Wdown0", "conv_w", "Wtarget")}
     with pytest.raises(ValueError):
         ip.forward(cfg, t["H"], t["X0"], t["Wgate"], t["Wup"], t["Wdown0"], t["conv_w"], t["Wtarget"])
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A device wait that nothing satisfies gives up after its limit and sets the
+    status word; the next layer call still runs."""
+    ip.selftest_wait_timeout(100_000_000)
+    assert ip.get_status() == 7
+    assert ip.get_status() == 0
+    cfg, inp = case(1, 256, 128, 128, 256)
+    out = gpu(cfg, inp, debug=False)
+    assert torch.isfinite(out.float()).all()
