@@ -124,6 +124,8 @@ struct Layout {
 // Apply tiles of `group` consecutive chunks share one launch, so that one launch
 // holds about kApplyTilesPerLaunch tiles (several even waves over the SMs).
 constexpr int kApplyTilesPerLaunch = 1280;
+// L2 budget for the Z/V slices of the chunks an update window walks through.
+constexpr size_t kUpdateWindowBytes = 512ull << 20;
 
 // Token rows of an apply or Gram tile: 128, or 64 for chunks that are odd
 // multiples of 64 (the MMA still spans 128 rows; the upper 64 are not used).
@@ -360,39 +362,48 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   sc.resid = (p.flags & IPTTT_FLAG_RESIDUAL) ? t.H : nullptr;
   sc.S = S;
   sc.nslots = G;
+  sc.dchunks = 1;
+  sc.dwin = 1;
   const bool need_final = t.Sfinal != nullptr || ss != nullptr;
-  const int delta_tiles = s.B * (s.d / 128) * (s.F / 128);
+  const int state_tiles = s.B * (s.d / 128) * (s.F / 128);
   const int apply_tiles_per_chunk = s.B * (s.C / arows) * (s.d / 128);
-  auto delta = [&](int j) -> ipttt_status {
+  // State updates of chunks [c0, c1) in one launch: each block keeps its state
+  // tiles through all of them and writes S_{c+1} snapshots into slot (c+1) % G.
+  // Z and V rows of one chunk (all batch rows): the slab every state tile reads.
+  const size_t slab = (size_t)s.B * s.C * (s.F + s.d) * 2;
+  auto update = [&](int c0, int c1) -> ipttt_status {
+    if (c1 <= c0) return IPTTT_OK;
     PhaseScope ph(st, PH_UPDATE);
     TcParams q = sc;
-    q.chunk = j;
-    q.write_snap = (j + 1 < s.k) ? 1 : 0;
+    q.chunk = c0;
+    q.dchunks = c1 - c0;
+    q.dwin = std::max(1, std::min(q.dchunks, (int)(kUpdateWindowBytes / slab)));
+    q.write_snap = 1;
     q.apply_chunk0 = 0;
     q.n_apply = 0;
-    q.n_tiles = delta_tiles;
+    q.n_tiles = state_tiles * q.dchunks;
     IP_CHECK(launch_tc(delta_fam, q, di->num_sms, st));
     counted(1);
     return IPTTT_OK;
   };
+  // Group [a, b) of G chunks: the updates of chunks a-1 .. b-2 produce S_a .. S_{b-1}
+  // (ring slots a % G .. (b-1) % G, which the previous group's applies have
+  // finished reading), then one launch applies chunks a .. b-1.
   for (int a = 0; a < s.k; a += G) {
     const int b = std::min(a + G, s.k);
-    for (int j = a; j + 1 < b; ++j)
-      if ((rc_ = delta(j)) != IPTTT_OK) return rc_;
-    {
-      PhaseScope ph(st, PH_APPLY);
-      TcParams q = sc;
-      q.chunk = 0;
-      q.write_snap = 0;
-      q.apply_chunk0 = a;
-      q.n_apply = (b - a) * apply_tiles_per_chunk;
-      q.n_tiles = q.n_apply;
-      IP_CHECK(launch_tc(apply_fam, q, di->num_sms, st));
-      counted(1);
-    }
-    if (b < s.k || need_final)
-      if ((rc_ = delta(b - 1)) != IPTTT_OK) return rc_;
+    if ((rc_ = update(std::max(a - 1, 0), b - 1)) != IPTTT_OK) return rc_;
+    PhaseScope ph(st, PH_APPLY);
+    TcParams q = sc;
+    q.chunk = 0;
+    q.dchunks = 1;
+    q.write_snap = 0;
+    q.apply_chunk0 = a;
+    q.n_apply = (b - a) * apply_tiles_per_chunk;
+    q.n_tiles = q.n_apply;
+    IP_CHECK(launch_tc(apply_fam, q, di->num_sms, st));
+    counted(1);
   }
+  if (need_final && (rc_ = update(s.k - 1, s.k)) != IPTTT_OK) return rc_;
   if (t.Sfinal) {
     IP_CHECK(aux::state_export(true, S, t.Sfinal, s, st));
     counted(1);

@@ -203,11 +203,12 @@ template <int KB>
 __device__ __forceinline__ void decode_delta(const TcParams& p, int tile, Job& j) {
   const int tiles_n = p.F / 128;
   const int per_row = (p.d / 128) * tiles_n;
+  const int X = tile / p.dchunks;  // state tile
   j.kind = K_DELTA;
-  j.chunk = p.chunk;
-  j.t0 = p.chunk * p.C;
-  j.b = tile / per_row;
-  const int r = tile % per_row;
+  j.chunk = p.chunk + tile % p.dchunks;
+  j.t0 = j.chunk * p.C;
+  j.b = X / per_row;
+  const int r = X % per_row;
   j.m0 = (r / tiles_n) * 128;     // d index
   j.n0 = (r % tiles_n) * 128;     // F index
   j.pair = 0;
@@ -231,6 +232,40 @@ __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
   else if constexpr (FAM == FAM_APPLY) decode_apply<0>(p, tile, j);
   else if constexpr (FAM == FAM_APPLY256) decode_apply<256>(p, tile, j);
   else decode_delta<Cfg<FAM>::KB>(p, tile, j);
+}
+
+// i-th tile of this block, or -1 past the end.  Update launches give each block
+// the state tiles X = blockIdx.x + m * gridDim.x; the chunks of the launch are
+// walked in windows of dwin chunks: every tile of the block goes through the
+// window (chunk by chunk, state kept in registers), then the next window, so a
+// window's Z and V slices stay in L2 while all tiles read them.
+template <int FAM>
+__device__ __forceinline__ int seq_tile(const TcParams& p, uint32_t i) {
+  if constexpr (is_delta<FAM>()) {
+    const int D = p.dchunks, g = p.dwin;
+    const int nX = p.n_tiles / D;
+    if ((int)blockIdx.x >= nX) return -1;
+    const int nXc = (nX - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const long long full = (long long)(D / g) * nXc * g;  // tiles in the full windows
+    int w, gw, r;
+    if ((long long)i < full) {
+      w = (int)(i / ((uint32_t)nXc * g));
+      gw = g;
+      r = (int)(i % ((uint32_t)nXc * g));
+    } else {
+      w = D / g;
+      gw = D % g;
+      r = (int)((long long)i - full);
+      if (gw == 0 || r >= nXc * gw) return -1;
+    }
+    const int m = r / gw;
+    const int c = w * g + r % gw;
+    const int X = (int)blockIdx.x + m * (int)gridDim.x;
+    return X * D + c;
+  } else {
+    const long long t = (long long)blockIdx.x + (long long)i * gridDim.x;
+    return t < p.n_tiles ? (int)t : -1;
+  }
 }
 
 // ------------------------------------------------------------------ producer
@@ -424,12 +459,13 @@ __device__ __forceinline__ void delta_load_old(const TcParams& p, int tile, int 
     old[q] = keep ? src[(16 * half + q) * 128 + row] : make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// State update of one 128 x 128 tile (d rows m0.., F columns n0..):
-// S_new = old + alpha eta acc, where `old` already holds S_old (or zeros after a
-// document start).  The bf16 snapshot of this warp's 32 x 64 block is staged in
-// the 128-byte-swizzled layout of a TMA box and stored by lane 0.
+// State update of one 128 x 128 tile (d rows m0.., F columns n0..) for one chunk:
+// S_new = old + alpha eta acc, where `old` holds S_old (or zeros after a document
+// start).  S_new replaces `old`; it goes to HBM only after the tile's last chunk of
+// the launch.  The bf16 snapshot of this warp's 32 x 64 block is staged in the
+// 128-byte-swizzled layout of a TMA box and stored by lane 0.
 __device__ __forceinline__ void delta_epilogue_tile(const TcParams& p, const Job& j, uint32_t tacc, int half,
-                                                    int quarter, int lane, const float4 (&old)[16],
+                                                    int quarter, int lane, float4 (&old)[16], bool store_fp32,
                                                     uint8_t* box) {
   const int row = quarter * 32 + lane;
   const float ae = p.alpha[(size_t)j.b * p.k + j.chunk] * p.eta;
@@ -448,7 +484,8 @@ __device__ __forceinline__ void delta_epilogue_tile(const TcParams& p, const Job
       nv.y = fmaf(ae, __uint_as_float(r[4 * q + 1]), o.y);
       nv.z = fmaf(ae, __uint_as_float(r[4 * q + 2]), o.z);
       nv.w = fmaf(ae, __uint_as_float(r[4 * q + 3]), o.w);
-      dst[(16 * half + 8 * g + q) * 128 + row] = nv;
+      if (store_fp32) dst[(16 * half + 8 * g + q) * 128 + row] = nv;
+      old[8 * g + q] = nv;  // the state this thread carries into the tile's next chunk
       packed[2 * q] = pack_bf16(nv.x, nv.y);
       packed[2 * q + 1] = pack_bf16(nv.z, nv.w);
     }
@@ -516,7 +553,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+      for (uint32_t i = 0; ok; ++i) {
+        const int tile = seq_tile<FAM>(p, i);
+        if (tile < 0) break;
         Job j;
         decode<FAM>(p, tile, j);
         for (int seg = 0; seg < j.nseg && ok; ++seg) {
@@ -537,7 +576,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++tcount) {
+      for (uint32_t i = 0; ok; ++i, ++tcount) {
+        const int tile = seq_tile<FAM>(p, i);
+        if (tile < 0) break;
         Job j;
         decode<FAM>(p, tile, j);
         const int buf = Cfg<FAM>::NBUF == 2 ? (tcount & 1) : 0;
@@ -589,9 +630,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     bool ok = true;
     float4 old[16];
     if constexpr (is_delta<FAM>()) {
-      if ((int)blockIdx.x < p.n_tiles) delta_load_old<Cfg<FAM>::KB>(p, blockIdx.x, half, row, old);
+      const int first = seq_tile<FAM>(p, 0);
+      if (first >= 0) delta_load_old<Cfg<FAM>::KB>(p, first, half, row, old);
     }
-    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++tcount) {
+    for (uint32_t i = 0;; ++i, ++tcount) {
+      const int tile = seq_tile<FAM>(p, i);
+      if (tile < 0) break;
       Job j;
       decode<FAM>(p, tile, j);
       const int buf = Cfg<FAM>::NBUF == 2 ? (tcount & 1) : 0;
@@ -606,15 +650,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
           if (lane == 0) bulk_wait_read<0>();  // the previous tile's store has read the box
           __syncwarp();
         }
-        delta_epilogue_tile(p, j, tacc, half, quarter, lane, old, box);
+        const int next = seq_tile<FAM>(p, i + 1);
+        // The tile's state goes back to HBM after its last chunk of this launch.
+        const bool last_chunk = next < 0 || next / p.dchunks != tile / p.dchunks;
+        delta_epilogue_tile(p, j, tacc, half, quarter, lane, old, last_chunk, box);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        // Start loading the next tile's old state now; it lands while that tile's
-        // MMAs run.
-        const int next = tile + gridDim.x;
-        if (next < p.n_tiles) delta_load_old<Cfg<FAM>::KB>(p, next, half, row, old);
-        if (p.write_snap) {
+        if (next >= 0) {
+          if (last_chunk) {
+            // next state tile: start loading its old state now, so it lands while
+            // that tile's MMAs run
+            delta_load_old<Cfg<FAM>::KB>(p, next, half, row, old);
+          } else {
+            Job jn;
+            decode_delta<Cfg<FAM>::KB>(p, next, jn);
+            if (p.meta[(size_t)jn.b * p.k + jn.chunk].has_start) {
+#pragma unroll
+              for (int q = 0; q < 16; ++q) old[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+          }
+        }
+        if (p.write_snap && j.chunk + 1 < p.k) {
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {

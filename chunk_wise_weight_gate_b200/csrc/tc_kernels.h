@@ -18,7 +18,11 @@ struct TcParams {
   int tr;            // token rows per apply / Gram tile: 128, or 64 when C % 128 != 0
   int ct;            // tiles per chunk (C / tr)
   int npairs;        // GRAM: tile pairs per chunk, ct (ct + 1) / 2
-  int chunk;         // SCAN: chunk whose state update the delta tiles perform
+  int chunk;         // DELTA: first chunk whose state update the launch performs
+  int dchunks;       // DELTA: consecutive chunks per launch (tile index = X * dchunks + c)
+  int dwin;          // DELTA: chunks per window; a block takes all of its state tiles
+                     //        through one window before the next, carrying each tile's
+                     //        state in registers inside the window
   int apply_chunk0;  // SCAN: first chunk of the apply tiles
   int n_apply;       // SCAN: apply tiles (chunks apply_chunk0.., all rows); delta tiles follow
   int n_tiles;
