@@ -312,7 +312,8 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
         !make_map_bf16(&v.map[1], t.Wt, s.d, s.d, 1, 64, 64))
       return IPTTT_ERR_CUDA;
     v.out0 = V;
-    v.n_tiles = s.B * ((s.T + 127) / 128) * (s.d / 128);
+    v.vn = s.d % 256 == 0 ? 256 : 128;
+    v.n_tiles = s.B * ((s.T + 127) / 128) * (s.d / v.vn);
     IP_CHECK(launch_tc(FAM_ZV, v, di->num_sms, st));
     counted(1);
   }

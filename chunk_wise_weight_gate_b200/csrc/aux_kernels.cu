@@ -92,7 +92,7 @@ cudaError_t build_meta(uint8_t* flags, ChunkMeta* meta, const Shape& s, const in
 // A thread owns VEC channels of one row over RUN consecutive tokens: it keeps
 // its 5 x VEC taps and a 5-row window of X0 in registers, so every X0 element
 // is read about once and a warp's loads and stores cover contiguous bytes.
-constexpr int kConvRun = 64;
+constexpr int kConvRun = 16;
 
 template <typename T, int VEC>
 __device__ __forceinline__ void load_vec(const T* p, float (&out)[VEC]) {

@@ -83,6 +83,7 @@ template <> struct Cfg<FAM_DELTA64> {
                        EPI_BYTES = NUM_EPI_WARPS * SNAP_BOX_BYTES, NBUF = 2;
 };
 template <int FAM> constexpr bool is_apply() { return FAM == FAM_APPLY || FAM == FAM_APPLY256; }
+template <int FAM> constexpr bool is_zv() { return FAM == FAM_ZV; }
 template <int FAM> constexpr bool is_delta() { return FAM == FAM_DELTA || FAM == FAM_DELTA64; }
 
 template <int FAM>
@@ -114,10 +115,12 @@ struct Job {
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 // ------------------------------------------------------------------ decoding
+template <int ROWS>
 __device__ __forceinline__ void decode_zv(const TcParams& p, int tile, Job& j) {
-  const int tiles_m = cdiv(p.T, BM);
+  const int tiles_m = cdiv(p.T, ROWS);
+  const int ncol = p.kind == K_GATEUP ? 128 : p.vn;  // gate/up: 128 gate + 128 up columns
   const int N = p.kind == K_GATEUP ? p.F : p.d;
-  const int tiles_n = N / 128;
+  const int tiles_n = N / ncol;
   const int M_all = p.B * tiles_m;
   constexpr int G = 16;  // m-tiles per raster group
   const int per_group = G * tiles_n;
@@ -128,8 +131,8 @@ __device__ __forceinline__ void decode_zv(const TcParams& p, int tile, Job& j) {
   const int nt = r / gm;
   j.kind = p.kind;
   j.b = mm / tiles_m;
-  j.m0 = (mm % tiles_m) * BM;
-  j.n0 = nt * 128;
+  j.m0 = (mm % tiles_m) * ROWS;
+  j.n0 = nt * ncol;
   j.t0 = 0;
   j.chunk = 0;
   j.pair = 0;
@@ -140,15 +143,16 @@ __device__ __forceinline__ void decode_zv(const TcParams& p, int tile, Job& j) {
   j.nsrc = 1;
   if (p.kind == K_GATEUP) {
     j.n_mma = 256;
-    j.tx = A_BYTES + 2 * 128 * BK * 2;
+    j.tx = ROWS * BK * 2 + 2 * 128 * BK * 2;
     j.a_mn = false;
     j.b_mn = false;
   } else {
-    j.n_mma = 128;
-    j.tx = A_BYTES + 128 * BK * 2;
+    j.n_mma = p.vn;
+    j.tx = A_BYTES + p.vn * BK * 2;
     j.a_mn = false;
     j.b_mn = true;
   }
+  j.halves = ROWS == 256 ? 2 : 1;
 }
 
 __device__ __forceinline__ void decode_gram(const TcParams& p, int tile, Job& j) {
@@ -227,7 +231,7 @@ __device__ __forceinline__ void decode_delta(const TcParams& p, int tile, Job& j
 template <int FAM>
 __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
   j.halves = 1;
-  if constexpr (FAM == FAM_ZV) decode_zv(p, tile, j);
+  if constexpr (FAM == FAM_ZV) decode_zv<128>(p, tile, j);
   else if constexpr (FAM == FAM_GRAM) decode_gram(p, tile, j);
   else if constexpr (FAM == FAM_APPLY) decode_apply<0>(p, tile, j);
   else if constexpr (FAM == FAM_APPLY256) decode_apply<256>(p, tile, j);
@@ -273,15 +277,16 @@ template <int FAM>
 __device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int seg, int kb, uint8_t* sa,
                                             uint8_t* sb, uint64_t* bar) {
   const int kx = kb * BK;
-  if constexpr (FAM == FAM_ZV) {
+  if constexpr (is_zv<FAM>()) {
     if (j.kind == K_GATEUP) {
       tma_load_3d(sa, &p.map[0], bar, kx, j.m0, j.b);              // H rows
+      if (j.halves == 2) tma_load_3d(sa + A_BYTES, &p.map[0], bar, kx, j.m0 + 128, j.b);
       tma_load_3d(sb, &p.map[1], bar, kx, j.n0, 0);                   // Wgate rows
       tma_load_3d(sb + 128 * BK * 2, &p.map[2], bar, kx, j.n0, 0);    // Wup rows
     } else {
       tma_load_3d(sa, &p.map[0], bar, kx, j.m0, j.b);              // U rows
-      tma_load_3d(sb, &p.map[1], bar, j.n0, kx, 0);                   // Wtarget[k][n], n contiguous
-      tma_load_3d(sb + 64 * BK * 2, &p.map[1], bar, j.n0 + 64, kx, 0);
+      for (int q = 0; q < p.vn / 64; ++q)                          // Wtarget[k][n], n contiguous
+        tma_load_3d(sb + q * 64 * BK * 2, &p.map[1], bar, j.n0 + 64 * q, kx, 0);
     }
   } else if constexpr (FAM == FAM_GRAM) {
     const CUtensorMap* m = seg == 0 ? &p.map[0] : &p.map[1];       // Z or V
@@ -333,13 +338,18 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
                                               int lane, int ew, float* red) {
   uint32_t r0[32], r1[32];
   float v[32];
-  if constexpr (FAM == FAM_ZV) {
-    const int t = j.m0 + row;
+  if constexpr (is_zv<FAM>()) {
+    // Two M halves (256-row gate/up tiles): this warp drains rows 128 half .. of
+    // all 128 output columns, from the accumulator 256 TMEM columns further up.
+    const bool two = j.halves == 2;
+    if (two) tacc += half * 256;
+    const int t = j.m0 + (two ? half * 128 : 0) + row;
     const bool valid = t < p.T;
     if (j.kind == K_GATEUP) {
       __nv_bfloat16* zrow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.F + j.n0;
+      const int c0 = two ? 0 : half * 64, c1 = two ? 128 : half * 64 + 64;
 #pragma unroll 1
-      for (int c = half * 64; c < half * 64 + 64; c += 32) {
+      for (int c = c0; c < c1; c += 32) {
         tmem_ld32(tacc + c, r0);
         tmem_ld32(tacc + 128 + c, r1);
         tmem_ld_wait();
@@ -351,8 +361,9 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
       const int chunk = t / p.C;
       const bool keep = valid && t >= p.meta[(size_t)j.b * p.k + min(chunk, p.k - 1)].last_start;
       __nv_bfloat16* vrow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.d + j.n0;
+      const int w = p.vn / 2;  // columns drained by this warp
 #pragma unroll 1
-      for (int c = half * 64; c < half * 64 + 64; c += 32) {
+      for (int c = half * w; c < half * w + w; c += 32) {
         tmem_ld32(tacc + c, r0);
         tmem_ld_wait();
 #pragma unroll

@@ -14,6 +14,7 @@ enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_DELTA = 3, FAM_DELTA6
 struct TcParams {
   CUtensorMap map[6];
   int kind;          // FAM_ZV: kind_gateup() or kind_vhat()
+  int vn;            // FAM_ZV target GEMM: output columns per tile (128 or 256)
   int B, T, d, F, C, k;
   int tr;            // token rows per apply / Gram tile: 128, or 64 when C % 128 != 0
   int ct;            // tiles per chunk (C / tr)

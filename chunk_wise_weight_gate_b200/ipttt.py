@@ -15,7 +15,8 @@ from dataclasses import dataclass
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libipttt.so")
+# IPTTT_LIB may name another build of the library (for example an instrumented one).
+LIB_PATH = os.environ.get("IPTTT_LIB") or os.path.join(_HERE, "libipttt.so")
 
 F32, BF16 = 0, 1
 STATUS = {0: "IPTTT_OK", 1: "IPTTT_ERR_ARG", 2: "IPTTT_ERR_SHAPE", 3: "IPTTT_ERR_ALIGN", 4: "IPTTT_ERR_DTYPE",
