@@ -124,8 +124,6 @@ struct Layout {
 // Apply tiles of `group` consecutive chunks share one launch, so that one launch
 // holds about kApplyTilesPerLaunch tiles (several even waves over the SMs).
 constexpr int kApplyTilesPerLaunch = 1280;
-// L2 budget for the Z/V slices of the chunks an update window walks through.
-constexpr size_t kUpdateWindowBytes = 512ull << 20;
 
 // Token rows of an apply or Gram tile: 128, or 64 for chunks that are odd
 // multiples of 64 (the MMA still spans 128 rows; the upper 64 are not used).
@@ -330,7 +328,9 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     g.n_tiles = s.B * s.k * tp.npairs;
     IP_CHECK(launch_tc(FAM_GRAM, g, di->num_sms, st));
     IP_CHECK(aux::alpha_from_partials(partials, alpha, s.B * s.k, tp.npairs, p.eta, tau, st));
-    counted(2);
+    // the state update accumulates alpha eta V^T Z: fold alpha eta into V's rows
+    IP_CHECK(aux::prescale_target(V, alpha, s, p.eta, st));
+    counted(3);
   }
   if (t.alpha) IP_CHECK(cudaMemcpyAsync(t.alpha, alpha, (size_t)s.B * s.k * 4, cudaMemcpyDeviceToDevice, st));
 
@@ -349,13 +349,11 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   TcParams sc = tp;
   const int arows = apply_rows(p);
   const int apply_fam = arows == 256 ? FAM_APPLY256 : FAM_APPLY;
-  const int delta_fam = s.C % 128 == 0 ? FAM_DELTA : FAM_DELTA64;
-  const int delta_kb = s.C % 128 == 0 ? 128 : 64;
   if (!make_map_bf16(&sc.map[0], Z, s.F, s.T, s.B, 64, arows == 256 ? 128 : tp.tr) ||
       !make_map_bf16(&sc.map[1], t.W0, s.F, s.d, 1, 64, 128) ||
       !make_map_bf16(&sc.map[2], snap, s.F, s.d, (uint64_t)G * s.B, 64, 128) ||
-      !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, delta_kb) ||
-      !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, delta_kb) ||
+      !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, 64) ||
+      !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, 64) ||
       !make_map_bf16(&sc.map[5], snap, s.F, s.d, (uint64_t)G * s.B, 64, 32))
     return IPTTT_ERR_CUDA;
   sc.out0 = t.O;
@@ -364,26 +362,23 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   sc.S = S;
   sc.nslots = G;
   sc.dchunks = 1;
-  sc.dwin = 1;
   const bool need_final = t.Sfinal != nullptr || ss != nullptr;
-  const int state_tiles = s.B * (s.d / 128) * (s.F / 128);
+  const int state_tiles = s.B * (s.d / 128) * ((s.F + 255) / 256);  // 128 x 256 tiles
   const int apply_tiles_per_chunk = s.B * (s.C / arows) * (s.d / 128);
   // State updates of chunks [c0, c1) in one launch: each block keeps its state
-  // tiles through all of them and writes S_{c+1} snapshots into slot (c+1) % G.
-  // Z and V rows of one chunk (all batch rows): the slab every state tile reads.
-  const size_t slab = (size_t)s.B * s.C * (s.F + s.d) * 2;
+  // tiles in TMEM through all of them and writes S_{c+1} snapshots into slot
+  // (c+1) % G.
   auto update = [&](int c0, int c1) -> ipttt_status {
     if (c1 <= c0) return IPTTT_OK;
     PhaseScope ph(st, PH_UPDATE);
     TcParams q = sc;
     q.chunk = c0;
     q.dchunks = c1 - c0;
-    q.dwin = std::max(1, std::min(q.dchunks, (int)(kUpdateWindowBytes / slab)));
     q.write_snap = 1;
     q.apply_chunk0 = 0;
     q.n_apply = 0;
-    q.n_tiles = state_tiles * q.dchunks;
-    IP_CHECK(launch_tc(delta_fam, q, di->num_sms, st));
+    q.n_tiles = state_tiles;
+    IP_CHECK(launch_update(q, di->num_sms, st));
     counted(1);
     return IPTTT_OK;
   };

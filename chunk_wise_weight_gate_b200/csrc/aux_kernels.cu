@@ -456,3 +456,33 @@ cudaError_t stream_advance(long long* pos, int32_t* cont, int B, int T, cudaStre
 
 }  // namespace aux
 }  // namespace ipttt
+
+namespace ipttt {
+namespace aux {
+
+// V[b,t,:] *= alpha[b, chunk(t)] * eta, in place (bf16), so that the state update's
+// MMAs accumulate alpha eta V^T Z directly.
+__global__ void k_prescale(__nv_bfloat16* V, const float* alpha, int B, int Tn, int d, int C, int k, float eta) {
+  const int groups = d / 8;
+  const size_t total = (size_t)B * Tn * groups;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t bt = i / groups;
+    const int t = (int)(bt % Tn);
+    const int b = (int)(bt / Tn);
+    const float sc = alpha[(size_t)b * k + t / C] * eta;
+    __nv_bfloat16* v = V + bt * d + (size_t)(i % groups) * 8;
+    float x[8];
+    load_vec<__nv_bfloat16, 8>(v, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] *= sc;
+    store_vec<__nv_bfloat16, 8>(v, x);
+  }
+}
+
+cudaError_t prescale_target(void* V, const float* alpha, const Shape& s, float eta, cudaStream_t st) {
+  k_prescale<<<148 * 8, 256, 0, st>>>((__nv_bfloat16*)V, alpha, s.B, s.T, s.d, s.C, s.k, eta);
+  return cudaGetLastError();
+}
+
+}  // namespace aux
+}  // namespace ipttt

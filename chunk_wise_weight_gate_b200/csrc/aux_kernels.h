@@ -53,5 +53,6 @@ namespace aux {
 cudaError_t mask_last_segment(int dtype, const void* in, void* out, const ChunkMeta* meta, const Shape& s,
                               cudaStream_t st);
 cudaError_t stream_advance(long long* pos, int32_t* cont, int B, int T, cudaStream_t st);
+cudaError_t prescale_target(void* V, const float* alpha, const Shape& s, float eta, cudaStream_t st);
 }  // namespace aux
 }  // namespace ipttt

@@ -20,14 +20,11 @@
 //            products side by side in one N=256 accumulator, S_i read from a bf16
 //            snapshot [notes, 步骤一 and 工程实现; iplexlaw.co.kr review §3: a chunk's output
 //            comes from the pre-update state].
-//   FAM_DELTA the state update of one chunk: S_{i+1} = keep_i S_i + alpha_i eta V_i^T Z_i
-//            on 128 x 128 tiles of the fp32 state (kept in a blocked layout whose
-//            rows match the TMEM lanes, so every warp access is 512 contiguous bytes;
-//            the next tile's old state is loaded into registers while the current
-//            tile's MMAs run), plus the bf16 snapshot of S_{i+1} stored with TMA
-//            [notes, 步骤二 and the Hebbian rule; iplexlaw.co.kr review §6 exclusive scan
-//            and document reset].  FAM_DELTA64 is the same with 64-token stages, for
-//            chunk sizes that are odd multiples of 64.
+// The state update S_{i+1} = keep_i S_i + alpha_i eta V_i^T Z_i runs in its own
+// kernel (upd_kernel, below): each block keeps two 128 x 256 fp32 state tiles in
+// TMEM as live accumulators and walks them through a group of chunks [notes,
+// 步骤二 and the Hebbian rule; iplexlaw.co.kr review §6 exclusive scan and document
+// reset].
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -71,28 +68,14 @@ template <> struct Cfg<FAM_APPLY256> {
   static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 64, B_OFF = 2 * A_BYTES, EPI_BYTES = 0,
                        NBUF = 1;
 };
-// The update contracts over tokens with MN-major operands; 128-token stages keep
-// every TMA box at 16 KB (128 rows of 128 bytes).  Chunks of 64 (mod 128) tokens
-// use 64-token stages.
-template <> struct Cfg<FAM_DELTA> {
-  static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 128, B_OFF = 32 * 1024,
-                       EPI_BYTES = NUM_EPI_WARPS * SNAP_BOX_BYTES, NBUF = 2;
-};
-template <> struct Cfg<FAM_DELTA64> {
-  static constexpr int STAGES = 5, STAGE_BYTES = 32 * 1024, KB = 64, B_OFF = 16 * 1024,
-                       EPI_BYTES = NUM_EPI_WARPS * SNAP_BOX_BYTES, NBUF = 2;
-};
 template <int FAM> constexpr bool is_apply() { return FAM == FAM_APPLY || FAM == FAM_APPLY256; }
 template <int FAM> constexpr bool is_zv() { return FAM == FAM_ZV; }
-template <int FAM> constexpr bool is_delta() { return FAM == FAM_DELTA || FAM == FAM_DELTA64; }
 
 template <int FAM>
 constexpr int smem_bytes() {
   return 1024 /*alignment slack*/ + Cfg<FAM>::STAGES * Cfg<FAM>::STAGE_BYTES + Cfg<FAM>::EPI_BYTES +
          256 /*barriers*/;
 }
-static_assert(smem_bytes<FAM_DELTA>() <= 232448, "delta kernel exceeds shared memory");
-static_assert(smem_bytes<FAM_DELTA64>() <= 232448, "delta kernel exceeds shared memory");
 static_assert(smem_bytes<FAM_ZV>() <= 232448, "kernel exceeds shared memory");
 
 struct Job {
@@ -203,73 +186,20 @@ __device__ __forceinline__ void decode_apply(const TcParams& p, int tile, Job& j
   j.b_mn = false;
 }
 
-template <int KB>
-__device__ __forceinline__ void decode_delta(const TcParams& p, int tile, Job& j) {
-  const int tiles_n = p.F / 128;
-  const int per_row = (p.d / 128) * tiles_n;
-  const int X = tile / p.dchunks;  // state tile
-  j.kind = K_DELTA;
-  j.chunk = p.chunk + tile % p.dchunks;
-  j.t0 = j.chunk * p.C;
-  j.b = X / per_row;
-  const int r = X % per_row;
-  j.m0 = (r / tiles_n) * 128;     // d index
-  j.n0 = (r % tiles_n) * 128;     // F index
-  j.pair = 0;
-  j.nseg = 1;
-  j.acc_col[0] = 0;
-  const int rows = min(p.C, p.T - j.t0);
-  j.kb0[0] = (p.meta[(size_t)j.b * p.k + j.chunk].last_start - j.t0) / KB;
-  j.kb1[0] = cdiv(rows, KB);
-  j.n_mma = 128;
-  j.nsrc = 1;
-  j.tx = 4 * 64 * KB * 2;  // two 64-column boxes of V and two of Z, KB token rows each
-  j.a_mn = true;
-  j.b_mn = true;
-}
-
 template <int FAM>
 __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
   j.halves = 1;
   if constexpr (FAM == FAM_ZV) decode_zv<128>(p, tile, j);
   else if constexpr (FAM == FAM_GRAM) decode_gram(p, tile, j);
   else if constexpr (FAM == FAM_APPLY) decode_apply<0>(p, tile, j);
-  else if constexpr (FAM == FAM_APPLY256) decode_apply<256>(p, tile, j);
-  else decode_delta<Cfg<FAM>::KB>(p, tile, j);
+  else decode_apply<256>(p, tile, j);
 }
 
-// i-th tile of this block, or -1 past the end.  Update launches give each block
-// the state tiles X = blockIdx.x + m * gridDim.x; the chunks of the launch are
-// walked in windows of dwin chunks: every tile of the block goes through the
-// window (chunk by chunk, state kept in registers), then the next window, so a
-// window's Z and V slices stay in L2 while all tiles read them.
+// i-th tile of this block (static round-robin schedule), or -1 past the end.
 template <int FAM>
 __device__ __forceinline__ int seq_tile(const TcParams& p, uint32_t i) {
-  if constexpr (is_delta<FAM>()) {
-    const int D = p.dchunks, g = p.dwin;
-    const int nX = p.n_tiles / D;
-    if ((int)blockIdx.x >= nX) return -1;
-    const int nXc = (nX - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-    const long long full = (long long)(D / g) * nXc * g;  // tiles in the full windows
-    int w, gw, r;
-    if ((long long)i < full) {
-      w = (int)(i / ((uint32_t)nXc * g));
-      gw = g;
-      r = (int)(i % ((uint32_t)nXc * g));
-    } else {
-      w = D / g;
-      gw = D % g;
-      r = (int)((long long)i - full);
-      if (gw == 0 || r >= nXc * gw) return -1;
-    }
-    const int m = r / gw;
-    const int c = w * g + r % gw;
-    const int X = (int)blockIdx.x + m * (int)gridDim.x;
-    return X * D + c;
-  } else {
-    const long long t = (long long)blockIdx.x + (long long)i * gridDim.x;
-    return t < p.n_tiles ? (int)t : -1;
-  }
+  const long long t = (long long)blockIdx.x + (long long)i * gridDim.x;
+  return t < p.n_tiles ? (int)t : -1;
 }
 
 // ------------------------------------------------------------------ producer
@@ -298,13 +228,6 @@ __device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int
     tma_load_3d(sb, &p.map[1], bar, kx, j.n0, 0);                 // Wdown0 rows
     if (j.nsrc == 2)
       tma_load_3d(sb + 128 * BK * 2, &p.map[2], bar, kx, j.n0, (j.chunk % p.nslots) * p.B + j.b);  // S_i rows
-  } else {
-    constexpr int KB = Cfg<FAM>::KB;
-    const int ty = j.t0 + kb * KB;                                 // token rows = K
-    tma_load_3d(sa, &p.map[3], bar, j.m0, ty, j.b);                // V[t][d], d contiguous
-    tma_load_3d(sa + 64 * KB * 2, &p.map[3], bar, j.m0 + 64, ty, j.b);
-    tma_load_3d(sb, &p.map[4], bar, j.n0, ty, j.b);                // Z[t][f], f contiguous
-    tma_load_3d(sb + 64 * KB * 2, &p.map[4], bar, j.n0 + 64, ty, j.b);
   }
 }
 
@@ -451,64 +374,6 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
   }
 }
 
-__device__ __forceinline__ float4* state_tile(const TcParams& p, const Job& j) {
-  return reinterpret_cast<float4*>(p.S + (size_t)j.b * p.d * p.F +
-                                   ((size_t)(j.m0 / 128) * (p.F / 128) + j.n0 / 128) * (128 * 128));
-}
-
-// This thread's 64 old state values of tile `tile` (row `row`, columns
-// 64*half..64*half+63), or zeros when the chunk resets the state.  In the blocked
-// layout a warp's 16-byte loads cover 512 contiguous bytes.
-template <int KB>
-__device__ __forceinline__ void delta_load_old(const TcParams& p, int tile, int half, int row, float4 (&old)[16]) {
-  Job j;
-  decode_delta<KB>(p, tile, j);
-  const bool keep = !p.meta[(size_t)j.b * p.k + j.chunk].has_start;
-  const float4* src = state_tile(p, j);
-#pragma unroll
-  for (int q = 0; q < 16; ++q)
-    old[q] = keep ? src[(16 * half + q) * 128 + row] : make_float4(0.f, 0.f, 0.f, 0.f);
-}
-
-// State update of one 128 x 128 tile (d rows m0.., F columns n0..) for one chunk:
-// S_new = old + alpha eta acc, where `old` holds S_old (or zeros after a document
-// start).  S_new replaces `old`; it goes to HBM only after the tile's last chunk of
-// the launch.  The bf16 snapshot of this warp's 32 x 64 block is staged in the
-// 128-byte-swizzled layout of a TMA box and stored by lane 0.
-__device__ __forceinline__ void delta_epilogue_tile(const TcParams& p, const Job& j, uint32_t tacc, int half,
-                                                    int quarter, int lane, float4 (&old)[16], bool store_fp32,
-                                                    uint8_t* box) {
-  const int row = quarter * 32 + lane;
-  const float ae = p.alpha[(size_t)j.b * p.k + j.chunk] * p.eta;
-  float4* dst = state_tile(p, j);
-#pragma unroll
-  for (int g = 0; g < 2; ++g) {
-    uint32_t r[32];
-    tmem_ld32(tacc + half * 64 + g * 32, r);
-    tmem_ld_wait();
-    uint32_t packed[16];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 o = old[8 * g + q];
-      float4 nv;
-      nv.x = fmaf(ae, __uint_as_float(r[4 * q + 0]), o.x);
-      nv.y = fmaf(ae, __uint_as_float(r[4 * q + 1]), o.y);
-      nv.z = fmaf(ae, __uint_as_float(r[4 * q + 2]), o.z);
-      nv.w = fmaf(ae, __uint_as_float(r[4 * q + 3]), o.w);
-      if (store_fp32) dst[(16 * half + 8 * g + q) * 128 + row] = nv;
-      old[8 * g + q] = nv;  // the state this thread carries into the tile's next chunk
-      packed[2 * q] = pack_bf16(nv.x, nv.y);
-      packed[2 * q + 1] = pack_bf16(nv.z, nv.w);
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int chunk16 = g * 4 + e;  // 16-byte chunk of this row inside the 128-byte box row
-      *reinterpret_cast<uint4*>(box + lane * 128 + ((chunk16 ^ (lane & 7)) << 4)) =
-          make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
-    }
-  }
-}
-
 // ------------------------------------------------------------------ kernel
 template <int FAM>
 __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__ TcParams p) {
@@ -517,7 +382,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* epi = smem + STAGES * STAGE_BYTES;    // FAM_DELTA: per-warp snapshot staging boxes
+  uint8_t* epi = smem + STAGES * STAGE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(epi + Cfg<FAM>::EPI_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
@@ -547,9 +412,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    const int first = is_delta<FAM>() ? 3 : 0;
-    const int nmaps = is_delta<FAM>() ? 3 : (is_apply<FAM>() ? 3 : (FAM == FAM_GRAM ? 2 : (p.kind == K_GATEUP ? 3 : 2)));
-    for (int i = 0; i < nmaps; ++i) prefetch_tmap(&p.map[first + i]);
+    const int nmaps = is_apply<FAM>() ? 3 : (FAM == FAM_GRAM ? 2 : (p.kind == K_GATEUP ? 3 : 2));
+    for (int i = 0; i < nmaps; ++i) prefetch_tmap(&p.map[i]);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 2 * ACC_COLS);
@@ -636,14 +500,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     const int quarter = warp & 3;      // TMEM lanes this warp may access
     const int half = ew >> 2;          // which half of the columns this warp drains
     const int row = quarter * 32 + lane;
-    uint8_t* box = epi + ew * SNAP_BOX_BYTES;  // FAM_DELTA: this warp's snapshot staging box
     uint32_t tcount = 0;
     bool ok = true;
-    float4 old[16];
-    if constexpr (is_delta<FAM>()) {
-      const int first = seq_tile<FAM>(p, 0);
-      if (first >= 0) delta_load_old<Cfg<FAM>::KB>(p, first, half, row, old);
-    }
     for (uint32_t i = 0;; ++i, ++tcount) {
       const int tile = seq_tile<FAM>(p, i);
       if (tile < 0) break;
@@ -656,47 +514,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
       if (!mbar_wait(&acc_full[buf], aph)) { ok = false; break; }
       tc_fence_after();
       const uint32_t tacc = tmem_base + buf * ACC_COLS + ((uint32_t)(quarter * 32) << 16);
-      if constexpr (is_delta<FAM>()) {
-        if (tcount >= 1 && p.write_snap) {
-          if (lane == 0) bulk_wait_read<0>();  // the previous tile's store has read the box
-          __syncwarp();
-        }
-        const int next = seq_tile<FAM>(p, i + 1);
-        // The tile's state goes back to HBM after its last chunk of this launch.
-        const bool last_chunk = next < 0 || next / p.dchunks != tile / p.dchunks;
-        delta_epilogue_tile(p, j, tacc, half, quarter, lane, old, last_chunk, box);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        if (next >= 0) {
-          if (last_chunk) {
-            // next state tile: start loading its old state now, so it lands while
-            // that tile's MMAs run
-            delta_load_old<Cfg<FAM>::KB>(p, next, half, row, old);
-          } else {
-            Job jn;
-            decode_delta<Cfg<FAM>::KB>(p, next, jn);
-            if (p.meta[(size_t)jn.b * p.k + jn.chunk].has_start) {
-#pragma unroll
-              for (int q = 0; q < 16; ++q) old[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-          }
-        }
-        if (p.write_snap && j.chunk + 1 < p.k) {
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&p.map[5], box, j.n0 + 64 * half, j.m0 + 32 * quarter,
-                         ((j.chunk + 1) % p.nslots) * p.B + j.b);
-            bulk_commit();
-          }
-        }
-      } else {
-        epilogue_tile<FAM>(p, j, tacc, half, row, lane, ew, red);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
-      }
+      epilogue_tile<FAM>(p, j, tacc, half, row, lane, ew, red);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
     if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
     if (lane == 0) bulk_wait<0>();
@@ -714,6 +535,326 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     tc_fence_after();
     tmem_dealloc(tmem_base, 2 * ACC_COLS);
   }
+}
+
+// ------------------------------------------------------------------ state update
+// S_{c+1} = keep_c S_c + alpha_c eta V_c^T Z_c for the chunks c of one launch.
+// V arrives pre-scaled by alpha_c eta per row, so the MMAs accumulate the state
+// itself: each block keeps two 128 (d) x 256 (F) fp32 state tiles in TMEM (slots 0
+// and 1) and walks both through all chunks of the launch, alternating, so that
+// the epilogue reads one slot (bf16 snapshot of S_{c+1} for the apply) while the
+// MMAs run on the other.  A chunk holding a document start resets the tile (its
+// first MMA does not accumulate).  A tile's fp32 state comes in from HBM before
+// its first chunk (tcgen05.st) and goes back after its last.
+constexpr int UPD_STAGES = 4;
+constexpr int UPD_KB = 64;                            // tokens per stage
+constexpr int UPD_A_BYTES = 128 * UPD_KB * 2;         // V: 128 d columns
+constexpr int UPD_STAGE_BYTES = UPD_A_BYTES + 256 * UPD_KB * 2;  // + Z: 256 F columns
+constexpr int UPD_BOX_BYTES = 32 * 128;               // a warp's 32-row x 64-column snapshot box
+
+constexpr int upd_smem_bytes() {
+  return 1024 + UPD_STAGES * UPD_STAGE_BYTES + NUM_EPI_WARPS * UPD_BOX_BYTES + 256;
+}
+static_assert(upd_smem_bytes() <= 232448, "update kernel exceeds shared memory");
+
+struct UpdJob {
+  int X;      // state tile: (b, mt, nt2) of B x (d/128) x ceil(F/256)
+  int chunk;  // absolute chunk index
+  int slot;   // TMEM slot 0 or 1
+  int b, m0, n0;
+};
+
+// Job i of this block, or false past the end.  The block's tiles are
+// X_m = blockIdx.x + m gridDim.x, taken in pairs (X_2m on slot 0, X_2m+1 on
+// slot 1); a pair is walked chunk by chunk, both tiles per chunk.
+__device__ __forceinline__ bool upd_job(const TcParams& p, uint32_t i, UpdJob& jb) {
+  const int D = p.dchunks;
+  const int nX = p.n_tiles;
+  if ((int)blockIdx.x >= nX) return false;
+  const int nXc = (nX - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  const int pairs = nXc / 2;
+  const uint32_t in_pairs = (uint32_t)pairs * D * 2;
+  int m, c, sl;
+  if (i < in_pairs) {
+    m = (int)(i / (2u * D));
+    const int r = (int)(i % (2u * D));
+    c = r / 2;
+    sl = r % 2;
+  } else {
+    const uint32_t r = i - in_pairs;
+    if ((nXc & 1) == 0 || r >= (uint32_t)D) return false;
+    m = pairs;
+    c = (int)r;
+    sl = 0;
+  }
+  jb.X = (int)blockIdx.x + (2 * m + sl) * (int)gridDim.x;
+  jb.chunk = p.chunk + c;
+  jb.slot = sl;
+  const int nt2s = (p.F + 255) / 256;
+  const int per_row = (p.d / 128) * nt2s;
+  jb.b = jb.X / per_row;
+  const int r = jb.X % per_row;
+  jb.m0 = (r / nt2s) * 128;
+  jb.n0 = (r % nt2s) * 256;
+  return true;
+}
+
+__device__ __forceinline__ bool upd_next_on_slot(const TcParams& p, uint32_t i, int slot, UpdJob& jn) {
+  for (uint32_t k = 1; k <= 2; ++k) {
+    if (!upd_job(p, i + k, jn)) return false;
+    if (jn.slot == slot) return true;
+  }
+  return false;
+}
+
+// fp32 state, 128 x 128 blocked tiles; this thread's row of tile column block h.
+__device__ __forceinline__ float4* upd_state_block(const TcParams& p, const UpdJob& jb, int h) {
+  return reinterpret_cast<float4*>(p.S + (size_t)jb.b * p.d * p.F +
+                                   ((size_t)(jb.m0 / 128) * (p.F / 128) + jb.n0 / 128 + h) * (128 * 128));
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  uint8_t* boxes = smem + UPD_STAGES * UPD_STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(boxes + NUM_EPI_WARPS * UPD_BOX_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + UPD_STAGES;
+  uint64_t* st_ready = empty + UPD_STAGES;  // [2] epilogue -> MMA: slot holds the state to accumulate on
+  uint64_t* st_done = st_ready + 2;         // [2] MMA -> epilogue: the chunk's MMAs on the slot finished
+  uint64_t* drain = st_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < UPD_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&st_ready[s], NUM_EPI_WARPS);
+      mbar_init(&st_done[s], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    counters[0] = counters[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&p.map[3]);
+    prefetch_tmap(&p.map[4]);
+    prefetch_tmap(&p.map[5]);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * ACC_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      UpdJob jb;
+      for (uint32_t i = 0; ok && upd_job(p, i, jb); ++i) {
+        const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
+        const int t0 = jb.chunk * p.C;
+        const int kb0 = (m.last_start - t0) / UPD_KB;
+        const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % UPD_STAGES;
+          const uint32_t ph = (it / UPD_STAGES) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) { ok = false; break; }
+          uint8_t* sa = stages + s * UPD_STAGE_BYTES;
+          uint8_t* sb = sa + UPD_A_BYTES;
+          mbar_arrive_expect_tx(&full[s], UPD_STAGE_BYTES);
+          const int ty = t0 + kb * UPD_KB;
+          tma_load_3d(sa, &p.map[3], &full[s], jb.m0, ty, jb.b);             // V[t][d], d contiguous
+          tma_load_3d(sa + 64 * UPD_KB * 2, &p.map[3], &full[s], jb.m0 + 64, ty, jb.b);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)                                       // Z[t][f], f contiguous
+            tma_load_3d(sb + q * 64 * UPD_KB * 2, &p.map[4], &full[s], jb.n0 + 64 * q, ty, jb.b);
+        }
+      }
+      if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
+      counters[0] = it;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t it = 0, uses[2] = {0, 0};
+      bool ok = true;
+      UpdJob jb;
+      const uint32_t idesc = idesc_bf16(BM, 256, true, true);
+      for (uint32_t i = 0; ok && upd_job(p, i, jb); ++i) {
+        const int sl = jb.slot;
+        const uint32_t u = sl ? uses[1] : uses[0];
+        if (!mbar_wait(&st_ready[sl], u & 1) || *abort_flag) { ok = false; break; }
+        tc_fence_after();
+        const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
+        const int t0 = jb.chunk * p.C;
+        const int kb0 = (m.last_start - t0) / UPD_KB;
+        const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
+        const uint32_t tacc = tmem_base + sl * ACC_COLS;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % UPD_STAGES;
+          const uint32_t ph = (it / UPD_STAGES) & 1;
+          if (!mbar_wait(&full[s], ph) || *abort_flag) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(stages + s * UPD_STAGE_BYTES);
+          const uint32_t b_addr = a_addr + UPD_A_BYTES;
+#pragma unroll
+          for (int ks = 0; ks < UPD_KB / 16; ++ks) {
+            const uint64_t ad = sdesc_sw128(a_addr + ks * 2048, UPD_KB * 128, 1024);
+            const uint64_t bd = sdesc_sw128(b_addr + ks * 2048, UPD_KB * 128, 1024);
+            // A document start inside the chunk drops the carried state.
+            const uint32_t acc = (m.has_start && kb == kb0 && ks == 0) ? 0u : 1u;
+            mma_bf16(tacc, ad, bd, idesc, acc);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&st_done[sl]);
+        if (sl) ++uses[1]; else ++uses[0];
+      }
+      if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
+      counters[1] = it;
+      mma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+  } else {
+    const int ew = warp - 2;
+    const int quarter = warp & 3;   // TMEM lanes this warp may access
+    const int half = ew >> 2;       // 128-column half of the 256-column state tile
+    const int row = quarter * 32 + lane;
+    uint8_t* box = boxes + ew * UPD_BOX_BYTES;
+    bool ok = true;
+    int stores = 0;
+    uint32_t done[2] = {0, 0};
+
+    // Brings tile jb's old state into TMEM slot jb.slot (nothing when its chunk
+    // starts a document: the first MMA then overwrites the slot).
+    auto load_state = [&](const UpdJob& jb) {
+      if (p.meta[(size_t)jb.b * p.k + jb.chunk].has_start) return;
+      if (jb.n0 + 128 * half >= p.F) return;  // past the last column block
+      const float4* src = upd_state_block(p, jb, half);
+      const uint32_t tcol = tmem_base + jb.slot * ACC_COLS + ((uint32_t)(quarter * 32) << 16) + 128 * half;
+#pragma unroll 1
+      for (int g = 0; g < 4; ++g) {
+        uint32_t r[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 v = src[(8 * g + q) * 128 + row];
+          r[4 * q] = __float_as_uint(v.x);
+          r[4 * q + 1] = __float_as_uint(v.y);
+          r[4 * q + 2] = __float_as_uint(v.z);
+          r[4 * q + 3] = __float_as_uint(v.w);
+        }
+        tmem_st32(tcol + 32 * g, r);
+      }
+      tmem_st_wait();
+    };
+    auto release = [&](int sl) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&st_ready[sl]);
+    };
+
+    UpdJob jb;
+    for (uint32_t i = 0; i < 2; ++i)
+      if (upd_job(p, i, jb) && (int)i == jb.slot) {
+        load_state(jb);
+        release(jb.slot);
+      }
+    for (uint32_t i = 0; upd_job(p, i, jb); ++i) {
+      const int sl = jb.slot;
+      if (!mbar_wait(&st_done[sl], done[sl] & 1)) { ok = false; break; }
+      ++done[sl];
+      tc_fence_after();
+      UpdJob jn;
+      const bool has_next = upd_next_on_slot(p, i, sl, jn);
+      const bool last = !has_next || jn.X != jb.X;  // tile's last chunk of the launch
+      const bool snap = jb.chunk + 1 < p.k;
+      if (jb.n0 + 128 * half < p.F) {
+        const uint32_t tcol = tmem_base + sl * ACC_COLS + ((uint32_t)(quarter * 32) << 16) + 128 * half;
+        float4* dst = upd_state_block(p, jb, half);
+#pragma unroll 1
+        for (int bx = 0; bx < 2; ++bx) {  // two 64-column snapshot boxes per warp
+          if (snap && stores > 0) {
+            if (lane == 0) bulk_wait_read<0>();  // the previous box store has read the buffer
+            __syncwarp();
+          }
+#pragma unroll
+          for (int g2 = 0; g2 < 2; ++g2) {
+            const int g = 2 * bx + g2;
+            uint32_t r[32];
+            tmem_ld32(tcol + 32 * g, r);
+            tmem_ld_wait();
+            if (last) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                dst[(8 * g + q) * 128 + row] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                                           __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+            }
+            if (snap) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int chunk16 = g2 * 4 + e;  // 16-byte chunk of this row in the 128-byte box row
+                *reinterpret_cast<uint4*>(box + lane * 128 + ((chunk16 ^ (lane & 7)) << 4)) = make_uint4(
+                    pack_bf16(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
+                    pack_bf16(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
+                    pack_bf16(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
+                    pack_bf16(__uint_as_float(r[8 * e + 6]), __uint_as_float(r[8 * e + 7])));
+              }
+            }
+          }
+          if (snap) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&p.map[5], box, jb.n0 + 128 * half + 64 * bx, jb.m0 + 32 * quarter,
+                           ((jb.chunk + 1) % p.nslots) * p.B + jb.b);
+              bulk_commit();
+            }
+            ++stores;
+          }
+        }
+      }
+      if (has_next) {
+        if (jn.X != jb.X) load_state(jn);
+        release(sl);
+      }
+    }
+    if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    for (uint32_t it = counters[1]; it < counters[0]; ++it)
+      mbar_wait(&full[it % UPD_STAGES], (it / UPD_STAGES) & 1);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * ACC_COLS);
+  }
+}
+
+cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st) {
+  if (p.n_tiles <= 0 || p.dchunks <= 0) return cudaSuccess;
+  constexpr int smem = upd_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(upd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int grid = std::max(1, std::min(p.n_tiles, num_sms));
+  upd_kernel<<<grid, NTHREADS, smem, st>>>(p);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ failure-path self test
@@ -781,10 +922,8 @@ cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st) 
   switch (fam) {
     case FAM_ZV: return launch<FAM_ZV>(p, num_sms, st);
     case FAM_GRAM: return launch<FAM_GRAM>(p, num_sms, st);
-    case FAM_APPLY: return launch<FAM_APPLY>(p, num_sms, st);
-    case FAM_DELTA64: return launch<FAM_DELTA64>(p, num_sms, st);
     case FAM_APPLY256: return launch<FAM_APPLY256>(p, num_sms, st);
-    default: return launch<FAM_DELTA>(p, num_sms, st);
+    default: return launch<FAM_APPLY>(p, num_sms, st);
   }
 }
 

@@ -9,7 +9,7 @@
 namespace ipttt {
 namespace tck {
 
-enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_DELTA = 3, FAM_DELTA64 = 4, FAM_APPLY256 = 5 };
+enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_APPLY256 = 5 };
 
 struct TcParams {
   CUtensorMap map[6];
@@ -19,11 +19,8 @@ struct TcParams {
   int tr;            // token rows per apply / Gram tile: 128, or 64 when C % 128 != 0
   int ct;            // tiles per chunk (C / tr)
   int npairs;        // GRAM: tile pairs per chunk, ct (ct + 1) / 2
-  int chunk;         // DELTA: first chunk whose state update the launch performs
-  int dchunks;       // DELTA: consecutive chunks per launch (tile index = X * dchunks + c)
-  int dwin;          // DELTA: chunks per window; a block takes all of its state tiles
-                     //        through one window before the next, carrying each tile's
-                     //        state in registers inside the window
+  int chunk;         // update: first chunk whose state update the launch performs
+  int dchunks;       // update: consecutive chunks per launch
   int apply_chunk0;  // SCAN: first chunk of the apply tiles
   int n_apply;       // SCAN: apply tiles (chunks apply_chunk0.., all rows); delta tiles follow
   int n_tiles;
@@ -36,13 +33,16 @@ struct TcParams {
   void* out0;             // Z (gate/up), V (target), O (scan)
   float* out1;            // SCAN: optional fp32 D
   const void* resid;      // SCAN: optional residual H added to O
-  float* S;               // DELTA: fp32 state, blocked 128 x 128 tiles
+  float* S;               // update: fp32 state, blocked 128 x 128 tiles
   int* status;            // device status word
 };
 
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
                    uint32_t box_inner, uint32_t box_rows);
 cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st);
+// State update of chunks [p.chunk, p.chunk + p.dchunks) on p.n_tiles state tiles of
+// 128 x 256 (V pre-scaled by alpha eta); writes S_{c+1} snapshots and the fp32 state.
+cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st);
 int kind_gateup();
 int kind_vhat();
