@@ -629,6 +629,47 @@ const char* ipttt_strerror(ipttt_status s) {
 
 const char* ipttt_version(void) { return "0.1.0"; }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation forward
+// Scratch for ipttt_forward_noalloc: one static array per device that loads the
+// library.  In host code the symbol is only a stand-in for the device array, so
+// its device address is looked up (once per device, with that device current)
+// and that address is what the kernels get.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[IPTTT_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_addr[kMaxDevices] = {nullptr};
+std::mutex g_noalloc_mu;
+
+ipttt_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return IPTTT_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) return IPTTT_ERR_CUDA;
+    g_noalloc_addr[dev] = addr;
+  }
+  *out = g_noalloc_addr[dev];
+  return IPTTT_OK;
+}
+}  // namespace
+
+extern "C" {
+
+ipttt_status ipttt_forward_noalloc(const ipttt_params* p, const void* H, const void* X0, const void* Wgate,
+                                   const void* Wup, const void* Wdown0, const void* conv_w, const void* Wtarget,
+                                   const int32_t* doc_starts, int32_t n_doc_starts, void* O, void* stream) {
+  ipttt_status rc = check_params(p);
+  if (rc != IPTTT_OK) return rc;
+  if (layout_of(*p).total > IPTTT_NOALLOC_SCRATCH_BYTES) return IPTTT_ERR_SHAPE;
+  void* ws = nullptr;
+  if ((rc = noalloc_scratch(&ws)) != IPTTT_OK) return rc;
+  return ipttt_forward(p, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_starts, n_doc_starts, O, ws,
+                       IPTTT_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 void ipttt_profile_enable(int on) { g_profile_on.store(on ? 1 : 0); }
 
 int ipttt_profile_read(double* ms, uint64_t* launches, int n_phases) {

@@ -24,7 +24,7 @@ STATUS = {0: "IPTTT_OK", 1: "IPTTT_ERR_ARG", 2: "IPTTT_ERR_SHAPE", 3: "IPTTT_ERR
 EXPORTS = ("ipttt_workspace_size", "ipttt_forward", "ipttt_forward_ex", "ipttt_core", "ipttt_stream_state_size",
            "ipttt_stream_reset", "ipttt_stream_forward", "ipttt_stream_export", "ipttt_get_status",
            "ipttt_strerror", "ipttt_version", "ipttt_profile_enable", "ipttt_profile_read",
-           "ipttt_kernel_launches", "ipttt_selftest_wait_timeout")
+           "ipttt_kernel_launches", "ipttt_selftest_wait_timeout", "ipttt_forward_noalloc")
 PHASES = ("prep", "gate_up", "target", "gram", "apply", "update")
 DEBUG_OUTPUTS = ("D", "S_final", "alpha", "Z", "V")
 
@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.ipttt_kernel_launches.restype = ctypes.c_uint64
         L.ipttt_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
         L.ipttt_selftest_wait_timeout.restype = ctypes.c_int
+        L.ipttt_forward_noalloc.argtypes = [P] + [vp] * 7 + [vp, i32, vp, vp]
+        L.ipttt_forward_noalloc.restype = ctypes.c_int
         _lib = L
     return _lib
 

@@ -174,6 +174,31 @@ IPTTT_API void ipttt_profile_enable(int on);
 IPTTT_API int ipttt_profile_read(double* ms, uint64_t* launches, int n_phases);
 IPTTT_API uint64_t ipttt_kernel_launches(void);
 
+/* Forward without any allocation, for callers that cannot call cudaMalloc: code
+ * whose device memory belongs to another allocator (a framework's caching
+ * allocator, a serving runtime with a fixed memory budget) and may not grow it in
+ * the middle of a run, or a latency-critical path that cannot accept the implicit
+ * device synchronisation of cudaMalloc/cudaFree.  The paper has no counterpart;
+ * this is a packaging variant of ipttt_forward.
+ *
+ * Same arguments and result as ipttt_forward, minus the workspace: the library
+ * uses its own scratch, a static device array of IPTTT_NOALLOC_SCRATCH_BYTES that
+ * every GPU loading the library holds until the process exits.  Shapes whose
+ * ipttt_workspace_size exceeds that return IPTTT_ERR_SHAPE without launching.
+ * The scratch address is looked up once per device, on that device's first call
+ * (make that call before any stream capture); the call allocates nothing.  All
+ * calls on a device share the one scratch array and it keeps the last call's
+ * contents (every call initialises what it reads), so calls that may overlap on
+ * the GPU (different streams without ordering, or different host threads) race
+ * and must be serialised by the caller. */
+#define IPTTT_NOALLOC_SCRATCH_BYTES (32u << 20)
+IPTTT_API ipttt_status ipttt_forward_noalloc(const ipttt_params* p,
+                                   const void* H, const void* X0,
+                                   const void* Wgate, const void* Wup, const void* Wdown0,
+                                   const void* conv_w, const void* Wtarget,
+                                   const int32_t* doc_starts, int32_t n_doc_starts,
+                                   void* O, void* stream);
+
 /* Self-test of the device-side failure path: launches one block that waits, with
  * the same bounded wait the kernels use, on a barrier phase that nothing ever
  * completes.  After limit_ns nanoseconds (0: the kernels' own limit, 2 s) it gives
