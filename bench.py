@@ -172,12 +172,18 @@ def config_dict(w: synth.Workload, n: int) -> dict:
             "l2": "inputs larger than L2 (H and X0 are B*T*d bf16; Z is B*T*F bf16)"}
 
 
+def sample_chunks(w: synth.Workload, tokens: int) -> int:
+    """Whole chunks of row 0 covering at least `tokens` tokens (at least one chunk)."""
+    k = (w.T + w.C - 1) // w.C
+    return max(1, min(k, (max(1, tokens) + w.C - 1) // w.C))
+
+
 def run_reference(args, w: synth.Workload):
     world, rank, _ = dist_env()
     if rank != 0:
         return
     inp = synth.make_inputs(w.replace(B=1), seed=0)
-    chunks = max(1, args.cpu_sample_chunks)
+    chunks = sample_chunks(w, args.ref_sample_tokens)
     for _ in range(args.warmup):
         oracle_sample(w, inp, chunks)
     secs, toks = 0.0, 0
@@ -326,9 +332,10 @@ def run_ours(args, w: synth.Workload):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        secs, n = oracle_sample(w, layers[0], args.cpu_sample_chunks)
+        chunks = sample_chunks(w, args.cpu_sample_tokens)
+        secs, n = oracle_sample(w, layers[0], chunks)
         cpu = {"value": n / secs, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"first {args.cpu_sample_chunks} chunk(s) ({n} tokens) of row 0, one layer, "
+               "sample": f"first {chunks} chunk(s) ({n} tokens) of row 0, one layer, "
                          f"fp64 numpy oracle, {secs:.1f} s"}
 
     if rank == 0:
@@ -355,7 +362,10 @@ def main(argv=None):
     ap.add_argument("--chunk", type=int, default=None, help="override the chunk size C")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-chunks", type=int, default=2)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=16384,
+                    help="tokens of row 0 the oracle runs for cpu_baseline (whole chunks, about 10 s)")
+    ap.add_argument("--ref-sample-tokens", type=int, default=4096,
+                    help="tokens of row 0 per step of the reference arm (whole chunks)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
