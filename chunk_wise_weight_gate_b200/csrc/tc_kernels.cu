@@ -29,6 +29,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -540,38 +541,52 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
 // ------------------------------------------------------------------ state update
 // S_{c+1} = keep_c S_c + alpha_c eta V_c^T Z_c for the chunks c of one launch.
 // V arrives pre-scaled by alpha_c eta per row, so the MMAs accumulate the state
-// itself: each block keeps two 128 (d) x 256 (F) fp32 state tiles in TMEM (slots 0
-// and 1) and walks both through all chunks of the launch, alternating, so that
-// the epilogue reads one slot (bf16 snapshot of S_{c+1} for the apply) while the
-// MMAs run on the other.  A chunk holding a document start resets the tile (its
-// first MMA does not accumulate).  A tile's fp32 state comes in from HBM before
-// its first chunk (tcgen05.st) and goes back after its last.
-constexpr int UPD_STAGES = 4;
+// itself: the fp32 state tiles live in TMEM (slots 0 and 1, 256 columns each)
+// and are walked through all chunks of the launch, the two slots alternating, so
+// that the epilogue reads one slot (bf16 snapshot of S_{c+1} for the apply) while
+// the MMAs run on the other.  A chunk holding a document start resets the tile
+// (its first MMA does not accumulate).  A tile's fp32 state comes in from HBM
+// before its first chunk (tcgen05.st) and goes back after its last.
+//
+// Two forms of one kernel body:
+//   PAIR = false: one CTA per 128 (d) x 256 (F) state tile, M=128 MMAs.
+//   PAIR = true : a cluster of two CTAs per 256 x 256 tile, M=256 pair MMAs
+//                 (cta_group::2).  CTA r holds d rows m0 + 128 r .. +127 of the
+//                 tile in its TMEM and loads those V columns and Z columns
+//                 n0 + 128 r .. +127 per stage; the even CTA issues the MMAs.  Per
+//                 FLOP this moves 2/3 of the operand bytes of the single-CTA form.
 constexpr int UPD_KB = 64;                            // tokens per stage
-constexpr int UPD_A_BYTES = 128 * UPD_KB * 2;         // V: 128 d columns
-constexpr int UPD_STAGE_BYTES = UPD_A_BYTES + 256 * UPD_KB * 2;  // + Z: 256 F columns
 constexpr int UPD_BOX_BYTES = 32 * 128;               // a warp's 32-row x 64-column snapshot box
+constexpr int UPD_BOXES = 2;                          // per warp: box stores in flight while the next is filled
+static_assert(UPD_BOXES == 1 || UPD_BOXES == 2, "one or two snapshot boxes per warp");
 
-constexpr int upd_smem_bytes() {
-  return 1024 + UPD_STAGES * UPD_STAGE_BYTES + NUM_EPI_WARPS * UPD_BOX_BYTES + 256;
-}
-static_assert(upd_smem_bytes() <= 232448, "update kernel exceeds shared memory");
+template <bool PAIR> struct UpdCfg {
+  static constexpr int STAGES = PAIR ? 5 : 3;
+  static constexpr int A_BYTES = 128 * UPD_KB * 2;                        // V: 128 d columns
+  static constexpr int B_COLS = PAIR ? 128 : 256;                         // Z columns this CTA loads
+  static constexpr int STAGE_BYTES = A_BYTES + B_COLS * UPD_KB * 2;
+  static constexpr int TILE_ROWS = PAIR ? 256 : 128;                      // d rows per state tile
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + NUM_EPI_WARPS * UPD_BOXES * UPD_BOX_BYTES + 256;
+};
+static_assert(UpdCfg<false>::SMEM <= 232448, "update kernel exceeds shared memory");
+static_assert(UpdCfg<true>::SMEM <= 232448, "pair update kernel exceeds shared memory");
 
 struct UpdJob {
-  int X;      // state tile: (b, mt, nt2) of B x (d/128) x ceil(F/256)
+  int X;      // state tile: (b, mt, nt2) of B x (d/TILE_ROWS) x ceil(F/256)
   int chunk;  // absolute chunk index
   int slot;   // TMEM slot 0 or 1
   int b, m0, n0;
 };
 
-// Job i of this block, or false past the end.  The block's tiles are
-// X_m = blockIdx.x + m gridDim.x, taken in pairs (X_2m on slot 0, X_2m+1 on
+// Job i of worker w (a CTA, or a CTA pair) of nw, or false past the end.  The
+// worker's tiles are X_m = w + m nw, taken in pairs (X_2m on slot 0, X_2m+1 on
 // slot 1); a pair is walked chunk by chunk, both tiles per chunk.
-__device__ __forceinline__ bool upd_job(const TcParams& p, uint32_t i, UpdJob& jb) {
+template <bool PAIR>
+__device__ __forceinline__ bool upd_job(const TcParams& p, uint32_t i, int w, int nw, UpdJob& jb) {
   const int D = p.dchunks;
   const int nX = p.n_tiles;
-  if ((int)blockIdx.x >= nX) return false;
-  const int nXc = (nX - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  if (w >= nX) return false;
+  const int nXc = (nX - w + nw - 1) / nw;
   const int pairs = nXc / 2;
   const uint32_t in_pairs = (uint32_t)pairs * D * 2;
   int m, c, sl;
@@ -587,42 +602,48 @@ __device__ __forceinline__ bool upd_job(const TcParams& p, uint32_t i, UpdJob& j
     c = (int)r;
     sl = 0;
   }
-  jb.X = (int)blockIdx.x + (2 * m + sl) * (int)gridDim.x;
+  jb.X = w + (2 * m + sl) * nw;
   jb.chunk = p.chunk + c;
   jb.slot = sl;
   const int nt2s = (p.F + 255) / 256;
-  const int per_row = (p.d / 128) * nt2s;
+  const int per_row = (p.d / UpdCfg<PAIR>::TILE_ROWS) * nt2s;
   jb.b = jb.X / per_row;
   const int r = jb.X % per_row;
-  jb.m0 = (r / nt2s) * 128;
+  jb.m0 = (r / nt2s) * UpdCfg<PAIR>::TILE_ROWS;
   jb.n0 = (r % nt2s) * 256;
   return true;
 }
 
-__device__ __forceinline__ bool upd_next_on_slot(const TcParams& p, uint32_t i, int slot, UpdJob& jn) {
+template <bool PAIR>
+__device__ __forceinline__ bool upd_next_on_slot(const TcParams& p, uint32_t i, int w, int nw, int slot,
+                                                 UpdJob& jn) {
   for (uint32_t k = 1; k <= 2; ++k) {
-    if (!upd_job(p, i + k, jn)) return false;
+    if (!upd_job<PAIR>(p, i + k, w, nw, jn)) return false;
     if (jn.slot == slot) return true;
   }
   return false;
 }
 
-// fp32 state, 128 x 128 blocked tiles; this thread's row of tile column block h.
-__device__ __forceinline__ float4* upd_state_block(const TcParams& p, const UpdJob& jb, int h) {
-  return reinterpret_cast<float4*>(p.S + (size_t)jb.b * p.d * p.F +
-                                   ((size_t)(jb.m0 / 128) * (p.F / 128) + jb.n0 / 128 + h) * (128 * 128));
+// fp32 state, 128 x 128 blocked tiles; tile column block h of the 128-row block
+// starting at d row m0 (a multiple of 128).
+__device__ __forceinline__ float4* upd_state_block(const TcParams& p, int b, int m0, int n0, int h) {
+  return reinterpret_cast<float4*>(p.S + (size_t)b * p.d * p.F +
+                                   ((size_t)(m0 / 128) * (p.F / 128) + n0 / 128 + h) * (128 * 128));
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant__ TcParams p) {
+  using Cf = UpdCfg<PAIR>;
+  constexpr int STAGES = Cf::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* boxes = smem + UPD_STAGES * UPD_STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(boxes + NUM_EPI_WARPS * UPD_BOX_BYTES);
+  uint8_t* boxes = smem + STAGES * Cf::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(boxes + NUM_EPI_WARPS * UPD_BOXES * UPD_BOX_BYTES);
   uint64_t* full = bars;
-  uint64_t* empty = bars + UPD_STAGES;
-  uint64_t* st_ready = empty + UPD_STAGES;  // [2] epilogue -> MMA: slot holds the state to accumulate on
-  uint64_t* st_done = st_ready + 2;         // [2] MMA -> epilogue: the chunk's MMAs on the slot finished
+  uint64_t* empty = bars + STAGES;
+  uint64_t* st_ready = empty + STAGES;  // [2] epilogue -> MMA: slot holds the state to accumulate on
+  uint64_t* st_done = st_ready + 2;     // [2] MMA -> epilogue: the chunk's MMAs on the slot finished
   uint64_t* drain = st_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -630,13 +651,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const int wk = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;      // worker (pair) index
+  const int nwk = PAIR ? (int)cluster_count_x() : (int)gridDim.x;
+  const int rofs = PAIR ? 128 * (int)rank : 0;                      // this CTA's rows / Z columns in the tile
+
   if (threadIdx.x == 0) {
-    for (int s = 0; s < UPD_STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&st_ready[s], NUM_EPI_WARPS);
+      mbar_init(&st_ready[s], NUM_EPI_WARPS * (PAIR ? 2 : 1));
       mbar_init(&st_done[s], 1);
     }
     mbar_init(drain, 1);
@@ -650,11 +676,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
     prefetch_tmap(&p.map[5]);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * ACC_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, 2 * ACC_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, 2 * ACC_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -663,39 +694,51 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
       uint32_t it = 0;
       bool ok = true;
       UpdJob jb;
-      for (uint32_t i = 0; ok && upd_job(p, i, jb); ++i) {
+      const uint32_t full0 = PAIR ? map_to_rank(smem_u32(full), 0) : 0u;  // the leader's full[0]
+      for (uint32_t i = 0; ok && upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
         const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
         const int t0 = jb.chunk * p.C;
         const int kb0 = (m.last_start - t0) / UPD_KB;
         const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % UPD_STAGES;
-          const uint32_t ph = (it / UPD_STAGES) & 1;
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) { ok = false; break; }
-          uint8_t* sa = stages + s * UPD_STAGE_BYTES;
-          uint8_t* sb = sa + UPD_A_BYTES;
-          mbar_arrive_expect_tx(&full[s], UPD_STAGE_BYTES);
+          uint8_t* sa = stages + s * Cf::STAGE_BYTES;
+          uint8_t* sb = sa + Cf::A_BYTES;
           const int ty = t0 + kb * UPD_KB;
-          tma_load_3d(sa, &p.map[3], &full[s], jb.m0, ty, jb.b);             // V[t][d], d contiguous
-          tma_load_3d(sa + 64 * UPD_KB * 2, &p.map[3], &full[s], jb.m0 + 64, ty, jb.b);
+          if constexpr (PAIR) {
+            // both CTAs' bytes complete the leader's barrier; the leader arms it
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cf::STAGE_BYTES);
+            const uint32_t fb = full0 + 8u * s;
+            tma_load_3d_pair(sa, &p.map[3], fb, jb.m0 + rofs, ty, jb.b);             // V[t][d], d contiguous
+            tma_load_3d_pair(sa + 64 * UPD_KB * 2, &p.map[3], fb, jb.m0 + rofs + 64, ty, jb.b);
+            tma_load_3d_pair(sb, &p.map[4], fb, jb.n0 + rofs, ty, jb.b);             // Z[t][f], f contiguous
+            tma_load_3d_pair(sb + 64 * UPD_KB * 2, &p.map[4], fb, jb.n0 + rofs + 64, ty, jb.b);
+          } else {
+            mbar_arrive_expect_tx(&full[s], Cf::STAGE_BYTES);
+            tma_load_3d(sa, &p.map[3], &full[s], jb.m0, ty, jb.b);
+            tma_load_3d(sa + 64 * UPD_KB * 2, &p.map[3], &full[s], jb.m0 + 64, ty, jb.b);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)                                       // Z[t][f], f contiguous
-            tma_load_3d(sb + q * 64 * UPD_KB * 2, &p.map[4], &full[s], jb.n0 + 64 * q, ty, jb.b);
+            for (int q = 0; q < 4; ++q)
+              tma_load_3d(sb + q * 64 * UPD_KB * 2, &p.map[4], &full[s], jb.n0 + 64 * q, ty, jb.b);
+          }
         }
       }
       if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
       counters[0] = it;
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      uint32_t it = 0, uses[2] = {0, 0};
+    if (lane == 0 && rank == 0) {
+      uint32_t it = 0, uses0 = 0, uses1 = 0;
       bool ok = true;
       UpdJob jb;
-      const uint32_t idesc = idesc_bf16(BM, 256, true, true);
-      for (uint32_t i = 0; ok && upd_job(p, i, jb); ++i) {
+      const uint32_t idesc = idesc_bf16(PAIR ? 256 : 128, 256, true, true);
+      for (uint32_t i = 0; ok && upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
         const int sl = jb.slot;
-        const uint32_t u = sl ? uses[1] : uses[0];
-        if (!mbar_wait(&st_ready[sl], u & 1) || *abort_flag) { ok = false; break; }
+        const uint32_t u = sl ? uses1 : uses0;
+        const bool got = PAIR ? mbar_wait_cluster(&st_ready[sl], u & 1) : mbar_wait(&st_ready[sl], u & 1);
+        if (!got || *abort_flag) { ok = false; break; }
         tc_fence_after();
         const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
         const int t0 = jb.chunk * p.C;
@@ -703,29 +746,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
         const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
         const uint32_t tacc = tmem_base + sl * ACC_COLS;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % UPD_STAGES;
-          const uint32_t ph = (it / UPD_STAGES) & 1;
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(&full[s], ph) || *abort_flag) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(stages + s * UPD_STAGE_BYTES);
-          const uint32_t b_addr = a_addr + UPD_A_BYTES;
+          const uint32_t a_addr = smem_u32(stages + s * Cf::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + Cf::A_BYTES;
 #pragma unroll
           for (int ks = 0; ks < UPD_KB / 16; ++ks) {
             const uint64_t ad = sdesc_sw128(a_addr + ks * 2048, UPD_KB * 128, 1024);
             const uint64_t bd = sdesc_sw128(b_addr + ks * 2048, UPD_KB * 128, 1024);
             // A document start inside the chunk drops the carried state.
             const uint32_t acc = (m.has_start && kb == kb0 && ks == 0) ? 0u : 1u;
-            mma_bf16(tacc, ad, bd, idesc, acc);
+            if constexpr (PAIR) mma_bf16_pair(tacc, ad, bd, idesc, acc);
+            else mma_bf16(tacc, ad, bd, idesc, acc);
           }
-          mma_commit(&empty[s]);
+          if constexpr (PAIR) mma_commit_pair(&empty[s], 3); else mma_commit(&empty[s]);
         }
         if (!ok) break;
-        mma_commit(&st_done[sl]);
-        if (sl) ++uses[1]; else ++uses[0];
+        if constexpr (PAIR) mma_commit_pair(&st_done[sl], 3); else mma_commit(&st_done[sl]);
+        if (sl) ++uses1; else ++uses0;
       }
       if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
       counters[1] = it;
-      mma_commit(drain);
+      if constexpr (PAIR) mma_commit_pair(drain, 1); else mma_commit(drain);
       mbar_wait(drain, 0);
     }
   } else {
@@ -733,17 +777,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
     const int quarter = warp & 3;   // TMEM lanes this warp may access
     const int half = ew >> 2;       // 128-column half of the 256-column state tile
     const int row = quarter * 32 + lane;
-    uint8_t* box = boxes + ew * UPD_BOX_BYTES;
+    uint8_t* wboxes = boxes + ew * UPD_BOXES * UPD_BOX_BYTES;
     bool ok = true;
     int stores = 0;
-    uint32_t done[2] = {0, 0};
+    uint32_t done0 = 0, done1 = 0;
+    const uint32_t ready0 = PAIR ? map_to_rank(smem_u32(st_ready), 0) : 0u;  // the leader's st_ready[0]
 
-    // Brings tile jb's old state into TMEM slot jb.slot (nothing when its chunk
-    // starts a document: the first MMA then overwrites the slot).
+    // Brings tile jb's old state (this CTA's rows) into TMEM slot jb.slot (nothing
+    // when its chunk starts a document: the first MMA then overwrites the slot).
     auto load_state = [&](const UpdJob& jb) {
       if (p.meta[(size_t)jb.b * p.k + jb.chunk].has_start) return;
       if (jb.n0 + 128 * half >= p.F) return;  // past the last column block
-      const float4* src = upd_state_block(p, jb, half);
+      const float4* src = upd_state_block(p, jb.b, jb.m0 + rofs, jb.n0, half);
       const uint32_t tcol = tmem_base + jb.slot * ACC_COLS + ((uint32_t)(quarter * 32) << 16) + 128 * half;
 #pragma unroll 1
       for (int g = 0; g < 4; ++g) {
@@ -763,39 +808,47 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
     auto release = [&](int sl) {
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&st_ready[sl]);
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(ready0 + 8u * sl);
+        else mbar_arrive(&st_ready[sl]);
+      }
     };
 
     UpdJob jb;
     for (uint32_t i = 0; i < 2; ++i)
-      if (upd_job(p, i, jb) && (int)i == jb.slot) {
+      if (upd_job<PAIR>(p, i, wk, nwk, jb) && (int)i == jb.slot) {
         load_state(jb);
         release(jb.slot);
       }
-    for (uint32_t i = 0; upd_job(p, i, jb); ++i) {
+    for (uint32_t i = 0; upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
       const int sl = jb.slot;
-      if (!mbar_wait(&st_done[sl], done[sl] & 1)) { ok = false; break; }
-      ++done[sl];
+      if (!mbar_wait(&st_done[sl], (sl ? done1 : done0) & 1)) { ok = false; break; }
+      if (sl) ++done1; else ++done0;
       tc_fence_after();
       UpdJob jn;
-      const bool has_next = upd_next_on_slot(p, i, sl, jn);
+      const bool has_next = upd_next_on_slot<PAIR>(p, i, wk, nwk, sl, jn);
       const bool last = !has_next || jn.X != jb.X;  // tile's last chunk of the launch
       const bool snap = jb.chunk + 1 < p.k;
+      const int m0c = jb.m0 + rofs;
       if (jb.n0 + 128 * half < p.F) {
         const uint32_t tcol = tmem_base + sl * ACC_COLS + ((uint32_t)(quarter * 32) << 16) + 128 * half;
-        float4* dst = upd_state_block(p, jb, half);
+        float4* dst = upd_state_block(p, jb.b, m0c, jb.n0, half);
 #pragma unroll 1
         for (int bx = 0; bx < 2; ++bx) {  // two 64-column snapshot boxes per warp
+          uint8_t* box = wboxes + (bx % UPD_BOXES) * UPD_BOX_BYTES;
           if (snap && stores > 0) {
-            if (lane == 0) bulk_wait_read<0>();  // the previous box store has read the buffer
+            // the store issued from this buffer two boxes ago has read it
+            if (lane == 0) bulk_wait_read<UPD_BOXES - 1>();
             __syncwarp();
           }
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tcol + 64 * bx, r0);
+          tmem_ld32(tcol + 64 * bx + 32, r1);
+          tmem_ld_wait();
 #pragma unroll
           for (int g2 = 0; g2 < 2; ++g2) {
+            const uint32_t* r = g2 ? r1 : r0;
             const int g = 2 * bx + g2;
-            uint32_t r[32];
-            tmem_ld32(tcol + 32 * g, r);
-            tmem_ld_wait();
             if (last) {
 #pragma unroll
               for (int q = 0; q < 8; ++q)
@@ -818,7 +871,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_3d(&p.map[5], box, jb.n0 + 128 * half + 64 * bx, jb.m0 + 32 * quarter,
+              tma_store_3d(&p.map[5], box, jb.n0 + 128 * half + 64 * bx, m0c + 32 * quarter,
                            ((jb.chunk + 1) % p.nslots) * p.B + jb.b);
               bulk_commit();
             }
@@ -836,24 +889,85 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
   }
 
   __syncthreads();
-  if (*abort_flag && threadIdx.x == 0) {
+  // After a timeout: let this CTA's issued but never consumed loads land before
+  // the shared memory goes away (each wait is bounded).
+  if (*abort_flag && threadIdx.x == 0 && rank == 0) {
     for (uint32_t it = counters[1]; it < counters[0]; ++it)
-      mbar_wait(&full[it % UPD_STAGES], (it / UPD_STAGES) & 1);
+      mbar_wait(&full[it % STAGES], (it / STAGES) & 1);
   }
-  __syncthreads();
+  tc_fence_before();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * ACC_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, 2 * ACC_COLS);
+    else tmem_dealloc(tmem_base, 2 * ACC_COLS);
   }
+}
+
+// Pairs of CTAs that can be resident at once (a cluster needs two SMs of one
+// GPC); 0 when the device cannot run the pair kernel.
+static int max_pairs(cudaStream_t st) {
+  static int cached[64];
+  static bool have[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (have[dev]) return cached[dev];
+  int n = 0;
+  constexpr int smem = UpdCfg<true>::SMEM;
+  if (cudaFuncSetAttribute(upd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(NTHREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, upd_kernel<true>, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  cached[dev] = n;
+  have[dev] = true;
+  return n;
+}
+
+static bool pair_update_enabled() {
+  const char* e = getenv("IPTTT_UPDATE_CTAS");
+  return !(e && e[0] == '1');
 }
 
 cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st) {
   if (p.n_tiles <= 0 || p.dchunks <= 0) return cudaSuccess;
-  constexpr int smem = upd_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(upd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (p.d % 256 == 0 && pair_update_enabled()) {
+    const int np = max_pairs(st);
+    if (np > 0) {
+      TcParams q = p;
+      q.n_tiles = p.n_tiles / 2;  // 256-row tiles
+      constexpr int smem = UpdCfg<true>::SMEM;
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * std::max(1, std::min(q.n_tiles, np)), 1, 1);
+      cfg.blockDim = dim3(NTHREADS, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = st;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      return cudaLaunchKernelEx(&cfg, upd_kernel<true>, q);
+    }
+  }
+  constexpr int smem = UpdCfg<false>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(upd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(p.n_tiles, num_sms));
-  upd_kernel<<<grid, NTHREADS, smem, st>>>(p);
+  upd_kernel<false><<<grid, NTHREADS, smem, st>>>(p);
   return cudaGetLastError();
 }
 
