@@ -352,8 +352,8 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   if (!make_map_bf16(&sc.map[0], Z, s.F, s.T, s.B, 64, arows == 256 ? 128 : tp.tr) ||
       !make_map_bf16(&sc.map[1], t.W0, s.F, s.d, 1, 64, 128) ||
       !make_map_bf16(&sc.map[2], snap, s.F, s.d, (uint64_t)G * s.B, 64, 128) ||
-      !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, 64) ||
-      !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, 64) ||
+      !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, update_tokens_per_stage(s.C)) ||
+      !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, update_tokens_per_stage(s.C)) ||
       !make_map_bf16(&sc.map[5], snap, s.F, s.d, (uint64_t)G * s.B, 64, 32))
     return IPTTT_ERR_CUDA;
   sc.out0 = t.O;

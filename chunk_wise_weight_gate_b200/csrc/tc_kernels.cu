@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
           for (int kb = j.kb0[seg]; kb < j.kb1[seg]; ++kb, ++it) {
             const int s = it % STAGES;
             const uint32_t ph = (it / STAGES) & 1;
-            if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) { ok = false; break; }
+            if (!mbar_wait_or_abort(&empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
             uint8_t* sa = stages + s * STAGE_BYTES;
             mbar_arrive_expect_tx(&full[s], j.tx);
             issue_loads<FAM>(p, j, seg, kb, sa, sa + Cfg<FAM>::B_OFF, &full[s]);
@@ -452,6 +452,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
+      bool ready = mbar_try_wait(&full[0], 0);
       for (uint32_t i = 0; ok; ++i, ++tcount) {
         const int tile = seq_tile<FAM>(p, i);
         if (tile < 0) break;
@@ -459,7 +460,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
         decode<FAM>(p, tile, j);
         const int buf = Cfg<FAM>::NBUF == 2 ? (tcount & 1) : 0;
         const uint32_t aph = Cfg<FAM>::NBUF == 2 ? ((tcount >> 1) & 1) : (tcount & 1);
-        if (!mbar_wait(&acc_empty[buf], aph ^ 1) || *abort_flag) { ok = false; break; }
+        if (!mbar_wait_or_abort(&acc_empty[buf], aph ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tacc = tmem_base + buf * ACC_COLS;
         const uint32_t idesc = idesc_bf16(BM, j.n_mma, j.a_mn, j.b_mn);
@@ -467,8 +468,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
           for (int kb = j.kb0[seg]; kb < j.kb1[seg]; ++kb, ++it) {
             const int s = it % STAGES;
             const uint32_t ph = (it / STAGES) & 1;
-            if (!mbar_wait(&full[s], ph) || *abort_flag) { ok = false; break; }
-            tc_fence_after();
+            if (!ready && !mbar_wait_or_abort(&full[s], ph, abort_flag)) { ok = false; break; }
+            // peek at the next stage while this one's MMAs are queued
+            ready = mbar_try_wait(&full[(it + 1) % STAGES], ((it + 1) / STAGES) & 1);
             const uint32_t a_addr = smem_u32(stages + s * STAGE_BYTES);
             const uint32_t b_addr = a_addr + Cfg<FAM>::B_OFF;
             constexpr int KB = Cfg<FAM>::KB;
@@ -555,21 +557,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
 //                 tile in its TMEM and loads those V columns and Z columns
 //                 n0 + 128 r .. +127 per stage; the even CTA issues the MMAs.  Per
 //                 FLOP this moves 2/3 of the operand bytes of the single-CTA form.
-constexpr int UPD_KB = 64;                            // tokens per stage
 constexpr int UPD_BOX_BYTES = 32 * 128;               // a warp's 32-row x 64-column snapshot box
-constexpr int UPD_BOXES = 2;                          // per warp: box stores in flight while the next is filled
-static_assert(UPD_BOXES == 1 || UPD_BOXES == 2, "one or two snapshot boxes per warp");
 
-template <bool PAIR> struct UpdCfg {
-  static constexpr int STAGES = PAIR ? 5 : 3;
-  static constexpr int A_BYTES = 128 * UPD_KB * 2;                        // V: 128 d columns
+// KB tokens per stage: 128 (8 MMAs per stage; the per-stage issue overhead is
+// paid half as often) when the chunk length is a multiple of 128, else 64 (a
+// stage never straddles two chunks).  BOXES snapshot boxes per warp: with two,
+// a box store stays in flight while the next box is filled.
+template <bool PAIR, int KB> struct UpdCfg {
+  static constexpr int STAGES = KB == 128 ? (PAIR ? 3 : 2) : (PAIR ? 5 : 3);
+  static constexpr int BOXES = KB == 128 ? 1 : 2;
+  static constexpr int A_BYTES = 128 * KB * 2;                            // V: 128 d columns
   static constexpr int B_COLS = PAIR ? 128 : 256;                         // Z columns this CTA loads
-  static constexpr int STAGE_BYTES = A_BYTES + B_COLS * UPD_KB * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_COLS * KB * 2;
   static constexpr int TILE_ROWS = PAIR ? 256 : 128;                      // d rows per state tile
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + NUM_EPI_WARPS * UPD_BOXES * UPD_BOX_BYTES + 256;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + NUM_EPI_WARPS * BOXES * UPD_BOX_BYTES + 256;
 };
-static_assert(UpdCfg<false>::SMEM <= 232448, "update kernel exceeds shared memory");
-static_assert(UpdCfg<true>::SMEM <= 232448, "pair update kernel exceeds shared memory");
+static_assert(UpdCfg<false, 64>::SMEM <= 232448 && UpdCfg<true, 64>::SMEM <= 232448 &&
+                  UpdCfg<false, 128>::SMEM <= 232448 && UpdCfg<true, 128>::SMEM <= 232448,
+              "update kernel exceeds shared memory");
 
 struct UpdJob {
   int X;      // state tile: (b, mt, nt2) of B x (d/TILE_ROWS) x ceil(F/256)
@@ -606,10 +611,10 @@ __device__ __forceinline__ bool upd_job(const TcParams& p, uint32_t i, int w, in
   jb.chunk = p.chunk + c;
   jb.slot = sl;
   const int nt2s = (p.F + 255) / 256;
-  const int per_row = (p.d / UpdCfg<PAIR>::TILE_ROWS) * nt2s;
+  const int per_row = (p.d / (PAIR ? 256 : 128)) * nt2s;
   jb.b = jb.X / per_row;
   const int r = jb.X % per_row;
-  jb.m0 = (r / nt2s) * UpdCfg<PAIR>::TILE_ROWS;
+  jb.m0 = (r / nt2s) * (PAIR ? 256 : 128);
   jb.n0 = (r % nt2s) * 256;
   return true;
 }
@@ -631,10 +636,12 @@ __device__ __forceinline__ float4* upd_state_block(const TcParams& p, int b, int
                                    ((size_t)(m0 / 128) * (p.F / 128) + n0 / 128 + h) * (128 * 128));
 }
 
-template <bool PAIR>
+template <bool PAIR, int KB>
 __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant__ TcParams p) {
-  using Cf = UpdCfg<PAIR>;
+  using Cf = UpdCfg<PAIR, KB>;
   constexpr int STAGES = Cf::STAGES;
+  constexpr int UPD_KB = KB;
+  constexpr int UPD_BOXES = Cf::BOXES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
@@ -906,6 +913,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
 
 // Pairs of CTAs that can be resident at once (a cluster needs two SMs of one
 // GPC); 0 when the device cannot run the pair kernel.
+template <int KB>
 static int max_pairs(cudaStream_t st) {
   static int cached[64];
   static bool have[64];
@@ -913,8 +921,9 @@ static int max_pairs(cudaStream_t st) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (have[dev]) return cached[dev];
   int n = 0;
-  constexpr int smem = UpdCfg<true>::SMEM;
-  if (cudaFuncSetAttribute(upd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+  constexpr int smem = UpdCfg<true, KB>::SMEM;
+  if (cudaFuncSetAttribute(upd_kernel<true, KB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
+      cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -927,7 +936,7 @@ static int max_pairs(cudaStream_t st) {
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, upd_kernel<true>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, upd_kernel<true, KB>, &cfg) != cudaSuccess) n = 0;
   }
   cudaGetLastError();
   cached[dev] = n;
@@ -940,14 +949,14 @@ static bool pair_update_enabled() {
   return !(e && e[0] == '1');
 }
 
-cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st) {
-  if (p.n_tiles <= 0 || p.dchunks <= 0) return cudaSuccess;
+template <int KB>
+static cudaError_t launch_update_kb(const TcParams& p, int num_sms, cudaStream_t st) {
   if (p.d % 256 == 0 && pair_update_enabled()) {
-    const int np = max_pairs(st);
+    const int np = max_pairs<KB>(st);
     if (np > 0) {
       TcParams q = p;
       q.n_tiles = p.n_tiles / 2;  // 256-row tiles
-      constexpr int smem = UpdCfg<true>::SMEM;
+      constexpr int smem = UpdCfg<true, KB>::SMEM;
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -960,15 +969,23 @@ cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st) {
       cfg.stream = st;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      return cudaLaunchKernelEx(&cfg, upd_kernel<true>, q);
+      return cudaLaunchKernelEx(&cfg, upd_kernel<true, KB>, q);
     }
   }
-  constexpr int smem = UpdCfg<false>::SMEM;
-  cudaError_t e = cudaFuncSetAttribute(upd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  constexpr int smem = UpdCfg<false, KB>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(upd_kernel<false, KB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(p.n_tiles, num_sms));
-  upd_kernel<false><<<grid, NTHREADS, smem, st>>>(p);
+  upd_kernel<false, KB><<<grid, NTHREADS, smem, st>>>(p);
   return cudaGetLastError();
+}
+
+int update_tokens_per_stage(int C) { return C % 128 == 0 ? 128 : 64; }
+
+cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st) {
+  if (p.n_tiles <= 0 || p.dchunks <= 0) return cudaSuccess;
+  return update_tokens_per_stage(p.C) == 128 ? launch_update_kb<128>(p, num_sms, st)
+                                             : launch_update_kb<64>(p, num_sms, st);
 }
 
 // ------------------------------------------------------------------ failure-path self test

@@ -43,6 +43,9 @@ cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st);
 // State update of chunks [p.chunk, p.chunk + p.dchunks) on p.n_tiles state tiles of
 // 128 x 256 (V pre-scaled by alpha eta); writes S_{c+1} snapshots and the fp32 state.
 cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st);
+// Tokens per pipeline stage of the state update for chunk length C: the V and Z
+// tensor maps (map[3], map[4]) carry boxes of that many rows.
+int update_tokens_per_stage(int C);
 cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st);
 int kind_gateup();
 int kind_vhat();
