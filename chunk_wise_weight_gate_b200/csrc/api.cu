@@ -10,6 +10,7 @@
 // §3 (a chunk's output always comes from the pre-update state).
 #include <cuda_runtime.h>
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -245,6 +246,12 @@ StreamState state_of(const ipttt_params& p, void* state) {
     if (e_ != cudaSuccess) return IPTTT_ERR_CUDA;       \
   } while (0)
 
+// Pair (cluster of two) GEMMs can be switched off with IPTTT_GEMM_CTAS=1.
+bool pair_gemms_enabled() {
+  const char* e = getenv("IPTTT_GEMM_CTAS");
+  return !(e && e[0] == '1');
+}
+
 ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, const Layout& L, StreamState* ss,
                       DeviceInfo* di, cudaStream_t st) {
   using namespace tck;
@@ -289,6 +296,11 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   tp.alpha = alpha;
   tp.status = di->status;
 
+  // Gate/up and target GEMMs on CTA pairs (256-row tiles) where the device runs
+  // clusters of two, else one CTA per 128-row tile.
+  const bool pair_gemm = pair_gemms_enabled() && pair_gemm_workers(st) > 0;
+  const int zv_fam = pair_gemm ? FAM_ZV2 : FAM_ZV;
+  const int zv_rows = pair_gemm ? 256 : 128;
   if (!t.Zin) {
     PhaseScope ph(st, PH_GATEUP);
     TcParams g = tp;
@@ -298,8 +310,8 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
         !make_map_bf16(&g.map[2], t.Wu, s.d, s.F, 1, 64, 128))
       return IPTTT_ERR_CUDA;
     g.out0 = Z;
-    g.n_tiles = s.B * ((s.T + 127) / 128) * (s.F / 128);
-    IP_CHECK(launch_tc(FAM_ZV, g, di->num_sms, st));
+    g.n_tiles = s.B * ((s.T + zv_rows - 1) / zv_rows) * (s.F / 128);
+    IP_CHECK(launch_tc(zv_fam, g, di->num_sms, st));
     counted(1);
   }
   if (!t.Zin) {
@@ -307,12 +319,12 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     TcParams v = tp;
     v.kind = kind_vhat();
     if (!make_map_bf16(&v.map[0], U, s.d, s.T, s.B, 64, 128) ||
-        !make_map_bf16(&v.map[1], t.Wt, s.d, s.d, 1, 64, 64))
+        !make_map_bf16(&v.map[1], t.Wt, s.d, s.d, 1, 64, pair_gemm ? 128 : 64))
       return IPTTT_ERR_CUDA;
     v.out0 = V;
     v.vn = s.d % 256 == 0 ? 256 : 128;
-    v.n_tiles = s.B * ((s.T + 127) / 128) * (s.d / v.vn);
-    IP_CHECK(launch_tc(FAM_ZV, v, di->num_sms, st));
+    v.n_tiles = s.B * ((s.T + zv_rows - 1) / zv_rows) * (s.d / v.vn);
+    IP_CHECK(launch_tc(zv_fam, v, di->num_sms, st));
     counted(1);
   }
   if (t.Zout) IP_CHECK(cudaMemcpyAsync(t.Zout, Z, (size_t)s.B * s.T * s.F * 2, cudaMemcpyDeviceToDevice, st));

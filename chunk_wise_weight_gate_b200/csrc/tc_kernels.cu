@@ -69,8 +69,16 @@ template <> struct Cfg<FAM_APPLY256> {
   static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 64, B_OFF = 2 * A_BYTES, EPI_BYTES = 0,
                        NBUF = 1;
 };
+// Pair gate/up and target: CTA r of the cluster holds A rows m0 + 128 r .. of the
+// 256-row tile and half of the N operand; 128 K per stage (two 64-wide boxes),
+// 8 pair MMAs per stage.
+template <> struct Cfg<FAM_ZV2> {
+  static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 128, B_OFF = 2 * A_BYTES, EPI_BYTES = 0,
+                       NBUF = 2;
+};
 template <int FAM> constexpr bool is_apply() { return FAM == FAM_APPLY || FAM == FAM_APPLY256; }
-template <int FAM> constexpr bool is_zv() { return FAM == FAM_ZV; }
+template <int FAM> constexpr bool is_zv() { return FAM == FAM_ZV || FAM == FAM_ZV2; }
+template <int FAM> constexpr bool is_pair() { return FAM == FAM_ZV2; }
 
 template <int FAM>
 constexpr int smem_bytes() {
@@ -191,6 +199,14 @@ template <int FAM>
 __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
   j.halves = 1;
   if constexpr (FAM == FAM_ZV) decode_zv<128>(p, tile, j);
+  else if constexpr (FAM == FAM_ZV2) {
+    // 256-row pair tile; each CTA moves its A half and its half of the N operand,
+    // 128 K per stage; the leader's barrier counts both CTAs' bytes.
+    decode_zv<256>(p, tile, j);
+    j.halves = 1;
+    j.kb1[0] = p.d / 128;
+    j.tx = 2 * (128 * 128 * 2 + (j.n_mma / 2) * 128 * 2);
+  }
   else if constexpr (FAM == FAM_GRAM) decode_gram(p, tile, j);
   else if constexpr (FAM == FAM_APPLY) decode_apply<0>(p, tile, j);
   else decode_apply<256>(p, tile, j);
@@ -199,7 +215,9 @@ __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
 // i-th tile of this block (static round-robin schedule), or -1 past the end.
 template <int FAM>
 __device__ __forceinline__ int seq_tile(const TcParams& p, uint32_t i) {
-  const long long t = (long long)blockIdx.x + (long long)i * gridDim.x;
+  const long long w = is_pair<FAM>() ? (long long)cluster_id_x() : (long long)blockIdx.x;
+  const long long nw = is_pair<FAM>() ? (long long)cluster_count_x() : (long long)gridDim.x;
+  const long long t = w + (long long)i * nw;
   return t < p.n_tiles ? (int)t : -1;
 }
 
@@ -208,7 +226,25 @@ template <int FAM>
 __device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int seg, int kb, uint8_t* sa,
                                             uint8_t* sb, uint64_t* bar) {
   const int kx = kb * BK;
-  if constexpr (is_zv<FAM>()) {
+  if constexpr (is_pair<FAM>()) {
+    // 128 K per stage: two 64-wide K boxes of this CTA's 128 A rows, then its half
+    // of the N operand (gate rows on CTA 0, up rows on CTA 1; or target columns).
+    const uint32_t r = cluster_rank();
+    const uint32_t fb = map_to_rank(smem_u32(bar), 0);
+    const int k0 = kb * 128;
+    const int arow = j.m0 + 128 * (int)r;
+    tma_load_3d_pair(sa, &p.map[0], fb, k0, arow, j.b);
+    tma_load_3d_pair(sa + A_BYTES, &p.map[0], fb, k0 + 64, arow, j.b);
+    if (j.kind == K_GATEUP) {
+      const CUtensorMap* wm = r == 0 ? &p.map[1] : &p.map[2];
+      tma_load_3d_pair(sb, wm, fb, k0, j.n0, 0);
+      tma_load_3d_pair(sb + 128 * BK * 2, wm, fb, k0 + 64, j.n0, 0);
+    } else {
+      const int nh = p.vn / 2;                                     // Wtarget[k][n], n contiguous
+      for (int q = 0; q < nh / 64; ++q)
+        tma_load_3d_pair(sb + q * 64 * 128 * 2, &p.map[1], fb, j.n0 + (int)r * nh + 64 * q, k0, 0);
+    }
+  } else if constexpr (is_zv<FAM>()) {
     if (j.kind == K_GATEUP) {
       tma_load_3d(sa, &p.map[0], bar, kx, j.m0, j.b);              // H rows
       if (j.halves == 2) tma_load_3d(sa + A_BYTES, &p.map[0], bar, kx, j.m0 + 128, j.b);
@@ -397,6 +433,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  constexpr bool PAIR = is_pair<FAM>();
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -405,7 +443,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], NUM_EPI_WARPS);
+      mbar_init(&acc_empty[a], NUM_EPI_WARPS * (PAIR ? 2 : 1));
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -417,11 +455,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     for (int i = 0; i < nmaps; ++i) prefetch_tmap(&p.map[i]);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * ACC_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, 2 * ACC_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, 2 * ACC_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -440,7 +483,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
             const uint32_t ph = (it / STAGES) & 1;
             if (!mbar_wait_or_abort(&empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
             uint8_t* sa = stages + s * STAGE_BYTES;
-            mbar_arrive_expect_tx(&full[s], j.tx);
+            if (!PAIR || rank == 0) mbar_arrive_expect_tx(&full[s], j.tx);
             issue_loads<FAM>(p, j, seg, kb, sa, sa + Cfg<FAM>::B_OFF, &full[s]);
           }
         }
@@ -449,7 +492,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
       counters[0] = it;
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       bool ready = mbar_try_wait(&full[0], 0);
@@ -460,10 +503,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
         decode<FAM>(p, tile, j);
         const int buf = Cfg<FAM>::NBUF == 2 ? (tcount & 1) : 0;
         const uint32_t aph = Cfg<FAM>::NBUF == 2 ? ((tcount >> 1) & 1) : (tcount & 1);
-        if (!mbar_wait_or_abort(&acc_empty[buf], aph ^ 1, abort_flag)) { ok = false; break; }
+        const bool got = PAIR ? mbar_wait_cluster(&acc_empty[buf], aph ^ 1)
+                              : mbar_wait_or_abort(&acc_empty[buf], aph ^ 1, abort_flag);
+        if (!got || (PAIR && *abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tacc = tmem_base + buf * ACC_COLS;
-        const uint32_t idesc = idesc_bf16(BM, j.n_mma, j.a_mn, j.b_mn);
+        const uint32_t idesc = idesc_bf16(PAIR ? 256 : BM, j.n_mma, j.a_mn, j.b_mn);
         for (int seg = 0; seg < j.nseg && ok; ++seg) {
           for (int kb = j.kb0[seg]; kb < j.kb1[seg]; ++kb, ++it) {
             const int s = it % STAGES;
@@ -477,25 +522,34 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
 #pragma unroll
             for (int ks = 0; ks < KB / 16; ++ks) {
               // MN-major: 16 K rows of 128 B per step, MN blocks KB rows apart.
+              // K-major: 32 B per step inside a 64-wide K box; boxes of 128 rows
+              // (16 KB) follow each other when a stage holds 128 K.
+              const uint32_t kofs = (ks / 4) * 16384 + (ks % 4) * 32;
               const uint64_t ad = j.a_mn ? sdesc_sw128(a_addr + ks * 2048, KB * 128, 1024)
-                                         : sdesc_sw128(a_addr + ks * 32, 16, 1024);
+                                         : sdesc_sw128(a_addr + kofs, 16, 1024);
               const uint64_t bd = j.b_mn ? sdesc_sw128(b_addr + ks * 2048, KB * 128, 1024)
-                                         : sdesc_sw128(b_addr + ks * 32, 16, 1024);
+                                         : sdesc_sw128(b_addr + kofs, 16, 1024);
               const uint32_t acc_flag = (kb > j.kb0[seg] || ks > 0) ? 1u : 0u;
+              if constexpr (PAIR) {
+                mma_bf16_pair(tacc + j.acc_col[seg], ad, bd, idesc, acc_flag);
+                continue;
+              }
               mma_bf16(tacc + j.acc_col[seg], ad, bd, idesc, acc_flag);
               if (j.halves == 2)  // rows 128..255 of A (K-major, 16 KB further), next 256 columns
                 mma_bf16(tacc + 256 + j.acc_col[seg], sdesc_sw128(a_addr + A_BYTES + ks * 32, 16, 1024), bd,
                          idesc, acc_flag);
             }
-            mma_commit(&empty[s]);
+            if constexpr (PAIR) mma_commit_pair(&empty[s], 3); else mma_commit(&empty[s]);
           }
         }
-        if (ok) mma_commit(&acc_full[buf]);
+        if (ok) {
+          if constexpr (PAIR) mma_commit_pair(&acc_full[buf], 3); else mma_commit(&acc_full[buf]);
+        }
       }
       if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
       counters[1] = it;
       // Let every MMA issued by this thread finish before TMEM is released.
-      mma_commit(drain);
+      if constexpr (PAIR) mma_commit_pair(drain, 1); else mma_commit(drain);
       mbar_wait(drain, 0);
     }
   } else {
@@ -505,6 +559,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     const int row = quarter * 32 + lane;
     uint32_t tcount = 0;
     bool ok = true;
+    const uint32_t empty0 = PAIR ? map_to_rank(smem_u32(acc_empty), 0) : 0u;  // the leader's acc_empty[0]
     for (uint32_t i = 0;; ++i, ++tcount) {
       const int tile = seq_tile<FAM>(p, i);
       if (tile < 0) break;
@@ -517,26 +572,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
       if (!mbar_wait(&acc_full[buf], aph)) { ok = false; break; }
       tc_fence_after();
       const uint32_t tacc = tmem_base + buf * ACC_COLS + ((uint32_t)(quarter * 32) << 16);
+      if constexpr (PAIR) j.m0 += 128 * (int)rank;  // this CTA's rows of the pair tile
       epilogue_tile<FAM>(p, j, tacc, half, row, lane, ew, red);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(empty0 + 8u * buf);
+        else mbar_arrive(&acc_empty[buf]);
+      }
     }
     if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
     if (lane == 0) bulk_wait<0>();
   }
 
   __syncthreads();
-  if (*abort_flag && threadIdx.x == 0) {
+  if (*abort_flag && threadIdx.x == 0 && rank == 0) {
     // Wait (bounded) for copies that were issued but never consumed, so no TMA
     // write lands in shared memory after the block has exited.
     for (uint32_t it = counters[1]; it < counters[0]; ++it)
       mbar_wait(&full[it % STAGES], (it / STAGES) & 1);
   }
-  __syncthreads();
+  tc_fence_before();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * ACC_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, 2 * ACC_COLS);
+    else tmem_dealloc(tmem_base, 2 * ACC_COLS);
   }
 }
 
@@ -1034,15 +1095,52 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ro
   return r == CUDA_SUCCESS;
 }
 
+static cudaLaunchConfig_t pair_config(int grid, int smem, cudaStream_t st, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(NTHREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+int pair_gemm_workers(cudaStream_t st) {
+  static int cached[64];
+  static bool have[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (have[dev]) return cached[dev];
+  int n = 0;
+  constexpr int smem = smem_bytes<FAM_ZV2>();
+  if (cudaFuncSetAttribute(tc_kernel<FAM_ZV2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pair_config(2, smem, st, attr);
+    if (cudaOccupancyMaxActiveClusters(&n, tc_kernel<FAM_ZV2>, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  cached[dev] = n;
+  have[dev] = true;
+  return n;
+}
+
 template <int FAM>
 static cudaError_t launch(const TcParams& p, int num_sms, cudaStream_t st) {
-  static bool attr_set[16] = {false};
-  const int dev_slot = 0;
-  (void)dev_slot;
   constexpr int smem = smem_bytes<FAM>();
   cudaError_t e = cudaFuncSetAttribute(tc_kernel<FAM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  (void)attr_set;
+  if constexpr (is_pair<FAM>()) {
+    const int np = pair_gemm_workers(st);
+    if (np <= 0) return cudaErrorInvalidConfiguration;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pair_config(2 * std::max(1, std::min(p.n_tiles, np)), smem, st, attr);
+    return cudaLaunchKernelEx(&cfg, tc_kernel<FAM>, p);
+  }
   const int grid = std::max(1, std::min(p.n_tiles, num_sms));
   tc_kernel<FAM><<<grid, NTHREADS, smem, st>>>(p);
   return cudaGetLastError();
@@ -1052,6 +1150,7 @@ cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st) 
   if (p.n_tiles <= 0) return cudaSuccess;
   switch (fam) {
     case FAM_ZV: return launch<FAM_ZV>(p, num_sms, st);
+    case FAM_ZV2: return launch<FAM_ZV2>(p, num_sms, st);
     case FAM_GRAM: return launch<FAM_GRAM>(p, num_sms, st);
     case FAM_APPLY256: return launch<FAM_APPLY256>(p, num_sms, st);
     default: return launch<FAM_APPLY>(p, num_sms, st);

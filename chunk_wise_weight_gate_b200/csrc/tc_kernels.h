@@ -9,7 +9,9 @@
 namespace ipttt {
 namespace tck {
 
-enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_APPLY256 = 5 };
+// FAM_ZV2: the gate/up and target GEMMs of FAM_ZV on CTA pairs (256-row tiles,
+// M=256 pair MMAs, 128 K per stage); launched as clusters of two.
+enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_APPLY256 = 5, FAM_ZV2 = 6 };
 
 struct TcParams {
   CUtensorMap map[6];
@@ -40,6 +42,9 @@ struct TcParams {
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
                    uint32_t box_inner, uint32_t box_rows);
 cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st);
+// Whether FAM_ZV2 can run on this device (a cluster of two fits), and the
+// number of CTA pairs resident at once.
+int pair_gemm_workers(cudaStream_t st);
 // State update of chunks [p.chunk, p.chunk + p.dchunks) on p.n_tiles state tiles of
 // 128 x 256 (V pre-scaled by alpha eta); writes S_{c+1} snapshots and the fp32 state.
 cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st);
