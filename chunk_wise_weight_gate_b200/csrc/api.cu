@@ -333,13 +333,21 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   {
     PhaseScope ph(st, PH_GRAM);
     TcParams g = tp;
-    if (!make_map_bf16(&g.map[0], Z, s.F, s.T, s.B, 64, tp.tr) ||
-        !make_map_bf16(&g.map[1], V, s.d, s.T, s.B, 64, tp.tr))
+    // On CTA pairs: 256 x 256 token-block pairs, two partials (one per CTA) each.
+    const bool gram2 = pair_gemm && s.C % 256 == 0;
+    if (gram2) {
+      g.tr = 256;
+      g.ct = s.C / 256;
+      g.npairs = g.ct * (g.ct + 1) / 2;
+    }
+    if (!make_map_bf16(&g.map[0], Z, s.F, s.T, s.B, 64, gram2 ? 128 : tp.tr) ||
+        !make_map_bf16(&g.map[1], V, s.d, s.T, s.B, 64, gram2 ? 128 : tp.tr))
       return IPTTT_ERR_CUDA;
     g.partials = partials;
-    g.n_tiles = s.B * s.k * tp.npairs;
-    IP_CHECK(launch_tc(FAM_GRAM, g, di->num_sms, st));
-    IP_CHECK(aux::alpha_from_partials(partials, alpha, s.B * s.k, tp.npairs, p.eta, tau, st));
+    g.n_tiles = s.B * s.k * g.npairs;
+    IP_CHECK(launch_tc(gram2 ? FAM_GRAM2 : FAM_GRAM, g, di->num_sms, st));
+    IP_CHECK(aux::alpha_from_partials(partials, alpha, s.B * s.k, gram2 ? 2 * g.npairs : tp.npairs, p.eta, tau,
+                                      st));
     // the state update accumulates alpha eta V^T Z: fold alpha eta into V's rows
     IP_CHECK(aux::prescale_target(V, alpha, s, p.eta, st));
     counted(3);

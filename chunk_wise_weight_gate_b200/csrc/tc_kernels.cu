@@ -76,9 +76,16 @@ template <> struct Cfg<FAM_ZV2> {
   static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 128, B_OFF = 2 * A_BYTES, EPI_BYTES = 0,
                        NBUF = 2;
 };
+// Pair Gram: the ZZ^T and VV^T accumulators of a 256 x 256 block pair take all of
+// TMEM (2 x 256 columns per CTA), so one accumulator set.
+template <> struct Cfg<FAM_GRAM2> {
+  static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 128, B_OFF = 2 * A_BYTES, EPI_BYTES = 0,
+                       NBUF = 1;
+};
 template <int FAM> constexpr bool is_apply() { return FAM == FAM_APPLY || FAM == FAM_APPLY256; }
 template <int FAM> constexpr bool is_zv() { return FAM == FAM_ZV || FAM == FAM_ZV2; }
-template <int FAM> constexpr bool is_pair() { return FAM == FAM_ZV2; }
+template <int FAM> constexpr bool is_pair() { return FAM == FAM_ZV2 || FAM == FAM_GRAM2; }
+template <int FAM> constexpr bool is_gram() { return FAM == FAM_GRAM || FAM == FAM_GRAM2; }
 
 template <int FAM>
 constexpr int smem_bytes() {
@@ -208,6 +215,15 @@ __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
     j.tx = 2 * (128 * 128 * 2 + (j.n_mma / 2) * 128 * 2);
   }
   else if constexpr (FAM == FAM_GRAM) decode_gram(p, tile, j);
+  else if constexpr (FAM == FAM_GRAM2) {
+    // p.tr = 256, p.ct = C / 256, p.npairs = ct (ct + 1) / 2; 128 K per stage
+    decode_gram(p, tile, j);
+    j.kb1[0] = p.F / 128;
+    j.kb1[1] = p.d / 128;
+    j.acc_col[1] = 256;
+    j.n_mma = 256;
+    j.tx = 2 * (2 * 128 * 128 * 2);
+  }
   else if constexpr (FAM == FAM_APPLY) decode_apply<0>(p, tile, j);
   else decode_apply<256>(p, tile, j);
 }
@@ -232,10 +248,15 @@ __device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int
     const uint32_t r = cluster_rank();
     const uint32_t fb = map_to_rank(smem_u32(bar), 0);
     const int k0 = kb * 128;
-    const int arow = j.m0 + 128 * (int)r;
-    tma_load_3d_pair(sa, &p.map[0], fb, k0, arow, j.b);
-    tma_load_3d_pair(sa + A_BYTES, &p.map[0], fb, k0 + 64, arow, j.b);
-    if (j.kind == K_GATEUP) {
+    const int arow = (is_gram<FAM>() ? j.t0 : 0) + j.m0 + 128 * (int)r;
+    const CUtensorMap* am = is_gram<FAM>() && seg == 1 ? &p.map[1] : &p.map[0];   // Gram: Z, then V
+    tma_load_3d_pair(sa, am, fb, k0, arow, j.b);
+    tma_load_3d_pair(sa + A_BYTES, am, fb, k0 + 64, arow, j.b);
+    if constexpr (is_gram<FAM>()) {                                 // rows of the other token block
+      const int brow = j.t0 + j.n0 + 128 * (int)r;
+      tma_load_3d_pair(sb, am, fb, k0, brow, j.b);
+      tma_load_3d_pair(sb + 128 * BK * 2, am, fb, k0 + 64, brow, j.b);
+    } else if (j.kind == K_GATEUP) {
       const CUtensorMap* wm = r == 0 ? &p.map[1] : &p.map[2];
       tma_load_3d_pair(sb, wm, fb, k0, j.n0, 0);
       tma_load_3d_pair(sb + 128 * BK * 2, wm, fb, k0 + 64, j.n0, 0);
@@ -331,6 +352,30 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
         if (valid) st_bf16x32(vrow + c, v);
       }
     }
+  } else if constexpr (FAM == FAM_GRAM2) {
+    // This CTA's 128 rows of the 256 x 256 block pair; warp half h sums columns
+    // [128 h, 128 h + 128) of (Z Z^T) * (V V^T).  Diagonal pairs count once, the
+    // others twice (the mirrored pair is not computed).
+    float s = 0.0f;
+#pragma unroll 1
+    for (int c = half * 128; c < half * 128 + 128; c += 32) {
+      tmem_ld32(tacc + c, r0);
+      tmem_ld32(tacc + 256 + c, r1);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s = fmaf(__uint_as_float(r0[i]), __uint_as_float(r1[i]), s);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) red[ew] = s;
+    epi_sync();
+    if (ew == 0 && lane == 0) {
+      float tot = 0.0f;
+      for (int w = 0; w < NUM_EPI_WARPS; ++w) tot += red[w];
+      const float wgt = (j.m0 / 256) == (j.n0 / 256) ? 1.0f : 2.0f;
+      p.partials[(((size_t)j.b * p.k + j.chunk) * p.npairs + j.pair) * 2 + cluster_rank()] = wgt * tot;
+    }
+    epi_sync();
   } else if constexpr (FAM == FAM_GRAM) {
     // Only rows and columns below tr hold Gram entries of this tile pair.
     float s = 0.0f;
@@ -451,7 +496,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    const int nmaps = is_apply<FAM>() ? 3 : (FAM == FAM_GRAM ? 2 : (p.kind == K_GATEUP ? 3 : 2));
+    const int nmaps = is_apply<FAM>() ? 3 : (is_gram<FAM>() ? 2 : (p.kind == K_GATEUP ? 3 : 2));
     for (int i = 0; i < nmaps; ++i) prefetch_tmap(&p.map[i]);
   }
   if (warp == 1) {
@@ -1151,6 +1196,7 @@ cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st) 
   switch (fam) {
     case FAM_ZV: return launch<FAM_ZV>(p, num_sms, st);
     case FAM_ZV2: return launch<FAM_ZV2>(p, num_sms, st);
+    case FAM_GRAM2: return launch<FAM_GRAM2>(p, num_sms, st);
     case FAM_GRAM: return launch<FAM_GRAM>(p, num_sms, st);
     case FAM_APPLY256: return launch<FAM_APPLY256>(p, num_sms, st);
     default: return launch<FAM_APPLY>(p, num_sms, st);

@@ -11,7 +11,9 @@ namespace tck {
 
 // FAM_ZV2: the gate/up and target GEMMs of FAM_ZV on CTA pairs (256-row tiles,
 // M=256 pair MMAs, 128 K per stage); launched as clusters of two.
-enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_APPLY256 = 5, FAM_ZV2 = 6 };
+// FAM_GRAM2: the Gram pass on 256 x 256 token-block pairs, one cluster of two per
+// block pair; each CTA writes its own partial (2 per pair, npairs = pairs per chunk).
+enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_APPLY256 = 5, FAM_ZV2 = 6, FAM_GRAM2 = 8 };
 
 struct TcParams {
   CUtensorMap map[6];
