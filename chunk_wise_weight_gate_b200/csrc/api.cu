@@ -547,6 +547,9 @@ ipttt_status run(const ipttt_params* pp, const Tensors& t, void* workspace, size
 }
 
 }  // namespace
+
+ipttt_status validate_params(const ipttt_params* p) { return check_params(p); }
+
 }  // namespace ipttt
 
 using namespace ipttt;

@@ -10,6 +10,9 @@
 
 namespace ipttt {
 
+// The argument checks every entry point runs first (IPTTT_OK or the error code).
+ipttt_status validate_params(const ipttt_params* p);
+
 // Kernels report errors they cannot return (bad doc_starts, a bounded wait that
 // gave up) by setting a per-device status word, passed to them as a pointer; the
 // first error wins.  ipttt_get_status reads and clears it.

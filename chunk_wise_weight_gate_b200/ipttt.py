@@ -24,7 +24,8 @@ STATUS = {0: "IPTTT_OK", 1: "IPTTT_ERR_ARG", 2: "IPTTT_ERR_SHAPE", 3: "IPTTT_ERR
 EXPORTS = ("ipttt_workspace_size", "ipttt_forward", "ipttt_forward_ex", "ipttt_core", "ipttt_stream_state_size",
            "ipttt_stream_reset", "ipttt_stream_forward", "ipttt_stream_export", "ipttt_get_status",
            "ipttt_strerror", "ipttt_version", "ipttt_profile_enable", "ipttt_profile_read",
-           "ipttt_kernel_launches", "ipttt_selftest_wait_timeout", "ipttt_forward_noalloc")
+           "ipttt_kernel_launches", "ipttt_selftest_wait_timeout", "ipttt_forward_noalloc",
+           "ipttt_forward_host_size", "ipttt_forward_host")
 PHASES = ("prep", "gate_up", "target", "gram", "apply", "update")
 DEBUG_OUTPUTS = ("D", "S_final", "alpha", "Z", "V")
 
@@ -88,6 +89,10 @@ def lib() -> ctypes.CDLL:
         L.ipttt_selftest_wait_timeout.restype = ctypes.c_int
         L.ipttt_forward_noalloc.argtypes = [P] + [vp] * 7 + [vp, i32, vp, vp]
         L.ipttt_forward_noalloc.restype = ctypes.c_int
+        L.ipttt_forward_host_size.argtypes = [P, i32, i32]
+        L.ipttt_forward_host_size.restype = sz
+        L.ipttt_forward_host.argtypes = [P] + [vp] * 7 + [vp, i32, vp, vp, sz, i32, vp]
+        L.ipttt_forward_host.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -229,6 +234,54 @@ def core(cfg: LayerConfig, Z, V, Wdown0, doc_starts=None, *, workspace=None, str
                             out["alpha"].data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)),
            "ipttt_core")
     return out
+
+
+def forward_host_size(cfg: LayerConfig, piece_tokens: int = 0, n_doc_starts: int = 0) -> int:
+    """Device bytes ipttt_forward_host needs (0 for an invalid piece length)."""
+    return int(lib().ipttt_forward_host_size(ctypes.byref(cfg.params()), piece_tokens, n_doc_starts))
+
+
+def _host_ptr(t: torch.Tensor, dtype, name: str) -> int:
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def forward_host(cfg: LayerConfig, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_starts=None, *, O=None,
+                 piece_tokens: int = 0, buffer=None, stream=None):
+    """One layer forward with H, X0 and O in host memory (page-locked tensors let
+    the copies overlap the compute) and the weights on the device; the sequence is
+    pipelined through the streaming path in pieces of piece_tokens tokens (0: about
+    T/8).  Returns O, a host tensor that is complete once `stream` has finished."""
+    dt = cfg.torch_dtype
+    for name, t in (("H", H), ("X0", X0)):
+        if tuple(t.shape) != (cfg.B, cfg.T, cfg.d):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {(cfg.B, cfg.T, cfg.d)}")
+    _shape_check(cfg, Wgate=Wgate, Wup=Wup, Wdown0=Wdown0, conv_w=conv_w, Wtarget=Wtarget)
+    dev = Wgate.device
+    if O is None:
+        O = torch.empty(cfg.B, cfg.T, cfg.d, dtype=dt, pin_memory=H.is_pinned())
+    ds = None
+    if doc_starts is not None:
+        ds = doc_starts if isinstance(doc_starts, torch.Tensor) else torch.as_tensor(doc_starts, dtype=torch.int32)
+        ds = ds.to(device="cpu", dtype=torch.int32).contiguous()
+    nd = 0 if ds is None else ds.numel()
+    need = forward_host_size(cfg, piece_tokens, nd)
+    if need == 0:
+        raise ValueError(f"invalid piece length {piece_tokens} for chunk {cfg.C}")
+    if buffer is None:
+        buffer = torch.empty(need, dtype=torch.uint8, device=dev)
+    p = cfg.params()
+    _check(lib().ipttt_forward_host(ctypes.byref(p), _host_ptr(H, dt, "H"), _host_ptr(X0, dt, "X0"),
+                                    _ptr(Wgate, dt, "Wgate"), _ptr(Wup, dt, "Wup"), _ptr(Wdown0, dt, "Wdown0"),
+                                    _ptr(conv_w, dt, "conv_w"), _ptr(Wtarget, dt, "Wtarget"),
+                                    ds.data_ptr() if nd else None, nd, _host_ptr(O, dt, "O"), buffer.data_ptr(),
+                                    buffer.numel(), piece_tokens, _stream(stream)), "ipttt_forward_host")
+    return O
 
 
 class StreamState:

@@ -206,6 +206,33 @@ IPTTT_API ipttt_status ipttt_forward_noalloc(const ipttt_params* p,
  * ipttt_get_status); the context stays usable.  Meant for tests. */
 IPTTT_API ipttt_status ipttt_selftest_wait_timeout(uint32_t limit_ns, void* stream);
 
+/* Host-buffer forward.  Same result as ipttt_forward, but H, X0 and O are HOST
+ * arrays [B, T, d] (page-locked memory lets the copies overlap the compute; with
+ * pageable memory the result is the same, only slower) and doc_starts is a HOST
+ * int32 array with the meaning given above.  The weights are device pointers.
+ * The pages have no counterpart: this is the way to feed a sequence that sits in
+ * host memory without waiting for the whole of it to be copied first.
+ *
+ * The sequence runs through ipttt_stream_reset / ipttt_stream_forward in pieces of
+ * piece_tokens tokens of every row (a multiple of C; 0 picks about T/8 in whole
+ * chunks): while piece i computes on `stream`, piece i+1 is copied in and piece
+ * i-1 copied out on two streams the call creates and releases.  device_buffer is
+ * caller-owned device memory, 256-byte aligned, of ipttt_forward_host_size(p,
+ * piece_tokens, n_doc_starts) bytes (two device copies of a piece of H, X0 and O,
+ * the pieces' document starts, the streaming state and a workspace); the call
+ * allocates no device memory.  Document starts are checked on the host (out of
+ * range or out of order: IPTTT_ERR_ARG, nothing launched).  The call returns once
+ * everything is queued; later work on `stream` sees O complete.  H, X0, O and
+ * device_buffer must stay untouched until then; doc_starts may be released when
+ * the call returns. */
+IPTTT_API size_t ipttt_forward_host_size(const ipttt_params* p, int32_t piece_tokens, int32_t n_doc_starts);
+IPTTT_API ipttt_status ipttt_forward_host(const ipttt_params* p, const void* H_host, const void* X0_host,
+                                          const void* Wgate, const void* Wup, const void* Wdown0,
+                                          const void* conv_w, const void* Wtarget,
+                                          const int32_t* doc_starts_host, int32_t n_doc_starts,
+                                          void* O_host, void* device_buffer, size_t device_bytes,
+                                          int32_t piece_tokens, void* stream);
+
 /* Library version, "major.minor.patch". */
 IPTTT_API const char* ipttt_version(void);
 

@@ -87,3 +87,25 @@ def test_fp32_path_accepts_any_shape():
     L = ip.lib()
     p = params(dtype=ip.F32, d=67, F=131, C=7, T=50)
     assert L.ipttt_workspace_size(ctypes.byref(p)) > 0
+
+
+def test_forward_host_size_and_argument_errors():
+    L = ip.lib()
+    p = params(B=2, T=777)
+    size = L.ipttt_forward_host_size(ctypes.byref(p), 256, 3)
+    assert size > 0 and size % 256 == 0
+    assert L.ipttt_forward_host_size(ctypes.byref(p), 100, 3) == 0           # piece not a multiple of C
+    assert L.ipttt_forward_host_size(ctypes.byref(params(C=96)), 0, 0) == 0  # unsupported shape
+    fake = [0x10000 + 256 * i for i in range(5)]
+    host = ctypes.create_string_buffer(16)
+    buf = 0x100000
+    # null host buffers, a bad piece length, an unsupported shape, a short device buffer
+    assert L.ipttt_forward_host(ctypes.byref(p), None, None, *fake, None, 0, None, buf, size, 256, None) == 1
+    assert L.ipttt_forward_host(ctypes.byref(p), host, host, *fake, None, 0, host, buf, size, 100, None) == 1
+    assert L.ipttt_forward_host(ctypes.byref(params(C=96)), host, host, *fake, None, 0, host, buf, size, 0,
+                                None) == 5
+    assert L.ipttt_forward_host(ctypes.byref(p), host, host, *fake, None, 0, host, buf, size - 256, 256,
+                                None) == 8
+    # document starts are checked on the host: out of order
+    docs = (ctypes.c_int32 * 2)(300, 200)
+    assert L.ipttt_forward_host(ctypes.byref(p), host, host, *fake, docs, 2, host, buf, size, 256, None) == 1
