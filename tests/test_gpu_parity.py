@@ -76,6 +76,8 @@ BF16_CASES = {
     "chunk64_docs_ragged": dict(B=2, T=700, C=64, d=256, F=384, eta=2e-2, clip=0.0,
                                 docs=[70, 200, 201, 700 + 64, 700 + 450]),
     "chunk192_clip": dict(B=1, T=1000, C=192, d=128, F=256, eta=1e-3, clip=1e-5),
+    "chunk256_docs_ragged": dict(B=2, T=1000, C=256, d=256, F=512, eta=2e-2, clip=0.0,
+                                 docs=[100, 300, 301, 1000 + 256, 1000 + 700]),
 }
 
 
