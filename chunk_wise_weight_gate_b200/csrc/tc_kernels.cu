@@ -683,7 +683,7 @@ static_assert(UpdCfg<false, 64>::SMEM <= 232448 && UpdCfg<true, 64>::SMEM <= 232
               "update kernel exceeds shared memory");
 
 struct UpdJob {
-  int X;      // state tile: (b, mt, nt2) of B x (d/TILE_ROWS) x ceil(F/256)
+  int X;      // state tile: (b, nt2, mt) of B x ceil(F/256) x (d/TILE_ROWS), mt fastest
   int chunk;  // absolute chunk index
   int slot;   // TMEM slot 0 or 1
   int b, m0, n0;
@@ -716,12 +716,16 @@ __device__ __forceinline__ bool upd_job(const TcParams& p, uint32_t i, int w, in
   jb.X = w + (2 * m + sl) * nw;
   jb.chunk = p.chunk + c;
   jb.slot = sl;
+  // Row blocks vary fastest: the tiles in flight at one time (about two per
+  // worker) then cover few column blocks, so each chunk's Z columns come from DRAM
+  // about once (V, four times smaller, once per tile group).
   const int nt2s = (p.F + 255) / 256;
-  const int per_row = (p.d / (PAIR ? 256 : 128)) * nt2s;
+  const int mts = p.d / (PAIR ? 256 : 128);
+  const int per_row = mts * nt2s;
   jb.b = jb.X / per_row;
   const int r = jb.X % per_row;
-  jb.m0 = (r / nt2s) * (PAIR ? 256 : 128);
-  jb.n0 = (r % nt2s) * 256;
+  jb.m0 = (r % mts) * (PAIR ? 256 : 128);
+  jb.n0 = (r / mts) * 256;
   return true;
 }
 
