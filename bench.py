@@ -172,6 +172,12 @@ def config_dict(w: synth.Workload, n: int) -> dict:
             "l2": "inputs larger than L2 (H and X0 are B*T*d bf16; Z is B*T*F bf16)"}
 
 
+# DRAM bytes (read + written) per launch of a kernel, measured by one ncu capture of
+# that launch on the named workload (profiles/apply_traffic_qwen3_4b_128k.md).  The
+# roofline object carries it only for the kernel and workload it was taken on.
+MEASURED_TRAFFIC = {("qwen3_4b_128k", "apply"): 2.21e9 + 81.19e6}
+
+
 def sample_chunks(w: synth.Workload, tokens: int) -> int:
     """Whole chunks of row 0 covering at least `tokens` tokens (at least one chunk)."""
     k = (w.T + w.C - 1) // w.C
@@ -300,7 +306,8 @@ def run_ours(args, w: synth.Workload):
         achieved = total / (dom_ms / 1000.0) / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "launches": dom_launches,
+                "frac": achieved / peak, "traffic": MEASURED_TRAFFIC.get((w.name, dom)), "traffic_unit": "bytes",
+                "launches": dom_launches,
                 "avg_launch_ms": dom_ms / max(1, dom_launches),
                 "peak_note": f"sustained bf16 ({peak_src}); burst {peaks['bf16_tflops']}"}
     phase_report = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
