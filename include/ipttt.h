@@ -44,7 +44,10 @@
  *  - dtype IPTTT_F32 runs an all-fp32 path (SIMT FMA) for any shape.  dtype
  *    IPTTT_BF16 runs the tensor-core path (tcgen05, fp32 accumulation, fp32 fast
  *    weight state) and needs d % 128 == 0, F % 128 == 0, C % 64 == 0; other shapes
- *    return IPTTT_ERR_UNSUPPORTED.
+ *    return IPTTT_ERR_UNSUPPORTED.  Where the device runs clusters of two CTAs, the
+ *    gate/up and target GEMMs, the Gram pass (C % 256 == 0) and the state update
+ *    (d % 256 == 0) run on CTA pairs; the environment variables IPTTT_GEMM_CTAS=1
+ *    and IPTTT_UPDATE_CTAS=1 select the single-CTA kernels instead.
  */
 #ifndef IPTTT_H_
 #define IPTTT_H_

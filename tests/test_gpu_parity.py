@@ -101,8 +101,9 @@ def test_bf16_eta_zero_is_plain_gated_mlp():
     assert maxrel(to_np(out["O"]), ref["O"]) <= TOL_O_BF16
 
 
-def test_bf16_deterministic():
-    cfg, inp = case(2, 640, 128, 256, 512, docs=[200, 640 + 333])
+@pytest.mark.parametrize("C", [128, 256])
+def test_bf16_deterministic(C):
+    cfg, inp = case(2, 640, C, 256, 512, docs=[200, 640 + 333])
     a = gpu(cfg, inp)
     b = gpu(cfg, inp)
     for key in ("O", "D", "S_final", "alpha", "Z", "V"):
