@@ -122,9 +122,14 @@ struct Layout {
   int group;  // bf16 path: chunks whose apply tiles share one launch (= snapshot ring slots)
 };
 
-// Apply tiles of `group` consecutive chunks share one launch, so that one launch
-// holds about kApplyTilesPerLaunch tiles (several even waves over the SMs).
+// Apply tiles of `group` consecutive chunks share one launch (and the snapshot
+// ring has `group` slots).  A launch holds at least kApplyTilesPerLaunch tiles;
+// beyond that the group is the smallest one that minimises the apply's waves over
+// kWaveCtas CTAs (the SMs of a B200) summed over all launches, within a ring of
+// at most kRingBytesMax.
 constexpr int kApplyTilesPerLaunch = 1280;
+constexpr int kWaveCtas = 148;
+constexpr size_t kRingBytesMax = size_t(8) << 30;
 
 // Token rows of an apply or Gram tile: 128, or 64 for chunks that are odd
 // multiples of 64 (the MMA still spans 128 rows; the upper 64 are not used).
@@ -135,12 +140,26 @@ int tile_rows(const ipttt_params& p) { return p.C % 128 == 0 ? 128 : 64; }
 int apply_rows(const ipttt_params& p) { return p.C % 256 == 0 ? 256 : tile_rows(p); }
 
 int apply_group(const ipttt_params& p) {
-  const int k = (p.T + p.C - 1) / p.C;
+  const long long k = (p.T + p.C - 1) / p.C;
   const long long per_chunk = (long long)p.B * (p.C / apply_rows(p)) * (p.d / 128);
-  long long g = (kApplyTilesPerLaunch + per_chunk - 1) / per_chunk;
-  if (g < 1) g = 1;
-  if (g > k) g = k;
-  return (int)g;
+  const long long slot_bytes = (long long)p.B * p.d * p.F * 2;
+  auto waves = [&](long long g) {
+    const long long full = k / g, rest = k % g;
+    return full * ((g * per_chunk + kWaveCtas - 1) / kWaveCtas) +
+           (rest ? (rest * per_chunk + kWaveCtas - 1) / kWaveCtas : 0);
+  };
+  long long gmin = (kApplyTilesPerLaunch + per_chunk - 1) / per_chunk;
+  gmin = std::max(1LL, std::min(gmin, k));
+  const long long gmax = std::max(gmin, std::min(k, (long long)(kRingBytesMax / std::max(1LL, slot_bytes))));
+  long long best = gmin, best_waves = waves(gmin);
+  for (long long g = gmin + 1; g <= gmax; ++g) {
+    const long long w = waves(g);
+    if (w < best_waves) {
+      best = g;
+      best_waves = w;
+    }
+  }
+  return (int)best;
 }
 
 bool is_bf16(const ipttt_params& p) { return p.dtype == IPTTT_BF16; }
