@@ -172,10 +172,10 @@ def config_dict(w: synth.Workload, n: int) -> dict:
             "l2": "inputs larger than L2 (H and X0 are B*T*d bf16; Z is B*T*F bf16)"}
 
 
-# DRAM bytes (read + written) per launch of a kernel, measured by one ncu capture of
-# that launch on the named workload (profiles/apply_traffic_qwen3_4b_128k.md).  The
+# DRAM bytes (read + written) per launch of a kernel, the mean over the launches of
+# one step captured by ncu on the named workload (profiles/apply_traffic_qwen3_4b_128k.md).  The
 # roofline object carries it only for the kernel and workload it was taken on.
-MEASURED_TRAFFIC = {("qwen3_4b_128k", "apply"): 2.21e9 + 81.19e6}
+MEASURED_TRAFFIC = {("qwen3_4b_128k", "apply"): 2.577e9 + 104.45e6}
 
 
 def sample_chunks(w: synth.Workload, tokens: int) -> int:
