@@ -413,9 +413,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     TcParams q = sc;
     q.chunk = c0;
     q.dchunks = c1 - c0;
-    q.write_snap = 1;
     q.apply_chunk0 = 0;
-    q.n_apply = 0;
     q.n_tiles = state_tiles;
     IP_CHECK(launch_update(q, di->num_sms, st));
     counted(1);
@@ -431,10 +429,8 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     TcParams q = sc;
     q.chunk = 0;
     q.dchunks = 1;
-    q.write_snap = 0;
     q.apply_chunk0 = a;
-    q.n_apply = (b - a) * apply_tiles_per_chunk;
-    q.n_tiles = q.n_apply;
+    q.n_tiles = (b - a) * apply_tiles_per_chunk;
     IP_CHECK(launch_tc(apply_fam, q, di->num_sms, st));
     counted(1);
   }

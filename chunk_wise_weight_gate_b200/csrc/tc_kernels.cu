@@ -1,30 +1,35 @@
 // Tensor-core (tcgen05) kernels of the bf16 path of the In-Place TTT MLP layer.
 //
-// One persistent, warp-specialised kernel template serves every contraction of
-// the layer.  Per CTA (one per SM): warp 0 issues TMA loads into a ring of
-// shared-memory stages, warp 1 allocates TMEM and one thread of it issues
-// tcgen05.mma into a double-buffered fp32 accumulator (2 x 256 TMEM columns),
+// One persistent, warp-specialised kernel template serves the GEMMs of the layer.
+// Per CTA: warp 0 issues TMA loads into a ring of shared-memory stages, warp 1
+// allocates TMEM and one thread of it issues tcgen05.mma into fp32 accumulators,
 // and 8 epilogue warps drain finished accumulators with tcgen05.ld.  Tiles are
-// handed out statically: tile = blockIdx.x + j * gridDim.x, and every role
-// decodes the same tile index into the same Job.
+// handed out statically (tile = worker + j * workers, a worker being a CTA or a
+// cluster of two) and every role decodes the same tile index into the same Job.
+// The pair families run as clusters of two CTAs: the even CTA issues M=256
+// tcgen05.mma.cta_group::2, each CTA loads its 128 A rows and half of the N
+// operand into its own shared memory (completion counted on the even CTA's
+// barrier), MMA completions are multicast to both CTAs' barriers, and both CTAs'
+// epilogues release the accumulator on the even CTA's barrier.
 //
 // Families (template parameter FAM):
-//   FAM_ZV   gate/up GEMM with the SiLU-product epilogue, Z = SiLU(H Wg^T) * (H Wu^T)
-//            [notes "In-Place Test-Time Training", 方法 › 原地自适应], and the
-//            target GEMM V = U Wtarget with rows outside each chunk's last document
-//            segment zeroed [notes, 对齐语言模型的目标函数].
-//   FAM_GRAM per-chunk Gram pass: ||V_L^T Z_L||_F^2 = sum_{s,t}(V V^T)_{st}(Z Z^T)_{st},
-//            written as deterministic partial sums per 128x128 tile pair; the clip
-//            factor follows [cloud.tencent.com "榨干MLP的剩余价值", 详细步骤 4].
-//   FAM_APPLY apply tiles of a group of chunks: O_i = Z_i W0^T + M_i (Z_i S_i^T), both
-//            products side by side in one N=256 accumulator, S_i read from a bf16
-//            snapshot [notes, 步骤一 and 工程实现; iplexlaw.co.kr review §3: a chunk's output
-//            comes from the pre-update state].
+//   FAM_ZV / FAM_ZV2 (pairs)  gate/up GEMM with the SiLU-product epilogue,
+//            Z = SiLU(H Wg^T) * (H Wu^T) [notes "In-Place Test-Time Training",
+//            方法 › 原地自适应], and the target GEMM V = U Wtarget with rows outside
+//            each chunk's last document segment zeroed [notes, 对齐语言模型的目标函数].
+//   FAM_GRAM / FAM_GRAM2 (pairs)  per-chunk Gram pass:
+//            ||V_L^T Z_L||_F^2 = sum_{s,t}(V V^T)_{st}(Z Z^T)_{st}, written as
+//            deterministic partial sums per tile pair; the clip factor follows
+//            [cloud.tencent.com "榨干MLP的剩余价值", 详细步骤 4].
+//   FAM_APPLY / FAM_APPLY256  apply tiles of a group of chunks:
+//            O_i = Z_i W0^T + M_i (Z_i S_i^T), both products side by side in one
+//            N=256 accumulator, S_i read from a bf16 snapshot [notes, 步骤一 and
+//            工程实现; iplexlaw.co.kr review §3: a chunk's output comes from the
+//            pre-update state].
 // The state update S_{i+1} = keep_i S_i + alpha_i eta V_i^T Z_i runs in its own
-// kernel (upd_kernel, below): each block keeps two 128 x 256 fp32 state tiles in
-// TMEM as live accumulators and walks them through a group of chunks [notes,
-// 步骤二 and the Hebbian rule; iplexlaw.co.kr review §6 exclusive scan and document
-// reset].
+// kernel (upd_kernel, below): each worker keeps two fp32 state tiles in TMEM as
+// live accumulators and walks them through a group of chunks [notes, 步骤二 and the
+// Hebbian rule; iplexlaw.co.kr review §6 exclusive scan and document reset].
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -48,7 +53,7 @@ constexpr int NTHREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr int ACC_COLS = 256;           // per accumulator buffer
 constexpr int SNAP_BOX_BYTES = 32 * 128;     // 32 rows x 64 bf16 columns (one warp's snapshot box)
 
-enum Kind { K_GATEUP = 0, K_VHAT = 1, K_GRAM = 2, K_APPLY = 3, K_DELTA = 4 };
+enum Kind { K_GATEUP = 0, K_VHAT = 1, K_GRAM = 2, K_APPLY = 3 };
 
 // Per family: pipeline stages, bytes per stage, K elements per stage (KB), offset
 // of the B operand inside a stage, and shared memory for the epilogue.
@@ -98,7 +103,7 @@ struct Job {
   int kind;
   int b;
   int m0, n0;     // tile origin: rows / columns of the accumulator in the operand index spaces
-  int t0;         // first token of the tile's chunk (GRAM, SCAN)
+  int t0;         // first token of the tile's chunk (Gram, apply)
   int chunk;
   int pair;       // GRAM: tile pair index
   int nseg;

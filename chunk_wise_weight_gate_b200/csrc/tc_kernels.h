@@ -25,18 +25,16 @@ struct TcParams {
   int npairs;        // GRAM: tile pairs per chunk, ct (ct + 1) / 2
   int chunk;         // update: first chunk whose state update the launch performs
   int dchunks;       // update: consecutive chunks per launch
-  int apply_chunk0;  // SCAN: first chunk of the apply tiles
-  int n_apply;       // SCAN: apply tiles (chunks apply_chunk0.., all rows); delta tiles follow
+  int apply_chunk0;  // apply: first chunk of the launch's tiles
   int n_tiles;
-  int write_snap;    // SCAN: delta tiles store the bf16 snapshot of S_{chunk+1}
-  int nslots;        // SCAN: snapshot ring slots; S_i lives in slot i % nslots
+  int nslots;        // apply, update: snapshot ring slots; S_i lives in slot i % nslots
   float eta;
   const ChunkMeta* meta;  // [B][k]
   const float* alpha;     // [B][k]
   float* partials;        // GRAM output [B][k][npairs]
-  void* out0;             // Z (gate/up), V (target), O (scan)
-  float* out1;            // SCAN: optional fp32 D
-  const void* resid;      // SCAN: optional residual H added to O
+  void* out0;             // Z (gate/up), V (target), O (apply)
+  float* out1;            // apply: optional fp32 D
+  const void* resid;      // apply: optional residual H added to O
   float* S;               // update: fp32 state, blocked 128 x 128 tiles
   int* status;            // device status word
 };
