@@ -367,6 +367,9 @@ def run_ours(args, w: synth.Workload):
                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w, world),
                "tflops": tflops, "frac_of_peak": tflops / world / peaks.get("bf16_tflops_sustained", 1.0),
+               "flops_per_token": ip.flops_per_token(w.d, w.F),
+               # the count for exact arithmetic, where W0 + S_i would be one operand: 8dF + 2d^2
+               "tflops_exact_arith_count": tflops * (8 * w.d * w.F + 2 * w.d * w.d) / ip.flops_per_token(w.d, w.F),
                "frac_of_burst_peak": tflops / world / peaks["bf16_tflops"], "peak_source": peak_src,
                "roofline": roof, "phases": phase_report, "clocks": clocks, "e2e": e2e,
                "gpu_launches": launches, "cpu_baseline": cpu, "device_status": status}
