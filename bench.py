@@ -379,6 +379,69 @@ def run_ours(args, w: synth.Workload):
         pg.destroy_process_group()
 
 
+def run_decode(args, w: synth.Workload):
+    """Token-by-token decoding of --decode-batch rows at the workload's d, F and C:
+    --steps chunks of C tokens after --warmup chunks, each chunk's commit included.
+    The per-token kernels read Wgate, Wup, Wdown0 and every row's bf16 state copy;
+    their roofline is HBM bandwidth."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B = args.decode_batch
+    wd = w.replace(B=B, T=w.C)
+    inp = synth.make_inputs(wd, seed=rank)
+    cfg = ip.LayerConfig(B=B, T=1, d=w.d, F=w.F, C=w.C, eta=w.eta, clip=w.clip)
+    wts = [inp[k].to(dev) for k in WEIGHTS]
+    H = inp["H"].to(dev)      # [B, C, d]: one chunk of tokens, reused every chunk
+    X0 = inp["X0"].to(dev)
+    hs = [H[:, t].contiguous() for t in range(w.C)]
+    xs = [X0[:, t].contiguous() for t in range(w.C)]
+    o = torch.empty(B, w.d, dtype=torch.bfloat16, device=dev)
+    st = ip.DecodeState(cfg, dev)
+    stream = torch.cuda.current_stream()
+
+    def chunk():
+        for t in range(w.C):
+            st.step(hs[t], xs[t], *wts, None, o=o)
+
+    for _ in range(max(1, args.warmup)):
+        chunk()
+    torch.cuda.synchronize()
+    ip.profile_read()
+    ip.profile_enable(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        chunk()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ip.profile_enable(False)
+    commit_ms = sum(v[0] for v in ip.profile_read().values()) / args.steps  # the chunk commits (streaming path)
+    ms = e0.elapsed_time(e1) / args.steps                                  # per chunk of C tokens
+    status = ip.get_status()
+    tokens = B * w.C
+    per_token_ms = (ms - commit_ms) / w.C
+    bytes_per_step = (3 * w.d * w.F + B * w.d * w.F) * 2 + 4 * B * w.d * 2 + 2 * B * w.F * 2
+    peaks, peak_src = load_peaks()
+    achieved = bytes_per_step / (per_token_ms / 1000.0) / 1e9
+    out = {"metric": "In-Place TTT MLP layer decode tokens/s (token-by-token, chunk commits included)",
+           "value": tokens / (ms / 1000.0), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": f"decode_{w.name}", "batch": B, "chunk": w.C, "d_model": w.d, "d_ff": w.F,
+                      "step": f"one chunk of {w.C} tokens per row", "l2": "weights and state copies larger than L2"},
+           "per_token_ms": per_token_ms, "commit_ms_per_chunk": commit_ms,
+           "roofline": {"kernel": "decode per-token kernels", "bound": "hbm", "achieved": achieved,
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                        "traffic": None, "bytes_per_token_step": bytes_per_step, "peak_source": peak_src},
+           "device_status": status}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -387,6 +450,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--chunk", type=int, default=None, help="override the chunk size C")
+    ap.add_argument("--mode", choices=("prefill", "decode"), default="prefill",
+                    help="decode: token-by-token decoding of --decode-batch rows instead of the prefill step")
+    ap.add_argument("--decode-batch", type=int, default=8)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--piece-tokens", type=int, default=0,
                     help="e2e: tokens per pipelined piece of the host-buffer call (0: about T/8)")
@@ -403,6 +469,8 @@ def main(argv=None):
         w = w.replace(C=args.chunk)
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.mode == "decode":
+        run_decode(args, w)
     else:
         run_ours(args, w)
 

@@ -1,0 +1,319 @@
+// Token-by-token decoding of the In-Place TTT MLP layer (bf16 path).
+//
+// A chunk's delta reaches only the chunks after it, and a chunk's outputs come
+// from the state before it [iplexlaw.co.kr review of arXiv 2604.06169, §3 and
+// §9.1; notes "In-Place Test-Time Training", 方法 › 步骤一/步骤二].  So a token
+// decoded inside chunk i needs only the committed state S_i: per token, for every
+// row b of the batch,
+//   z_t = SiLU(Wgate h_t) * (Wup h_t)                    (rounded to bf16, as Z is)
+//   o_t = Wdown0 z_t + m_b (S_i z_t)                       (one fp32 sum, then bf16)
+// with m_b = 1 when the token's document began before the chunk.  The chunk's H
+// and X0 rows are kept on the device; when the chunk is full, the streaming entry
+// point runs on it and commits S_{i+1} exactly as a prefill over the same tokens
+// would (target, clip and update need the whole chunk, the conv looks ahead up to
+// the chunk end).  The review notes the paper left the decode stage unmeasured
+// (§7.5, §8).
+//
+// The two per-token kernels are batched matrix-vector products bound by HBM: each
+// reads Wgate, Wup, Wdown0 once for all rows and every row's bf16 state snapshot.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "aux_kernels.h"
+#include "common.cuh"
+
+namespace ipttt {
+namespace {
+
+constexpr int kDecodeMaxRows = 16;  // rows per decode batch
+constexpr int kWarps = 8;           // warps per block; one output row (f or j) per warp
+constexpr int kFChunk = 2048;       // z columns staged in shared memory at a time
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Dot product of the 8 bf16 in one 16-byte word with the 8 bf16 in another, in fp32.
+__device__ __forceinline__ float dot8(const uint4 w, const uint4 x) {
+  const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+  const uint32_t b[4] = {x.x, x.y, x.z, x.w};
+  float s = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a[e]));
+    const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b[e]));
+    s = fmaf(fa.x, fb.x, s);
+    s = fmaf(fa.y, fb.y, s);
+  }
+  return s;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// z[b][f] = bf16(SiLU(Wg[f] . h_b) * (Wu[f] . h_b)); one warp per f, h in shared memory.
+__global__ void __launch_bounds__(kWarps * 32) k_decode_gateup(const __nv_bfloat16* __restrict__ h,
+                                                             const __nv_bfloat16* __restrict__ Wg,
+                                                             const __nv_bfloat16* __restrict__ Wu,
+                                                             __nv_bfloat16* __restrict__ z, int B, int d, int F) {
+  extern __shared__ uint4 hs[];  // [B][d / 8]
+  const int dv = d / 8;
+  for (int i = threadIdx.x; i < B * dv; i += blockDim.x) hs[i] = reinterpret_cast<const uint4*>(h)[i];
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f = blockIdx.x * kWarps + warp;
+  if (f >= F) return;
+  const uint4* wg = reinterpret_cast<const uint4*>(Wg + (size_t)f * d);
+  const uint4* wu = reinterpret_cast<const uint4*>(Wu + (size_t)f * d);
+  float g[kDecodeMaxRows], u[kDecodeMaxRows];
+#pragma unroll
+  for (int b = 0; b < kDecodeMaxRows; ++b) g[b] = u[b] = 0.0f;
+  for (int k = lane; k < dv; k += 32) {
+    const uint4 a = wg[k], c = wu[k];
+#pragma unroll
+    for (int b = 0; b < kDecodeMaxRows; ++b)
+      if (b < B) {
+        const uint4 x = hs[b * dv + k];
+        g[b] += dot8(a, x);
+        u[b] += dot8(c, x);
+      }
+  }
+#pragma unroll
+  for (int b = 0; b < kDecodeMaxRows; ++b)
+    if (b < B) {
+      const float gs = warp_sum(g[b]), us = warp_sum(u[b]);
+      if (lane == 0) z[(size_t)b * F + f] = __float2bfloat16_rn(silu_fast(gs) * us);
+    }
+}
+
+// o[b][j] = bf16(W0[j] . z_b + (m_b ? snap_b[j] . z_b : 0)); one warp per j, z staged
+// in shared memory kFChunk columns at a time.
+__global__ void __launch_bounds__(kWarps * 32) k_decode_apply(const __nv_bfloat16* __restrict__ z,
+                                                            const __nv_bfloat16* __restrict__ W0,
+                                                            const __nv_bfloat16* __restrict__ snap,
+                                                            uint32_t mask, __nv_bfloat16* __restrict__ o, int B,
+                                                            int d, int F) {
+  extern __shared__ uint4 zs[];  // [B][kFChunk / 8]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * kWarps + warp;
+  float a0[kDecodeMaxRows], a1[kDecodeMaxRows];
+#pragma unroll
+  for (int b = 0; b < kDecodeMaxRows; ++b) a0[b] = a1[b] = 0.0f;
+  for (int f0 = 0; f0 < F; f0 += kFChunk) {
+    const int fn = min(kFChunk, F - f0) / 8;
+    __syncthreads();
+    for (int i = threadIdx.x; i < B * fn; i += blockDim.x) {
+      const int b = i / fn, k = i % fn;
+      zs[b * (kFChunk / 8) + k] = reinterpret_cast<const uint4*>(z + (size_t)b * F + f0)[k];
+    }
+    __syncthreads();
+    if (j < d) {
+      const uint4* w = reinterpret_cast<const uint4*>(W0 + (size_t)j * F + f0);
+      for (int k = lane; k < fn; k += 32) {
+        const uint4 wv = w[k];
+#pragma unroll
+        for (int b = 0; b < kDecodeMaxRows; ++b)
+          if (b < B) {
+            const uint4 x = zs[b * (kFChunk / 8) + k];
+            a0[b] += dot8(wv, x);
+            if (mask >> b & 1u) {
+              const uint4 sv = reinterpret_cast<const uint4*>(snap + ((size_t)b * d + j) * F + f0)[k];
+              a1[b] += dot8(sv, x);
+            }
+          }
+      }
+    }
+  }
+  if (j >= d) return;
+#pragma unroll
+  for (int b = 0; b < kDecodeMaxRows; ++b)
+    if (b < B) {
+      const float s0 = warp_sum(a0[b]), s1 = warp_sum(a1[b]);
+      if (lane == 0) o[(size_t)b * d + j] = __float2bfloat16_rn(s0 + s1);
+    }
+}
+
+// Host bookkeeping of a decode state (lives in the caller's host buffer).
+struct DecodeHost {
+  int32_t B, C, d, F;
+  int32_t n;           // tokens of the current chunk already decoded
+  int32_t n_starts;    // document starts recorded in the current chunk
+  int64_t chunks;      // chunks committed since the reset
+  uint32_t cont_mask;  // rows whose current document began before the chunk
+  int32_t starts[1];   // [B * C] piece-relative offsets b*C + t of the chunk's starts
+};
+
+struct DecodeLayout {
+  size_t stream_state, H, X0, Oscr, snap, z, docs, ws, ws_bytes, total;
+};
+
+ipttt_params chunk_params(const ipttt_params& p) {
+  ipttt_params pc = p;
+  pc.T = p.C;
+  return pc;
+}
+
+bool decode_layout(const ipttt_params& p, DecodeLayout& L) {
+  const ipttt_params pc = chunk_params(p);
+  const size_t st = ipttt_stream_state_size(&pc), ws = ipttt_workspace_size(&pc);
+  if (st == 0 || ws == 0) return false;
+  const size_t rows = (size_t)p.B * p.C * p.d * 2;
+  size_t off = 0;
+  L.stream_state = off; off += al256(st);
+  L.H = off;            off += al256(rows);
+  L.X0 = off;           off += al256(rows);
+  L.Oscr = off;         off += al256(rows);
+  L.snap = off;         off += al256((size_t)p.B * p.d * p.F * 2);
+  L.z = off;            off += al256((size_t)p.B * p.F * 2);
+  L.docs = off;         off += al256((size_t)p.B * p.C * 4);
+  L.ws = off;           off += al256(ws);
+  L.ws_bytes = ws;
+  L.total = off;
+  return true;
+}
+
+ipttt_status decode_check(const ipttt_params* p) {
+  const ipttt_status rc = validate_params(p);
+  if (rc != IPTTT_OK) return rc;
+  if (p->dtype != IPTTT_BF16 || p->B > kDecodeMaxRows || p->d % 8 != 0 || p->F % 8 != 0)
+    return IPTTT_ERR_UNSUPPORTED;
+  return IPTTT_OK;
+}
+
+size_t host_bytes(const ipttt_params& p) { return sizeof(DecodeHost) + sizeof(int32_t) * (size_t)p.B * p.C; }
+
+}  // namespace
+}  // namespace ipttt
+
+using namespace ipttt;
+
+extern "C" {
+
+size_t ipttt_decode_state_size(const ipttt_params* p) {
+  if (decode_check(p) != IPTTT_OK) return 0;
+  DecodeLayout L;
+  return decode_layout(*p, L) ? L.total : 0;
+}
+
+size_t ipttt_decode_host_size(const ipttt_params* p) {
+  if (decode_check(p) != IPTTT_OK) return 0;
+  return host_bytes(*p);
+}
+
+ipttt_status ipttt_decode_reset(const ipttt_params* p, void* state, void* host_state, void* stream) {
+  const ipttt_status rc = decode_check(p);
+  if (rc != IPTTT_OK) return rc;
+  if (!state || !host_state) return IPTTT_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(state) % 256 != 0) return IPTTT_ERR_ALIGN;
+  DecodeLayout L;
+  if (!decode_layout(*p, L)) return IPTTT_ERR_SHAPE;
+  uint8_t* base = static_cast<uint8_t*>(state);
+  const ipttt_params pc = chunk_params(*p);
+  const ipttt_status r2 = ipttt_stream_reset(&pc, base + L.stream_state, stream);
+  if (r2 != IPTTT_OK) return r2;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(base + L.snap, 0, (size_t)p->B * p->d * p->F * 2, st) != cudaSuccess) return IPTTT_ERR_CUDA;
+  DecodeHost* hs = static_cast<DecodeHost*>(host_state);
+  hs->B = p->B;
+  hs->C = p->C;
+  hs->d = p->d;
+  hs->F = p->F;
+  hs->n = 0;
+  hs->n_starts = 0;
+  hs->chunks = 0;
+  hs->cont_mask = 0;
+  return IPTTT_OK;
+}
+
+ipttt_status ipttt_decode_step(const ipttt_params* p, void* state, void* host_state, const void* h, const void* x0,
+                               const int32_t* starts_host, const void* Wgate, const void* Wup, const void* Wdown0,
+                               const void* conv_w, const void* Wtarget, void* o, void* stream) {
+  const ipttt_status rc = decode_check(p);
+  if (rc != IPTTT_OK) return rc;
+  if (!state || !host_state || !h || !x0 || !Wgate || !Wup || !Wdown0 || !conv_w || !Wtarget || !o)
+    return IPTTT_ERR_ARG;
+  DecodeHost* hs = static_cast<DecodeHost*>(host_state);
+  if (hs->B != p->B || hs->C != p->C || hs->d != p->d || hs->F != p->F) return IPTTT_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(h) | reinterpret_cast<uintptr_t>(x0) | reinterpret_cast<uintptr_t>(o)) % 16 != 0)
+    return IPTTT_ERR_ALIGN;
+  DecodeLayout L;
+  if (!decode_layout(*p, L)) return IPTTT_ERR_SHAPE;
+  uint8_t* base = static_cast<uint8_t*>(state);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int B = p->B, C = p->C, d = p->d, F = p->F;
+  const size_t row = (size_t)d * 2;
+
+  // A document start on a row ends its continuation of the previous document.
+  if (starts_host)
+    for (int b = 0; b < B; ++b)
+      if (starts_host[b]) {
+        hs->cont_mask &= ~(1u << b);
+        hs->starts[hs->n_starts++] = b * C + hs->n;
+      }
+
+  // keep this token's inputs for the chunk's update
+  if (cudaMemcpy2DAsync(base + L.H + hs->n * row, (size_t)C * row, h, row, row, B, cudaMemcpyDeviceToDevice, st) !=
+          cudaSuccess ||
+      cudaMemcpy2DAsync(base + L.X0 + hs->n * row, (size_t)C * row, x0, row, row, B, cudaMemcpyDeviceToDevice,
+                        st) != cudaSuccess)
+    return IPTTT_ERR_CUDA;
+
+  __nv_bfloat16* z = reinterpret_cast<__nv_bfloat16*>(base + L.z);
+  {
+    const int smem = B * d * 2;
+    if (cudaFuncSetAttribute(k_decode_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return IPTTT_ERR_CUDA;
+    k_decode_gateup<<<(F + kWarps - 1) / kWarps, kWarps * 32, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(Wgate),
+        static_cast<const __nv_bfloat16*>(Wup), z, B, d, F);
+  }
+  {
+    const int smem = B * kFChunk * 2;
+    if (cudaFuncSetAttribute(k_decode_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return IPTTT_ERR_CUDA;
+    k_decode_apply<<<(d + kWarps - 1) / kWarps, kWarps * 32, smem, st>>>(
+        z, static_cast<const __nv_bfloat16*>(Wdown0), reinterpret_cast<const __nv_bfloat16*>(base + L.snap),
+        hs->cont_mask, static_cast<__nv_bfloat16*>(o), B, d, F);
+  }
+  if (cudaGetLastError() != cudaSuccess) return IPTTT_ERR_CUDA;
+
+  if (++hs->n < C) return IPTTT_OK;
+
+  // The chunk is complete: commit its update through the streaming entry point (the
+  // chunk's outputs it also computes are not needed), then refresh the snapshot.
+  std::sort(hs->starts, hs->starts + hs->n_starts);
+  int32_t* docs = reinterpret_cast<int32_t*>(base + L.docs);
+  if (hs->n_starts > 0 &&
+      cudaMemcpyAsync(docs, hs->starts, sizeof(int32_t) * hs->n_starts, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return IPTTT_ERR_CUDA;
+  const ipttt_params pc = chunk_params(*p);
+  const ipttt_status r2 =
+      ipttt_stream_forward(&pc, base + L.stream_state, base + L.H, base + L.X0, Wgate, Wup, Wdown0, conv_w, Wtarget,
+                           hs->n_starts > 0 ? docs : nullptr, hs->n_starts, base + L.Oscr, base + L.ws, L.ws_bytes,
+                           stream);
+  if (r2 != IPTTT_OK) return r2;
+  const Shape s{B, C, d, F, C, 1};
+  if (aux::state_snapshot(reinterpret_cast<const float*>(base + L.stream_state), base + L.snap, s, st) !=
+      cudaSuccess)
+    return IPTTT_ERR_CUDA;
+  hs->n = 0;
+  hs->n_starts = 0;
+  hs->chunks += 1;
+  hs->cont_mask = (B >= 32) ? 0xffffffffu : ((1u << B) - 1u);  // every row continues into the next chunk
+  return IPTTT_OK;
+}
+
+ipttt_status ipttt_decode_export(const ipttt_params* p, const void* state, float* S_out, void* stream) {
+  const ipttt_status rc = decode_check(p);
+  if (rc != IPTTT_OK) return rc;
+  if (!state || !S_out) return IPTTT_ERR_ARG;
+  DecodeLayout L;
+  if (!decode_layout(*p, L)) return IPTTT_ERR_SHAPE;
+  const ipttt_params pc = chunk_params(*p);
+  return ipttt_stream_export(&pc, static_cast<const uint8_t*>(state) + L.stream_state, S_out, stream);
+}
+
+}  // extern "C"

@@ -25,7 +25,8 @@ EXPORTS = ("ipttt_workspace_size", "ipttt_forward", "ipttt_forward_ex", "ipttt_c
            "ipttt_stream_reset", "ipttt_stream_forward", "ipttt_stream_export", "ipttt_get_status",
            "ipttt_strerror", "ipttt_version", "ipttt_profile_enable", "ipttt_profile_read",
            "ipttt_kernel_launches", "ipttt_selftest_wait_timeout", "ipttt_forward_noalloc",
-           "ipttt_forward_host_size", "ipttt_forward_host")
+           "ipttt_forward_host_size", "ipttt_forward_host", "ipttt_decode_state_size", "ipttt_decode_host_size",
+           "ipttt_decode_reset", "ipttt_decode_step", "ipttt_decode_export")
 PHASES = ("prep", "gate_up", "target", "gram", "apply", "update")
 DEBUG_OUTPUTS = ("D", "S_final", "alpha", "Z", "V")
 
@@ -93,6 +94,16 @@ def lib() -> ctypes.CDLL:
         L.ipttt_forward_host_size.restype = sz
         L.ipttt_forward_host.argtypes = [P] + [vp] * 7 + [vp, i32, vp, vp, sz, i32, vp]
         L.ipttt_forward_host.restype = ctypes.c_int
+        L.ipttt_decode_state_size.argtypes = [P]
+        L.ipttt_decode_state_size.restype = sz
+        L.ipttt_decode_host_size.argtypes = [P]
+        L.ipttt_decode_host_size.restype = sz
+        L.ipttt_decode_reset.argtypes = [P, vp, vp, vp]
+        L.ipttt_decode_reset.restype = ctypes.c_int
+        L.ipttt_decode_step.argtypes = [P, vp, vp, vp, vp, vp] + [vp] * 5 + [vp, vp]
+        L.ipttt_decode_step.restype = ctypes.c_int
+        L.ipttt_decode_export.argtypes = [P, vp, vp, vp]
+        L.ipttt_decode_export.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -321,6 +332,54 @@ class StreamState:
         S = torch.empty(self.cfg.B, self.cfg.d, self.cfg.F, dtype=torch.float32, device=self.buf.device)
         _check(lib().ipttt_stream_export(ctypes.byref(self.cfg.params()), self.buf.data_ptr(), S.data_ptr(),
                                          _stream(stream)), "ipttt_stream_export")
+        return S
+
+
+class DecodeState:
+    """Token-by-token decoding of B rows (bf16, B <= 16): a device state buffer and
+    the host bookkeeping the library keeps between steps.  cfg.T is ignored."""
+
+    def __init__(self, cfg: LayerConfig, device="cuda", stream=None):
+        self.cfg = cfg
+        p = cfg.params()
+        n = int(lib().ipttt_decode_state_size(ctypes.byref(p)))
+        nh = int(lib().ipttt_decode_host_size(ctypes.byref(p)))
+        if n == 0 or nh == 0:
+            raise ValueError("decoding needs bf16 and at most 16 rows")
+        self.buf = torch.empty(n, dtype=torch.uint8, device=device)
+        self.host = ctypes.create_string_buffer(nh)
+        self.reset(stream)
+
+    def reset(self, stream=None):
+        _check(lib().ipttt_decode_reset(ctypes.byref(self.cfg.params()), self.buf.data_ptr(), self.host,
+                                        _stream(stream)), "ipttt_decode_reset")
+
+    def step(self, h, x0, Wgate, Wup, Wdown0, conv_w, Wtarget, starts=None, *, o=None, stream=None):
+        """One token of every row: h, x0 [B, d] on the device; starts: B flags (a
+        document begins at this token), or None.  Returns o [B, d]."""
+        cfg = self.cfg
+        dt = cfg.torch_dtype
+        for name, t in (("h", h), ("x0", x0)):
+            if tuple(t.shape) != (cfg.B, cfg.d):
+                raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {(cfg.B, cfg.d)}")
+        _shape_check(cfg, Wgate=Wgate, Wup=Wup, Wdown0=Wdown0, conv_w=conv_w, Wtarget=Wtarget)
+        if o is None:
+            o = torch.empty(cfg.B, cfg.d, dtype=dt, device=h.device)
+        flags = None
+        if starts is not None:
+            flags = (ctypes.c_int32 * cfg.B)(*[int(bool(x)) for x in starts])
+        _check(lib().ipttt_decode_step(ctypes.byref(cfg.params()), self.buf.data_ptr(), self.host,
+                                       _ptr(h, dt, "h"), _ptr(x0, dt, "x0"), flags, _ptr(Wgate, dt, "Wgate"),
+                                       _ptr(Wup, dt, "Wup"), _ptr(Wdown0, dt, "Wdown0"), _ptr(conv_w, dt, "conv_w"),
+                                       _ptr(Wtarget, dt, "Wtarget"), _ptr(o, dt, "o"), _stream(stream)),
+               "ipttt_decode_step")
+        return o
+
+    def export(self, stream=None) -> torch.Tensor:
+        """The committed fp32 state [B, d, F]."""
+        S = torch.empty(self.cfg.B, self.cfg.d, self.cfg.F, dtype=torch.float32, device=self.buf.device)
+        _check(lib().ipttt_decode_export(ctypes.byref(self.cfg.params()), self.buf.data_ptr(), S.data_ptr(),
+                                         _stream(stream)), "ipttt_decode_export")
         return S
 
 

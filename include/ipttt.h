@@ -236,6 +236,38 @@ IPTTT_API ipttt_status ipttt_forward_host(const ipttt_params* p, const void* H_h
                                           void* O_host, void* device_buffer, size_t device_bytes,
                                           int32_t piece_tokens, void* stream);
 
+/* Token-by-token decoding (bf16, B <= 16 rows decoded together).  The pages leave
+ * the decode stage unmeasured (iplexlaw.co.kr review of arXiv 2604.06169, §7.5 and
+ * §8); what it must compute follows from the ordering (§3, §9.1): a token inside
+ * chunk i is output with the state committed before the chunk, and a chunk's delta
+ * is committed once the chunk is complete.  Per step, for every row b:
+ *   z = SiLU(Wgate h_b) * (Wup h_b)  (rounded to bf16),
+ *   o_b = Wdown0 z + m_b (S_i z)     (one fp32 sum, rounded to bf16),
+ * m_b = 1 while the row's document began before the current chunk.  When C tokens
+ * have been decoded, the chunk's H and X0 rows (kept in the state) go through
+ * ipttt_stream_forward, which commits S_{i+1} exactly as a prefill would; the
+ * outputs then equal ipttt_forward's up to the fp32 summation order.
+ *
+ * State: a device buffer of ipttt_decode_state_size(p) bytes (256-byte aligned:
+ * streaming state, the chunk's H and X0 rows, a bf16 copy of the committed state,
+ * a workspace) and a host buffer of ipttt_decode_host_size(p) bytes (positions and
+ * the chunk's document starts); p->T is ignored.  ipttt_decode_reset starts every
+ * row afresh.  ipttt_decode_step takes h, x0 and writes o, DEVICE [B, d] bf16;
+ * starts_host (HOST int32 [B], or NULL) flags rows whose token begins a new
+ * document.  The step that completes a chunk copies that chunk's document starts
+ * from the host buffer (pageable), so it first waits for work queued on `stream`.
+ * Other shapes or dtypes: IPTTT_ERR_UNSUPPORTED.  ipttt_decode_export copies the
+ * committed fp32 state [B, d, F] to S_out (device). */
+IPTTT_API size_t ipttt_decode_state_size(const ipttt_params* p);
+IPTTT_API size_t ipttt_decode_host_size(const ipttt_params* p);
+IPTTT_API ipttt_status ipttt_decode_reset(const ipttt_params* p, void* state, void* host_state, void* stream);
+IPTTT_API ipttt_status ipttt_decode_step(const ipttt_params* p, void* state, void* host_state,
+                                         const void* h, const void* x0, const int32_t* starts_host,
+                                         const void* Wgate, const void* Wup, const void* Wdown0,
+                                         const void* conv_w, const void* Wtarget, void* o, void* stream);
+IPTTT_API ipttt_status ipttt_decode_export(const ipttt_params* p, const void* state, float* S_out,
+                                           void* stream);
+
 /* Library version, "major.minor.patch". */
 IPTTT_API const char* ipttt_version(void);
 

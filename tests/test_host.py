@@ -109,3 +109,20 @@ def test_forward_host_size_and_argument_errors():
     # document starts are checked on the host: out of order
     docs = (ctypes.c_int32 * 2)(300, 200)
     assert L.ipttt_forward_host(ctypes.byref(p), host, host, *fake, docs, 2, host, buf, size, 256, None) == 1
+
+
+def test_decode_sizes_and_argument_errors():
+    L = ip.lib()
+    p = params(B=4, T=1, C=128)
+    assert L.ipttt_decode_state_size(ctypes.byref(p)) > 0
+    assert L.ipttt_decode_host_size(ctypes.byref(p)) >= 4 * 128 * 4
+    # more than 16 rows, or fp32: not supported by the decode kernels
+    assert L.ipttt_decode_state_size(ctypes.byref(params(B=17))) == 0
+    assert L.ipttt_decode_state_size(ctypes.byref(params(dtype=ip.F32))) == 0
+    host = ctypes.create_string_buffer(L.ipttt_decode_host_size(ctypes.byref(p)))
+    assert L.ipttt_decode_reset(ctypes.byref(params(B=17)), 0x100000, host, None) == 5
+    assert L.ipttt_decode_reset(ctypes.byref(p), None, host, None) == 1
+    assert L.ipttt_decode_reset(ctypes.byref(p), 0x100010, host, None) == 3  # misaligned state
+    fake = [0x10000 + 256 * i for i in range(8)]
+    # h missing
+    assert L.ipttt_decode_step(ctypes.byref(p), 0x100000, host, None, fake[0], None, *fake[1:6], fake[6], None) == 1
