@@ -71,6 +71,7 @@ __global__ void __launch_bounds__(kWarps * 32) k_decode_gateup(const __nv_bfloat
   float g[kDecodeMaxRows], u[kDecodeMaxRows];
 #pragma unroll
   for (int b = 0; b < kDecodeMaxRows; ++b) g[b] = u[b] = 0.0f;
+#pragma unroll 4
   for (int k = lane; k < dv; k += 32) {
     const uint4 a = wg[k], c = wu[k];
 #pragma unroll
@@ -89,16 +90,18 @@ __global__ void __launch_bounds__(kWarps * 32) k_decode_gateup(const __nv_bfloat
     }
 }
 
-// o[b][j] = bf16(W0[j] . z_b + (m_b ? snap_b[j] . z_b : 0)); one warp per j, z staged
-// in shared memory kFChunk columns at a time.
+// o[b][j] = bf16(W0[j] . z_b + (m_b ? snap_b[j] . z_b : 0)).  A block holds kWarps/2
+// rows j, two warps per row, each summing half of every staged z chunk (kFChunk
+// columns at a time); the two halves are added in a fixed order at the end.
 __global__ void __launch_bounds__(kWarps * 32) k_decode_apply(const __nv_bfloat16* __restrict__ z,
                                                             const __nv_bfloat16* __restrict__ W0,
                                                             const __nv_bfloat16* __restrict__ snap,
                                                             uint32_t mask, __nv_bfloat16* __restrict__ o, int B,
                                                             int d, int F) {
-  extern __shared__ uint4 zs[];  // [B][kFChunk / 8]
+  extern __shared__ uint4 zs[];  // [B][kFChunk / 8], then the halves' partial sums
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * kWarps + warp;
+  const int j = blockIdx.x * (kWarps / 2) + (warp >> 1);
+  const int part = warp & 1;
   float a0[kDecodeMaxRows], a1[kDecodeMaxRows];
 #pragma unroll
   for (int b = 0; b < kDecodeMaxRows; ++b) a0[b] = a1[b] = 0.0f;
@@ -112,7 +115,9 @@ __global__ void __launch_bounds__(kWarps * 32) k_decode_apply(const __nv_bfloat1
     __syncthreads();
     if (j < d) {
       const uint4* w = reinterpret_cast<const uint4*>(W0 + (size_t)j * F + f0);
-      for (int k = lane; k < fn; k += 32) {
+      const int k_lo = part * (fn / 2), k_hi = part ? fn : fn / 2;
+#pragma unroll 4
+      for (int k = k_lo + lane; k < k_hi; k += 32) {
         const uint4 wv = w[k];
 #pragma unroll
         for (int b = 0; b < kDecodeMaxRows; ++b)
@@ -127,13 +132,22 @@ __global__ void __launch_bounds__(kWarps * 32) k_decode_apply(const __nv_bfloat1
       }
     }
   }
-  if (j >= d) return;
+  // halves: warp 2r+1 hands its sums to warp 2r through shared memory
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(zs);  // [kWarps / 2][kDecodeMaxRows]
 #pragma unroll
   for (int b = 0; b < kDecodeMaxRows; ++b)
     if (b < B) {
-      const float s0 = warp_sum(a0[b]), s1 = warp_sum(a1[b]);
-      if (lane == 0) o[(size_t)b * d + j] = __float2bfloat16_rn(s0 + s1);
+      const float s = warp_sum(a0[b]) + warp_sum(a1[b]);
+      if (part == 1 && lane == 0) red[(warp >> 1) * kDecodeMaxRows + b] = s;
+      a0[b] = s;
     }
+  __syncthreads();
+  if (part == 0 && lane == 0 && j < d) {
+#pragma unroll
+    for (int b = 0; b < kDecodeMaxRows; ++b)
+      if (b < B) o[(size_t)b * d + j] = __float2bfloat16_rn(a0[b] + red[(warp >> 1) * kDecodeMaxRows + b]);
+  }
 }
 
 // Host bookkeeping of a decode state (lives in the caller's host buffer).
@@ -274,7 +288,7 @@ ipttt_status ipttt_decode_step(const ipttt_params* p, void* state, void* host_st
     const int smem = B * kFChunk * 2;
     if (cudaFuncSetAttribute(k_decode_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return IPTTT_ERR_CUDA;
-    k_decode_apply<<<(d + kWarps - 1) / kWarps, kWarps * 32, smem, st>>>(
+    k_decode_apply<<<(d + kWarps / 2 - 1) / (kWarps / 2), kWarps * 32, smem, st>>>(
         z, static_cast<const __nv_bfloat16*>(Wdown0), reinterpret_cast<const __nv_bfloat16*>(base + L.snap),
         hs->cont_mask, static_cast<__nv_bfloat16*>(o), B, d, F);
   }
