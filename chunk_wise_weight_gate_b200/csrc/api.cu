@@ -119,6 +119,7 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 
 struct Layout {
   size_t flags, meta, alpha, partials, Z, U, V, S, snap, raw, dpart, total;
+  size_t cp_docs, cp_plan;  // context-parallel calls: local document starts, per-row plan
   int group;  // bf16 path: chunks whose apply tiles share one launch (= snapshot ring slots)
 };
 
@@ -175,7 +176,10 @@ Shape shape_of(const ipttt_params& p) {
   return s;
 }
 
-Layout layout_of(const ipttt_params& p) {
+// cp: the layout of the context-parallel calls, whose snapshot ring holds every
+// chunk's S_i (k + 1 slots: the apply runs after all the shard's updates) and
+// which keep the shard's document starts and per-row plan on the device.
+Layout layout_of(const ipttt_params& p, bool cp = false) {
   const Shape s = shape_of(p);
   const size_t B = s.B, T = s.T, d = s.d, F = s.F, k = s.k;
   Layout L{};
@@ -195,7 +199,7 @@ Layout layout_of(const ipttt_params& p) {
     L.U = take(B * T * d * 2);
     L.V = take(B * T * d * 2);
     L.S = take(B * d * F * 4);
-    L.group = apply_group(p);
+    L.group = cp ? s.k + 1 : apply_group(p);
     L.snap = take((size_t)L.group * B * d * F * 2);
     L.raw = L.dpart = 0;
   } else {
@@ -207,6 +211,11 @@ Layout layout_of(const ipttt_params& p) {
     L.raw = take(B * d * F * 4);
     L.dpart = take(B * 64 * sizeof(double));
     L.snap = 0;
+  }
+  L.cp_docs = L.cp_plan = 0;
+  if (cp) {
+    L.cp_docs = take(B * T * sizeof(int32_t));
+    L.cp_plan = take(4 * B * sizeof(int32_t));
   }
   L.total = off;
   return L;
@@ -244,6 +253,23 @@ struct StreamState {
   int32_t* cont;
 };
 
+// The two context-parallel stages (ipttt_cp_begin / ipttt_cp_finish).
+//   begin : the shard's forward up to its state updates, from a zero state, with the
+//           first chunk continuing the row's document where plan row_cont says so;
+//           the fp32 state (= the shard's aggregate) is the caller's `agg`.
+//   finish: S_in from the gathered aggregates, folded into the snapshots of the
+//           chunks that continue the incoming document, then the apply of every
+//           chunk and the final state.
+enum CpStageKind { kCpBegin = 1, kCpFinish = 2 };
+struct CpArgs {
+  int stage;
+  int world, rank;
+  const int32_t* plan;     // device [4][B]: row_cont, first_rank, prefix_chunks, keep
+  float* agg;              // begin: the state / aggregate [B][d][F] (blocked tiles)
+  const float* gathered;   // finish: [world][B][d][F], every rank's aggregate
+  float* Sfinal;           // finish: optional row-major S_final [B][d][F]
+};
+
 size_t state_bytes(const ipttt_params& p) {
   const size_t B = p.B;
   return align256(B * p.d * (size_t)p.F * 4) + align256(B * 8) + align256(B * 4);
@@ -272,7 +298,7 @@ bool pair_gemms_enabled() {
 }
 
 ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, const Layout& L, StreamState* ss,
-                      DeviceInfo* di, cudaStream_t st) {
+                      DeviceInfo* di, cudaStream_t st, const CpArgs* cp = nullptr) {
   using namespace tck;
   const Shape s = shape_of(p);
   uint8_t* flags = ws + L.flags;
@@ -282,14 +308,17 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   void* Z = t.Zin ? const_cast<void*>(t.Zin) : static_cast<void*>(ws + L.Z);
   void* U = ws + L.U;
   void* V = ws + L.V;
-  float* S = ss ? ss->S : reinterpret_cast<float*>(ws + L.S);
+  float* S = ss ? ss->S : cp ? cp->agg : reinterpret_cast<float*>(ws + L.S);
   void* snap = ws + L.snap;
   const float tau = (p.clip_thresh > 0.0f && isfinite(p.clip_thresh)) ? p.clip_thresh : 0.0f;
   ipttt_status rc_ = IPTTT_OK;
+  // A context-parallel finish reuses everything its begin left in the workspace.
+  const bool cp_finish = cp && cp->stage == kCpFinish;
 
-  {
+  if (!cp_finish) {
     PhaseScope ph(st, PH_PREP);
-    IP_CHECK(aux::build_meta(flags, meta, s, t.doc, t.n_doc, ss ? ss->cont : nullptr, di->status, st));
+    IP_CHECK(aux::build_meta(flags, meta, s, t.doc, t.n_doc, ss ? ss->cont : cp ? cp->plan : nullptr, di->status,
+                             st));
     counted(3);
     if (!t.Zin) {
       IP_CHECK(aux::conv_target(IPTTT_BF16, t.X0, t.cw, flags, U, s, st));
@@ -320,7 +349,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   const bool pair_gemm = pair_gemms_enabled() && pair_gemm_workers(st) > 0;
   const int zv_fam = pair_gemm ? FAM_ZV2 : FAM_ZV;
   const int zv_rows = pair_gemm ? 256 : 128;
-  if (!t.Zin) {
+  if (!t.Zin && !cp_finish) {
     PhaseScope ph(st, PH_GATEUP);
     TcParams g = tp;
     g.kind = kind_gateup();
@@ -333,7 +362,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     IP_CHECK(launch_tc(zv_fam, g, di->num_sms, st));
     counted(1);
   }
-  if (!t.Zin) {
+  if (!t.Zin && !cp_finish) {
     PhaseScope ph(st, PH_TARGET);
     TcParams v = tp;
     v.kind = kind_vhat();
@@ -349,7 +378,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   if (t.Zout) IP_CHECK(cudaMemcpyAsync(t.Zout, Z, (size_t)s.B * s.T * s.F * 2, cudaMemcpyDeviceToDevice, st));
   if (t.Vout) IP_CHECK(cudaMemcpyAsync(t.Vout, V, (size_t)s.B * s.T * s.d * 2, cudaMemcpyDeviceToDevice, st));
 
-  {
+  if (!cp_finish) {
     PhaseScope ph(st, PH_GRAM);
     TcParams g = tp;
     // On CTA pairs: 256 x 256 token-block pairs, two partials (one per CTA) each.
@@ -373,6 +402,12 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   }
   if (t.alpha) IP_CHECK(cudaMemcpyAsync(t.alpha, alpha, (size_t)s.B * s.k * 4, cudaMemcpyDeviceToDevice, st));
 
+  // A context-parallel shard starts from a zero state: S_0 (snapshot slot 0) and
+  // the fp32 state are cleared; the incoming state is added in the finish.
+  if (cp && !cp_finish) {
+    IP_CHECK(cudaMemsetAsync(S, 0, (size_t)s.B * s.d * s.F * 4, st));
+    IP_CHECK(cudaMemsetAsync(snap, 0, (size_t)s.B * s.d * s.F * 2, st));
+  }
   // A streaming piece that continues a row starts from the carried state S.
   if (ss) {
     PhaseScope ph(st, PH_UPDATE);
@@ -389,7 +424,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   const int arows = apply_rows(p);
   const int apply_fam = arows == 256 ? FAM_APPLY256 : FAM_APPLY;
   if (!make_map_bf16(&sc.map[0], Z, s.F, s.T, s.B, 64, arows == 256 ? 128 : tp.tr) ||
-      !make_map_bf16(&sc.map[1], t.W0, s.F, s.d, 1, 64, 128) ||
+      (t.W0 && !make_map_bf16(&sc.map[1], t.W0, s.F, s.d, 1, 64, 128)) ||  // no W0: a context-parallel begin
       !make_map_bf16(&sc.map[2], snap, s.F, s.d, (uint64_t)G * s.B, 64, 128) ||
       !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, update_tokens_per_stage(s.C)) ||
       !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, update_tokens_per_stage(s.C)) ||
@@ -419,6 +454,26 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     counted(1);
     return IPTTT_OK;
   };
+  if (cp) {
+    // begin: every chunk's update in one launch, S_1 .. S_k into slots 1 .. k and
+    // the shard's aggregate left in the state.  finish: the incoming state into
+    // S_0 .. S_{prefix-1} (and S_final), then the apply of all k chunks.
+    if (!cp_finish) return update(0, s.k);
+    {
+      PhaseScope ph(st, PH_UPDATE);
+      IP_CHECK(aux::cp_combine(cp->gathered, cp->world, cp->rank, cp->plan, snap, G, cp->Sfinal, s, st));
+      counted(1);
+    }
+    PhaseScope ph(st, PH_APPLY);
+    TcParams q = sc;
+    q.chunk = 0;
+    q.dchunks = 1;
+    q.apply_chunk0 = 0;
+    q.n_tiles = s.k * apply_tiles_per_chunk;
+    IP_CHECK(launch_tc(apply_fam, q, di->num_sms, st));
+    counted(1);
+    return IPTTT_OK;
+  }
   // Group [a, b) of G chunks: the updates of chunks a-1 .. b-2 produce S_a .. S_{b-1}
   // (ring slots a % G .. (b-1) % G, which the previous group's applies have
   // finished reading), then one launch applies chunks a .. b-1.
@@ -633,6 +688,137 @@ ipttt_status ipttt_stream_export(const ipttt_params* p, const void* state, float
   if (!aligned(state, 256) || !aligned(S_out, 16)) return IPTTT_ERR_ALIGN;
   const StreamState ss = state_of(*p, const_cast<void*>(state));
   return cuda_status(aux::state_export(is_bf16(*p), ss.S, S_out, shape_of(*p), static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------- context parallelism
+size_t ipttt_cp_workspace_size(const ipttt_params* p) {
+  if (check_params(p) != IPTTT_OK || p->dtype != IPTTT_BF16) return 0;
+  return layout_of(*p, true).total;
+}
+
+ipttt_status ipttt_cp_plan(const ipttt_params* p, int32_t world, int32_t rank, const int32_t* doc_starts_host,
+                           int32_t n_doc_starts, int32_t* local_starts, int32_t* n_local, int32_t* plan) {
+  ipttt_status rc = check_params(p);
+  if (rc != IPTTT_OK) return rc;
+  if (world < 1 || rank < 0 || rank >= world || n_doc_starts < 0 || (n_doc_starts > 0 && !doc_starts_host) ||
+      !n_local || !plan)
+    return IPTTT_ERR_ARG;
+  const long long B = p->B, T = p->T, C = p->C;
+  const long long Tg = T * world;
+  if (B * Tg > 0x7fffffffLL) return IPTTT_ERR_SHAPE;
+  if (world > 1 && T % C != 0) return IPTTT_ERR_SHAPE;
+  const long long k = (T + C - 1) / C;
+  int32_t* row_cont = plan;
+  int32_t* first_rank = plan + B;
+  int32_t* prefix = plan + 2 * B;
+  int32_t* keep = plan + 3 * B;
+  // last[b]: the last rank before this one whose shard of row b holds a start (the
+  // row start counts for rank 0); first[b]: this shard's first local start or -1.
+  std::vector<long long> last(B, 0), first(B, -1);
+  long long prev = -1;
+  int32_t m = 0;
+  for (int32_t i = 0; i < n_doc_starts; ++i) {
+    const long long g = doc_starts_host[i];
+    if (g < 0 || g >= B * Tg || g <= prev) return IPTTT_ERR_ARG;
+    prev = g;
+    const long long b = g / Tg, t = g % Tg, owner = t / T;
+    if (owner < rank) last[b] = std::max(last[b], owner);
+    if (owner == rank) {
+      if (first[b] < 0) first[b] = t - rank * T;
+      if (local_starts) local_starts[m] = (int32_t)(b * T + (t - rank * T));
+      ++m;
+    }
+  }
+  *n_local = m;
+  for (long long b = 0; b < B; ++b) {
+    const bool starts_at_0 = rank == 0 || first[b] == 0;
+    row_cont[b] = starts_at_0 ? 0 : 1;
+    first_rank[b] = rank == 0 ? 0 : (int32_t)last[b];
+    prefix[b] = starts_at_0 ? 0 : (int32_t)(first[b] < 0 ? k : first[b] / C + 1);
+    keep[b] = (!starts_at_0 && first[b] < 0) ? 1 : 0;
+  }
+  return IPTTT_OK;
+}
+
+}  // extern "C"
+
+namespace ipttt {
+namespace {
+ipttt_status cp_run(const ipttt_params* p, int32_t world, int32_t rank, const int32_t* doc_starts_host,
+                    int32_t n_doc_starts, const Tensors& t, CpArgs cp, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  ipttt_status rc = check_params(p);
+  if (rc != IPTTT_OK) return rc;
+  if (p->dtype != IPTTT_BF16) return IPTTT_ERR_UNSUPPORTED;
+  const Layout L = layout_of(*p, true);
+  if (!workspace || workspace_bytes < L.total) return IPTTT_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return IPTTT_ERR_ALIGN;
+  int32_t n_local = 0;
+  std::vector<int32_t> plan(4 * (size_t)p->B);
+  if ((rc = ipttt_cp_plan(p, world, rank, doc_starts_host, n_doc_starts, nullptr, &n_local, plan.data())) !=
+      IPTTT_OK)
+    return rc;
+  std::vector<int32_t> local((size_t)std::max(n_local, 1));
+  if ((rc = ipttt_cp_plan(p, world, rank, doc_starts_host, n_doc_starts, local.data(), &n_local, plan.data())) !=
+      IPTTT_OK)
+    return rc;
+  DeviceInfo* di = nullptr;
+  if ((rc = device_info(&di)) != IPTTT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* plan_dev = reinterpret_cast<int32_t*>(ws + L.cp_plan);
+  int32_t* docs_dev = reinterpret_cast<int32_t*>(ws + L.cp_docs);
+  // pageable sources: the copies have taken the bytes when they return
+  IP_CHECK(cudaMemcpyAsync(plan_dev, plan.data(), plan.size() * 4, cudaMemcpyHostToDevice, st));
+  if (cp.stage == kCpBegin && n_local > 0)
+    IP_CHECK(cudaMemcpyAsync(docs_dev, local.data(), (size_t)n_local * 4, cudaMemcpyHostToDevice, st));
+  Tensors tt = t;
+  tt.doc = n_local > 0 ? docs_dev : nullptr;
+  tt.n_doc = n_local;
+  cp.world = world;
+  cp.rank = rank;
+  cp.plan = plan_dev;
+  rc = run_bf16(*p, tt, ws, L, nullptr, di, st, &cp);
+  if (rc == IPTTT_OK && cudaPeekAtLastError() != cudaSuccess) rc = IPTTT_ERR_CUDA;
+  return rc;
+}
+}  // namespace
+}  // namespace ipttt
+
+extern "C" {
+
+ipttt_status ipttt_cp_begin(const ipttt_params* p, int32_t world, int32_t rank, const int32_t* doc_starts_host,
+                            int32_t n_doc_starts, const void* H, const void* X0, const void* Wgate, const void* Wup,
+                            const void* conv_w, const void* Wtarget, float* agg, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  ipttt_status rc;
+  const void* must[] = {H, X0, Wgate, Wup, conv_w, Wtarget, agg};
+  for (const void* q : must)
+    if ((rc = check_tensor(q)) != IPTTT_OK) return rc;
+  Tensors t{H, X0, Wgate, Wup, nullptr, conv_w, Wtarget, nullptr, nullptr, nullptr, 0, nullptr,
+            nullptr, nullptr, nullptr, nullptr, nullptr};
+  CpArgs cp{};
+  cp.stage = kCpBegin;
+  cp.agg = agg;
+  return cp_run(p, world, rank, doc_starts_host, n_doc_starts, t, cp, workspace, workspace_bytes, stream);
+}
+
+ipttt_status ipttt_cp_finish(const ipttt_params* p, int32_t world, int32_t rank, const int32_t* doc_starts_host,
+                             int32_t n_doc_starts, const void* H, const void* Wdown0, const float* gathered,
+                             void* O, float* S_final_opt, void* workspace, size_t workspace_bytes, void* stream) {
+  ipttt_status rc;
+  if (p && (p->flags & IPTTT_FLAG_RESIDUAL) && O == H) return IPTTT_ERR_ARG;
+  const void* must[] = {H, Wdown0, gathered, O};
+  for (const void* q : must)
+    if ((rc = check_tensor(q)) != IPTTT_OK) return rc;
+  if (S_final_opt && !aligned(S_final_opt, 16)) return IPTTT_ERR_ALIGN;
+  Tensors t{H, nullptr, nullptr, nullptr, Wdown0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, O,
+            nullptr, nullptr, nullptr, nullptr, nullptr};
+  CpArgs cp{};
+  cp.stage = kCpFinish;
+  cp.gathered = gathered;
+  cp.Sfinal = S_final_opt;
+  return cp_run(p, world, rank, doc_starts_host, n_doc_starts, t, cp, workspace, workspace_bytes, stream);
 }
 
 ipttt_status ipttt_get_status(void* stream) {

@@ -440,6 +440,105 @@ cudaError_t mask_last_segment(int dtype, const void* in, void* out, const ChunkM
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ context parallelism
+// One block per (row b, 128 x 128 state tile, quarter of 32 tile rows).  With plan
+// = [row_cont | first_rank | prefix_chunks | keep] (each [B]):
+//   S_in      = sum over ranks j in [first_rank[b], rank) of gathered[j][b]
+//   snapshot S_i (ring slot i, bf16, row-major) += S_in   for chunks i < prefix_chunks[b]
+//   S_final   = gathered[rank][b] + (keep[b] ? S_in : 0)   (row-major fp32, optional)
+// The aggregates are in the state's blocked order, where the 32 rows of a quarter
+// and 4 columns form one 512-byte run, so the reads are whole runs; the rows go
+// through shared memory (rows padded to 33 float4) to the row-major writes.  The
+// sum runs in rank order, the same on every rank.
+__global__ void __launch_bounds__(256) k_cp_combine(const float* __restrict__ gathered, int rank,
+                                                    const int32_t* __restrict__ plan, __nv_bfloat16* snap,
+                                                    int nslots, float* Sfinal, int B, int d, int F) {
+  __shared__ float4 s_in[32][33];
+  __shared__ float4 s_fin[32][33];
+  const int ntn = F / 128;
+  const int q = blockIdx.x & 3;
+  const int tile_all = blockIdx.x >> 2;
+  const int per_row = (d / 128) * ntn;
+  const int b = tile_all / per_row;
+  const int tile = tile_all % per_row;
+  const int mt = tile / ntn, nt = tile % ntn;
+  const int j0 = plan[B + b], pre = plan[2 * B + b], keep = plan[3 * B + b];
+  const size_t per = (size_t)d * F;
+  const size_t tbase = (size_t)b * per + (size_t)tile * 16384;
+  const int r = threadIdx.x & 31;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int g = (threadIdx.x >> 5) + 8 * it;  // 4-column group of the tile
+    const size_t idx = tbase + ((size_t)g * 128 + q * 32 + r) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = j0; j < rank; ++j) {
+      const float4 v = *reinterpret_cast<const float4*>(gathered + (size_t)j * B * per + idx);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    s_in[r][g] = acc;
+    if (Sfinal) {
+      float4 a = *reinterpret_cast<const float4*>(gathered + (size_t)rank * B * per + idx);
+      if (keep) {
+        a.x += acc.x;
+        a.y += acc.y;
+        a.z += acc.z;
+        a.w += acc.w;
+      }
+      s_fin[r][g] = a;
+    }
+  }
+  __syncthreads();
+  const int wr = threadIdx.x >> 3;   // tile row of the quarter
+  const int part = threadIdx.x & 7;  // 16 columns
+  const size_t grow = (size_t)mt * 128 + q * 32 + wr;
+  const size_t gcol = (size_t)nt * 128 + part * 16;
+  if (Sfinal) {
+    float4* dst = reinterpret_cast<float4*>(Sfinal + (size_t)b * per + grow * F + gcol);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) dst[u] = s_fin[wr][part * 4 + u];
+  }
+  if (pre <= 0) return;
+  float add[16];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float4 v = s_in[wr][part * 4 + u];
+    add[4 * u] = v.x;
+    add[4 * u + 1] = v.y;
+    add[4 * u + 2] = v.z;
+    add[4 * u + 3] = v.w;
+  }
+  for (int i = 0; i < pre; ++i) {
+    uint4* p = reinterpret_cast<uint4*>(snap + ((size_t)(i % nslots) * B + b) * per + grow * F + gcol);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint4 w = p[h];
+      uint32_t* e = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        __nv_bfloat162 v2 = *reinterpret_cast<__nv_bfloat162*>(&e[x]);
+        const float lo = __low2float(v2) + add[8 * h + 2 * x];
+        const float hi = __high2float(v2) + add[8 * h + 2 * x + 1];
+        v2 = __floats2bfloat162_rn(lo, hi);
+        e[x] = *reinterpret_cast<uint32_t*>(&v2);
+      }
+      p[h] = w;
+    }
+  }
+}
+
+cudaError_t cp_combine(const float* gathered, int world, int rank, const int32_t* plan, void* snap, int nslots,
+                       float* Sfinal, const Shape& s, cudaStream_t st) {
+  if (rank < 0 || rank >= world || s.d % 128 != 0 || s.F % 128 != 0) return cudaErrorInvalidValue;
+  const long long blocks = (long long)s.B * (s.d / 128) * (s.F / 128) * 4;
+  if (blocks <= 0 || blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  k_cp_combine<<<(unsigned)blocks, 256, 0, st>>>(gathered, rank, plan, (__nv_bfloat16*)snap, nslots, Sfinal, s.B,
+                                                 s.d, s.F);
+  return cudaGetLastError();
+}
+
 // Streaming bookkeeping: every row has now consumed `T` more tokens.
 __global__ void k_stream_advance(long long* pos, int32_t* cont, int B, int T) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;

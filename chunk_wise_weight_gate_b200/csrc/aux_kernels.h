@@ -53,6 +53,11 @@ namespace aux {
 cudaError_t mask_last_segment(int dtype, const void* in, void* out, const ChunkMeta* meta, const Shape& s,
                               cudaStream_t st);
 cudaError_t stream_advance(long long* pos, int32_t* cont, int B, int T, cudaStream_t st);
+// Context parallelism: S_in from the gathered shard aggregates (ranks
+// [first_rank, rank) of each row), added to the snapshots of the chunks that
+// continue the incoming document, and S_final (optional); plan is [4][B] int32.
+cudaError_t cp_combine(const float* gathered, int world, int rank, const int32_t* plan, void* snap, int nslots,
+                       float* Sfinal, const Shape& s, cudaStream_t st);
 cudaError_t prescale_target(void* V, const float* alpha, const Shape& s, float eta, cudaStream_t st);
 }  // namespace aux
 }  // namespace ipttt

@@ -26,7 +26,8 @@ EXPORTS = ("ipttt_workspace_size", "ipttt_forward", "ipttt_forward_ex", "ipttt_c
            "ipttt_strerror", "ipttt_version", "ipttt_profile_enable", "ipttt_profile_read",
            "ipttt_kernel_launches", "ipttt_selftest_wait_timeout", "ipttt_forward_noalloc",
            "ipttt_forward_host_size", "ipttt_forward_host", "ipttt_decode_state_size", "ipttt_decode_host_size",
-           "ipttt_decode_reset", "ipttt_decode_step", "ipttt_decode_export")
+           "ipttt_decode_reset", "ipttt_decode_step", "ipttt_decode_export", "ipttt_cp_workspace_size",
+           "ipttt_cp_plan", "ipttt_cp_begin", "ipttt_cp_finish")
 PHASES = ("prep", "gate_up", "target", "gram", "apply", "update")
 DEBUG_OUTPUTS = ("D", "S_final", "alpha", "Z", "V")
 
@@ -104,6 +105,14 @@ def lib() -> ctypes.CDLL:
         L.ipttt_decode_step.restype = ctypes.c_int
         L.ipttt_decode_export.argtypes = [P, vp, vp, vp]
         L.ipttt_decode_export.restype = ctypes.c_int
+        L.ipttt_cp_workspace_size.argtypes = [P]
+        L.ipttt_cp_workspace_size.restype = sz
+        L.ipttt_cp_plan.argtypes = [P, i32, i32, vp, i32, vp, vp, vp]
+        L.ipttt_cp_plan.restype = ctypes.c_int
+        L.ipttt_cp_begin.argtypes = [P, i32, i32, vp, i32] + [vp] * 6 + [vp, vp, sz, vp]
+        L.ipttt_cp_begin.restype = ctypes.c_int
+        L.ipttt_cp_finish.argtypes = [P, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.ipttt_cp_finish.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -293,6 +302,110 @@ def forward_host(cfg: LayerConfig, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, d
                                     ds.data_ptr() if nd else None, nd, _host_ptr(O, dt, "O"), buffer.data_ptr(),
                                     buffer.numel(), piece_tokens, _stream(stream)), "ipttt_forward_host")
     return O
+
+
+# ---------------------------------------------------------------- context parallelism
+# cfg.T is the shard length: rank r of `world` holds tokens [r*T, (r+1)*T) of every
+# row; doc_starts are offsets b*(world*T) + t over the whole sequence, on the host.
+
+def _host_docs(doc_starts) -> torch.Tensor:
+    if doc_starts is None:
+        return torch.zeros(0, dtype=torch.int32)
+    ds = doc_starts if isinstance(doc_starts, torch.Tensor) else torch.as_tensor(doc_starts, dtype=torch.int32)
+    return ds.to(device="cpu", dtype=torch.int32).contiguous()
+
+
+def cp_workspace_size(cfg: LayerConfig) -> int:
+    n = lib().ipttt_cp_workspace_size(ctypes.byref(cfg.params()))
+    if n == 0:
+        raise ValueError(f"invalid context-parallel configuration {cfg}")
+    return int(n)
+
+
+def cp_plan(cfg: LayerConfig, world: int, rank: int, doc_starts=None):
+    """Host side of the split (no GPU needed): this rank's document starts as
+    offsets within the shard, and the per-row plan dict (row_cont, first_rank,
+    prefix_chunks, keep), each a list of B ints."""
+    ds = _host_docs(doc_starts)
+    nd = ds.numel()
+    local = torch.zeros(max(nd, 1), dtype=torch.int32)
+    plan = torch.zeros(4, cfg.B, dtype=torch.int32)
+    n_local = ctypes.c_int32(0)
+    p = cfg.params()
+    _check(lib().ipttt_cp_plan(ctypes.byref(p), int(world), int(rank), ds.data_ptr() if nd else None, nd,
+                               local.data_ptr(), ctypes.addressof(n_local), plan.data_ptr()), "ipttt_cp_plan")
+    names = ("row_cont", "first_rank", "prefix_chunks", "keep")
+    return local[:n_local.value].tolist(), {n: plan[i].tolist() for i, n in enumerate(names)}
+
+
+def cp_begin(cfg: LayerConfig, world: int, rank: int, H, X0, Wgate, Wup, conv_w, Wtarget, doc_starts=None, *,
+             agg=None, workspace=None, stream=None):
+    """First stage on one rank: the shard's forward up to its state updates.
+    Returns (agg, workspace); agg [B, d, F] fp32 is what the ranks exchange, and
+    the workspace goes unchanged to cp_finish."""
+    dt = cfg.torch_dtype
+    _shape_check(cfg, H=H, X0=X0, Wgate=Wgate, Wup=Wup, conv_w=conv_w, Wtarget=Wtarget)
+    dev = H.device
+    if agg is None:
+        agg = torch.empty(cfg.B, cfg.d, cfg.F, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(cp_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    ds = _host_docs(doc_starts)
+    nd = ds.numel()
+    p = cfg.params()
+    _check(lib().ipttt_cp_begin(ctypes.byref(p), int(world), int(rank), ds.data_ptr() if nd else None, nd,
+                                _ptr(H, dt, "H"), _ptr(X0, dt, "X0"), _ptr(Wgate, dt, "Wgate"), _ptr(Wup, dt, "Wup"),
+                                _ptr(conv_w, dt, "conv_w"), _ptr(Wtarget, dt, "Wtarget"),
+                                _ptr(agg, torch.float32, "agg"), workspace.data_ptr(), workspace.numel(),
+                                _stream(stream)), "ipttt_cp_begin")
+    return agg, workspace
+
+
+def cp_exchange(agg: torch.Tensor, group=None) -> torch.Tensor:
+    """The one exchange: every rank's aggregate, gathered in rank order
+    ([world, B, d, F]), through torch.distributed (NCCL on GPUs)."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    flat = torch.empty(world * agg.numel(), dtype=agg.dtype, device=agg.device)
+    dist.all_gather_into_tensor(flat, agg.contiguous().view(-1), group=group)
+    return flat.view(world, *agg.shape)
+
+
+def cp_finish(cfg: LayerConfig, world: int, rank: int, H, Wdown0, gathered, workspace, doc_starts=None, *, O=None,
+              S_final=False, residual=False, stream=None):
+    """Second stage on one rank: returns this shard's O (and S_final, the state
+    after the shard's last chunk, when S_final=True)."""
+    dt = cfg.torch_dtype
+    _shape_check(cfg, H=H, Wdown0=Wdown0, O=O)
+    if tuple(gathered.shape) != (world, cfg.B, cfg.d, cfg.F):
+        raise ValueError(f"gathered has shape {tuple(gathered.shape)}, expected {(world, cfg.B, cfg.d, cfg.F)}")
+    dev = H.device
+    if O is None:
+        O = torch.empty(cfg.B, cfg.T, cfg.d, dtype=dt, device=dev)
+    if residual and O.data_ptr() == H.data_ptr():
+        raise ValueError("O must not alias H when residual=True")
+    Sf = torch.empty(cfg.B, cfg.d, cfg.F, dtype=torch.float32, device=dev) if S_final else None
+    ds = _host_docs(doc_starts)
+    nd = ds.numel()
+    p = cfg.params(FLAG_RESIDUAL if residual else 0)
+    _check(lib().ipttt_cp_finish(ctypes.byref(p), int(world), int(rank), ds.data_ptr() if nd else None, nd,
+                                 _ptr(H, dt, "H"), _ptr(Wdown0, dt, "Wdown0"),
+                                 _ptr(gathered, torch.float32, "gathered"), _ptr(O, dt, "O"),
+                                 Sf.data_ptr() if Sf is not None else None, workspace.data_ptr(), workspace.numel(),
+                                 _stream(stream)), "ipttt_cp_finish")
+    return (O, Sf) if S_final else O
+
+
+def cp_forward(cfg: LayerConfig, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_starts=None, *, group=None,
+               S_final=False, residual=False, stream=None):
+    """This rank's shard of a context-parallel forward over the ranks of `group`:
+    begin, one all-gather of the shard aggregates, finish."""
+    import torch.distributed as dist
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    agg, ws = cp_begin(cfg, world, rank, H, X0, Wgate, Wup, conv_w, Wtarget, doc_starts, stream=stream)
+    gathered = cp_exchange(agg, group)
+    return cp_finish(cfg, world, rank, H, Wdown0, gathered, ws, doc_starts, S_final=S_final, residual=residual,
+                     stream=stream)
 
 
 class StreamState:

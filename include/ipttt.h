@@ -158,6 +158,54 @@ IPTTT_API ipttt_status ipttt_stream_forward(const ipttt_params* p, void* state,
 IPTTT_API ipttt_status ipttt_stream_export(const ipttt_params* p, const void* state, float* S_out,
                                  void* stream);
 
+/* Context parallelism: the batch's sequences split along T over `world` ranks
+ * (one process per GPU), rank r holding tokens [r*T, (r+1)*T) of every row, with
+ * params->T the shard length (a multiple of C when world > 1, so that no conv tap
+ * and no chunk crosses a shard).  The chunk deltas are independent of the state, so
+ * each shard computes its own; the fast weight a shard starts from is the
+ * segmented exclusive sum of the earlier shards' aggregates, restarted at the last
+ * shard that holds a document start (lijianxiong.blog notes "In-Place Test-Time
+ * Training", 工程实现: deltas in parallel, then a prefix sum; iplexlaw.co.kr
+ * review §6: exclusive scan with document resets).  One exchange:
+ *   ipttt_cp_begin   the shard's Z, V, clip factors and state updates from a zero
+ *                    state; leaves the shard's aggregate in agg [B, d, F] fp32 (an
+ *                    opaque tile order, the same on every rank);
+ *   (caller)         all-gather agg in rank order into gathered [world, B, d, F];
+ *   ipttt_cp_finish  adds the incoming state to the state the shard's chunks of the
+ *                    continuing document see, applies every chunk (O [B, T, d] =
+ *                    this shard's rows of the full forward) and optionally writes
+ *                    S_final [B, d, F] (row-major fp32): the state after the shard's
+ *                    last chunk (on the last rank, after the whole sequence).
+ * doc_starts_host: HOST int32, n_doc_starts strictly increasing offsets
+ * b*(world*T) + t over the whole sequence (every rank passes the same list).  Both
+ * calls of a rank take the same params, world, rank, doc starts and workspace
+ * (ipttt_cp_workspace_size bytes, 256-byte aligned; its snapshot ring holds the
+ * state of every chunk of the shard), which must not be touched in between.
+ * bf16 only (IPTTT_ERR_UNSUPPORTED otherwise).  Bad doc starts, world or rank
+ * return IPTTT_ERR_ARG before anything is launched.  The incoming state is added
+ * to the bf16 copy of each continuing chunk's state, one extra rounding against a
+ * single-device forward.  H is read by the finish only with IPTTT_FLAG_RESIDUAL. */
+IPTTT_API size_t ipttt_cp_workspace_size(const ipttt_params* p);
+/* The host side of the split, run by both calls (pure host function): this rank's
+ * document starts as offsets b*T + t within the shard (local_starts, room for
+ * n_doc_starts entries, or NULL to count only; their number in *n_local), and
+ * plan [4, B]: row_cont (the shard's first token continues a document), first_rank
+ * (the first rank of the row's segmented sum), prefix_chunks (the shard's chunks
+ * that see the incoming state) and keep (the incoming state reaches S_final). */
+IPTTT_API ipttt_status ipttt_cp_plan(const ipttt_params* p, int32_t world, int32_t rank,
+                                     const int32_t* doc_starts_host, int32_t n_doc_starts,
+                                     int32_t* local_starts, int32_t* n_local, int32_t* plan);
+IPTTT_API ipttt_status ipttt_cp_begin(const ipttt_params* p, int32_t world, int32_t rank,
+                                      const int32_t* doc_starts_host, int32_t n_doc_starts,
+                                      const void* H, const void* X0, const void* Wgate, const void* Wup,
+                                      const void* conv_w, const void* Wtarget, float* agg,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+IPTTT_API ipttt_status ipttt_cp_finish(const ipttt_params* p, int32_t world, int32_t rank,
+                                       const int32_t* doc_starts_host, int32_t n_doc_starts,
+                                       const void* H, const void* Wdown0, const float* gathered,
+                                       void* O, float* S_final_opt,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
 /* Waits for `stream`, then returns and clears the per-device status word that
  * kernels set on device-side errors (IPTTT_OK if none). */
 IPTTT_API ipttt_status ipttt_get_status(void* stream);

@@ -57,6 +57,24 @@ int main(void) {
   expect(ipttt_decode_reset(&p, NULL, host, NULL) == IPTTT_ERR_ARG, "decode reset without a state");
   expect(ipttt_stream_reset(&bad, dev, NULL) == IPTTT_ERR_UNSUPPORTED, "stream reset, unsupported shape");
 
+  /* context parallelism: the host plan of rank 1 of 2 (shards of 2048 tokens) for a
+   * row whose document begins at token 1000 and continues through shard 1 */
+  int32_t starts[1] = {1000};
+  int32_t local[1] = {-1};
+  int32_t n_local = -1;
+  int32_t plan[4] = {-1, -1, -1, -1};
+  expect(ipttt_cp_workspace_size(&p) > ws, "context-parallel workspace holds every chunk's state");
+  expect(ipttt_cp_plan(&p, 2, 1, starts, 1, local, &n_local, plan) == IPTTT_OK, "cp plan");
+  expect(n_local == 0 && plan[0] == 1 && plan[1] == 0 && plan[2] == 8 && plan[3] == 1,
+         "cp plan: shard continues shard 0's document through all 8 chunks");
+  expect(ipttt_cp_plan(&p, 2, 2, starts, 1, local, &n_local, plan) == IPTTT_ERR_ARG, "cp plan, rank out of range");
+  expect(ipttt_cp_begin(&p, 2, 0, NULL, 0, NULL, dev, dev, dev, dev, dev, (float*)dev, dev, 1u << 30, NULL) ==
+             IPTTT_ERR_ARG,
+         "cp begin with a null H");
+  expect(ipttt_cp_finish(&p, 2, 0, NULL, 0, dev, dev, (const float*)dev, NULL, NULL, dev, 1u << 30, NULL) ==
+             IPTTT_ERR_ARG,
+         "cp finish with a null O");
+
   if (failures == 0) printf("C ABI checks passed\n");
   return failures == 0 ? 0 : 1;
 }
