@@ -442,6 +442,112 @@ def run_decode(args, w: synth.Workload):
         print(json.dumps(out), flush=True)
 
 
+def run_cp(args, w: synth.Workload):
+    """Context parallelism: the workload's sequences split along T over the N
+    ranks (strong scaling: the total work is fixed).  A step is every rank's
+    ipttt_cp_begin, one NCCL all-gather of the shard aggregates and ipttt_cp_finish;
+    with one rank there is no exchange."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    if w.T % world or (w.T // world) % w.C:
+        raise ValueError(f"T={w.T} does not split into {world} shards of whole {w.C}-token chunks")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+        pg = dist
+    TL = w.T // world
+    inp = synth.make_inputs(w, seed=0)           # the same sequence and weights on every rank
+    sl = slice(rank * TL, (rank + 1) * TL)
+    H = inp["H"][:, sl].contiguous().to(dev)
+    X0 = inp["X0"][:, sl].contiguous().to(dev)
+    wts = {k: inp[k].to(dev) for k in WEIGHTS}
+    docs = inp["doc_starts"].to(torch.int32).contiguous()
+    del inp
+    cfg = ip.LayerConfig(B=w.B, T=TL, d=w.d, F=w.F, C=w.C, eta=w.eta, clip=w.clip, dtype=w.dtype)
+    ws = torch.empty(ip.cp_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    agg = torch.empty(w.B, w.d, w.F, dtype=torch.float32, device=dev)
+    # one rank: its own aggregate is the whole gathered set
+    gathered = torch.empty(world, w.B, w.d, w.F, dtype=torch.float32, device=dev) if world > 1 else agg.view(1, *agg.shape)
+    O = torch.empty(w.B, TL, w.d, dtype=cfg.torch_dtype, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ip.cp_begin(cfg, world, rank, H, X0, wts["Wgate"], wts["Wup"], wts["conv_w"], wts["Wtarget"], docs,
+                    agg=agg, workspace=ws)
+        if pg:
+            ip.cp_exchange(agg, out=gathered)
+        ip.cp_finish(cfg, world, rank, H, wts["Wdown0"], gathered, ws, docs, O=O)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ip.get_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+    gpu_id = str(local)
+    try:
+        gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
+        if not gpu_id.startswith("GPU-"):
+            gpu_id = "GPU-" + gpu_id
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    ip.profile_read()
+    ip.profile_enable(True)
+    launches0 = ip.kernel_launches()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if pg:
+        pg.barrier()
+    ip.profile_enable(False)
+    launches = ip.kernel_launches() - launches0
+    phases = ip.profile_read()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, pg, dev)
+    status = ip.get_status()
+    tokens = w.B * w.T
+    peaks, peak_src = load_peaks()
+    pf = phase_flops(w.replace(T=TL))
+    dom = max(phases, key=lambda k: phases[k][0])
+    dom_ms, dom_launches = phases[dom]
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    achieved = pf.get(dom, 0) * args.steps / (dom_ms / 1000.0) / 1e12 if dom in pf else None
+    roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak if achieved else None, "traffic": None, "launches": dom_launches,
+            "peak_note": f"sustained bf16 ({peak_src}); rank {rank}'s phases"}
+    phase_report = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
+                    for k, v in phases.items()}
+    if rank == 0:
+        cfgd = config_dict(w, world)
+        cfgd.update({"workload": f"cp_{w.name}", "parallelism": f"cp{world}", "shard_tokens": TL, "global_batch": w.B,
+                     "exchange": "NCCL all-gather of the fp32 shard aggregates" if world > 1 else "none"})
+        out = {"metric": METRIC + " (one sequence split over the GPUs)", "value": tokens / (ms / 1000.0),
+               "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+               "dtype": "bf16", "data": "synthetic", "config": cfgd,
+               "tflops": layer_flops(w) / (ms / 1000.0) / 1e12, "roofline": roof, "phases": phase_report,
+               "clocks": clocks, "e2e": None, "gpu_launches": launches, "cpu_baseline": None,
+               "device_status": status}
+        print(json.dumps(out), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -450,8 +556,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--chunk", type=int, default=None, help="override the chunk size C")
-    ap.add_argument("--mode", choices=("prefill", "decode"), default="prefill",
-                    help="decode: token-by-token decoding of --decode-batch rows instead of the prefill step")
+    ap.add_argument("--mode", choices=("prefill", "decode", "cp"), default="prefill",
+                    help="decode: token-by-token decoding of --decode-batch rows instead of the prefill step; "
+                         "cp: the sequence split along T over the GPUs (context parallelism)")
     ap.add_argument("--decode-batch", type=int, default=8)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--piece-tokens", type=int, default=0,
@@ -471,6 +578,8 @@ def main(argv=None):
         run_reference(args, w)
     elif args.mode == "decode":
         run_decode(args, w)
+    elif args.mode == "cp":
+        run_cp(args, w)
     else:
         run_ours(args, w)
 

@@ -361,14 +361,18 @@ def cp_begin(cfg: LayerConfig, world: int, rank: int, H, X0, Wgate, Wup, conv_w,
     return agg, workspace
 
 
-def cp_exchange(agg: torch.Tensor, group=None) -> torch.Tensor:
+def cp_exchange(agg: torch.Tensor, group=None, out: torch.Tensor | None = None) -> torch.Tensor:
     """The one exchange: every rank's aggregate, gathered in rank order
-    ([world, B, d, F]), through torch.distributed (NCCL on GPUs)."""
+    ([world, B, d, F]; into `out` when given), through torch.distributed (NCCL on
+    GPUs)."""
     import torch.distributed as dist
     world = dist.get_world_size(group)
-    flat = torch.empty(world * agg.numel(), dtype=agg.dtype, device=agg.device)
-    dist.all_gather_into_tensor(flat, agg.contiguous().view(-1), group=group)
-    return flat.view(world, *agg.shape)
+    if out is None:
+        out = torch.empty(world, *agg.shape, dtype=agg.dtype, device=agg.device)
+    if tuple(out.shape) != (world, *agg.shape) or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {(world, *agg.shape)} tensor")
+    dist.all_gather_into_tensor(out.view(-1), agg.contiguous().view(-1), group=group)
+    return out
 
 
 def cp_finish(cfg: LayerConfig, world: int, rank: int, H, Wdown0, gathered, workspace, doc_starts=None, *, O=None,
