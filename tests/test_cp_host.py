@@ -111,7 +111,21 @@ def draw(seed, world):
     }
 
 
-def shard_forward(inp, world, rank, docs):
+def median_chunk_norm(inp, world, docs):
+    """The median ||eta P_i|| over the chunks of the whole sequence: a threshold at
+    which about half the chunks clip."""
+    Tg = TL * world
+    flags = fw.start_flags(B, Tg, docs)
+    norms = []
+    for b in range(B):
+        Z = fw.gated_activation(inp["H"][b], inp["Wgate"], inp["Wup"])
+        V = fw.lm_target(inp["X0"][b], inp["conv_w"], inp["Wtarget"], C, flags[b])
+        for (s, e, f, l, cont, has_start) in fw.chunk_segments(flags[b], C):
+            norms.append(np.linalg.norm(fw.hebbian_delta(Z[l:e], V[l:e], ETA)))
+    return float(np.median(norms))
+
+
+def shard_forward(inp, world, rank, docs, tau=TAU):
     """One rank: the oracle forward of the shard from a zero state, the first chunk
     continuing the row's document where the plan says so, then the exchange, then
     the incoming state on the rows before the shard's first start."""
@@ -129,7 +143,7 @@ def shard_forward(inp, world, rank, docs):
                 flags[g % TL] = True
         Z = fw.gated_activation(inp["H"][b, sl], inp["Wgate"], inp["Wup"])
         V = fw.lm_target(inp["X0"][b, sl], inp["conv_w"], inp["Wtarget"], C, flags)
-        O[b], _, S_loc[b], _ = fw.core_sequential(Z, V, inp["Wdown0"], C, flags, ETA, TAU)
+        O[b], _, S_loc[b], _ = fw.core_sequential(Z, V, inp["Wdown0"], C, flags, ETA, tau)
         Z_all[b] = Z
     gathered = ip.cp_exchange(torch.from_numpy(S_loc)).numpy()
     assert gathered.shape == (world, B, d, F)
@@ -145,31 +159,35 @@ def shard_forward(inp, world, rank, docs):
     return O, S_final
 
 
-def _worker(rank, world, port, docs, out):
+def _worker(rank, world, port, docs, tau, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         inp = draw(7, world)
-        O, S_final = shard_forward(inp, world, rank, docs)
+        O, S_final = shard_forward(inp, world, rank, docs, tau)
         out[rank] = (O, S_final)
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,docs", [
-    (2, []),                                   # one document over both shards
-    (2, [TL, 2 * TL + 50]),                    # row 0 restarts on the shard boundary; row 1 inside shard 0
-    (3, [100, 3 * TL + TL + 70]),              # row 0: start in shard 0 carries into 1 and 2
-    (3, [TL + 10, 2 * TL + 64, 3 * TL + 5]),   # starts inside shards, one on a chunk boundary
+@pytest.mark.parametrize("world,docs,clip", [
+    (2, [], False),                                  # one document over both shards
+    (2, [TL, 2 * TL + 50], False),                   # row 0 restarts on the shard boundary; row 1 inside shard 0
+    (3, [100, 3 * TL + TL + 70], False),             # row 0: start in shard 0 carries into 1 and 2
+    (3, [TL + 10, 2 * TL + 64, 3 * TL + 5], False),  # starts inside shards, one on a chunk boundary
+    (3, [100, 3 * TL + TL + 70], True),              # the clip active on about half the chunks
 ])
-def test_context_parallel_equals_single_sequence(world, docs):
+def test_context_parallel_equals_single_sequence(world, docs, clip):
+    inp = draw(7, world)
+    tau = median_chunk_norm(inp, world, docs) if clip else TAU
     with mp.Manager() as m:
         out = m.dict()
-        mp.spawn(_worker, args=(world, free_port(), docs, out), nprocs=world, join=True)
+        mp.spawn(_worker, args=(world, free_port(), docs, tau, out), nprocs=world, join=True)
         res = dict(out)
-    inp = draw(7, world)
     full = fw.layer_forward(inp["H"], inp["X0"], inp["Wgate"], inp["Wup"], inp["Wdown0"], inp["conv_w"],
-                            inp["Wtarget"], C, docs, ETA, TAU)
+                            inp["Wtarget"], C, docs, ETA, tau)
+    if clip:
+        assert np.any(full["alpha"] < 1.0) and np.any(full["alpha"] == 1.0)
     D_scale = np.max(np.abs(full["D"])) if np.any(full["D"]) else 1.0
     for r in range(world):
         O, S_final = res[r]
