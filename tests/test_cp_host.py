@@ -197,3 +197,20 @@ def test_context_parallel_equals_single_sequence(world, docs, clip):
     np.testing.assert_allclose(res[world - 1][1], full["S_final"], rtol=1e-10, atol=1e-12)
     # the case is one where the carried state matters
     assert D_scale > 1e-3
+
+
+def test_binding_refuses_host_tensors_and_wrong_shapes():
+    # the product path has no CPU fallback: host tensors are refused before any call
+    cfg = cfg_for()
+    H = torch.zeros(B, TL, d, dtype=torch.bfloat16)
+    Wg = torch.zeros(F, d, dtype=torch.bfloat16)
+    cw = torch.zeros(d, 5, dtype=torch.bfloat16)
+    Wt = torch.zeros(d, d, dtype=torch.bfloat16)
+    agg = torch.zeros(B, d, F)
+    ws = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA"):
+        ip.cp_begin(cfg, 2, 0, H, H, Wg, Wg, cw, Wt, [], agg=agg, workspace=ws)
+    with pytest.raises(ValueError, match="gathered"):
+        ip.cp_finish(cfg, 2, 0, H, Wg.T.contiguous(), torch.zeros(3, B, d, F), ws, [])
+    with pytest.raises(ValueError, match="shape"):
+        ip.cp_begin(cfg, 2, 0, H[:, :64], H, Wg, Wg, cw, Wt, [], agg=agg, workspace=ws)
