@@ -250,6 +250,20 @@ def test_document_isolation_unaligned():
     assert np.any(o[:, 9:17] != base[:, 9:17])
 
 
+def test_hand_worked_stack():
+    """stack_forward against a two-layer residual chain worked by hand."""
+    for case in json.load(open(GOLD))["stack_cases"]:
+        layers = [{k: np.asarray(v, float) for k, v in l.items()} for l in case["layers"]]
+        H0 = np.asarray(case["H0"], float)[None]
+        X0 = np.asarray(case["X0"], float)[None]
+        Hout, outs = orc.stack_forward(layers, X0, H0, case["C"], case["doc_starts"], case["eta"], case["tau"])
+        np.testing.assert_allclose(Hout[0], np.asarray(case["H_out"], float), rtol=1e-13, atol=1e-13)
+        for l, r in enumerate(outs):
+            np.testing.assert_allclose(r["O"][0], np.asarray(case["O"][l], float), rtol=1e-13, atol=1e-13)
+            np.testing.assert_allclose(r["S_final"][0], np.asarray(case["S_final"][l], float), rtol=1e-13,
+                                       atol=1e-13)
+
+
 def test_stack_residual():
     H, X0, Wg, Wu, W0, cw, Wt = small_layer(24, T=12, C=4)
     p = dict(Wgate=Wg, Wup=Wu, Wdown0=W0, conv_w=cw, Wtarget=Wt)
