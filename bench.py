@@ -128,16 +128,59 @@ def phase_flops(w: synth.Workload) -> dict:
     """Algorithmic flops per call of each phase (per layer)."""
     B, T, d, F, C = w.B, w.T, w.d, w.F, w.C
     k = (T + C - 1) // C
-    ct = C // 128
+    ct = max(1, C // 256) if C % 256 == 0 else max(1, C // 128)
+    tr = C // ct
     return {
-        "prep": 10 * B * T * d,
+        "prep": 0,
         "gate_up": 4 * B * T * d * F,
-        "target": 2 * B * T * d * d,
-        "gram": 2 * B * k * (ct * (ct + 1) // 2) * 128 * 128 * (d + F),
+        "target": 2 * B * T * d * d + 10 * B * T * d,
+        "gram": 2 * B * k * (ct * (ct + 1) // 2) * tr * tr * (d + F),
         "apply": 4 * B * T * d * F,
         "update": 2 * B * T * d * F,
-        "scan": 6 * B * T * d * F,
     }
+
+
+def phase_bytes(w: synth.Workload, phase: str, launches: float) -> float:
+    """Algorithmic DRAM bytes per call of a phase (per layer): every input read once,
+    every output written once.  `launches` is the phase's launch count per layer (the
+    state update reads and writes the fp32 state once per launch; the apply reads
+    Wdown0 once per launch)."""
+    B, T, d, F, C = w.B, w.T, w.d, w.F, w.C
+    k = (T + C - 1) // C
+    e = 2  # bf16
+    if phase == "prep":
+        return 2 * B * T
+    if phase == "gate_up":
+        return B * T * d * e + 2 * F * d * e + B * T * F * e
+    if phase == "target":
+        return B * T * d * e + d * d * e + 5 * d * e + B * T * d * e
+    if phase == "gram":  # Z and V read; V read and written again by the pre-scale
+        return B * T * (F + d) * e + 2 * B * T * d * e
+    if phase == "update":  # V, Z read; a bf16 snapshot per chunk; the fp32 state per launch
+        return B * T * (F + d) * e + B * (k - 1) * d * F * e + launches * B * d * F * 4 * 2
+    if phase == "apply":  # Z and every snapshot read, Wdown0 per launch, O written (H read: residual)
+        return B * T * F * e + B * (k - 1) * d * F * e + launches * d * F * e + B * T * d * e * (2 if w.layers > 1 else 1)
+    return 0.0
+
+
+def phase_roofline(w: synth.Workload, phase: str, ms: float, launches: float, steps: int, peaks: dict) -> dict:
+    """Achieved rate of one phase against the bound that limits it: the tensor time
+    (algorithmic flops at the sustained bf16 peak) or the HBM time (algorithmic bytes
+    at the measured copy bandwidth), whichever is longer."""
+    per = launches / max(1, steps * w.layers)
+    fl = phase_flops(w).get(phase, 0) * w.layers * steps
+    by = phase_bytes(w, phase, per) * w.layers * steps
+    tflops = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    t_tensor = fl / (tflops * 1e12)
+    t_hbm = by / (peaks["hbm_gbs"] * 1e9)
+    sec = ms / 1000.0
+    if t_tensor >= t_hbm:
+        ach = fl / sec / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s", "frac": ach / tflops,
+                "algorithmic_bytes_per_step": by / steps}
+    ach = by / sec / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+            "algorithmic_bytes_per_step": by / steps, "tflops": fl / sec / 1e12}
 
 
 def oracle_sample(w: synth.Workload, inp: dict, chunks: int) -> tuple[float, int]:
@@ -173,9 +216,10 @@ def config_dict(w: synth.Workload, n: int) -> dict:
 
 
 # DRAM bytes (read + written) per launch of a kernel, the mean over the launches of
-# one step captured by ncu on the named workload (profiles/apply_traffic_qwen3_4b_128k.md).  The
-# roofline object carries it only for the kernel and workload it was taken on.
-MEASURED_TRAFFIC = {("qwen3_4b_128k", "apply"): 2.577e9 + 104.45e6}
+# one step captured by ncu, keyed by (workload, chunk size, phase); the summaries in
+# profiles/ give the commands.  The roofline object carries a figure only for the
+# kernel and workload it was taken on.
+MEASURED_TRAFFIC = {("qwen3_4b_128k", 1024, "apply"): 2.577e9 + 104.45e6}
 
 
 def sample_chunks(w: synth.Workload, tokens: int) -> int:
@@ -293,25 +337,17 @@ def run_ours(args, w: synth.Workload):
     peaks, peak_src = load_peaks()
 
     # roofline of the dominant kernel (the phase with the largest share of device time)
-    pf = phase_flops(w)
     dom = max(phases, key=lambda k: phases[k][0])
     dom_ms, dom_launches = phases[dom]
-    if dom in ("prep",):
-        algo_bytes = w.B * w.T * w.d * 2 * 2 * w.layers * args.steps
-        achieved = algo_bytes / (dom_ms / 1000.0) / 1e9
-        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None}
-    else:
-        total = pf[dom] * w.layers * args.steps
-        achieved = total / (dom_ms / 1000.0) / 1e12
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": MEASURED_TRAFFIC.get((w.name, dom)), "traffic_unit": "bytes",
-                "launches": dom_launches,
-                "avg_launch_ms": dom_ms / max(1, dom_launches),
-                "peak_note": f"sustained bf16 ({peak_src}); burst {peaks['bf16_tflops']}"}
-    phase_report = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
-                    for k, v in phases.items()}
+    roof = {"kernel": dom, **phase_roofline(w, dom, dom_ms, dom_launches, args.steps, peaks),
+            "launches": dom_launches, "avg_launch_ms": dom_ms / max(1, dom_launches),
+            "peak_note": f"sustained bf16 and copy bandwidth ({peak_src}); burst bf16 {peaks['bf16_tflops']}"}
+    traffic = MEASURED_TRAFFIC.get((w.name, w.C, dom))
+    roof["traffic"] = traffic
+    roof["traffic_unit"] = "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
+    phase_report = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps,
+                        **phase_roofline(w, k, v[0], v[1], args.steps, peaks)}
+                    for k, v in phases.items() if v[1] > 0}
 
     # end to end through the public API: pinned host inputs in, result read back, every step
     e2e = None
@@ -521,14 +557,11 @@ def run_cp(args, w: synth.Workload):
     status = ip.get_status()
     tokens = w.B * w.T
     peaks, peak_src = load_peaks()
-    pf = phase_flops(w.replace(T=TL))
+    wl = w.replace(T=TL)
     dom = max(phases, key=lambda k: phases[k][0])
     dom_ms, dom_launches = phases[dom]
-    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    achieved = pf.get(dom, 0) * args.steps / (dom_ms / 1000.0) / 1e12 if dom in pf else None
-    roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak if achieved else None, "traffic": None, "launches": dom_launches,
-            "peak_note": f"sustained bf16 ({peak_src}); rank {rank}'s phases"}
+    roof = {"kernel": dom, **phase_roofline(wl, dom, dom_ms, dom_launches, args.steps, peaks), "traffic": None,
+            "launches": dom_launches, "peak_note": f"sustained bf16 and copy bandwidth ({peak_src}); rank {rank}'s phases"}
     phase_report = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
                     for k, v in phases.items()}
     if rank == 0:

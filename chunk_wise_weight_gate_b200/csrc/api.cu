@@ -2,14 +2,16 @@
 // carve-up, and the order of kernel launches for one In-Place TTT MLP layer.
 //
 // Launch order (bf16 path), all on the caller's stream:
-//   metadata -> masked conv U -> Z = SiLU(H Wg^T)*(H Wu^T) -> V = U Wt (last-segment
-//   rows) -> Gram partials -> alpha -> for each chunk i: one scan launch holding the
-//   apply tiles of chunk i (reads S_i) and the delta tiles (S_i -> S_{i+1}).
+//   metadata -> Z = SiLU(H Wg^T)*(H Wu^T) -> V = conv(X0) Wt (the masked conv in the
+//   target GEMM's producer; last-segment rows) -> Gram partials -> alpha and the
+//   pre-scale of V -> per group of chunks: the state updates (S_i -> S_{i+1}, bf16
+//   snapshots) and one launch of the group's apply tiles (reads S_i).
 // The chunk order follows lijianxiong.blog notes "In-Place Test-Time Training",
 // 方法 (apply with the current fast weight, then update) and iplexlaw.co.kr review
 // §3 (a chunk's output always comes from the pre-update state).
 #include <cuda_runtime.h>
 #include <math.h>
+#include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -119,6 +121,8 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 
 struct Layout {
   size_t flags, meta, alpha, partials, Z, U, V, S, snap, raw, dpart, total;
+  size_t gmeta, glo, P, E;  // grouped scan: group metadata, per-token group offsets, within-group terms
+  bool grouped;
   size_t cp_docs, cp_plan;  // context-parallel calls: local document starts, per-row plan
   int group;  // bf16 path: chunks whose apply tiles share one launch (= snapshot ring slots)
 };
@@ -165,6 +169,32 @@ int apply_group(const ipttt_params& p) {
 
 bool is_bf16(const ipttt_params& p) { return p.dtype == IPTTT_BF16; }
 
+// Chunks of 64 or 128 tokens are scanned kGroupTokens at a time (groups of 4 or 2
+// chunks): the state is carried, snapshotted and applied per group, and the
+// chunks of a group see each other's deltas through the within-group term
+//   E[t] = sum_{u in an earlier chunk of t's group, in t's document} (z_t . z_u) v'_u
+// (v' = alpha eta v on the rows that feed the update).  That equals the
+// chunk-by-chunk scan (the apply is linear in the state), with one bf16 state
+// snapshot written and read per group instead of per chunk.
+constexpr int kGroupTokens = 256;
+// IPTTT_GROUPED_SCAN=0 scans such chunks one by one instead.
+bool grouped_scan(const ipttt_params& p) {
+  const char* e = getenv("IPTTT_GROUPED_SCAN");
+  if (e && e[0] == '0') return false;
+  return is_bf16(p) && (p.C == 64 || p.C == 128) && p.T > p.C;
+}
+}  // namespace
+
+int scan_unit_tokens(const ipttt_params& p) { return grouped_scan(p) ? kGroupTokens : p.C; }
+
+namespace {
+
+ipttt_params group_params(const ipttt_params& p) {
+  ipttt_params g = p;
+  g.C = kGroupTokens;
+  return g;
+}
+
 Shape shape_of(const ipttt_params& p) {
   Shape s;
   s.B = p.B;
@@ -199,10 +229,21 @@ Layout layout_of(const ipttt_params& p, bool cp = false) {
     L.U = take(B * T * d * 2);
     L.V = take(B * T * d * 2);
     L.S = take(B * d * F * 4);
-    L.group = cp ? s.k + 1 : apply_group(p);
+    L.grouped = grouped_scan(p);
+    const size_t kg = (T + kGroupTokens - 1) / kGroupTokens;
+    L.group = cp ? (int)(L.grouped ? kg : s.k) + 1 : apply_group(L.grouped ? group_params(p) : p);
     L.snap = take((size_t)L.group * B * d * F * 2);
     L.raw = L.dpart = 0;
+    L.gmeta = L.glo = L.P = L.E = 0;
+    if (L.grouped) {
+      L.gmeta = take(B * kg * sizeof(ChunkMeta));
+      L.glo = take(B * T);
+      L.P = take(B * T * kGroupTokens * 2);
+      L.E = take(B * T * d * 2);
+    }
   } else {
+    L.grouped = false;
+    L.gmeta = L.glo = L.P = L.E = 0;
     L.partials = 0;
     L.Z = take(B * T * F * 4);
     L.U = take(B * T * d * 4);
@@ -285,16 +326,30 @@ StreamState state_of(const ipttt_params& p, void* state) {
   return s;
 }
 
+// The detail behind the last IPTTT_ERR_CUDA of this thread (ipttt_last_error_detail).
+thread_local char g_err_detail[320];
+
+ipttt_status cuda_fail(const char* step, cudaError_t e) {
+  snprintf(g_err_detail, sizeof(g_err_detail), "%s: %s (%s)", step, cudaGetErrorName(e), cudaGetErrorString(e));
+  return IPTTT_ERR_CUDA;
+}
+
 #define IP_CHECK(expr)                                  \
   do {                                                  \
     cudaError_t e_ = (expr);                            \
-    if (e_ != cudaSuccess) return IPTTT_ERR_CUDA;       \
+    if (e_ != cudaSuccess) return cuda_fail(#expr, e_); \
   } while (0)
 
 // Pair (cluster of two) GEMMs can be switched off with IPTTT_GEMM_CTAS=1.
 bool pair_gemms_enabled() {
   const char* e = getenv("IPTTT_GEMM_CTAS");
   return !(e && e[0] == '1');
+}
+
+// Whether this call scans its chunks in groups: the layout allows it and the
+// within-group products can run (CTA pairs).
+bool scan_grouped(const Layout& L, cudaStream_t st) {
+  return L.grouped && pair_gemms_enabled() && tck::pair_gemm_workers(st) > 0;
 }
 
 ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, const Layout& L, StreamState* ss,
@@ -315,17 +370,38 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   // A context-parallel finish reuses everything its begin left in the workspace.
   const bool cp_finish = cp && cp->stage == kCpFinish;
 
+  // Gate/up and target GEMMs on CTA pairs (256-row tiles) where the device runs
+  // clusters of two, else one CTA per 128-row tile.  On pairs the masked conv is
+  // computed inside the target GEMM (U never reaches HBM); otherwise a conv kernel
+  // writes U first.
+  const bool pair_gemm = pair_gemms_enabled() && pair_gemm_workers(st) > 0;
+  const bool fused_target = pair_gemm && fused_target_supported(s.d) && fused_target_workers(st) > 0;
+  // the grouped scan's within-group products run on CTA pairs
+  const bool grouped = scan_grouped(L, st);
+  Shape gs = s;
+  gs.C = kGroupTokens;
+  gs.k = (s.T + kGroupTokens - 1) / kGroupTokens;
+  const Shape& sq = grouped ? gs : s;  // the chunking of the scan
+  ChunkMeta* gmeta = grouped ? reinterpret_cast<ChunkMeta*>(ws + L.gmeta) : meta;
+  uint8_t* glo = ws + L.glo;
+  void* Pw = ws + L.P;
+  void* Ew = ws + L.E;
   if (!cp_finish) {
     PhaseScope ph(st, PH_PREP);
     IP_CHECK(aux::build_meta(flags, meta, s, t.doc, t.n_doc, ss ? ss->cont : cp ? cp->plan : nullptr, di->status,
                              st));
     counted(3);
-    if (!t.Zin) {
-      IP_CHECK(aux::conv_target(IPTTT_BF16, t.X0, t.cw, flags, U, s, st));
-    } else {
-      IP_CHECK(aux::mask_last_segment(IPTTT_BF16, t.Vin, V, meta, s, st));
+    if (grouped) {
+      IP_CHECK(aux::group_meta(flags, gmeta, glo, gs, st));
+      counted(2);
     }
-    counted(1);
+    if (t.Zin) {
+      IP_CHECK(aux::mask_last_segment(IPTTT_BF16, t.Vin, V, meta, s, st));
+      counted(1);
+    } else if (!fused_target) {
+      IP_CHECK(aux::conv_target(IPTTT_BF16, t.X0, t.cw, flags, U, s, st));
+      counted(1);
+    }
   }
 
   TcParams tp;
@@ -344,9 +420,6 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   tp.alpha = alpha;
   tp.status = di->status;
 
-  // Gate/up and target GEMMs on CTA pairs (256-row tiles) where the device runs
-  // clusters of two, else one CTA per 128-row tile.
-  const bool pair_gemm = pair_gemms_enabled() && pair_gemm_workers(st) > 0;
   const int zv_fam = pair_gemm ? FAM_ZV2 : FAM_ZV;
   const int zv_rows = pair_gemm ? 256 : 128;
   if (!t.Zin && !cp_finish) {
@@ -356,19 +429,31 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     if (!make_map_bf16(&g.map[0], t.H, s.d, s.T, s.B, 64, 128) ||
         !make_map_bf16(&g.map[1], t.Wg, s.d, s.F, 1, 64, 128) ||
         !make_map_bf16(&g.map[2], t.Wu, s.d, s.F, 1, 64, 128))
-      return IPTTT_ERR_CUDA;
+      return cuda_fail("tensor maps of the gate/up GEMM", cudaErrorInvalidValue);
     g.out0 = Z;
     g.n_tiles = s.B * ((s.T + zv_rows - 1) / zv_rows) * (s.F / 128);
     IP_CHECK(launch_tc(zv_fam, g, di->num_sms, st));
     counted(1);
   }
-  if (!t.Zin && !cp_finish) {
+  if (!t.Zin && !cp_finish && fused_target) {
+    PhaseScope ph(st, PH_TARGET);
+    TcParams v = tp;
+    if (!make_map_bf16(&v.map[0], t.Wt, s.d, s.d, 1, 64, 64))
+      return cuda_fail("tensor map of the fused target GEMM", cudaErrorInvalidValue);
+    v.src0 = t.X0;
+    v.src1 = t.cw;
+    v.flags = flags;
+    v.out0 = V;
+    v.n_tiles = s.B * ((s.T + 255) / 256) * ((s.d + 511) / 512);
+    IP_CHECK(launch_fused_target(v, st));
+    counted(1);
+  } else if (!t.Zin && !cp_finish) {
     PhaseScope ph(st, PH_TARGET);
     TcParams v = tp;
     v.kind = kind_vhat();
     if (!make_map_bf16(&v.map[0], U, s.d, s.T, s.B, 64, 128) ||
         !make_map_bf16(&v.map[1], t.Wt, s.d, s.d, 1, 64, pair_gemm ? 128 : 64))
-      return IPTTT_ERR_CUDA;
+      return cuda_fail("tensor maps of the target GEMM", cudaErrorInvalidValue);
     v.out0 = V;
     v.vn = s.d % 256 == 0 ? 256 : 128;
     v.n_tiles = s.B * ((s.T + zv_rows - 1) / zv_rows) * (s.d / v.vn);
@@ -390,7 +475,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     }
     if (!make_map_bf16(&g.map[0], Z, s.F, s.T, s.B, 64, gram2 ? 128 : tp.tr) ||
         !make_map_bf16(&g.map[1], V, s.d, s.T, s.B, 64, gram2 ? 128 : tp.tr))
-      return IPTTT_ERR_CUDA;
+      return cuda_fail("tensor maps of the Gram pass", cudaErrorInvalidValue);
     g.partials = partials;
     g.n_tiles = s.B * s.k * g.npairs;
     IP_CHECK(launch_tc(gram2 ? FAM_GRAM2 : FAM_GRAM, g, di->num_sms, st));
@@ -399,6 +484,28 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     // the state update accumulates alpha eta V^T Z: fold alpha eta into V's rows
     IP_CHECK(aux::prescale_target(V, alpha, s, p.eta, st));
     counted(3);
+  }
+  if (grouped && !cp_finish) {
+    // within-group term: P = masked Z Z^T per group of 256 tokens, then E = P V'
+    PhaseScope ph(st, PH_APPLY);
+    TcParams z = tp;
+    if (!make_map_bf16(&z.map[0], Z, s.F, s.T, s.B, 64, 128))
+      return cuda_fail("tensor map of the within-group products", cudaErrorInvalidValue);
+    z.glo = glo;
+    z.cs = s.C;
+    z.out0 = Pw;
+    z.n_tiles = s.B * gs.k;
+    IP_CHECK(launch_tc(FAM_PZ, z, di->num_sms, st));
+    TcParams e = tp;
+    e.kind = kind_intra();
+    e.vn = s.d % 256 == 0 ? 256 : 128;
+    if (!make_map_bf16(&e.map[0], Pw, kGroupTokens, s.T, s.B, 64, 128) ||
+        !make_map_bf16(&e.map[1], V, s.d, s.T, s.B, 64, 128))
+      return cuda_fail("tensor maps of the within-group term", cudaErrorInvalidValue);
+    e.out0 = Ew;
+    e.n_tiles = s.B * gs.k * (s.d / e.vn);
+    IP_CHECK(launch_tc(FAM_ZV2, e, di->num_sms, st));
+    counted(2);
   }
   if (t.alpha) IP_CHECK(cudaMemcpyAsync(t.alpha, alpha, (size_t)s.B * s.k * 4, cudaMemcpyDeviceToDevice, st));
 
@@ -421,15 +528,23 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   // then the update of chunk b-1 (writes S_b into the slot S_a has left).
   const int G = L.group;
   TcParams sc = tp;
-  const int arows = apply_rows(p);
+  if (grouped) {
+    sc.C = gs.C;
+    sc.k = gs.k;
+    sc.tr = tile_rows(group_params(p));
+    sc.meta = gmeta;
+    sc.upd_kb = update_tokens_per_stage(s.C);  // a stage never spans two chunks of the group
+    sc.intra = Ew;
+  }
+  const int arows = grouped ? apply_rows(group_params(p)) : apply_rows(p);
   const int apply_fam = arows == 256 ? FAM_APPLY256 : FAM_APPLY;
-  if (!make_map_bf16(&sc.map[0], Z, s.F, s.T, s.B, 64, arows == 256 ? 128 : tp.tr) ||
+  if (!make_map_bf16(&sc.map[0], Z, s.F, s.T, s.B, 64, arows == 256 ? 128 : sc.tr) ||
       (t.W0 && !make_map_bf16(&sc.map[1], t.W0, s.F, s.d, 1, 64, 128)) ||  // no W0: a context-parallel begin
       !make_map_bf16(&sc.map[2], snap, s.F, s.d, (uint64_t)G * s.B, 64, 128) ||
       !make_map_bf16(&sc.map[3], V, s.d, s.T, s.B, 64, update_tokens_per_stage(s.C)) ||
       !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, update_tokens_per_stage(s.C)) ||
       !make_map_bf16(&sc.map[5], snap, s.F, s.d, (uint64_t)G * s.B, 64, 32))
-    return IPTTT_ERR_CUDA;
+    return cuda_fail("tensor maps of the chunk scan", cudaErrorInvalidValue);
   sc.out0 = t.O;
   sc.out1 = t.D;
   sc.resid = (p.flags & IPTTT_FLAG_RESIDUAL) ? t.H : nullptr;
@@ -438,7 +553,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   sc.dchunks = 1;
   const bool need_final = t.Sfinal != nullptr || ss != nullptr;
   const int state_tiles = s.B * (s.d / 128) * ((s.F + 255) / 256);  // 128 x 256 tiles
-  const int apply_tiles_per_chunk = s.B * (s.C / arows) * (s.d / 128);
+  const int apply_tiles_per_chunk = s.B * (sq.C / arows) * (s.d / 128);
   // State updates of chunks [c0, c1) in one launch: each block keeps its state
   // tiles in TMEM through all of them and writes S_{c+1} snapshots into slot
   // (c+1) % G.
@@ -458,7 +573,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     // begin: every chunk's update in one launch, S_1 .. S_k into slots 1 .. k and
     // the shard's aggregate left in the state.  finish: the incoming state into
     // S_0 .. S_{prefix-1} (and S_final), then the apply of all k chunks.
-    if (!cp_finish) return update(0, s.k);
+    if (!cp_finish) return update(0, sq.k);
     {
       PhaseScope ph(st, PH_UPDATE);
       IP_CHECK(aux::cp_combine(cp->gathered, cp->world, cp->rank, cp->plan, snap, G, cp->Sfinal, s, st));
@@ -469,7 +584,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     q.chunk = 0;
     q.dchunks = 1;
     q.apply_chunk0 = 0;
-    q.n_tiles = s.k * apply_tiles_per_chunk;
+    q.n_tiles = sq.k * apply_tiles_per_chunk;
     IP_CHECK(launch_tc(apply_fam, q, di->num_sms, st));
     counted(1);
     return IPTTT_OK;
@@ -477,8 +592,8 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   // Group [a, b) of G chunks: the updates of chunks a-1 .. b-2 produce S_a .. S_{b-1}
   // (ring slots a % G .. (b-1) % G, which the previous group's applies have
   // finished reading), then one launch applies chunks a .. b-1.
-  for (int a = 0; a < s.k; a += G) {
-    const int b = std::min(a + G, s.k);
+  for (int a = 0; a < sq.k; a += G) {
+    const int b = std::min(a + G, sq.k);
     if ((rc_ = update(std::max(a - 1, 0), b - 1)) != IPTTT_OK) return rc_;
     PhaseScope ph(st, PH_APPLY);
     TcParams q = sc;
@@ -489,7 +604,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     IP_CHECK(launch_tc(apply_fam, q, di->num_sms, st));
     counted(1);
   }
-  if (need_final && (rc_ = update(s.k - 1, s.k)) != IPTTT_OK) return rc_;
+  if (need_final && (rc_ = update(sq.k - 1, sq.k)) != IPTTT_OK) return rc_;
   if (t.Sfinal) {
     IP_CHECK(aux::state_export(true, S, t.Sfinal, s, st));
     counted(1);
@@ -611,8 +726,9 @@ ipttt_status run(const ipttt_params* pp, const Tensors& t, void* workspace, size
     ssp = &ss;
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  g_err_detail[0] = 0;
   rc = is_bf16(p) ? run_bf16(p, t, ws, L, ssp, di, st) : run_f32(p, t, ws, L, ssp, di, st);
-  if (rc == IPTTT_OK && cudaPeekAtLastError() != cudaSuccess) rc = IPTTT_ERR_CUDA;
+  if (rc == IPTTT_OK && cudaPeekAtLastError() != cudaSuccess) rc = cuda_fail("kernel launch", cudaGetLastError());
   return rc;
 }
 
@@ -766,6 +882,14 @@ ipttt_status cp_run(const ipttt_params* p, int32_t world, int32_t rank, const in
   if ((rc = device_info(&di)) != IPTTT_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (scan_grouped(L, static_cast<cudaStream_t>(stream))) {
+    // the incoming state reaches the groups up to the one holding the shard's
+    // first document start (the plan counts chunks)
+    for (int32_t b = 0; b < p->B; ++b) {
+      int32_t& pre = plan[2 * (size_t)p->B + b];
+      if (pre > 0) pre = (int32_t)(((long long)(pre - 1) * p->C) / kGroupTokens + 1);
+    }
+  }
   int32_t* plan_dev = reinterpret_cast<int32_t*>(ws + L.cp_plan);
   int32_t* docs_dev = reinterpret_cast<int32_t*>(ws + L.cp_docs);
   // pageable sources: the copies have taken the bytes when they return
@@ -778,8 +902,9 @@ ipttt_status cp_run(const ipttt_params* p, int32_t world, int32_t rank, const in
   cp.world = world;
   cp.rank = rank;
   cp.plan = plan_dev;
+  g_err_detail[0] = 0;
   rc = run_bf16(*p, tt, ws, L, nullptr, di, st, &cp);
-  if (rc == IPTTT_OK && cudaPeekAtLastError() != cudaSuccess) rc = IPTTT_ERR_CUDA;
+  if (rc == IPTTT_OK && cudaPeekAtLastError() != cudaSuccess) rc = cuda_fail("kernel launch", cudaGetLastError());
   return rc;
 }
 }  // namespace
@@ -851,7 +976,9 @@ const char* ipttt_strerror(ipttt_status s) {
   return "unknown status";
 }
 
-const char* ipttt_version(void) { return "0.1.0"; }
+const char* ipttt_version(void) { return "0.2.0"; }
+
+const char* ipttt_last_error_detail(void) { return g_err_detail; }
 
 }  // extern "C"
 

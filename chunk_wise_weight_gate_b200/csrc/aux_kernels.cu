@@ -578,6 +578,34 @@ __global__ void k_prescale(__nv_bfloat16* V, const float* alpha, int B, int Tn, 
   }
 }
 
+// One block of 256 threads per (row, group of 256 tokens): thread i holds token
+// g0 + i; an inclusive max-scan of (start flag ? i : 0) gives the offset of the
+// last document start at or before the token inside the group (0 if none).
+__global__ void __launch_bounds__(256) k_group_lo(const uint8_t* flags, uint8_t* glo, int Tn, int groups) {
+  __shared__ int wmax[8];
+  const int b = blockIdx.x / groups, g = blockIdx.x % groups;
+  const int i = threadIdx.x, t = g * 256 + i;
+  const int lane = i & 31, w = i >> 5;
+  int v = (t < Tn && flags[(size_t)b * Tn + t]) ? i : 0;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v = max(v, u);
+  }
+  if (lane == 31) wmax[w] = v;
+  __syncthreads();
+  int pre = 0;
+  for (int q = 0; q < w; ++q) pre = max(pre, wmax[q]);
+  v = max(v, pre);
+  if (t < Tn) glo[(size_t)b * Tn + t] = (uint8_t)v;
+}
+
+cudaError_t group_meta(const uint8_t* flags, ChunkMeta* gmeta, uint8_t* glo, const Shape& gs, cudaStream_t st) {
+  k_chunk_meta<<<gs.B * gs.k, 256, 0, st>>>(flags, gmeta, gs.B, gs.T, gs.C, gs.k);
+  k_group_lo<<<gs.B * gs.k, 256, 0, st>>>(flags, glo, gs.T, gs.k);
+  return cudaGetLastError();
+}
+
 cudaError_t prescale_target(void* V, const float* alpha, const Shape& s, float eta, cudaStream_t st) {
   k_prescale<<<148 * 8, 256, 0, st>>>((__nv_bfloat16*)V, alpha, s.B, s.T, s.d, s.C, s.k, eta);
   return cudaGetLastError();

@@ -22,11 +22,14 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t elem_bytes(const ipttt_params& p) { return p.dtype == IPTTT_BF16 ? 2 : 4; }
 
-// Piece length: the caller's, else about an eighth of the sequence in whole chunks.
+// Piece length: the caller's, else about an eighth of the sequence in whole scan
+// steps (chunks, or groups of chunks), which keeps the result bit-identical to one
+// call over the whole sequence.
 int32_t piece_tokens_of(const ipttt_params& p, int32_t piece) {
   if (piece > 0) return piece;
-  const int32_t k = (p.T + p.C - 1) / p.C;
-  return std::max<int32_t>(1, k / 8) * p.C;
+  const int32_t unit = ipttt::scan_unit_tokens(p);
+  const int32_t k = (p.T + unit - 1) / unit;
+  return std::max<int32_t>(1, k / 8) * unit;
 }
 
 struct HostLayout {

@@ -27,8 +27,9 @@
 //            工程实现; iplexlaw.co.kr review §3: a chunk's output comes from the
 //            pre-update state].
 // The state update S_{i+1} = keep_i S_i + alpha_i eta V_i^T Z_i runs in its own
-// kernel (upd_kernel, below): each worker keeps two fp32 state tiles in TMEM as
-// live accumulators and walks them through a group of chunks [notes, 步骤二 and the
+// kernel (upd_kernel, below): the MMAs form each chunk's delta from zero in TMEM,
+// and the epilogue warps hold the fp32 state of one tile in registers and add the
+// deltas to it, walking the tile through a group of chunks [notes, 步骤二 and the
 // Hebbian rule; iplexlaw.co.kr review §6 exclusive scan and document reset].
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -51,9 +52,8 @@ constexpr int A_BYTES = BM * BK * 2;    // 16 KB
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int NTHREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr int ACC_COLS = 256;           // per accumulator buffer
-constexpr int SNAP_BOX_BYTES = 32 * 128;     // 32 rows x 64 bf16 columns (one warp's snapshot box)
 
-enum Kind { K_GATEUP = 0, K_VHAT = 1, K_GRAM = 2, K_APPLY = 3 };
+enum Kind { K_GATEUP = 0, K_VHAT = 1, K_GRAM = 2, K_APPLY = 3, K_INTRA = 4 };
 
 // Per family: pipeline stages, bytes per stage, K elements per stage (KB), offset
 // of the B operand inside a stage, and shared memory for the epilogue.
@@ -87,9 +87,17 @@ template <> struct Cfg<FAM_GRAM2> {
   static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 128, B_OFF = 2 * A_BYTES, EPI_BYTES = 0,
                        NBUF = 1;
 };
+// Within-group products of the grouped scan: one 256 x 256 accumulator per group,
+// two of them in TMEM (the epilogue of one overlaps the MMAs of the next).
+template <> struct Cfg<FAM_PZ> {
+  static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 128, B_OFF = 2 * A_BYTES, EPI_BYTES = 0,
+                       NBUF = 2;
+};
 template <int FAM> constexpr bool is_apply() { return FAM == FAM_APPLY || FAM == FAM_APPLY256; }
 template <int FAM> constexpr bool is_zv() { return FAM == FAM_ZV || FAM == FAM_ZV2; }
-template <int FAM> constexpr bool is_pair() { return FAM == FAM_ZV2 || FAM == FAM_GRAM2; }
+template <int FAM> constexpr bool is_pair() { return FAM == FAM_ZV2 || FAM == FAM_GRAM2 || FAM == FAM_PZ; }
+// token-block families: A and B rows both come from the tile's own tokens
+template <int FAM> constexpr bool is_tokblk() { return FAM == FAM_GRAM || FAM == FAM_GRAM2 || FAM == FAM_PZ; }
 template <int FAM> constexpr bool is_gram() { return FAM == FAM_GRAM || FAM == FAM_GRAM2; }
 
 template <int FAM>
@@ -216,7 +224,7 @@ __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
     // 128 K per stage; the leader's barrier counts both CTAs' bytes.
     decode_zv<256>(p, tile, j);
     j.halves = 1;
-    j.kb1[0] = p.d / 128;
+    j.kb1[0] = (p.kind == K_INTRA ? 256 : p.d) / 128;  // K: d, or the group's 256 tokens
     j.tx = 2 * (128 * 128 * 2 + (j.n_mma / 2) * 128 * 2);
   }
   else if constexpr (FAM == FAM_GRAM) decode_gram(p, tile, j);
@@ -228,6 +236,23 @@ __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
     j.acc_col[1] = 256;
     j.n_mma = 256;
     j.tx = 2 * (2 * 128 * 128 * 2);
+  }
+  else if constexpr (FAM == FAM_PZ) {
+    // one group of 256 tokens of one row: its rows against its columns, K = d_ff
+    const int groups = cdiv(p.T, 256);
+    j.kind = K_GRAM;
+    j.b = tile / groups;
+    j.t0 = (tile % groups) * 256;
+    j.m0 = j.n0 = 0;
+    j.chunk = j.pair = 0;
+    j.nseg = 1;
+    j.kb0[0] = 0;
+    j.kb1[0] = p.F / 128;
+    j.acc_col[0] = 0;
+    j.n_mma = 256;
+    j.nsrc = 1;
+    j.tx = 2 * (2 * 128 * 128 * 2);
+    j.a_mn = j.b_mn = false;
   }
   else if constexpr (FAM == FAM_APPLY) decode_apply<0>(p, tile, j);
   else decode_apply<256>(p, tile, j);
@@ -253,11 +278,11 @@ __device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int
     const uint32_t r = cluster_rank();
     const uint32_t fb = map_to_rank(smem_u32(bar), 0);
     const int k0 = kb * 128;
-    const int arow = (is_gram<FAM>() ? j.t0 : 0) + j.m0 + 128 * (int)r;
+    const int arow = (is_tokblk<FAM>() ? j.t0 : 0) + j.m0 + 128 * (int)r;
     const CUtensorMap* am = is_gram<FAM>() && seg == 1 ? &p.map[1] : &p.map[0];   // Gram: Z, then V
     tma_load_3d_pair(sa, am, fb, k0, arow, j.b);
     tma_load_3d_pair(sa + A_BYTES, am, fb, k0 + 64, arow, j.b);
-    if constexpr (is_gram<FAM>()) {                                 // rows of the other token block
+    if constexpr (is_tokblk<FAM>()) {                               // rows of the other token block
       const int brow = j.t0 + j.n0 + 128 * (int)r;
       tma_load_3d_pair(sb, am, fb, k0, brow, j.b);
       tma_load_3d_pair(sb + 128 * BK * 2, am, fb, k0 + 64, brow, j.b);
@@ -266,9 +291,12 @@ __device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int
       tma_load_3d_pair(sb, wm, fb, k0, j.n0, 0);
       tma_load_3d_pair(sb + 128 * BK * 2, wm, fb, k0 + 64, j.n0, 0);
     } else {
-      const int nh = p.vn / 2;                                     // Wtarget[k][n], n contiguous
+      // Wtarget[k][n] (or, within-group term, V'[b][group token k][n]), n contiguous
+      const int nh = p.vn / 2;
+      const bool intra = j.kind == K_INTRA;
       for (int q = 0; q < nh / 64; ++q)
-        tma_load_3d_pair(sb + q * 64 * 128 * 2, &p.map[1], fb, j.n0 + (int)r * nh + 64 * q, k0, 0);
+        tma_load_3d_pair(sb + q * 64 * 128 * 2, &p.map[1], fb, j.n0 + (int)r * nh + 64 * q, (intra ? j.m0 : 0) + k0,
+                         intra ? j.b : 0);
     }
   } else if constexpr (is_zv<FAM>()) {
     if (j.kind == K_GATEUP) {
@@ -345,7 +373,9 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
       }
     } else {
       const int chunk = t / p.C;
-      const bool keep = valid && t >= p.meta[(size_t)j.b * p.k + min(chunk, p.k - 1)].last_start;
+      // the target keeps the rows of each chunk's last document segment; the
+      // within-group term keeps every row
+      const bool keep = valid && (j.kind == K_INTRA || t >= p.meta[(size_t)j.b * p.k + min(chunk, p.k - 1)].last_start);
       __nv_bfloat16* vrow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.d + j.n0;
       const int w = p.vn / 2;  // columns drained by this warp
 #pragma unroll 1
@@ -356,6 +386,26 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
         for (int i = 0; i < 32; ++i) v[i] = keep ? __uint_as_float(r0[i]) : 0.0f;
         if (valid) st_bf16x32(vrow + c, v);
       }
+    }
+  } else if constexpr (FAM == FAM_PZ) {
+    // Row t of the group (this CTA's 128, j.m0 holds the CTA's offset) against
+    // columns u of [128 half, 128 half + 128): z_t . z_u is kept where u lies in
+    // t's document (u >= lo(t)) and in an earlier chunk (u < the start of t's chunk).
+    const int t = j.t0 + j.m0 + row;
+    const bool valid = t < p.T;
+    const int lo = valid ? j.t0 + (int)p.glo[(size_t)j.b * p.T + t] : 0;
+    const int hi = valid ? (t / p.cs) * p.cs : 0;
+    __nv_bfloat16* prow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * 256;
+#pragma unroll 1
+    for (int c = half * 128; c < half * 128 + 128; c += 32) {
+      tmem_ld32(tacc + c, r0);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int u = j.t0 + c + i;
+        v[i] = (u >= lo && u < hi) ? __uint_as_float(r0[i]) : 0.0f;
+      }
+      if (valid) st_bf16x32(prow + c, v);
     }
   } else if constexpr (FAM == FAM_GRAM2) {
     // This CTA's 128 rows of the 256 x 256 block pair; warp half h sums columns
@@ -422,14 +472,35 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
     const __nv_bfloat16* hrow =
         p.resid ? reinterpret_cast<const __nv_bfloat16*>(p.resid) + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
     float* drow = p.out1 ? p.out1 + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
+    const __nv_bfloat16* erow =
+        p.intra ? reinterpret_cast<const __nv_bfloat16*>(p.intra) + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
 #pragma unroll 1
     for (int c = c_begin; c < c_end; c += 32) {
       tmem_ld32(tacc + c, r0);
       if (j.nsrc == 2) tmem_ld32(tacc + 128 + c, r1);
       tmem_ld_wait();
+      float e[32];
+      if (erow && valid) {
+        // the grouped scan's within-group term joins the fast-weight part
+        const uint4* e4 = reinterpret_cast<const uint4*>(erow + c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 ev = e4[q];
+          const uint32_t ew4[4] = {ev.x, ev.y, ev.z, ev.w};
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&ew4[x]);
+            e[8 * q + 2 * x] = __low2float(h2);
+            e[8 * q + 2 * x + 1] = __high2float(h2);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) e[i] = 0.0f;
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float dv = carry ? __uint_as_float(r1[i]) : 0.0f;
+        const float dv = (carry ? __uint_as_float(r1[i]) : 0.0f) + e[i];
         v[i] = __uint_as_float(r0[i]) + dv;
         r1[i] = __float_as_uint(dv);
       }
@@ -501,7 +572,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    const int nmaps = is_apply<FAM>() ? 3 : (is_gram<FAM>() ? 2 : (p.kind == K_GATEUP ? 3 : 2));
+    const int nmaps = is_apply<FAM>() ? 3 : FAM == FAM_PZ ? 1 : (is_gram<FAM>() ? 2 : (p.kind == K_GATEUP ? 3 : 2));
     for (int i = 0; i < nmaps; ++i) prefetch_tmap(&p.map[i]);
   }
   if (warp == 1) {
@@ -653,13 +724,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
 
 // ------------------------------------------------------------------ state update
 // S_{c+1} = keep_c S_c + alpha_c eta V_c^T Z_c for the chunks c of one launch.
-// V arrives pre-scaled by alpha_c eta per row, so the MMAs accumulate the state
-// itself: the fp32 state tiles live in TMEM (slots 0 and 1, 256 columns each)
-// and are walked through all chunks of the launch, the two slots alternating, so
-// that the epilogue reads one slot (bf16 snapshot of S_{c+1} for the apply) while
-// the MMAs run on the other.  A chunk holding a document start resets the tile
-// (its first MMA does not accumulate).  A tile's fp32 state comes in from HBM
-// before its first chunk (tcgen05.st) and goes back after its last.
+// V arrives pre-scaled by alpha_c eta per row.  The MMAs form each chunk's delta
+// from zero in one of two TMEM slots (256 fp32 columns each, taken in turn chunk
+// by chunk), so the tensor cores never add a small delta onto a large running
+// sum.  The fp32 state of the worker's current tile lives in the registers of
+// the epilogue warps (one TMEM lane row, 128 columns per thread) and takes each
+// delta with an ordinary fp32 add, rounded to nearest.  While the epilogue folds
+// chunk c's delta and writes the bf16 snapshot of S_{c+1} for the apply, the MMAs
+// of chunk c+1 fill the other slot.  A chunk holding a document start drops the
+// carried state before its delta is added.  A tile's fp32 state comes in from HBM
+// before its first chunk of the launch and goes back after its last.
 //
 // Two forms of one kernel body:
 //   PAIR = false: one CTA per 128 (d) x 256 (F) state tile, M=128 MMAs.
@@ -669,6 +743,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
 //                 n0 + 128 r .. +127 per stage; the even CTA issues the MMAs.  Per
 //                 FLOP this moves 2/3 of the operand bytes of the single-CTA form.
 constexpr int UPD_BOX_BYTES = 32 * 128;               // a warp's 32-row x 64-column snapshot box
+// Three warpgroups: warps 0-7 the epilogue (each thread holds 128 fp32 state
+// values), warp 8 the TMA producer, warp 9 the MMA issuer, warps 10-11 idle.
+// Twelve warps put three on each SM sub-partition, which caps a thread at 168
+// registers at launch; the third warpgroup then drops to UPD_REGS_LOW and the two
+// epilogue warpgroups rise to UPD_REGS_EPI, an exact trade:
+// 128 x (168 - 56) = 256 x (224 - 168).  The launcher checks that the kernel was
+// compiled to 168 registers, the count this balance assumes.
+constexpr int UPD_THREADS = 384;
+constexpr int UPD_WARP_TMA = 8, UPD_WARP_MMA = 9;
+constexpr int UPD_REGS_LAUNCH = 168, UPD_REGS_LOW = 56, UPD_REGS_EPI = 224;
+static_assert((UPD_THREADS - 32 * NUM_EPI_WARPS) * (UPD_REGS_LAUNCH - UPD_REGS_LOW) ==
+                  32 * NUM_EPI_WARPS * (UPD_REGS_EPI - UPD_REGS_LAUNCH),
+              "the register trade of the update kernel must balance");
 
 // KB tokens per stage: 128 (8 MMAs per stage; the per-stage issue overhead is
 // paid half as often) when the chunk length is a multiple of 128, else 64 (a
@@ -689,41 +776,25 @@ static_assert(UpdCfg<false, 64>::SMEM <= 232448 && UpdCfg<true, 64>::SMEM <= 232
 
 struct UpdJob {
   int X;      // state tile: (b, nt2, mt) of B x ceil(F/256) x (d/TILE_ROWS), mt fastest
+  int c;      // chunk of the launch, 0 .. dchunks-1
   int chunk;  // absolute chunk index
-  int slot;   // TMEM slot 0 or 1
   int b, m0, n0;
 };
 
 // Job i of worker w (a CTA, or a CTA pair) of nw, or false past the end.  The
-// worker's tiles are X_m = w + m nw, taken in pairs (X_2m on slot 0, X_2m+1 on
-// slot 1); a pair is walked chunk by chunk, both tiles per chunk.
+// worker's tiles are X_m = w + m nw; each is walked through every chunk of the
+// launch before the next.  The delta of job i goes to TMEM slot i % 2.
 template <bool PAIR>
 __device__ __forceinline__ bool upd_job(const TcParams& p, uint32_t i, int w, int nw, UpdJob& jb) {
-  const int D = p.dchunks;
-  const int nX = p.n_tiles;
-  if (w >= nX) return false;
-  const int nXc = (nX - w + nw - 1) / nw;
-  const int pairs = nXc / 2;
-  const uint32_t in_pairs = (uint32_t)pairs * D * 2;
-  int m, c, sl;
-  if (i < in_pairs) {
-    m = (int)(i / (2u * D));
-    const int r = (int)(i % (2u * D));
-    c = r / 2;
-    sl = r % 2;
-  } else {
-    const uint32_t r = i - in_pairs;
-    if ((nXc & 1) == 0 || r >= (uint32_t)D) return false;
-    m = pairs;
-    c = (int)r;
-    sl = 0;
-  }
-  jb.X = w + (2 * m + sl) * nw;
-  jb.chunk = p.chunk + c;
-  jb.slot = sl;
-  // Row blocks vary fastest: the tiles in flight at one time (about two per
-  // worker) then cover few column blocks, so each chunk's Z columns come from DRAM
-  // about once (V, four times smaller, once per tile group).
+  const uint32_t D = (uint32_t)p.dchunks;
+  const long long X = (long long)w + (long long)(i / D) * nw;
+  if (X >= p.n_tiles) return false;
+  jb.X = (int)X;
+  jb.c = (int)(i % D);
+  jb.chunk = p.chunk + jb.c;
+  // Row blocks vary fastest: the tiles in flight at one time (one per worker)
+  // then cover few column blocks, so each chunk's Z columns come from DRAM about
+  // once per launch (V, four times smaller, once per round of tiles).
   const int nt2s = (p.F + 255) / 256;
   const int mts = p.d / (PAIR ? 256 : 128);
   const int per_row = mts * nt2s;
@@ -734,25 +805,17 @@ __device__ __forceinline__ bool upd_job(const TcParams& p, uint32_t i, int w, in
   return true;
 }
 
-template <bool PAIR>
-__device__ __forceinline__ bool upd_next_on_slot(const TcParams& p, uint32_t i, int w, int nw, int slot,
-                                                 UpdJob& jn) {
-  for (uint32_t k = 1; k <= 2; ++k) {
-    if (!upd_job<PAIR>(p, i + k, w, nw, jn)) return false;
-    if (jn.slot == slot) return true;
-  }
-  return false;
-}
-
 // fp32 state, 128 x 128 blocked tiles; tile column block h of the 128-row block
-// starting at d row m0 (a multiple of 128).
+// starting at d row m0 (a multiple of 128).  Inside a block, element (row, c) sits
+// at float4 index (c / 4) * 128 + row, so a warp holding 32 consecutive rows moves
+// 512 contiguous bytes per float4 column.
 __device__ __forceinline__ float4* upd_state_block(const TcParams& p, int b, int m0, int n0, int h) {
   return reinterpret_cast<float4*>(p.S + (size_t)b * p.d * p.F +
                                    ((size_t)(m0 / 128) * (p.F / 128) + n0 / 128 + h) * (128 * 128));
 }
 
 template <bool PAIR, int KB>
-__global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_constant__ TcParams p) {
   using Cf = UpdCfg<PAIR, KB>;
   constexpr int STAGES = Cf::STAGES;
   constexpr int UPD_KB = KB;
@@ -764,9 +827,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
   uint64_t* bars = reinterpret_cast<uint64_t*>(boxes + NUM_EPI_WARPS * UPD_BOXES * UPD_BOX_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
-  uint64_t* st_ready = empty + STAGES;  // [2] epilogue -> MMA: slot holds the state to accumulate on
-  uint64_t* st_done = st_ready + 2;     // [2] MMA -> epilogue: the chunk's MMAs on the slot finished
-  uint64_t* drain = st_done + 2;
+  uint64_t* slot_free = empty + STAGES;  // [2] epilogue -> MMA: the slot's delta has been read
+  uint64_t* slot_full = slot_free + 2;   // [2] MMA -> epilogue: the chunk's delta is complete
+  uint64_t* drain = slot_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* counters = reinterpret_cast<uint32_t*>(tmem_slot + 2);
@@ -784,20 +847,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
       mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&st_ready[s], NUM_EPI_WARPS * (PAIR ? 2 : 1));
-      mbar_init(&st_done[s], 1);
+      mbar_init(&slot_free[s], NUM_EPI_WARPS * (PAIR ? 2 : 1));
+      mbar_init(&slot_full[s], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     counters[0] = counters[1] = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == UPD_WARP_TMA && lane == 0) {
     prefetch_tmap(&p.map[3]);
     prefetch_tmap(&p.map[4]);
     prefetch_tmap(&p.map[5]);
   }
-  if (warp == 1) {
+  if (warp == UPD_WARP_MMA) {
     if constexpr (PAIR) {
       tmem_alloc_pair(tmem_slot, 2 * ACC_COLS);
       tmem_relinquish_pair();
@@ -811,205 +874,189 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      uint32_t it = 0;
-      bool ok = true;
-      UpdJob jb;
-      const uint32_t full0 = PAIR ? map_to_rank(smem_u32(full), 0) : 0u;  // the leader's full[0]
-      for (uint32_t i = 0; ok && upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
-        const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
-        const int t0 = jb.chunk * p.C;
-        const int kb0 = (m.last_start - t0) / UPD_KB;
-        const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) { ok = false; break; }
-          uint8_t* sa = stages + s * Cf::STAGE_BYTES;
-          uint8_t* sb = sa + Cf::A_BYTES;
-          const int ty = t0 + kb * UPD_KB;
-          if constexpr (PAIR) {
-            // both CTAs' bytes complete the leader's barrier; the leader arms it
-            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cf::STAGE_BYTES);
-            const uint32_t fb = full0 + 8u * s;
-            tma_load_3d_pair(sa, &p.map[3], fb, jb.m0 + rofs, ty, jb.b);             // V[t][d], d contiguous
-            tma_load_3d_pair(sa + 64 * UPD_KB * 2, &p.map[3], fb, jb.m0 + rofs + 64, ty, jb.b);
-            tma_load_3d_pair(sb, &p.map[4], fb, jb.n0 + rofs, ty, jb.b);             // Z[t][f], f contiguous
-            tma_load_3d_pair(sb + 64 * UPD_KB * 2, &p.map[4], fb, jb.n0 + rofs + 64, ty, jb.b);
-          } else {
-            mbar_arrive_expect_tx(&full[s], Cf::STAGE_BYTES);
-            tma_load_3d(sa, &p.map[3], &full[s], jb.m0, ty, jb.b);
-            tma_load_3d(sa + 64 * UPD_KB * 2, &p.map[3], &full[s], jb.m0 + 64, ty, jb.b);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              tma_load_3d(sb + q * 64 * UPD_KB * 2, &p.map[4], &full[s], jb.n0 + 64 * q, ty, jb.b);
-          }
-        }
-      }
-      if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
-      counters[0] = it;
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
-      uint32_t it = 0, uses0 = 0, uses1 = 0;
-      bool ok = true;
-      UpdJob jb;
-      const uint32_t idesc = idesc_bf16(PAIR ? 256 : 128, 256, true, true);
-      for (uint32_t i = 0; ok && upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
-        const int sl = jb.slot;
-        const uint32_t u = sl ? uses1 : uses0;
-        const bool got = PAIR ? mbar_wait_cluster(&st_ready[sl], u & 1) : mbar_wait(&st_ready[sl], u & 1);
-        if (!got || *abort_flag) { ok = false; break; }
-        tc_fence_after();
-        const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
-        const int t0 = jb.chunk * p.C;
-        const int kb0 = (m.last_start - t0) / UPD_KB;
-        const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
-        const uint32_t tacc = tmem_base + sl * ACC_COLS;
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&full[s], ph) || *abort_flag) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(stages + s * Cf::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + Cf::A_BYTES;
-#pragma unroll
-          for (int ks = 0; ks < UPD_KB / 16; ++ks) {
-            const uint64_t ad = sdesc_sw128(a_addr + ks * 2048, UPD_KB * 128, 1024);
-            const uint64_t bd = sdesc_sw128(b_addr + ks * 2048, UPD_KB * 128, 1024);
-            // A document start inside the chunk drops the carried state.
-            const uint32_t acc = (m.has_start && kb == kb0 && ks == 0) ? 0u : 1u;
-            if constexpr (PAIR) mma_bf16_pair(tacc, ad, bd, idesc, acc);
-            else mma_bf16(tacc, ad, bd, idesc, acc);
-          }
-          if constexpr (PAIR) mma_commit_pair(&empty[s], 3); else mma_commit(&empty[s]);
-        }
-        if (!ok) break;
-        if constexpr (PAIR) mma_commit_pair(&st_done[sl], 3); else mma_commit(&st_done[sl]);
-        if (sl) ++uses1; else ++uses0;
-      }
-      if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
-      counters[1] = it;
-      if constexpr (PAIR) mma_commit_pair(drain, 1); else mma_commit(drain);
-      mbar_wait(drain, 0);
-    }
-  } else {
-    const int ew = warp - 2;
+  if (warp < NUM_EPI_WARPS) {
+    // the epilogue warpgroups take the registers the third warpgroup gives up
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(UPD_REGS_EPI));
+    const int ew = warp;
     const int quarter = warp & 3;   // TMEM lanes this warp may access
     const int half = ew >> 2;       // 128-column half of the 256-column state tile
     const int row = quarter * 32 + lane;
     uint8_t* wboxes = boxes + ew * UPD_BOXES * UPD_BOX_BYTES;
     bool ok = true;
     int stores = 0;
-    uint32_t done0 = 0, done1 = 0;
-    const uint32_t ready0 = PAIR ? map_to_rank(smem_u32(st_ready), 0) : 0u;  // the leader's st_ready[0]
-
-    // Brings tile jb's old state (this CTA's rows) into TMEM slot jb.slot (nothing
-    // when its chunk starts a document: the first MMA then overwrites the slot).
-    auto load_state = [&](const UpdJob& jb) {
-      if (p.meta[(size_t)jb.b * p.k + jb.chunk].has_start) return;
-      if (jb.n0 + 128 * half >= p.F) return;  // past the last column block
-      const float4* src = upd_state_block(p, jb.b, jb.m0 + rofs, jb.n0, half);
-      const uint32_t tcol = tmem_base + jb.slot * ACC_COLS + ((uint32_t)(quarter * 32) << 16) + 128 * half;
-#pragma unroll 1
-      for (int g = 0; g < 4; ++g) {
-        uint32_t r[32];
+    const uint32_t free0 = PAIR ? map_to_rank(smem_u32(slot_free), 0) : 0u;  // the leader's slot_free[0]
+    // This thread's row of the current tile's state: columns 128 half .. +127.
+    float st[128];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 v = src[(8 * g + q) * 128 + row];
-          r[4 * q] = __float_as_uint(v.x);
-          r[4 * q + 1] = __float_as_uint(v.y);
-          r[4 * q + 2] = __float_as_uint(v.z);
-          r[4 * q + 3] = __float_as_uint(v.w);
+    for (int e = 0; e < 128; ++e) st[e] = 0.0f;
+
+    UpdJob jb;
+    for (uint32_t i = 0; upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
+      const int sl = (int)(i & 1);
+      const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
+      const int m0c = jb.m0 + rofs;
+      const bool cols = jb.n0 + 128 * half < p.F;  // this warp's half lies inside the state
+      // what the delta is added to: nothing (a document starts in the chunk: the
+      // carried state is dropped), the state in registers, or (the tile's first
+      // chunk of the launch) the state as the previous launch or the caller left it
+      const int base = m.has_start ? 0 : (jb.c == 0 ? 2 : 1);
+      if (!mbar_wait(&slot_full[sl], (i >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      if (cols) {
+        const uint32_t tcol = tmem_base + sl * ACC_COLS + ((uint32_t)(quarter * 32) << 16) + 128 * half;
+        const float4* src = upd_state_block(p, jb.b, m0c, jb.n0, half);
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          uint32_t r[16];
+          tmem_ld16(tcol + 16 * g, r);
+          float o[16];
+          if (base == 2) {
+            const float* sf = reinterpret_cast<const float*>(src);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) o[q] = sf[((4 * g + q / 4) * 128 + row) * 4 + (q & 3)];
+          }
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const int c = 16 * g + q;
+            const float old = base == 2 ? o[q] : base == 1 ? st[c] : 0.0f;
+            st[c] = old + __uint_as_float(r[q]);
+          }
         }
-        tmem_st32(tcol + 32 * g, r);
       }
-      tmem_st_wait();
-    };
-    auto release = [&](int sl) {
+      // the slot's delta is in registers: the MMAs may overwrite it
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if constexpr (PAIR) mbar_arrive_cluster(ready0 + 8u * sl);
-        else mbar_arrive(&st_ready[sl]);
+        if constexpr (PAIR) mbar_arrive_cluster(free0 + 8u * sl);
+        else mbar_arrive(&slot_free[sl]);
       }
-    };
-
-    UpdJob jb;
-    for (uint32_t i = 0; i < 2; ++i)
-      if (upd_job<PAIR>(p, i, wk, nwk, jb) && (int)i == jb.slot) {
-        load_state(jb);
-        release(jb.slot);
-      }
-    for (uint32_t i = 0; upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
-      const int sl = jb.slot;
-      if (!mbar_wait(&st_done[sl], (sl ? done1 : done0) & 1)) { ok = false; break; }
-      if (sl) ++done1; else ++done0;
-      tc_fence_after();
-      UpdJob jn;
-      const bool has_next = upd_next_on_slot<PAIR>(p, i, wk, nwk, sl, jn);
-      const bool last = !has_next || jn.X != jb.X;  // tile's last chunk of the launch
-      const bool snap = jb.chunk + 1 < p.k;
-      const int m0c = jb.m0 + rofs;
-      if (jb.n0 + 128 * half < p.F) {
-        const uint32_t tcol = tmem_base + sl * ACC_COLS + ((uint32_t)(quarter * 32) << 16) + 128 * half;
-        float4* dst = upd_state_block(p, jb.b, m0c, jb.n0, half);
-#pragma unroll 1
-        for (int bx = 0; bx < 2; ++bx) {  // two 64-column snapshot boxes per warp
+      if (!cols) continue;
+      if (jb.chunk + 1 < p.k) {
+        // bf16 snapshot of S_{chunk+1} (what the apply of chunk+1 reads), two boxes
+        // of 32 rows x 64 columns per warp, 128-byte swizzled for the TMA store
+#pragma unroll
+        for (int bx = 0; bx < 2; ++bx) {
           uint8_t* box = wboxes + (bx % UPD_BOXES) * UPD_BOX_BYTES;
-          if (snap && stores > 0) {
-            // the store issued from this buffer two boxes ago has read it
+          if (stores > 0) {
+            // the store issued from this buffer UPD_BOXES boxes ago has read it
             if (lane == 0) bulk_wait_read<UPD_BOXES - 1>();
             __syncwarp();
           }
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tcol + 64 * bx, r0);
-          tmem_ld32(tcol + 64 * bx + 32, r1);
-          tmem_ld_wait();
 #pragma unroll
-          for (int g2 = 0; g2 < 2; ++g2) {
-            const uint32_t* r = g2 ? r1 : r0;
-            const int g = 2 * bx + g2;
-            if (last) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                dst[(8 * g + q) * 128 + row] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                                           __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
-            }
-            if (snap) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int chunk16 = g2 * 4 + e;  // 16-byte chunk of this row in the 128-byte box row
-                *reinterpret_cast<uint4*>(box + lane * 128 + ((chunk16 ^ (lane & 7)) << 4)) = make_uint4(
-                    pack_bf16(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
-                    pack_bf16(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
-                    pack_bf16(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
-                    pack_bf16(__uint_as_float(r[8 * e + 6]), __uint_as_float(r[8 * e + 7])));
-              }
-            }
+          for (int e = 0; e < 8; ++e) {
+            const int c = 64 * bx + 8 * e;
+            *reinterpret_cast<uint4*>(box + lane * 128 + ((e ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16(st[c], st[c + 1]), pack_bf16(st[c + 2], st[c + 3]),
+                           pack_bf16(st[c + 4], st[c + 5]), pack_bf16(st[c + 6], st[c + 7]));
           }
-          if (snap) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_3d(&p.map[5], box, jb.n0 + 128 * half + 64 * bx, m0c + 32 * quarter,
-                           ((jb.chunk + 1) % p.nslots) * p.B + jb.b);
-              bulk_commit();
-            }
-            ++stores;
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&p.map[5], box, jb.n0 + 128 * half + 64 * bx, m0c + 32 * quarter,
+                         ((jb.chunk + 1) % p.nslots) * p.B + jb.b);
+            bulk_commit();
           }
+          ++stores;
         }
       }
-      if (has_next) {
-        if (jn.X != jb.X) load_state(jn);
-        release(sl);
+      if (jb.c == p.dchunks - 1) {
+        // the tile's last chunk of the launch: the fp32 state goes back to HBM
+        float4* dst = upd_state_block(p, jb.b, m0c, jb.n0, half);
+        float* df = reinterpret_cast<float*>(dst);
+#pragma unroll
+        for (int q = 0; q < 128; ++q) df[((q / 4) * 128 + row) * 4 + (q & 3)] = st[q];
       }
     }
     if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
     if (lane == 0) bulk_wait<0>();
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(UPD_REGS_LOW));
+    if (warp == UPD_WARP_TMA) {
+      if (lane == 0) {
+        uint32_t it = 0;
+        bool ok = true;
+        UpdJob jb;
+        const uint32_t full0 = PAIR ? map_to_rank(smem_u32(full), 0) : 0u;  // the leader's full[0]
+        for (uint32_t i = 0; ok && upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
+          const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
+          const int t0 = jb.chunk * p.C;
+          const int kb0 = (m.last_start - t0) / UPD_KB;
+          const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
+          for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) { ok = false; break; }
+            uint8_t* sa = stages + s * Cf::STAGE_BYTES;
+            uint8_t* sb = sa + Cf::A_BYTES;
+            const int ty = t0 + kb * UPD_KB;
+            if constexpr (PAIR) {
+              // both CTAs' bytes complete the leader's barrier; the leader arms it
+              if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cf::STAGE_BYTES);
+              const uint32_t fb = full0 + 8u * s;
+              tma_load_3d_pair(sa, &p.map[3], fb, jb.m0 + rofs, ty, jb.b);             // V[t][d], d contiguous
+              tma_load_3d_pair(sa + 64 * UPD_KB * 2, &p.map[3], fb, jb.m0 + rofs + 64, ty, jb.b);
+              tma_load_3d_pair(sb, &p.map[4], fb, jb.n0 + rofs, ty, jb.b);             // Z[t][f], f contiguous
+              tma_load_3d_pair(sb + 64 * UPD_KB * 2, &p.map[4], fb, jb.n0 + rofs + 64, ty, jb.b);
+            } else {
+              mbar_arrive_expect_tx(&full[s], Cf::STAGE_BYTES);
+              tma_load_3d(sa, &p.map[3], &full[s], jb.m0, ty, jb.b);
+              tma_load_3d(sa + 64 * UPD_KB * 2, &p.map[3], &full[s], jb.m0 + 64, ty, jb.b);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                tma_load_3d(sb + q * 64 * UPD_KB * 2, &p.map[4], &full[s], jb.n0 + 64 * q, ty, jb.b);
+            }
+          }
+        }
+        if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
+        counters[0] = it;
+      }
+    } else if (warp == UPD_WARP_MMA) {
+      if (lane == 0 && rank == 0) {
+        uint32_t it = 0;
+        bool ok = true;
+        UpdJob jb;
+        const uint32_t idesc = idesc_bf16(PAIR ? 256 : 128, 256, true, true);
+        for (uint32_t i = 0; ok && upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
+          const int sl = (int)(i & 1);
+          const uint32_t u = i >> 1;  // earlier uses of this slot
+          const bool got =
+              PAIR ? mbar_wait_cluster(&slot_free[sl], (u & 1) ^ 1) : mbar_wait(&slot_free[sl], (u & 1) ^ 1);
+          if (!got || *abort_flag) { ok = false; break; }
+          tc_fence_after();
+          const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
+          const int t0 = jb.chunk * p.C;
+          const int kb0 = (m.last_start - t0) / UPD_KB;
+          const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
+          const uint32_t tacc = tmem_base + sl * ACC_COLS;
+          for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!mbar_wait(&full[s], ph) || *abort_flag) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(stages + s * Cf::STAGE_BYTES);
+            const uint32_t b_addr = a_addr + Cf::A_BYTES;
+#pragma unroll
+            for (int ks = 0; ks < UPD_KB / 16; ++ks) {
+              const uint64_t ad = sdesc_sw128(a_addr + ks * 2048, UPD_KB * 128, 1024);
+              const uint64_t bd = sdesc_sw128(b_addr + ks * 2048, UPD_KB * 128, 1024);
+              // the chunk's first MMA overwrites the slot: every delta starts from zero
+              const uint32_t acc = (kb == kb0 && ks == 0) ? 0u : 1u;
+              if constexpr (PAIR) mma_bf16_pair(tacc, ad, bd, idesc, acc);
+              else mma_bf16(tacc, ad, bd, idesc, acc);
+            }
+            if constexpr (PAIR) mma_commit_pair(&empty[s], 3); else mma_commit(&empty[s]);
+          }
+          if (!ok) break;
+          if constexpr (PAIR) mma_commit_pair(&slot_full[sl], 3); else mma_commit(&slot_full[sl]);
+        }
+        if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
+        counters[1] = it;
+        if constexpr (PAIR) mma_commit_pair(drain, 1); else mma_commit(drain);
+        mbar_wait(drain, 0);
+      }
+    }
   }
-
   __syncthreads();
   // After a timeout: let this CTA's issued but never consumed loads land before
   // the shared memory goes away (each wait is bounded).
@@ -1019,7 +1066,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) upd_kernel(const __grid_constant_
   }
   tc_fence_before();
   if constexpr (PAIR) cluster_sync(); else __syncthreads();
-  if (warp == 1) {
+  if (warp == UPD_WARP_MMA) {
     tc_fence_after();
     if constexpr (PAIR) tmem_dealloc_pair(tmem_base, 2 * ACC_COLS);
     else tmem_dealloc(tmem_base, 2 * ACC_COLS);
@@ -1046,7 +1093,7 @@ static int max_pairs(cudaStream_t st) {
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(NTHREADS, 1, 1);
+    cfg.blockDim = dim3(UPD_THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = attr;
@@ -1064,8 +1111,22 @@ static bool pair_update_enabled() {
   return !(e && e[0] == '1');
 }
 
+// The update kernel's register trade (setmaxnreg) balances only at the launch
+// register count it was written for; any other count could leave a warpgroup
+// waiting for registers, so such a build is refused.
+template <bool PAIR, int KB>
+static bool upd_regs_ok() {
+  cudaFuncAttributes a;
+  if (cudaFuncGetAttributes(&a, upd_kernel<PAIR, KB>) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.numRegs == UPD_REGS_LAUNCH;
+}
+
 template <int KB>
 static cudaError_t launch_update_kb(const TcParams& p, int num_sms, cudaStream_t st) {
+  if (!upd_regs_ok<true, KB>() || !upd_regs_ok<false, KB>()) return cudaErrorInvalidDeviceFunction;
   if (p.d % 256 == 0 && pair_update_enabled()) {
     const int np = max_pairs<KB>(st);
     if (np > 0) {
@@ -1079,7 +1140,7 @@ static cudaError_t launch_update_kb(const TcParams& p, int num_sms, cudaStream_t
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.gridDim = dim3(2 * std::max(1, std::min(q.n_tiles, np)), 1, 1);
-      cfg.blockDim = dim3(NTHREADS, 1, 1);
+      cfg.blockDim = dim3(UPD_THREADS, 1, 1);
       cfg.dynamicSmemBytes = smem;
       cfg.stream = st;
       cfg.attrs = attr;
@@ -1091,7 +1152,7 @@ static cudaError_t launch_update_kb(const TcParams& p, int num_sms, cudaStream_t
   cudaError_t e = cudaFuncSetAttribute(upd_kernel<false, KB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(p.n_tiles, num_sms));
-  upd_kernel<false, KB><<<grid, NTHREADS, smem, st>>>(p);
+  upd_kernel<false, KB><<<grid, UPD_THREADS, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -1099,8 +1160,8 @@ int update_tokens_per_stage(int C) { return C % 128 == 0 ? 128 : 64; }
 
 cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st) {
   if (p.n_tiles <= 0 || p.dchunks <= 0) return cudaSuccess;
-  return update_tokens_per_stage(p.C) == 128 ? launch_update_kb<128>(p, num_sms, st)
-                                             : launch_update_kb<64>(p, num_sms, st);
+  const int kb = p.upd_kb ? p.upd_kb : update_tokens_per_stage(p.C);
+  return kb == 128 ? launch_update_kb<128>(p, num_sms, st) : launch_update_kb<64>(p, num_sms, st);
 }
 
 // ------------------------------------------------------------------ failure-path self test
@@ -1206,6 +1267,7 @@ cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st) 
     case FAM_ZV: return launch<FAM_ZV>(p, num_sms, st);
     case FAM_ZV2: return launch<FAM_ZV2>(p, num_sms, st);
     case FAM_GRAM2: return launch<FAM_GRAM2>(p, num_sms, st);
+    case FAM_PZ: return launch<FAM_PZ>(p, num_sms, st);
     case FAM_GRAM: return launch<FAM_GRAM>(p, num_sms, st);
     case FAM_APPLY256: return launch<FAM_APPLY256>(p, num_sms, st);
     default: return launch<FAM_APPLY>(p, num_sms, st);
@@ -1214,6 +1276,7 @@ cudaError_t launch_tc(int fam, const TcParams& p, int num_sms, cudaStream_t st) 
 
 int kind_gateup() { return K_GATEUP; }
 int kind_vhat() { return K_VHAT; }
+int kind_intra() { return K_INTRA; }
 
 }  // namespace tck
 }  // namespace ipttt

@@ -13,7 +13,11 @@ namespace tck {
 // M=256 pair MMAs, 128 K per stage); launched as clusters of two.
 // FAM_GRAM2: the Gram pass on 256 x 256 token-block pairs, one cluster of two per
 // block pair; each CTA writes its own partial (2 per pair, npairs = pairs per chunk).
-enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_APPLY256 = 5, FAM_ZV2 = 6, FAM_GRAM2 = 8 };
+// FAM_PZ: per group of 256 tokens of a row, the masked token-token products
+// P[t][u] = z_t . z_u for u in t's document and in an earlier chunk of the group
+// (cta pairs, K = d_ff), written as bf16 [B][T][256]; the grouped scan's
+// within-group term.
+enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_APPLY256 = 5, FAM_ZV2 = 6, FAM_GRAM2 = 8, FAM_PZ = 9 };
 
 struct TcParams {
   CUtensorMap map[6];
@@ -37,6 +41,13 @@ struct TcParams {
   const void* resid;      // apply: optional residual H added to O
   float* S;               // update: fp32 state, blocked 128 x 128 tiles
   int* status;            // device status word
+  const void* src0;       // fused target: X0 [B][T][d]
+  const void* src1;       // fused target: conv_w [d][5]
+  const uint8_t* flags;   // fused target: document-start flags [B][T]
+  const uint8_t* glo;     // FAM_PZ: per token, its document's first token within its group (offset)
+  int cs;                 // FAM_PZ: chunk length (the group holds 256 / cs chunks)
+  const void* intra;      // apply: optional within-group term E [B][T][d] bf16, added to the fast-weight part
+  int upd_kb;             // update: tokens per stage (0: update_tokens_per_stage(C))
 };
 
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
@@ -51,9 +62,17 @@ cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st);
 // Tokens per pipeline stage of the state update for chunk length C: the V and Z
 // tensor maps (map[3], map[4]) carry boxes of that many rows.
 int update_tokens_per_stage(int C);
+// Target GEMM with the masked conv in its producer (tgt_kernel.cu): V = conv(X0)
+// Wtarget, rows outside each chunk's last segment zeroed.  map[0]: Wtarget, box
+// {64, 64}; src0 X0, src1 conv_w, flags, meta, out0 V; n_tiles = B ceil(T/256)
+// ceil(d/512).  Needs clusters of two and d % 256 == 0.
+bool fused_target_supported(int d);
+int fused_target_workers(cudaStream_t st);
+cudaError_t launch_fused_target(const TcParams& p, cudaStream_t st);
 cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st);
 int kind_gateup();
 int kind_vhat();
+int kind_intra();
 
 }  // namespace tck
 }  // namespace ipttt

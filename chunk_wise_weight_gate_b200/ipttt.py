@@ -27,7 +27,7 @@ EXPORTS = ("ipttt_workspace_size", "ipttt_forward", "ipttt_forward_ex", "ipttt_c
            "ipttt_kernel_launches", "ipttt_selftest_wait_timeout", "ipttt_forward_noalloc",
            "ipttt_forward_host_size", "ipttt_forward_host", "ipttt_decode_state_size", "ipttt_decode_host_size",
            "ipttt_decode_reset", "ipttt_decode_step", "ipttt_decode_export", "ipttt_cp_workspace_size",
-           "ipttt_cp_plan", "ipttt_cp_begin", "ipttt_cp_finish")
+           "ipttt_cp_plan", "ipttt_cp_begin", "ipttt_cp_finish", "ipttt_last_error_detail")
 PHASES = ("prep", "gate_up", "target", "gram", "apply", "update")
 DEBUG_OUTPUTS = ("D", "S_final", "alpha", "Z", "V")
 
@@ -44,7 +44,8 @@ FLAG_RESIDUAL = 1
 class IptttError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {STATUS.get(code, code)} ({strerror(code)})")
+        detail = last_error_detail() if code == 6 else ""
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({strerror(code)})" + (f": {detail}" if detail else ""))
 
 
 _lib = None
@@ -80,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.ipttt_strerror.restype = ctypes.c_char_p
         L.ipttt_version.argtypes = []
         L.ipttt_version.restype = ctypes.c_char_p
+        L.ipttt_last_error_detail.argtypes = []
+        L.ipttt_last_error_detail.restype = ctypes.c_char_p
         L.ipttt_profile_enable.argtypes = [ctypes.c_int]
         L.ipttt_profile_enable.restype = None
         L.ipttt_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64),
@@ -122,6 +125,14 @@ def strerror(code: int) -> str:
         return lib().ipttt_strerror(code).decode()
     except Exception:  # library missing while formatting an error
         return "?"
+
+
+def last_error_detail() -> str:
+    """The CUDA error behind this thread's last IPTTT_ERR_CUDA ("" if none)."""
+    try:
+        return lib().ipttt_last_error_detail().decode()
+    except Exception:
+        return ""
 
 
 def _check(code: int, where: str):

@@ -140,7 +140,12 @@ IPTTT_API ipttt_status ipttt_core(const ipttt_params* p, const void* Z, const vo
  * position between calls, so a long sequence can be fed in pieces; the result
  * equals one call over the whole sequence.  params->T is the piece length and
  * must be a multiple of C except for the final piece of a sequence (the conv
- * look-ahead and the update both close at chunk ends).  doc_starts are offsets
+ * look-ahead and the update both close at chunk ends).  The bf16 path scans
+ * chunks of 64 or 128 tokens in groups of 256 tokens, starting at each call's
+ * first token; pieces whose lengths are multiples of the scan group (256 tokens
+ * then, else C) give one call's result bit for bit, other whole-chunk pieces give
+ * it up to rounding (the state sums and snapshots are grouped differently).
+ * doc_starts are offsets
  * b*T + t within the piece; a piece start is a document start only when the row
  * has consumed nothing yet or when doc_starts lists it.
  * State layout (opaque, 256-byte aligned): fp32 S[B][d][F], then per-row int64
@@ -213,8 +218,14 @@ IPTTT_API ipttt_status ipttt_get_status(void* stream);
 /* Static description of a status code. */
 IPTTT_API const char* ipttt_strerror(ipttt_status s);
 
+/* The CUDA error behind the last IPTTT_ERR_CUDA returned on the calling thread:
+ * the failing step and the CUDA runtime's error name and text ("" if none).  The
+ * string belongs to the library and stays valid until the thread's next call. */
+IPTTT_API const char* ipttt_last_error_detail(void);
+
 /* Diagnostics.  While profiling is on, every call records CUDA events on its own
- * stream around each phase: 0 metadata + conv, 1 gate/up GEMM, 2 target GEMM,
+ * stream around each phase: 0 metadata (and, without CTA pairs, the conv), 1 gate/up
+ * GEMM, 2 target GEMM (with the conv in its producer on CTA pairs),
  * 3 Gram pass + clip factors, 4 apply launches of the chunk scan, 5 state-update
  * launches of the chunk scan.  ipttt_profile_read waits for the recorded events
  * and returns, per phase, the milliseconds and kernel launches accumulated since
@@ -266,7 +277,8 @@ IPTTT_API ipttt_status ipttt_selftest_wait_timeout(uint32_t limit_ns, void* stre
  *
  * The sequence runs through ipttt_stream_reset / ipttt_stream_forward in pieces of
  * piece_tokens tokens of every row (a multiple of C; 0 picks about T/8 in whole
- * chunks): while piece i computes on `stream`, piece i+1 is copied in and piece
+ * scan groups, so that the result is ipttt_forward's bit for bit, see streaming
+ * above): while piece i computes on `stream`, piece i+1 is copied in and piece
  * i-1 copied out on two streams the call creates and releases.  device_buffer is
  * caller-owned device memory, 256-byte aligned, of ipttt_forward_host_size(p,
  * piece_tokens, n_doc_starts) bytes (two device copies of a piece of H, X0 and O,

@@ -31,6 +31,7 @@ int main(void) {
 
   expect(strlen(ipttt_version()) >= 5, "version string");
   expect(strcmp(ipttt_strerror(IPTTT_OK), ipttt_strerror(IPTTT_ERR_ARG)) != 0, "distinct error strings");
+  expect(ipttt_last_error_detail() != NULL && ipttt_last_error_detail()[0] == 0, "no CUDA error detail yet");
 
   const size_t ws = ipttt_workspace_size(&p);
   expect(ws > 0 && ws % 256 == 0, "workspace size of a valid shape");

@@ -57,3 +57,21 @@ def gpu(cfg, inp, debug=True, **kw):
     torch.cuda.synchronize()
     assert ip.get_status() == 0
     return out
+
+
+# Largest scale error allowed on a fast-weight state, as the error's component
+# along the reference state (scale_bias).  Rounding the bf16 operands turns every
+# delta by a small random angle, which leaves a component of the order of the
+# squared normwise error (about 1e-5 here: measured |bias| <= 1.8e-5 on the
+# workloads' shapes); summing the deltas in fp32 (round to nearest) adds k u at
+# most.  A state update that lets the tensor cores add each small delta onto the
+# large running sum loses the addends' low bits and shrinks the state instead:
+# measured -7.2e-5 over 1024 chunks.
+BIAS_TOL = 4e-5
+
+
+def scale_bias(x, ref):
+    """<x - ref, ref> / <ref, ref>: the relative error of x along ref."""
+    x, ref = np.asarray(x, np.float64).ravel(), np.asarray(ref, np.float64).ravel()
+    den = float(ref @ ref)
+    return float((x - ref) @ ref) / den if den > 0 else 0.0

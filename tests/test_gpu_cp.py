@@ -143,29 +143,3 @@ def test_cp_shards_starting_documents_need_no_exchange():
     O, _ = cp_emulated(cfg, inp, world)
     ref = single(cfg, inp)
     assert torch.equal(O.cpu(), ref["O"].cpu())
-
-
-@pytest.mark.slow
-@pytest.mark.parametrize("name,world", [("qwen3_4b_128k", 8), ("packed_8x8k", 4)])
-def test_cp_full_size(name, world):
-    """The benchmark's workloads split over ranks: rank 0 is the single-device result
-    bit for bit, every rank is within 1e-2 of it (the single-device forward at these
-    sizes is held to the oracle by test_gpu_fullsize.py), and the last rank's state
-    is the single-device state after the whole sequence within 1e-5 normwise."""
-    from chunk_wise_weight_gate_b200 import synth
-    w = synth.WORKLOADS[name]
-    inp = synth.make_inputs(w, seed=0)
-    cfg = ip.LayerConfig(B=w.B, T=w.T, d=w.d, F=w.F, C=w.C, eta=w.eta, clip=w.clip)
-    O, finals = cp_emulated(cfg, inp, world)
-    last = finals[-1]
-    del finals
-    torch.cuda.empty_cache()
-    ref = single(cfg, inp)
-    TL = w.T // world
-    # compared on the device: bf16 values and their differences are exact in fp32
-    Of, Rf = O.float(), ref["O"].float()
-    assert torch.isfinite(Of).all()
-    assert torch.equal(O[:, :TL], ref["O"][:, :TL])
-    assert ((Of - Rf).abs().max() / Rf.abs().max()).item() <= 1e-2
-    S_ref = ref["S_final"].double()
-    assert (torch.linalg.vector_norm(last.double() - S_ref) / torch.linalg.vector_norm(S_ref)).item() <= 1e-5

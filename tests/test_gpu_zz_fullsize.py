@@ -1,13 +1,15 @@
 """Parity at the full sizes of the layer's headline workloads, run in the same
-launch configuration the benchmark times.
+launch configuration the benchmark times.  Collected after the small-shape parity
+tests, so a failure here never hides them.
 
-The oracle cannot redo a 128k-token scan in a test, so three checks that hold at
-any size stand in for the full comparison:
+Checks against the fp64 oracle:
   * prefix: outputs depend only on earlier tokens (apply before update, conv looks
     at most to the chunk end), so the oracle run on the first chunks of a row
-    reproduces exactly the GPU outputs on those chunks (O, D, alpha);
-  * clip factors are chunk-local: the oracle run on one late chunk alone gives
-    that chunk's alpha;
+    reproduces the GPU outputs on those chunks (O, D, alpha);
+  * the whole state walk: the oracle's chunk-by-chunk scan of a row
+    (tests/fullsize_ref.py) gives every chunk's alpha, the final state S_final and
+    the state a late chunk is applied with, hence that chunk's fast-weight term D;
+    S_final and D are held to the bf16 bars, and S_final to carry no scale bias;
   * late output rows: O[t] = z_t W0^T + D[t] with |D[t]| <= |z_t| * sum_i alpha_i
     ||dW_i||_F <= |z_t| k tau, so sampled rows of the last chunk must lie within the
     bf16 tolerance plus that bound of the oracle's z_t W0^T.
@@ -21,7 +23,8 @@ import torch
 from chunk_wise_weight_gate_b200 import ipttt as ip
 from chunk_wise_weight_gate_b200 import synth
 from oracle import ipttt_oracle as orc
-from tests.gpu_util import WEIGHTS, maxrel, normrel
+from tests import fullsize_ref
+from tests.gpu_util import BIAS_TOL, WEIGHTS, maxrel, normrel, scale_bias
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -101,16 +104,38 @@ def check_late_chunks(out, inp, w, b, chunks):
     assert np.all(err <= TOL_O * scale + bound), float(np.max(err - bound))
 
 
+def check_state_walk(out, w, name, b):
+    """S_final, every alpha and the last chunk's D of row b against the oracle's scan."""
+    k = (w.T + w.C - 1) // w.C
+    late = k - 1
+    S_ref, a_ref, states = fullsize_ref.scan_row(name, b, (late,))
+    np.testing.assert_allclose(f64(out["alpha"][b]), a_ref, rtol=1e-2)
+    S = f64(out["S_final"][b])
+    _, D_ref = states[late]
+    D = f64(out["D"][b, late * w.C:min(k * w.C, w.T)])
+    print(f"{name} row {b}: S_final normrel {normrel(S, S_ref):.3e}, scale bias {scale_bias(S, S_ref):+.3e}; "
+          f"chunk {late} D normrel {normrel(D, D_ref):.3e} maxrel {maxrel(D, D_ref):.3e}")
+    assert normrel(S, S_ref) <= 2e-2
+    assert abs(scale_bias(S, S_ref)) <= BIAS_TOL
+    if np.any(D_ref != 0):
+        assert normrel(D, D_ref) <= 2e-2
+        assert maxrel(D, D_ref) <= 5e-2
+    else:
+        assert np.all(D == 0)
+
+
 @pytest.mark.parametrize("name", ["qwen3_4b_32k", "qwen3_4b_128k", "packed_8x8k"])
 def test_full_size_layer(name):
     w = synth.WORKLOADS[name]
-    inp = synth.make_inputs(w, seed=0)
-    out = run_layer(w, inp)
+    inp = fullsize_ref.inputs(name)
+    out = run_layer(w, inp, debug=("D", "alpha", "S_final"))
     assert torch.isfinite(out["O"].float()).all()
     rows = list(range(w.B)) if w.B <= 2 else [0, w.B // 2, w.B - 1]
     check_prefix(out, inp, w, rows)
     k = (w.T + w.C - 1) // w.C
     check_late_chunks(out, inp, w, rows[-1], [k // 2, k - 1])
+    for b in (rows[0], rows[-1]) if len(rows) > 1 else rows:
+        check_state_walk(out, w, name, b)
     if w.clip > 0 and w.docs == "single":
         # every chunk's update has norm tau after the clip, so |S| <= k tau
         assert np.all(f64(out["alpha"]) < 1.0)
