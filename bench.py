@@ -140,13 +140,19 @@ def phase_flops(w: synth.Workload) -> dict:
     }
 
 
+def scan_step_tokens(w: synth.Workload) -> int:
+    """Tokens per step of the library's chunk scan: chunks of 64 or 128 tokens are
+    scanned in groups of 256 tokens (one state snapshot per group), others one by one."""
+    return 256 if w.dtype == "bf16" and w.C in (64, 128) and w.T > w.C else w.C
+
+
 def phase_bytes(w: synth.Workload, phase: str, launches: float) -> float:
     """Algorithmic DRAM bytes per call of a phase (per layer): every input read once,
     every output written once.  `launches` is the phase's launch count per layer (the
     state update reads and writes the fp32 state once per launch; the apply reads
     Wdown0 once per launch)."""
-    B, T, d, F, C = w.B, w.T, w.d, w.F, w.C
-    k = (T + C - 1) // C
+    B, T, d, F = w.B, w.T, w.d, w.F
+    k = (T + scan_step_tokens(w) - 1) // scan_step_tokens(w)  # state snapshots per row (+1)
     e = 2  # bf16
     if phase == "prep":
         return 2 * B * T

@@ -900,29 +900,57 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
       // carried state is dropped), the state in registers, or (the tile's first
       // chunk of the launch) the state as the previous launch or the caller left it
       const int base = m.has_start ? 0 : (jb.c == 0 ? 2 : 1);
+      const bool snap = jb.chunk + 1 < p.k;
+      const float* sf = reinterpret_cast<const float*>(upd_state_block(p, jb.b, m0c, jb.n0, half));
+      // Folds 64 columns of the delta (two 32-column TMEM loads) into st[64 hb ..].
+      auto fold = [&](const int hb, const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+          const int c = 64 * hb + q;
+          const float old = base == 2 ? sf[((c / 4) * 128 + row) * 4 + (c & 3)] : base == 1 ? st[c] : 0.0f;
+          st[c] = old + __uint_as_float(q < 32 ? ra[q & 31] : rb[q & 31]);
+        }
+      };
+      // Snapshot box hb: 32 rows x 64 columns of bf16(S_{chunk+1}) (what the apply of
+      // chunk+1 reads), 128-byte swizzled, stored by TMA.
+      auto store_box = [&](const int hb) {
+        uint8_t* box = wboxes + (hb % UPD_BOXES) * UPD_BOX_BYTES;
+        if (stores > 0) {
+          // the store issued from this buffer UPD_BOXES boxes ago has read it
+          if (lane == 0) bulk_wait_read<UPD_BOXES - 1>();
+          __syncwarp();
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int c = 64 * hb + 8 * e;
+          *reinterpret_cast<uint4*>(box + lane * 128 + ((e ^ (lane & 7)) << 4)) =
+              make_uint4(pack_bf16(st[c], st[c + 1]), pack_bf16(st[c + 2], st[c + 3]),
+                         pack_bf16(st[c + 4], st[c + 5]), pack_bf16(st[c + 6], st[c + 7]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&p.map[5], box, jb.n0 + 128 * half + 64 * hb, m0c + 32 * quarter,
+                       ((jb.chunk + 1) % p.nslots) * p.B + jb.b);
+          bulk_commit();
+        }
+        ++stores;
+      };
       if (!mbar_wait(&slot_full[sl], (i >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
+      // Two halves of the warp's 128 columns, one TMEM round trip each: the second
+      // half's loads are in flight while the first is folded and stored.
+      uint32_t x0[32], x1[32], y0[32], y1[32];
+      const uint32_t tcol = tmem_base + sl * ACC_COLS + ((uint32_t)(quarter * 32) << 16) + 128 * half;
       if (cols) {
-        const uint32_t tcol = tmem_base + sl * ACC_COLS + ((uint32_t)(quarter * 32) << 16) + 128 * half;
-        const float4* src = upd_state_block(p, jb.b, m0c, jb.n0, half);
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          uint32_t r[16];
-          tmem_ld16(tcol + 16 * g, r);
-          float o[16];
-          if (base == 2) {
-            const float* sf = reinterpret_cast<const float*>(src);
-#pragma unroll
-            for (int q = 0; q < 16; ++q) o[q] = sf[((4 * g + q / 4) * 128 + row) * 4 + (q & 3)];
-          }
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const int c = 16 * g + q;
-            const float old = base == 2 ? o[q] : base == 1 ? st[c] : 0.0f;
-            st[c] = old + __uint_as_float(r[q]);
-          }
-        }
+        tmem_ld32(tcol, x0);
+        tmem_ld32(tcol + 32, x1);
+        tmem_ld_wait();
+        fold(0, x0, x1);
+        tmem_ld32(tcol + 64, y0);
+        tmem_ld32(tcol + 96, y1);
+        if (snap) store_box(0);
+        tmem_ld_wait();
       }
       // the slot's delta is in registers: the MMAs may overwrite it
       tc_fence_before();
@@ -932,34 +960,8 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
         else mbar_arrive(&slot_free[sl]);
       }
       if (!cols) continue;
-      if (jb.chunk + 1 < p.k) {
-        // bf16 snapshot of S_{chunk+1} (what the apply of chunk+1 reads), two boxes
-        // of 32 rows x 64 columns per warp, 128-byte swizzled for the TMA store
-#pragma unroll
-        for (int bx = 0; bx < 2; ++bx) {
-          uint8_t* box = wboxes + (bx % UPD_BOXES) * UPD_BOX_BYTES;
-          if (stores > 0) {
-            // the store issued from this buffer UPD_BOXES boxes ago has read it
-            if (lane == 0) bulk_wait_read<UPD_BOXES - 1>();
-            __syncwarp();
-          }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int c = 64 * bx + 8 * e;
-            *reinterpret_cast<uint4*>(box + lane * 128 + ((e ^ (lane & 7)) << 4)) =
-                make_uint4(pack_bf16(st[c], st[c + 1]), pack_bf16(st[c + 2], st[c + 3]),
-                           pack_bf16(st[c + 4], st[c + 5]), pack_bf16(st[c + 6], st[c + 7]));
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&p.map[5], box, jb.n0 + 128 * half + 64 * bx, m0c + 32 * quarter,
-                         ((jb.chunk + 1) % p.nslots) * p.B + jb.b);
-            bulk_commit();
-          }
-          ++stores;
-        }
-      }
+      fold(1, y0, y1);
+      if (snap) store_box(1);
       if (jb.c == p.dchunks - 1) {
         // the tile's last chunk of the launch: the fp32 state goes back to HBM
         float4* dst = upd_state_block(p, jb.b, m0c, jb.n0, half);

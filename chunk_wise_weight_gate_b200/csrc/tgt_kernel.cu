@@ -13,16 +13,18 @@
 // output columns: per K step two M=256 x N=256 pair MMAs (tcgen05.mma.cta_group::2)
 // fill the whole TMEM of both CTAs (2 x 256 fp32 columns each).  Per 64-channel K
 // stage:
-//   warp 0, one thread : TMA of this CTA's half of the tile's Wtarget columns
+//   warp 8, one thread : TMA of this CTA's half of the tile's Wtarget columns
 //                        (64 x 64 MN-major boxes; completion counted on the even
 //                        CTA's barrier, no multicast);
-//   warp 1, one thread of the even CTA: the MMAs;
-//   warps 2-9          : U for this CTA's 128 rows and the stage's 64 channels, read
+//   warp 9, one thread of the even CTA: the MMAs;
+//   warps 0-7          : U for this CTA's 128 rows and the stage's 64 channels, read
 //                        from X0 in global memory (each thread 8 channels x 8 rows
-//                        through a 12-row window), written as bf16 in the 128-byte-
-//                        swizzled K-major layout the MMA reads, then made visible to
-//                        the tensor cores (proxy fence, release at cluster scope).
-//                        Warps 2-5 fill the even stages, warps 6-9 the odd ones.
+//                        through a 12-row window, the next stage's window loaded
+//                        while the current one is computed), written as bf16 in the
+//                        128-byte-swizzled K-major layout the MMA reads, then made
+//                        visible to the tensor cores (proxy fence, release at
+//                        cluster scope).  Warps 0-3 fill the even stages, 4-7 the
+//                        odd ones.
 // The conv arithmetic is that of the stand-alone conv kernel (fp32 FMAs in tap
 // order, one bf16 rounding), done two channels per instruction (fma.rn.f32x2).
 // There is one accumulator, so the MMAs of a tile wait for the previous tile's
@@ -51,7 +53,17 @@ constexpr int TG_BOX_BYTES = 64 * TG_KB * 2;  // one 64-column Wtarget box
 constexpr int TG_B_BYTES = 4 * TG_BOX_BYTES;  // 2 accumulators x this CTA's 128 columns
 constexpr int TG_STAGE_BYTES = TG_A_BYTES + TG_B_BYTES;
 constexpr int TG_EPI_WARPS = 8;
-constexpr int TG_THREADS = 64 + 32 * TG_EPI_WARPS;
+// Three warpgroups: warps 0-7 conv and epilogue, warp 8 TMA, warp 9 MMA, 10-11
+// idle.  Twelve warps cap a thread at 168 registers at launch; the third
+// warpgroup drops to 56 and the conv/epilogue warpgroups rise to 224 (an exact
+// trade: 128 x (168 - 56) = 256 x (224 - 168)), which holds a second X0 window
+// in flight.  The launcher checks the compiled register count.
+constexpr int TG_THREADS = 384;
+constexpr int TG_WARP_TMA = 8, TG_WARP_MMA = 9;
+constexpr int TG_REGS_LAUNCH = 168, TG_REGS_LOW = 56, TG_REGS_EPI = 224;
+static_assert((TG_THREADS - 32 * TG_EPI_WARPS) * (TG_REGS_LAUNCH - TG_REGS_LOW) ==
+                  32 * TG_EPI_WARPS * (TG_REGS_EPI - TG_REGS_LAUNCH),
+              "the register trade of the fused target kernel must balance");
 constexpr int TG_SMEM = 1024 + TG_STAGES * TG_STAGE_BYTES + 256;
 constexpr int TG_TAPS = 5;
 static_assert(TG_SMEM <= 232448, "fused target kernel exceeds shared memory");
@@ -139,8 +151,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
     counters[0] = counters[1] = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) prefetch_tmap(&p.map[0]);
-  if (warp == 1) {
+  if (warp == TG_WARP_TMA && lane == 0) prefetch_tmap(&p.map[0]);
+  if (warp == TG_WARP_MMA) {
     tmem_alloc_pair(tmem_slot, 512);
     tmem_relinquish_pair();
   }
@@ -150,67 +162,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t full0 = map_to_rank(smem_u32(full), 0);  // the even CTA's full[0]
 
-  if (warp == 0) {
-    if (lane == 0) {
-      uint32_t it = 0;
-      bool ok = true;
-      TgJob j;
-      for (uint32_t i = 0; ok && tg_job(p, i, wk, nwk, j); ++i) {
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % TG_STAGES;
-          const uint32_t ph = (it / TG_STAGES) & 1;
-          if (!mbar_wait_or_abort(&empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
-          uint8_t* sb = stages + s * TG_STAGE_BYTES + TG_A_BYTES;
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * j.nacc * 2 * TG_BOX_BYTES);
-          const uint32_t fb = full0 + 8u * s;
-          for (int a = 0; a < j.nacc; ++a)
-            for (int q = 0; q < 2; ++q)  // Wtarget[k][n], n contiguous: this CTA's columns of accumulator a
-              tma_load_3d_pair(sb + (2 * a + q) * TG_BOX_BYTES, &p.map[0], fb,
-                               j.n0 + 256 * a + 128 * (int)rank + 64 * q, kb * TG_KB, 0);
-        }
-      }
-      if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
-      counters[0] = it;
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
-      uint32_t it = 0, tcount = 0;
-      bool ok = true;
-      TgJob j;
-      const uint32_t idesc = idesc_bf16(256, 256, false, true);
-      for (uint32_t i = 0; ok && tg_job(p, i, wk, nwk, j); ++i, ++tcount) {
-        if (!mbar_wait_cluster(acc_empty, (tcount & 1) ^ 1) || *abort_flag) { ok = false; break; }
-        tc_fence_after();
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % TG_STAGES;
-          const uint32_t ph = (it / TG_STAGES) & 1;
-          if (!mbar_wait_cluster(&full[s], ph) || *abort_flag) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(stages + s * TG_STAGE_BYTES);
-          const uint32_t b_addr = a_addr + TG_A_BYTES;
-#pragma unroll
-          for (int ks = 0; ks < TG_KB / 16; ++ks) {
-            const uint64_t ad = sdesc_sw128(a_addr + ks * 32, 16, 1024);
-            const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
-            for (int a = 0; a < j.nacc; ++a) {
-              // MN-major: 16 K rows of 128 B per step; the two 64-column blocks of
-              // this CTA's half are TG_BOX_BYTES apart
-              const uint64_t bd = sdesc_sw128(b_addr + a * 2 * TG_BOX_BYTES + ks * 2048, TG_BOX_BYTES, 1024);
-              mma_bf16_pair(tmem_base + 256 * a, ad, bd, idesc, acc);
-            }
-          }
-          mma_commit_pair(&empty[s], 3);
-        }
-        if (!ok) break;
-        mma_commit_pair(acc_full, 3);
-      }
-      if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
-      counters[1] = it;
-      mma_commit_pair(drain, 1);
-      mbar_wait(drain, 0);
-    }
-  } else {
-    const int ew = warp - 2;
+  if (warp < TG_EPI_WARPS) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(TG_REGS_EPI));
+    const int ew = warp;
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int half = ew >> 2;      // epilogue: accumulator (256-column half); conv: even / odd stages
     const int erow = quarter * 32 + lane;
@@ -221,7 +175,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
     const __nv_bfloat16* cw = reinterpret_cast<const __nv_bfloat16*>(p.src1);
     const uint32_t acc_empty0 = map_to_rank(smem_u32(acc_empty), 0);
     bool ok = true;
-    uint32_t it = 0, tcount = 0;
+    uint32_t tcount = 0;
 
     // Drains the accumulator of tile jp: this warp's 32 rows, 256 columns.
     auto epilogue = [&](const TgJob& jp, uint32_t tc) -> bool {
@@ -260,13 +214,12 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
       return true;
     };
 
-    TgJob j, jprev;
-    bool have_prev = false;
-    for (uint32_t i = 0; ok && tg_job(p, i, wk, nwk, j); ++i) {
-      // taps in use for this thread's 8 rows (the same for every stage of the tile)
-      const int t0 = j.m0 + 128 * (int)rank + rg * 8;
-      const uint8_t* fl = p.flags + (size_t)j.b * p.T;
-      int ntap[8];
+    // Taps in use for this thread's 8 rows of tile jj (the same for every stage of
+    // the tile), 3 bits per row.
+    auto taps_of = [&](const TgJob& jj) -> uint32_t {
+      const int t0 = jj.m0 + 128 * (int)rank + rg * 8;
+      const uint8_t* fl = p.flags + (size_t)jj.b * p.T;
+      uint32_t packed = 0;
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const int t = t0 + r;
@@ -277,24 +230,52 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
           for (int o = 1; o < TG_TAPS; ++o)
             if (n == o && t + o < cend && !fl[t + o]) n = o + 1;
         }
-        ntap[r] = n;
+        packed |= (uint32_t)n << (3 * r);
       }
-      const __nv_bfloat16* xrow = X0 + ((size_t)j.b * p.T + t0) * p.d + cj * 8;
-      for (int kb = 0; kb < nk; ++kb, ++it) {
-        if (kb == TG_STAGES && have_prev) {
+      return packed;
+    };
+    // The 12-row X0 window (8 channels) of this thread for stage kb of tile jj.
+    auto load_window = [&](uint4 (&x)[12], const TgJob& jj, int kb) {
+      const int t0 = jj.m0 + 128 * (int)rank + rg * 8;
+      const __nv_bfloat16* xrow = X0 + ((size_t)jj.b * p.T + t0) * p.d + kb * TG_KB + cj * 8;
+#pragma unroll
+      for (int q = 0; q < 12; ++q)
+        x[q] = (t0 + q < p.T) ? *reinterpret_cast<const uint4*>(xrow + (size_t)q * p.d) : make_uint4(0u, 0u, 0u, 0u);
+    };
+
+    // This group's stages are kb = half, half + 2, ... of every tile (a tile has an
+    // even number of stages).  The X0 window of the next one is loaded while the
+    // current one is computed.
+    TgJob j, jn, jprev;
+    bool have_prev = false;
+    uint4 nx[12];
+    uint32_t ntp_n = 0;
+    bool have_j = tg_job(p, 0, wk, nwk, j);
+    if (have_j) {
+      ntp_n = taps_of(j);
+      load_window(nx, j, half);
+    }
+    for (uint32_t i = 0; ok && have_j; ++i) {
+      const uint32_t ntp = ntp_n;
+      const bool have_jn = tg_job(p, i + 1, wk, nwk, jn);
+      for (int kb = half; kb < nk; kb += 2) {
+        if (kb >= TG_STAGES && have_prev) {
           // the next tile's first stages are filled: drain the previous tile
           if (!epilogue(jprev, tcount - 1)) { ok = false; break; }
           have_prev = false;
         }
-        if ((int)(it & 1) != half) continue;  // the other group fills this stage
+        const uint32_t it = i * (uint32_t)nk + (uint32_t)kb;
         const int s = it % TG_STAGES;
         const uint32_t ph = (it / TG_STAGES) & 1;
-        // X0 window and conv taps of the stage (read before the stage is free)
         uint4 xr[12];
 #pragma unroll
-        for (int q = 0; q < 12; ++q)
-          xr[q] = (t0 + q < p.T) ? *reinterpret_cast<const uint4*>(xrow + (size_t)q * p.d + kb * TG_KB)
-                                 : make_uint4(0u, 0u, 0u, 0u);
+        for (int q = 0; q < 12; ++q) xr[q] = nx[q];
+        if (kb + 2 < nk) {
+          load_window(nx, j, kb + 2);
+        } else if (have_jn) {
+          ntp_n = taps_of(jn);
+          load_window(nx, jn, half);
+        }
         uint4 wr[5];
         const uint4* wsrc = reinterpret_cast<const uint4*>(cw + (size_t)(kb * TG_KB + cj * 8) * TG_TAPS);
 #pragma unroll
@@ -311,10 +292,11 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
         uint8_t* sa = stages + s * TG_STAGE_BYTES;
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
+          const int nt = (int)((ntp >> (3 * r)) & 7u);
           unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
           for (int o = 0; o < TG_TAPS; ++o) {
-            if (o < ntap[r]) {
+            if (o < nt) {
               const uint32_t xw[4] = {xr[r + o].x, xr[r + o].y, xr[r + o].z, xr[r + o].w};
 #pragma unroll
               for (int q = 0; q < 4; ++q) acc[q] = fma2(wp[o][q], bf2_to_f2(xw[q]), acc[q]);
@@ -335,17 +317,80 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
         if (lane == 0) mbar_arrive_release_cluster(full0 + 8u * s);
       }
       if (!ok) break;
-      if (have_prev) {  // a tile of fewer than STAGES + 1 stages
+      if (have_prev) {  // a tile of at most STAGES stages
         if (!epilogue(jprev, tcount - 1)) { ok = false; break; }
       }
       jprev = j;
       have_prev = true;
       ++tcount;
+      j = jn;
+      have_j = have_jn;
     }
     if (ok && have_prev && !epilogue(jprev, tcount - 1)) ok = false;
     if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
+    } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(TG_REGS_LOW));
+    if (warp == TG_WARP_TMA) {
+      if (lane == 0) {
+        uint32_t it = 0;
+        bool ok = true;
+        TgJob j;
+        for (uint32_t i = 0; ok && tg_job(p, i, wk, nwk, j); ++i) {
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = it % TG_STAGES;
+            const uint32_t ph = (it / TG_STAGES) & 1;
+            if (!mbar_wait_or_abort(&empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
+            uint8_t* sb = stages + s * TG_STAGE_BYTES + TG_A_BYTES;
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * j.nacc * 2 * TG_BOX_BYTES);
+            const uint32_t fb = full0 + 8u * s;
+            for (int a = 0; a < j.nacc; ++a)
+              for (int q = 0; q < 2; ++q)  // Wtarget[k][n], n contiguous: this CTA's columns of accumulator a
+                tma_load_3d_pair(sb + (2 * a + q) * TG_BOX_BYTES, &p.map[0], fb,
+                                 j.n0 + 256 * a + 128 * (int)rank + 64 * q, kb * TG_KB, 0);
+          }
+        }
+        if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
+        counters[0] = it;
+      }
+    } else if (warp == TG_WARP_MMA) {
+      if (lane == 0 && rank == 0) {
+        uint32_t it = 0, tcount = 0;
+        bool ok = true;
+        TgJob j;
+        const uint32_t idesc = idesc_bf16(256, 256, false, true);
+        for (uint32_t i = 0; ok && tg_job(p, i, wk, nwk, j); ++i, ++tcount) {
+          if (!mbar_wait_cluster(acc_empty, (tcount & 1) ^ 1) || *abort_flag) { ok = false; break; }
+          tc_fence_after();
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = it % TG_STAGES;
+            const uint32_t ph = (it / TG_STAGES) & 1;
+            if (!mbar_wait_cluster(&full[s], ph) || *abort_flag) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(stages + s * TG_STAGE_BYTES);
+            const uint32_t b_addr = a_addr + TG_A_BYTES;
+  #pragma unroll
+            for (int ks = 0; ks < TG_KB / 16; ++ks) {
+              const uint64_t ad = sdesc_sw128(a_addr + ks * 32, 16, 1024);
+              const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
+              for (int a = 0; a < j.nacc; ++a) {
+                // MN-major: 16 K rows of 128 B per step; the two 64-column blocks of
+                // this CTA's half are TG_BOX_BYTES apart
+                const uint64_t bd = sdesc_sw128(b_addr + a * 2 * TG_BOX_BYTES + ks * 2048, TG_BOX_BYTES, 1024);
+                mma_bf16_pair(tmem_base + 256 * a, ad, bd, idesc, acc);
+              }
+            }
+            mma_commit_pair(&empty[s], 3);
+          }
+          if (!ok) break;
+          mma_commit_pair(acc_full, 3);
+        }
+        if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
+        counters[1] = it;
+        mma_commit_pair(drain, 1);
+        mbar_wait(drain, 0);
+      }
+    }
   }
-
   __syncthreads();
   // After a timeout: let this CTA's issued but never consumed loads land before
   // the shared memory goes away (each wait is bounded).
@@ -354,7 +399,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
   }
   tc_fence_before();
   cluster_sync();
-  if (warp == 1) {
+  if (warp == TG_WARP_MMA) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, 512);
   }
@@ -371,7 +416,11 @@ int fused_target_workers(cudaStream_t st) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (have[dev]) return cached[dev];
   int n = 0;
-  if (cudaFuncSetAttribute(tgt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TG_SMEM) == cudaSuccess) {
+  // The register trade (setmaxnreg) balances only at the launch register count it
+  // was written for; a build compiled to another count is not used.
+  cudaFuncAttributes fa;
+  const bool regs_ok = cudaFuncGetAttributes(&fa, tgt_kernel) == cudaSuccess && fa.numRegs == TG_REGS_LAUNCH;
+  if (regs_ok && cudaFuncSetAttribute(tgt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TG_SMEM) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
