@@ -141,9 +141,10 @@ def phase_flops(w: synth.Workload) -> dict:
 
 
 def scan_step_tokens(w: synth.Workload) -> int:
-    """Tokens per step of the library's chunk scan: chunks of 64 or 128 tokens are
-    scanned in groups of 256 tokens (one state snapshot per group), others one by one."""
-    return 256 if w.dtype == "bf16" and w.C in (64, 128) and w.T > w.C else w.C
+    """Tokens per step of the library's chunk scan: chunks of 64, 128 or 256 tokens
+    are scanned in groups of 512 tokens (one state snapshot per group), others one
+    by one."""
+    return 512 if w.dtype == "bf16" and w.C < 512 and 512 % w.C == 0 and w.T > w.C else w.C
 
 
 def phase_bytes(w: synth.Workload, phase: str, launches: float) -> float:
@@ -169,6 +170,11 @@ def phase_bytes(w: synth.Workload, phase: str, launches: float) -> float:
     return 0.0
 
 
+def fp32_fma_tflops(sms: int, mhz: float) -> float:
+    """Peak fp32 rate of the CUDA cores: 128 fp32 lanes per SM, an FMA = 2 flops."""
+    return sms * 128 * 2 * mhz * 1e6 / 1e12
+
+
 def phase_roofline(w: synth.Workload, phase: str, ms: float, launches: float, steps: int, peaks: dict) -> dict:
     """Achieved rate of one phase against the bound that limits it: the tensor time
     (algorithmic flops at the sustained bf16 peak) or the HBM time (algorithmic bytes
@@ -179,7 +185,7 @@ def phase_roofline(w: synth.Workload, phase: str, ms: float, launches: float, st
     tflops = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     t_tensor = fl / (tflops * 1e12)
     t_hbm = by / (peaks["hbm_gbs"] * 1e9)
-    sec = ms / 1000.0
+    sec = max(ms, 1e-9) / 1000.0
     if t_tensor >= t_hbm:
         ach = fl / sec / 1e12
         return {"bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s", "frac": ach / tflops,
@@ -266,7 +272,7 @@ def run_ours(args, w: synth.Workload):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     pg = None
-    if world > 1:
+    if world > 1 and not emulated:
         import torch.distributed as dist
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
@@ -343,11 +349,25 @@ def run_ours(args, w: synth.Workload):
     peaks, peak_src = load_peaks()
 
     # roofline of the dominant kernel (the phase with the largest share of device time)
-    dom = max(phases, key=lambda k: phases[k][0])
-    dom_ms, dom_launches = phases[dom]
-    roof = {"kernel": dom, **phase_roofline(w, dom, dom_ms, dom_launches, args.steps, peaks),
-            "launches": dom_launches, "avg_launch_ms": dom_ms / max(1, dom_launches),
-            "peak_note": f"sustained bf16 and copy bandwidth ({peak_src}); burst bf16 {peaks['bf16_tflops']}"}
+    timed = {k: v for k, v in phases.items() if v[1] > 0}
+    if timed:
+        dom = max(timed, key=lambda k: timed[k][0])
+        dom_ms, dom_launches = phases[dom]
+        roof = {"kernel": dom, **phase_roofline(w, dom, dom_ms, dom_launches, args.steps, peaks),
+                "launches": dom_launches, "avg_launch_ms": dom_ms / max(1, dom_launches),
+                "peak_note": f"sustained bf16 and copy bandwidth ({peak_src}); burst bf16 {peaks['bf16_tflops']}"}
+    else:
+        # the fp32 path runs on the CUDA cores and does not time its phases: the
+        # whole step against the fp32 FMA rate of the device
+        dom = "step"
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        mhz = (clocks or {}).get("sm_max_mhz") or peaks.get("sm_max_mhz", 1965.0)
+        fp32_peak = fp32_fma_tflops(sms, mhz)
+        ach = flops / (ms / 1000.0) / 1e12
+        roof = {"kernel": "whole step (fp32 CUDA-core path)", "bound": "alu", "achieved": ach, "peak": fp32_peak,
+                "unit": "TFLOP/s", "frac": ach / fp32_peak, "launches": launches / max(1, args.steps),
+                "avg_launch_ms": ms / max(1, launches / max(1, args.steps)),
+                "peak_note": f"fp32 FMA rate: {sms} SMs x 128 lanes x 2 flops x {mhz:.0f} MHz"}
     traffic = MEASURED_TRAFFIC.get((w.name, w.C, dom))
     roof["traffic"] = traffic
     roof["traffic_unit"] = "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
@@ -492,12 +512,21 @@ def run_cp(args, w: synth.Workload):
     world, rank, local = dist_env()
     if not torch.cuda.is_available():
         raise RuntimeError("bench.py needs a CUDA device")
+    emulated = world == 1 and args.cp_world > 1
+    if emulated:
+        # one rank's share of an N-rank split, alone on this GPU: its begin and
+        # finish on its own shard, the gathered set filled with copies of its own
+        # aggregate (the finish reads N aggregates as it would after the exchange;
+        # the values are not a forward's, the bytes and launches are)
+        if not 0 <= args.cp_rank < args.cp_world:
+            raise ValueError("--cp-rank must lie in [0, --cp-world)")
+        world, rank = args.cp_world, args.cp_rank
     if w.T % world or (w.T // world) % w.C:
         raise ValueError(f"T={w.T} does not split into {world} shards of whole {w.C}-token chunks")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     pg = None
-    if world > 1:
+    if world > 1 and not emulated:
         import torch.distributed as dist
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
@@ -524,6 +553,11 @@ def run_cp(args, w: synth.Workload):
         if pg:
             ip.cp_exchange(agg, out=gathered)
         ip.cp_finish(cfg, world, rank, H, wts["Wdown0"], gathered, ws, docs, O=O)
+
+    if emulated:
+        ip.cp_begin(cfg, world, rank, H, X0, wts["Wgate"], wts["Wup"], wts["conv_w"], wts["Wtarget"], docs,
+                    agg=agg, workspace=ws)
+        gathered.copy_(agg.unsqueeze(0).expand_as(gathered))
 
     for _ in range(args.warmup):
         step()
@@ -561,7 +595,7 @@ def run_cp(args, w: synth.Workload):
     phases = ip.profile_read()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, pg, dev)
     status = ip.get_status()
-    tokens = w.B * w.T
+    tokens = w.B * (TL if emulated else w.T)
     peaks, peak_src = load_peaks()
     wl = w.replace(T=TL)
     dom = max(phases, key=lambda k: phases[k][0])
@@ -573,9 +607,12 @@ def run_cp(args, w: synth.Workload):
     if rank == 0:
         cfgd = config_dict(w, world)
         cfgd.update({"workload": f"cp_{w.name}", "parallelism": f"cp{world}", "shard_tokens": TL, "global_batch": w.B,
-                     "exchange": "NCCL all-gather of the fp32 shard aggregates" if world > 1 else "none"})
+                     "exchange": "NCCL all-gather of the fp32 shard aggregates" if pg else "none"})
+        if emulated:
+            cfgd.update({"emulated_rank": rank, "note": "one rank's share alone on one GPU; value = the rank's "
+                         "shard tokens / its step time"})
         out = {"metric": METRIC + " (one sequence split over the GPUs)", "value": tokens / (ms / 1000.0),
-               "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+               "unit": "tokens/s", "n_gpus": 1 if emulated else world, "steps": args.steps, "warmup": args.warmup,
                "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
                "dtype": "bf16", "data": "synthetic", "config": cfgd,
                "tflops": layer_flops(w) / (ms / 1000.0) / 1e12, "roofline": roof, "phases": phase_report,
@@ -599,6 +636,9 @@ def main(argv=None):
                     help="decode: token-by-token decoding of --decode-batch rows instead of the prefill step; "
                          "cp: the sequence split along T over the GPUs (context parallelism)")
     ap.add_argument("--decode-batch", type=int, default=8)
+    ap.add_argument("--cp-world", type=int, default=1,
+                    help="with --mode cp on one GPU: run one rank's share of a split over this many ranks")
+    ap.add_argument("--cp-rank", type=int, default=0, help="the rank that --cp-world runs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--piece-tokens", type=int, default=0,
                     help="e2e: tokens per pipelined piece of the host-buffer call (0: about T/8)")

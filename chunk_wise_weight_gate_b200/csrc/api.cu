@@ -2,10 +2,10 @@
 // carve-up, and the order of kernel launches for one In-Place TTT MLP layer.
 //
 // Launch order (bf16 path), all on the caller's stream:
-//   metadata -> Z = SiLU(H Wg^T)*(H Wu^T) -> V = conv(X0) Wt (the masked conv in the
-//   target GEMM's producer; last-segment rows) -> Gram partials -> alpha and the
-//   pre-scale of V -> per group of chunks: the state updates (S_i -> S_{i+1}, bf16
-//   snapshots) and one launch of the group's apply tiles (reads S_i).
+//   metadata, masked conv U -> Z = SiLU(H Wg^T)*(H Wu^T) -> V = U Wt (last-segment
+//   rows) -> Gram partials -> alpha and the pre-scale of V -> per group of chunks:
+//   the state updates (S_i -> S_{i+1}, bf16 snapshots) and one launch of the
+//   group's apply tiles (reads S_i).
 // The chunk order follows lijianxiong.blog notes "In-Place Test-Time Training",
 // 方法 (apply with the current fast weight, then update) and iplexlaw.co.kr review
 // §3 (a chunk's output always comes from the pre-update state).
@@ -169,19 +169,24 @@ int apply_group(const ipttt_params& p) {
 
 bool is_bf16(const ipttt_params& p) { return p.dtype == IPTTT_BF16; }
 
-// Chunks of 64 or 128 tokens are scanned kGroupTokens at a time (groups of 4 or 2
-// chunks): the state is carried, snapshotted and applied per group, and the
-// chunks of a group see each other's deltas through the within-group term
+// Chunks shorter than kGroupTokens (64, 128 or 256 tokens) are scanned
+// kGroupTokens at a time: the state is carried, snapshotted and applied per
+// group, and the chunks of a group see each other's deltas through the
+// within-group term
 //   E[t] = sum_{u in an earlier chunk of t's group, in t's document} (z_t . z_u) v'_u
 // (v' = alpha eta v on the rows that feed the update).  That equals the
 // chunk-by-chunk scan (the apply is linear in the state), with one bf16 state
 // snapshot written and read per group instead of per chunk.
-constexpr int kGroupTokens = 256;
-// IPTTT_GROUPED_SCAN=0 scans such chunks one by one instead.
+constexpr int kGroupTokens = 512;
+// The choice depends on the chunk length alone, never on T, so that a call over
+// a piece of a sequence (a streamed piece, a host-pipeline piece, a context shard)
+// does the same arithmetic as a call over the whole sequence: the grouped scan
+// rounds alpha eta v to bf16 before the update, the chunk-by-chunk scan scales
+// each fp32 delta instead.  IPTTT_GROUPED_SCAN=0 scans such chunks one by one.
 bool grouped_scan(const ipttt_params& p) {
   const char* e = getenv("IPTTT_GROUPED_SCAN");
   if (e && e[0] == '0') return false;
-  return is_bf16(p) && (p.C == 64 || p.C == 128) && p.T > p.C;
+  return is_bf16(p) && p.C < kGroupTokens && kGroupTokens % p.C == 0;
 }
 }  // namespace
 
@@ -237,7 +242,7 @@ Layout layout_of(const ipttt_params& p, bool cp = false) {
     L.gmeta = L.glo = L.P = L.E = 0;
     if (L.grouped) {
       L.gmeta = take(B * kg * sizeof(ChunkMeta));
-      L.glo = take(B * T);
+      L.glo = take(B * T * sizeof(uint16_t));
       L.P = take(B * T * kGroupTokens * 2);
       L.E = take(B * T * d * 2);
     }
@@ -371,11 +376,15 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   const bool cp_finish = cp && cp->stage == kCpFinish;
 
   // Gate/up and target GEMMs on CTA pairs (256-row tiles) where the device runs
-  // clusters of two, else one CTA per 128-row tile.  On pairs the masked conv is
-  // computed inside the target GEMM (U never reaches HBM); otherwise a conv kernel
-  // writes U first.
+  // clusters of two, else one CTA per 128-row tile; a conv kernel writes U first.
   const bool pair_gemm = pair_gemms_enabled() && pair_gemm_workers(st) > 0;
-  const bool fused_target = pair_gemm && fused_target_supported(s.d) && fused_target_workers(st) > 0;
+  // IPTTT_FUSED_TARGET=1: the target GEMM with the conv in its producer (U never
+  // reaches HBM; slower today than the conv kernel and the pair GEMM, whose U round
+  // trip costs less than the producer's conv arithmetic recomputed for every
+  // 512-column tile).
+  const char* fe = getenv("IPTTT_FUSED_TARGET");
+  const bool fused_target = pair_gemm && fe && fe[0] == '1' && fused_target_supported(s.d) &&
+                            fused_target_workers(st) > 0;
   // the grouped scan's within-group products run on CTA pairs
   const bool grouped = scan_grouped(L, st);
   Shape gs = s;
@@ -383,7 +392,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   gs.k = (s.T + kGroupTokens - 1) / kGroupTokens;
   const Shape& sq = grouped ? gs : s;  // the chunking of the scan
   ChunkMeta* gmeta = grouped ? reinterpret_cast<ChunkMeta*>(ws + L.gmeta) : meta;
-  uint8_t* glo = ws + L.glo;
+  uint16_t* glo = reinterpret_cast<uint16_t*>(ws + L.glo);
   void* Pw = ws + L.P;
   void* Ew = ws + L.E;
   if (!cp_finish) {
@@ -481,29 +490,37 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     IP_CHECK(launch_tc(gram2 ? FAM_GRAM2 : FAM_GRAM, g, di->num_sms, st));
     IP_CHECK(aux::alpha_from_partials(partials, alpha, s.B * s.k, gram2 ? 2 * g.npairs : tp.npairs, p.eta, tau,
                                       st));
-    // the state update accumulates alpha eta V^T Z: fold alpha eta into V's rows
-    IP_CHECK(aux::prescale_target(V, alpha, s, p.eta, st));
-    counted(3);
+    if (grouped) {
+      // a group's update sums several chunks' V^T Z in one accumulator, and the
+      // within-group term uses alpha eta v: fold alpha eta into V's rows
+      IP_CHECK(aux::prescale_target(V, alpha, s, p.eta, st));
+      counted(1);
+    }
+    counted(2);
   }
   if (grouped && !cp_finish) {
-    // within-group term: P = masked Z Z^T per group of 256 tokens, then E = P V'
+    // within-group term: P = masked Z Z^T per group (256 x 256 blocks on and below
+    // the diagonal), then E = P V'
     PhaseScope ph(st, PH_APPLY);
     TcParams z = tp;
     if (!make_map_bf16(&z.map[0], Z, s.F, s.T, s.B, 64, 128))
       return cuda_fail("tensor map of the within-group products", cudaErrorInvalidValue);
     z.glo = glo;
     z.cs = s.C;
+    z.gl = kGroupTokens;
     z.out0 = Pw;
-    z.n_tiles = s.B * gs.k;
+    constexpr int nb = kGroupTokens / 256;
+    z.n_tiles = s.B * gs.k * (nb * (nb + 1) / 2);
     IP_CHECK(launch_tc(FAM_PZ, z, di->num_sms, st));
     TcParams e = tp;
     e.kind = kind_intra();
+    e.gl = kGroupTokens;
     e.vn = s.d % 256 == 0 ? 256 : 128;
     if (!make_map_bf16(&e.map[0], Pw, kGroupTokens, s.T, s.B, 64, 128) ||
         !make_map_bf16(&e.map[1], V, s.d, s.T, s.B, 64, 128))
       return cuda_fail("tensor maps of the within-group term", cudaErrorInvalidValue);
     e.out0 = Ew;
-    e.n_tiles = s.B * gs.k * (s.d / e.vn);
+    e.n_tiles = s.B * ((s.T + 255) / 256) * (s.d / e.vn);
     IP_CHECK(launch_tc(FAM_ZV2, e, di->num_sms, st));
     counted(2);
   }
@@ -535,6 +552,8 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     sc.meta = gmeta;
     sc.upd_kb = update_tokens_per_stage(s.C);  // a stage never spans two chunks of the group
     sc.intra = Ew;
+  } else {
+    sc.upd_scale = 1;  // the update multiplies each chunk's delta by alpha eta
   }
   const int arows = grouped ? apply_rows(group_params(p)) : apply_rows(p);
   const int apply_fam = arows == 256 ? FAM_APPLY256 : FAM_APPLY;

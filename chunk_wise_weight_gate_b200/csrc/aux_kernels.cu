@@ -195,13 +195,104 @@ __global__ void __launch_bounds__(256) k_conv(const T* __restrict__ X0, const T*
   }
 }
 
+// bf16 masked depthwise conv: each thread 8 channels x kRun16 rows, its whole
+// (rows + 4)-row window requested at once so that every thread keeps 12 loads in
+// flight, two blocks of 256 threads per SM (the generic kernel above slides one
+// row at a time and waits on each);
+// two channels per FMA (fma.rn.f32x2), taps in order from zero, one bf16 rounding:
+// the generic kernel's arithmetic, bit for bit.
+constexpr int kRun16 = 8;
+
+__device__ __forceinline__ unsigned long long cv_f2pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ unsigned long long cv_fma2(unsigned long long a, unsigned long long b,
+                                                      unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__global__ void __launch_bounds__(256, 2) k_conv_bf16(const __nv_bfloat16* __restrict__ X0,
+                                                   const __nv_bfloat16* __restrict__ cw,
+                                                   const uint8_t* __restrict__ flags, __nv_bfloat16* __restrict__ U,
+                                                   int B, int Tn, int d, int C) {
+  const int groups = d / 8;
+  const int runs = (Tn + kRun16 - 1) / kRun16;
+  const size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (idx >= (size_t)B * runs * groups) return;
+  const int g = (int)(idx % groups);
+  const size_t rr = idx / groups;
+  const int run = (int)(rr % runs);
+  const int b = (int)(rr / runs);
+  const int t0 = run * kRun16;
+  const __nv_bfloat16* xb = X0 + ((size_t)b * Tn + t0) * d + (size_t)g * 8;
+  uint4 x[kRun16 + 4];
+#pragma unroll
+  for (int q = 0; q < kRun16 + 4; ++q)
+    x[q] = (t0 + q < Tn) ? __ldg(reinterpret_cast<const uint4*>(xb + (size_t)q * d)) : make_uint4(0u, 0u, 0u, 0u);
+  // taps: channel pairs (2p, 2p+1) of tap o as one fp32 pair
+  uint4 wr[5];
+  const uint4* wsrc = reinterpret_cast<const uint4*>(cw + (size_t)g * 8 * kTaps);
+#pragma unroll
+  for (int q = 0; q < 5; ++q) wr[q] = __ldg(wsrc + q);
+  const __nv_bfloat16* wb = reinterpret_cast<const __nv_bfloat16*>(wr);
+  unsigned long long wp[kTaps][4];
+#pragma unroll
+  for (int o = 0; o < kTaps; ++o)
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+      wp[o][p] = cv_f2pack(__bfloat162float(wb[(2 * p) * kTaps + o]), __bfloat162float(wb[(2 * p + 1) * kTaps + o]));
+  // start flags of rows t0 + 1 .. t0 + kRun16 + 3 (a tap past one of them is dropped)
+  const uint8_t* f = flags + (size_t)b * Tn;
+  uint32_t st = 0;
+#pragma unroll
+  for (int q = 1; q < kRun16 + 4; ++q)
+    if (t0 + q < Tn && f[t0 + q]) st |= 1u << q;
+  __nv_bfloat16* ub = U + ((size_t)b * Tn + t0) * d + (size_t)g * 8;
+#pragma unroll
+  for (int r = 0; r < kRun16; ++r) {
+    const int t = t0 + r;
+    if (t >= Tn) break;
+    const int cend = min((t / C + 1) * C, Tn);
+    int n = 1;
+#pragma unroll
+    for (int o = 1; o < kTaps; ++o)
+      if (n == o && t + o < cend && !((st >> (r + o)) & 1u)) n = o + 1;
+    unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int o = 0; o < kTaps; ++o) {
+      if (o < n) {
+        const uint32_t xw[4] = {x[r + o].x, x[r + o].y, x[r + o].z, x[r + o].w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          acc[p] = cv_fma2(wp[o][p], cv_f2pack(__uint_as_float(xw[p] << 16), __uint_as_float(xw[p] & 0xffff0000u)),
+                           acc[p]);
+      }
+    }
+    uint32_t ow[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      float lo, hi;
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc[p]));
+      __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+      ow[p] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(ub + (size_t)r * d) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+  }
+}
+
 cudaError_t conv_target(int dtype, const void* X0, const void* cw, const uint8_t* flags, void* U, const Shape& s,
                         cudaStream_t st) {
   const int blocks = 148 * 8;
-  if (dtype == IPTTT_BF16 && s.d % 8 == 0)
-    k_conv<__nv_bfloat16, 8><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)X0, (const __nv_bfloat16*)cw, flags,
-                                                       (__nv_bfloat16*)U, s.B, s.T, s.d, s.C);
-  else if (dtype == IPTTT_BF16)
+  if (dtype == IPTTT_BF16 && s.d % 8 == 0) {
+    const size_t threads = (size_t)s.B * ((s.T + kRun16 - 1) / kRun16) * (s.d / 8);
+    k_conv_bf16<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>((const __nv_bfloat16*)X0,
+                                                                  (const __nv_bfloat16*)cw, flags,
+                                                                  (__nv_bfloat16*)U, s.B, s.T, s.d, s.C);
+  } else if (dtype == IPTTT_BF16)
     k_conv<__nv_bfloat16, 1><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)X0, (const __nv_bfloat16*)cw, flags,
                                                        (__nv_bfloat16*)U, s.B, s.T, s.d, s.C);
   else if (s.d % 4 == 0)
@@ -578,13 +669,13 @@ __global__ void k_prescale(__nv_bfloat16* V, const float* alpha, int B, int Tn, 
   }
 }
 
-// One block of 256 threads per (row, group of 256 tokens): thread i holds token
-// g0 + i; an inclusive max-scan of (start flag ? i : 0) gives the offset of the
-// last document start at or before the token inside the group (0 if none).
-__global__ void __launch_bounds__(256) k_group_lo(const uint8_t* flags, uint8_t* glo, int Tn, int groups) {
-  __shared__ int wmax[8];
+// One block per (row, group of blockDim.x tokens): thread i holds token g0 + i; an
+// inclusive max-scan of (start flag ? i : 0) gives the offset of the last document
+// start at or before the token inside the group (0 if none).
+__global__ void __launch_bounds__(1024) k_group_lo(const uint8_t* flags, uint16_t* glo, int Tn, int groups) {
+  __shared__ int wmax[32];
   const int b = blockIdx.x / groups, g = blockIdx.x % groups;
-  const int i = threadIdx.x, t = g * 256 + i;
+  const int i = threadIdx.x, t = g * blockDim.x + i;
   const int lane = i & 31, w = i >> 5;
   int v = (t < Tn && flags[(size_t)b * Tn + t]) ? i : 0;
 #pragma unroll
@@ -597,12 +688,13 @@ __global__ void __launch_bounds__(256) k_group_lo(const uint8_t* flags, uint8_t*
   int pre = 0;
   for (int q = 0; q < w; ++q) pre = max(pre, wmax[q]);
   v = max(v, pre);
-  if (t < Tn) glo[(size_t)b * Tn + t] = (uint8_t)v;
+  if (t < Tn) glo[(size_t)b * Tn + t] = (uint16_t)v;
 }
 
-cudaError_t group_meta(const uint8_t* flags, ChunkMeta* gmeta, uint8_t* glo, const Shape& gs, cudaStream_t st) {
+cudaError_t group_meta(const uint8_t* flags, ChunkMeta* gmeta, uint16_t* glo, const Shape& gs, cudaStream_t st) {
+  if (gs.C % 32 != 0 || gs.C > 1024) return cudaErrorInvalidValue;
   k_chunk_meta<<<gs.B * gs.k, 256, 0, st>>>(flags, gmeta, gs.B, gs.T, gs.C, gs.k);
-  k_group_lo<<<gs.B * gs.k, 256, 0, st>>>(flags, glo, gs.T, gs.k);
+  k_group_lo<<<gs.B * gs.k, gs.C, 0, st>>>(flags, glo, gs.T, gs.k);
   return cudaGetLastError();
 }
 

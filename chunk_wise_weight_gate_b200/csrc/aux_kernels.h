@@ -59,9 +59,9 @@ cudaError_t stream_advance(long long* pos, int32_t* cont, int B, int T, cudaStre
 cudaError_t cp_combine(const float* gathered, int world, int rank, const int32_t* plan, void* snap, int nslots,
                        float* Sfinal, const Shape& s, cudaStream_t st);
 cudaError_t prescale_target(void* V, const float* alpha, const Shape& s, float eta, cudaStream_t st);
-// Grouped scan (chunks of 64 or 128 tokens taken 256 tokens at a time): metadata
-// of the 256-token groups (gs: the shape with C = 256) and, per token, the offset
-// in its group of the first token of its document within the group.
-cudaError_t group_meta(const uint8_t* flags, ChunkMeta* gmeta, uint8_t* glo, const Shape& gs, cudaStream_t st);
+// Grouped scan (short chunks taken gs.C tokens at a time, gs.C <= 1024): metadata
+// of the groups (gs: the shape with C = the group length) and, per token, the
+// offset in its group of the first token of its document within the group.
+cudaError_t group_meta(const uint8_t* flags, ChunkMeta* gmeta, uint16_t* glo, const Shape& gs, cudaStream_t st);
 }  // namespace aux
 }  // namespace ipttt

@@ -53,8 +53,8 @@ __device__ __forceinline__ float silu_precise(float x) { return x / (1.0f + expf
 
 // Host helpers (implemented in api.cu).
 ipttt_status cuda_status(cudaError_t e);
-// Tokens per step of the chunk scan: 256 when the bf16 path scans chunks of 64 or
-// 128 tokens in groups, else C.  Streaming pieces that are multiples of it give
+// Tokens per step of the chunk scan: 512 when the bf16 path scans chunks of 64,
+// 128 or 256 tokens in groups, else C.  Streaming pieces that are multiples of it give
 // one call's result bit for bit.
 int scan_unit_tokens(const ipttt_params& p);
 

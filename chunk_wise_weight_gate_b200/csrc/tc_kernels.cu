@@ -224,7 +224,9 @@ __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
     // 128 K per stage; the leader's barrier counts both CTAs' bytes.
     decode_zv<256>(p, tile, j);
     j.halves = 1;
-    j.kb1[0] = (p.kind == K_INTRA ? 256 : p.d) / 128;  // K: d, or the group's 256 tokens
+    // K: d; or, within-group term, the group's tokens up to the end of the tile's
+    // 256-row block (P is zero beyond)
+    j.kb1[0] = (p.kind == K_INTRA ? ((j.m0 % p.gl) / 256 + 1) * 256 : p.d) / 128;
     j.tx = 2 * (128 * 128 * 2 + (j.n_mma / 2) * 128 * 2);
   }
   else if constexpr (FAM == FAM_GRAM) decode_gram(p, tile, j);
@@ -238,12 +240,19 @@ __device__ __forceinline__ void decode(const TcParams& p, int tile, Job& j) {
     j.tx = 2 * (2 * 128 * 128 * 2);
   }
   else if constexpr (FAM == FAM_PZ) {
-    // one group of 256 tokens of one row: its rows against its columns, K = d_ff
-    const int groups = cdiv(p.T, 256);
+    // one 256 x 256 block (row block rb, column block cb <= rb) of one group of
+    // p.gl tokens of one row: its rows against its columns, K = d_ff
+    const int groups = cdiv(p.T, p.gl);
+    const int nb = p.gl / 256;
+    const int per_group = nb * (nb + 1) / 2;
+    const int g = tile / per_group;
+    int rb = 0, rem = tile % per_group;
+    while (rem > rb) { rem -= rb + 1; ++rb; }
     j.kind = K_GRAM;
-    j.b = tile / groups;
-    j.t0 = (tile % groups) * 256;
-    j.m0 = j.n0 = 0;
+    j.b = g / groups;
+    j.t0 = (g % groups) * p.gl;
+    j.m0 = rb * 256;
+    j.n0 = rem * 256;
     j.chunk = j.pair = 0;
     j.nseg = 1;
     j.kb0[0] = 0;
@@ -294,8 +303,9 @@ __device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int
       // Wtarget[k][n] (or, within-group term, V'[b][group token k][n]), n contiguous
       const int nh = p.vn / 2;
       const bool intra = j.kind == K_INTRA;
+      const int kofs = intra ? j.m0 - j.m0 % p.gl : 0;  // the group's first token
       for (int q = 0; q < nh / 64; ++q)
-        tma_load_3d_pair(sb + q * 64 * 128 * 2, &p.map[1], fb, j.n0 + (int)r * nh + 64 * q, (intra ? j.m0 : 0) + k0,
+        tma_load_3d_pair(sb + q * 64 * 128 * 2, &p.map[1], fb, j.n0 + (int)r * nh + 64 * q, kofs + k0,
                          intra ? j.b : 0);
     }
   } else if constexpr (is_zv<FAM>()) {
@@ -388,21 +398,22 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
       }
     }
   } else if constexpr (FAM == FAM_PZ) {
-    // Row t of the group (this CTA's 128, j.m0 holds the CTA's offset) against
-    // columns u of [128 half, 128 half + 128): z_t . z_u is kept where u lies in
-    // t's document (u >= lo(t)) and in an earlier chunk (u < the start of t's chunk).
+    // Row t of the group (j.m0: the row block and this CTA's offset) against
+    // columns u of the column block j.n0, [128 half, 128 half + 128): z_t . z_u is
+    // kept where u lies in t's document (u >= lo(t)) and in an earlier chunk (u <
+    // the start of t's chunk).
     const int t = j.t0 + j.m0 + row;
     const bool valid = t < p.T;
     const int lo = valid ? j.t0 + (int)p.glo[(size_t)j.b * p.T + t] : 0;
     const int hi = valid ? (t / p.cs) * p.cs : 0;
-    __nv_bfloat16* prow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * 256;
+    __nv_bfloat16* prow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.gl + j.n0;
 #pragma unroll 1
     for (int c = half * 128; c < half * 128 + 128; c += 32) {
       tmem_ld32(tacc + c, r0);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const int u = j.t0 + c + i;
+        const int u = j.t0 + j.n0 + c + i;
         v[i] = (u >= lo && u < hi) ? __uint_as_float(r0[i]) : 0.0f;
       }
       if (valid) st_bf16x32(prow + c, v);
@@ -903,12 +914,14 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
       const bool snap = jb.chunk + 1 < p.k;
       const float* sf = reinterpret_cast<const float*>(upd_state_block(p, jb.b, m0c, jb.n0, half));
       // Folds 64 columns of the delta (two 32-column TMEM loads) into st[64 hb ..].
+      // the chunk's clip factor times eta, when V was not pre-scaled by it
+      const float sc = p.upd_scale ? p.alpha[(size_t)jb.b * p.k + jb.chunk] * p.eta : 1.0f;
       auto fold = [&](const int hb, const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
 #pragma unroll
         for (int q = 0; q < 64; ++q) {
           const int c = 64 * hb + q;
           const float old = base == 2 ? sf[((c / 4) * 128 + row) * 4 + (c & 3)] : base == 1 ? st[c] : 0.0f;
-          st[c] = old + __uint_as_float(q < 32 ? ra[q & 31] : rb[q & 31]);
+          st[c] = fmaf(sc, __uint_as_float(q < 32 ? ra[q & 31] : rb[q & 31]), old);
         }
       };
       // Snapshot box hb: 32 rows x 64 columns of bf16(S_{chunk+1}) (what the apply of

@@ -13,10 +13,10 @@ namespace tck {
 // M=256 pair MMAs, 128 K per stage); launched as clusters of two.
 // FAM_GRAM2: the Gram pass on 256 x 256 token-block pairs, one cluster of two per
 // block pair; each CTA writes its own partial (2 per pair, npairs = pairs per chunk).
-// FAM_PZ: per group of 256 tokens of a row, the masked token-token products
-// P[t][u] = z_t . z_u for u in t's document and in an earlier chunk of the group
-// (cta pairs, K = d_ff), written as bf16 [B][T][256]; the grouped scan's
-// within-group term.
+// FAM_PZ: per group of gl tokens of a row (gl a multiple of 256), the masked
+// token-token products P[t][u] = z_t . z_u for u in t's document and in an
+// earlier chunk of the group (cta pairs, K = d_ff, 256 x 256 blocks on and below
+// the diagonal), written as bf16 [B][T][gl]; the grouped scan's within-group term.
 enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_APPLY256 = 5, FAM_ZV2 = 6, FAM_GRAM2 = 8, FAM_PZ = 9 };
 
 struct TcParams {
@@ -44,10 +44,12 @@ struct TcParams {
   const void* src0;       // fused target: X0 [B][T][d]
   const void* src1;       // fused target: conv_w [d][5]
   const uint8_t* flags;   // fused target: document-start flags [B][T]
-  const uint8_t* glo;     // FAM_PZ: per token, its document's first token within its group (offset)
-  int cs;                 // FAM_PZ: chunk length (the group holds 256 / cs chunks)
+  const uint16_t* glo;    // FAM_PZ: per token, its document's first token within its group (offset)
+  int cs;                 // FAM_PZ: chunk length
+  int gl;                 // FAM_PZ, K_INTRA: tokens per group of the grouped scan
   const void* intra;      // apply: optional within-group term E [B][T][d] bf16, added to the fast-weight part
   int upd_kb;             // update: tokens per stage (0: update_tokens_per_stage(C))
+  int upd_scale;          // update: 1 = V is not pre-scaled; the delta is scaled by alpha[b][chunk] eta
 };
 
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,

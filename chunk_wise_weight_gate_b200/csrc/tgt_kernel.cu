@@ -18,13 +18,12 @@
 //                        CTA's barrier, no multicast);
 //   warp 9, one thread of the even CTA: the MMAs;
 //   warps 0-7          : U for this CTA's 128 rows and the stage's 64 channels, read
-//                        from X0 in global memory (each thread 8 channels x 8 rows
-//                        through a 12-row window, the next stage's window loaded
-//                        while the current one is computed), written as bf16 in the
-//                        128-byte-swizzled K-major layout the MMA reads, then made
-//                        visible to the tensor cores (proxy fence, release at
-//                        cluster scope).  Warps 0-3 fill the even stages, 4-7 the
-//                        odd ones.
+//                        from X0 in global memory (each thread 8 channels x 16 rows
+//                        through a 20-row window), written as bf16 in the 128-byte-
+//                        swizzled K-major layout the MMA reads, then made visible to
+//                        the tensor cores (proxy fence, release at cluster scope).
+//                        Four groups of two warps take the stages in turn; a group
+//                        requests its next window right after publishing a stage.
 // The conv arithmetic is that of the stand-alone conv kernel (fp32 FMAs in tap
 // order, one bf16 rounding), done two channels per instruction (fma.rn.f32x2).
 // There is one accumulator, so the MMAs of a tile wait for the previous tile's
@@ -66,6 +65,10 @@ static_assert((TG_THREADS - 32 * TG_EPI_WARPS) * (TG_REGS_LAUNCH - TG_REGS_LOW) 
               "the register trade of the fused target kernel must balance");
 constexpr int TG_SMEM = 1024 + TG_STAGES * TG_STAGE_BYTES + 256;
 constexpr int TG_TAPS = 5;
+// conv producers: TG_GROUPS groups of two warps, group g filling the stages kb = g
+// mod TG_GROUPS; a thread computes TG_RUN rows x 8 channels of its 128 rows
+constexpr int TG_GROUPS = 4, TG_RUN = 16;
+static_assert(TG_GROUPS * 2 == TG_EPI_WARPS && 8 * TG_RUN == 128, "conv producer layout");
 static_assert(TG_SMEM <= 232448, "fused target kernel exceeds shared memory");
 
 struct TgJob {
@@ -123,7 +126,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TG_STAGES * TG_STAGE_BYTES);
-  uint64_t* full = bars;                   // [STAGES] even CTA: Wtarget bytes + 8 conv warps
+  uint64_t* full = bars;                   // [STAGES] even CTA: Wtarget bytes + the conv warps
   uint64_t* empty = bars + TG_STAGES;      // [STAGES] MMA -> producers, both CTAs
   uint64_t* acc_full = empty + TG_STAGES;  // MMA -> epilogue, both CTAs
   uint64_t* acc_empty = acc_full + 1;      // even CTA: 8 epilogue warps of each CTA
@@ -141,7 +144,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < TG_STAGES; ++s) {
-      mbar_init(&full[s], 1 + 2 * 4);
+      mbar_init(&full[s], 1 + 2 * (TG_EPI_WARPS / TG_GROUPS));  // TMA + the stage group's warps of both CTAs
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
@@ -166,11 +169,13 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(TG_REGS_EPI));
     const int ew = warp;
     const int quarter = warp & 3;  // TMEM lanes this warp may access
-    const int half = ew >> 2;      // epilogue: accumulator (256-column half); conv: even / odd stages
+    const int half = ew >> 2;      // epilogue: accumulator (256-column half)
     const int erow = quarter * 32 + lane;
-    // conv role: chunk of 8 channels and run of 8 rows of this CTA's 128
+    // conv role: stage group (stages kb = grp mod TG_GROUPS), chunk of 8 channels
+    // and run of TG_RUN rows of this CTA's 128
+    const int grp = ew >> 1;
     const int cj = lane & 7;
-    const int rg = (ew & 3) * 4 + (lane >> 3);
+    const int rg = (ew & 1) * 4 + (lane >> 3);
     const __nv_bfloat16* X0 = reinterpret_cast<const __nv_bfloat16*>(p.src0);
     const __nv_bfloat16* cw = reinterpret_cast<const __nv_bfloat16*>(p.src1);
     const uint32_t acc_empty0 = map_to_rank(smem_u32(acc_empty), 0);
@@ -214,14 +219,14 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
       return true;
     };
 
-    // Taps in use for this thread's 8 rows of tile jj (the same for every stage of
-    // the tile), 3 bits per row.
-    auto taps_of = [&](const TgJob& jj) -> uint32_t {
-      const int t0 = jj.m0 + 128 * (int)rank + rg * 8;
+    // Taps in use for this thread's rows of tile jj (the same for every stage of the
+    // tile), 3 bits per row.
+    auto taps_of = [&](const TgJob& jj) -> uint64_t {
+      const int t0 = jj.m0 + 128 * (int)rank + rg * TG_RUN;
       const uint8_t* fl = p.flags + (size_t)jj.b * p.T;
-      uint32_t packed = 0;
+      uint64_t packed = 0;
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
+      for (int r = 0; r < TG_RUN; ++r) {
         const int t = t0 + r;
         int n = 1;
         if (t < p.T) {
@@ -230,35 +235,37 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
           for (int o = 1; o < TG_TAPS; ++o)
             if (n == o && t + o < cend && !fl[t + o]) n = o + 1;
         }
-        packed |= (uint32_t)n << (3 * r);
+        packed |= (uint64_t)n << (3 * r);
       }
       return packed;
     };
-    // The 12-row X0 window (8 channels) of this thread for stage kb of tile jj.
-    auto load_window = [&](uint4 (&x)[12], const TgJob& jj, int kb) {
-      const int t0 = jj.m0 + 128 * (int)rank + rg * 8;
+    // The X0 window (8 channels, TG_RUN + 4 rows) of this thread for stage kb of tile jj.
+    auto load_window = [&](uint4 (&x)[TG_RUN + 4], const TgJob& jj, int kb) {
+      const int t0 = jj.m0 + 128 * (int)rank + rg * TG_RUN;
       const __nv_bfloat16* xrow = X0 + ((size_t)jj.b * p.T + t0) * p.d + kb * TG_KB + cj * 8;
 #pragma unroll
-      for (int q = 0; q < 12; ++q)
+      for (int q = 0; q < TG_RUN + 4; ++q)
         x[q] = (t0 + q < p.T) ? *reinterpret_cast<const uint4*>(xrow + (size_t)q * p.d) : make_uint4(0u, 0u, 0u, 0u);
     };
 
-    // This group's stages are kb = half, half + 2, ... of every tile (a tile has an
-    // even number of stages).  The X0 window of the next one is loaded while the
-    // current one is computed.
+    // This group's stages are kb = grp, grp + TG_GROUPS, ... of every tile (a tile's
+    // stage count is a multiple of TG_GROUPS).  The X0 window of the next one is
+    // requested right after this stage is published: the loads then have the
+    // other groups' stages to arrive in, and are not in flight when the release
+    // below orders this thread's memory operations.
     TgJob j, jn, jprev;
     bool have_prev = false;
-    uint4 nx[12];
-    uint32_t ntp_n = 0;
+    uint4 xr[TG_RUN + 4];
+    uint64_t ntp_n = 0;
     bool have_j = tg_job(p, 0, wk, nwk, j);
     if (have_j) {
       ntp_n = taps_of(j);
-      load_window(nx, j, half);
+      load_window(xr, j, grp);
     }
     for (uint32_t i = 0; ok && have_j; ++i) {
-      const uint32_t ntp = ntp_n;
+      const uint64_t ntp = ntp_n;
       const bool have_jn = tg_job(p, i + 1, wk, nwk, jn);
-      for (int kb = half; kb < nk; kb += 2) {
+      for (int kb = grp; kb < nk; kb += TG_GROUPS) {
         if (kb >= TG_STAGES && have_prev) {
           // the next tile's first stages are filled: drain the previous tile
           if (!epilogue(jprev, tcount - 1)) { ok = false; break; }
@@ -267,15 +274,6 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
         const uint32_t it = i * (uint32_t)nk + (uint32_t)kb;
         const int s = it % TG_STAGES;
         const uint32_t ph = (it / TG_STAGES) & 1;
-        uint4 xr[12];
-#pragma unroll
-        for (int q = 0; q < 12; ++q) xr[q] = nx[q];
-        if (kb + 2 < nk) {
-          load_window(nx, j, kb + 2);
-        } else if (have_jn) {
-          ntp_n = taps_of(jn);
-          load_window(nx, jn, half);
-        }
         uint4 wr[5];
         const uint4* wsrc = reinterpret_cast<const uint4*>(cw + (size_t)(kb * TG_KB + cj * 8) * TG_TAPS);
 #pragma unroll
@@ -291,7 +289,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
             wp[o][q] = f2pack(__bfloat162float(wb[(2 * q) * TG_TAPS + o]), __bfloat162float(wb[(2 * q + 1) * TG_TAPS + o]));
         uint8_t* sa = stages + s * TG_STAGE_BYTES;
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
+        for (int r = 0; r < TG_RUN; ++r) {
           const int nt = (int)((ntp >> (3 * r)) & 7u);
           unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -309,12 +307,18 @@ __global__ void __launch_bounds__(TG_THREADS, 1) tgt_kernel(const __grid_constan
             f2unpack(acc[q], lo, hi);
             ow[q] = pack_bf16x2(lo, hi);
           }
-          const int row = rg * 8 + r;
+          const int row = rg * TG_RUN + r;
           *reinterpret_cast<uint4*>(sa + row * 128 + ((cj ^ (row & 7)) << 4)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive_release_cluster(full0 + 8u * s);
+        if (kb + TG_GROUPS < nk) {
+          load_window(xr, j, kb + TG_GROUPS);
+        } else if (have_jn) {
+          ntp_n = taps_of(jn);
+          load_window(xr, jn, grp);
+        }
       }
       if (!ok) break;
       if (have_prev) {  // a tile of at most STAGES stages

@@ -141,10 +141,11 @@ IPTTT_API ipttt_status ipttt_core(const ipttt_params* p, const void* Z, const vo
  * equals one call over the whole sequence.  params->T is the piece length and
  * must be a multiple of C except for the final piece of a sequence (the conv
  * look-ahead and the update both close at chunk ends).  The bf16 path scans
- * chunks of 64 or 128 tokens in groups of 256 tokens, starting at each call's
- * first token; pieces whose lengths are multiples of the scan group (256 tokens
- * then, else C) give one call's result bit for bit, other whole-chunk pieces give
- * it up to rounding (the state sums and snapshots are grouped differently).
+ * chunks of 64, 128 or 256 tokens in groups of 512 tokens, starting at each
+ * call's first token; pieces whose lengths are multiples of the scan group (512
+ * tokens then, else C) give one call's result bit for bit, other whole-chunk
+ * pieces give it up to rounding (the state sums and snapshots are grouped
+ * differently).
  * doc_starts are offsets
  * b*T + t within the piece; a piece start is a document start only when the row
  * has consumed nothing yet or when doc_starts lists it.

@@ -52,7 +52,10 @@ def test_decode_equals_forward_and_oracle():
 
 
 def test_decode_commits_the_prefill_state():
-    B, C = 2, 256
+    # chunks of 512 tokens: a one-call forward then also scans chunk by chunk, as
+    # the decode commits do (shorter chunks are scanned in groups of 512 tokens,
+    # which agree with chunk-by-chunk commits up to rounding)
+    B, C = 2, 512
     T = 3 * C
     cfg, inp = case(B, T, C, 256, 512, eta=1e-3, clip=1e-5, docs=[300, T + 20])
     dev = torch.device("cuda")

@@ -118,6 +118,25 @@ def test_bf16_long_scan_state(name):
     assert abs(scale_bias(S, S_ref)) <= BIAS_TOL
 
 
+@pytest.mark.parametrize("name", ["clip_docs_ragged_multitile", "chunk256_docs_ragged"])
+def test_fused_target_kernel(name, monkeypatch):
+    """The target GEMM with the masked conv in its producer (IPTTT_FUSED_TARGET=1)
+    computes the conv with the conv kernel's arithmetic and feeds the same MMAs in
+    the same K order: V, and so every output, equals the default path's bit for bit;
+    both match the oracle."""
+    kw = dict(BF16_CASES[name])
+    if kw["d"] % 256:
+        kw["d"] = 512  # the fused kernel takes d % 256 == 0
+    cfg, inp = case(**kw)
+    ref = gpu(cfg, inp)
+    monkeypatch.setenv("IPTTT_FUSED_TARGET", "1")
+    out = gpu(cfg, inp)
+    monkeypatch.delenv("IPTTT_FUSED_TARGET")
+    for key in ("V", "O", "S_final"):
+        assert torch.equal(out[key], ref[key]), key
+    check_bf16(out, oracle(cfg, inp), cfg.clip)
+
+
 def test_bf16_eta_zero_is_plain_gated_mlp():
     cfg, inp = case(1, 384, 128, 256, 512, eta=0.0, clip=1e-5)
     out = gpu(cfg, inp)
@@ -169,7 +188,7 @@ def stream_pieces(cfg, inp, bounds):
 
 
 def test_bf16_streaming_pieces_of_part_groups():
-    """128-token chunks are scanned in groups of 256 tokens; a piece that splits a
+    """128-token chunks are scanned in groups of 512 tokens; a piece that splits a
     group regroups the state sums and snapshots: equal up to that rounding."""
     cfg, inp = case(2, 768, 128, 256, 512, eta=2e-2, clip=0.0, docs=[100, 300, 768 + 500])
     one = gpu(cfg, inp)
@@ -188,8 +207,8 @@ def test_bf16_streaming_equals_one_shot():
     st = ip.StreamState(cfg)
     outs = []
     docs = inp["doc_starts"].numpy()
-    # pieces of whole scan groups (256 tokens for 128-token chunks)
-    for a, b in ((0, 256), (256, 512), (512, 768)):
+    # pieces of whole scan groups (512 tokens for 128-token chunks)
+    for a, b in ((0, 512), (512, 768)):
         pc = ip.LayerConfig(B=2, T=b - a, d=cfg.d, F=cfg.F, C=cfg.C, eta=cfg.eta, clip=cfg.clip)
         pd = [int((g // cfg.T) * (b - a) + (g % cfg.T - a)) for g in docs if a <= g % cfg.T < b]
         H = inp["H"][:, a:b].contiguous().to(dev)
