@@ -231,7 +231,7 @@ def config_dict(w: synth.Workload, n: int) -> dict:
 # one step captured by ncu, keyed by (workload, chunk size, phase); the summaries in
 # profiles/ give the commands.  The roofline object carries a figure only for the
 # kernel and workload it was taken on.
-MEASURED_TRAFFIC = {("qwen3_4b_128k", 1024, "apply"): 2.577e9 + 104.45e6}
+MEASURED_TRAFFIC = {("qwen3_4b_128k", 1024, "apply"): 2452600192.0}
 
 
 def sample_chunks(w: synth.Workload, tokens: int) -> int:
@@ -272,7 +272,7 @@ def run_ours(args, w: synth.Workload):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     pg = None
-    if world > 1 and not emulated:
+    if world > 1:
         import torch.distributed as dist
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
@@ -295,7 +295,8 @@ def run_ours(args, w: synth.Workload):
 
     def step(H, X0, out):
         if w.layers == 1:
-            ip.forward(cfg, H, X0, *(dev_w[0][k] for k in WEIGHTS), docs_dev, O=out, workspace=ws)
+            ip.forward(cfg, H, X0, *(dev_w[0][k] for k in WEIGHTS), docs_dev, O=out, workspace=ws,
+                       state_clip=args.state_clip)
             return
         cur = H
         for l in range(w.layers):
@@ -417,7 +418,7 @@ def run_ours(args, w: synth.Workload):
                "d2h_bytes_per_step": o_host.numel() * o_host.element_size(), "ms_per_step": ems, "api": api}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.state_clip:
         chunks = sample_chunks(w, args.cpu_sample_tokens)
         secs, n = oracle_sample(w, layers[0], chunks)
         cpu = {"value": n / secs, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
@@ -427,7 +428,9 @@ def run_ours(args, w: synth.Workload):
     if rank == 0:
         out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-               "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w, world),
+               "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+               "config": {**config_dict(w, world),
+                          **({"clip_on": "accumulated state (ablation)"} if args.state_clip else {})},
                "tflops": tflops, "frac_of_peak": tflops / world / peaks.get("bf16_tflops_sustained", 1.0),
                "flops_per_token": ip.flops_per_token(w.d, w.F),
                # the count for exact arithmetic, where W0 + S_i would be one operand: 8dF + 2d^2
@@ -604,7 +607,7 @@ def run_cp(args, w: synth.Workload):
             "launches": dom_launches, "peak_note": f"sustained bf16 and copy bandwidth ({peak_src}); rank {rank}'s phases"}
     phase_report = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
                     for k, v in phases.items()}
-    if rank == 0:
+    if rank == 0 or emulated:
         cfgd = config_dict(w, world)
         cfgd.update({"workload": f"cp_{w.name}", "parallelism": f"cp{world}", "shard_tokens": TL, "global_batch": w.B,
                      "exchange": "NCCL all-gather of the fp32 shard aggregates" if pg else "none"})
@@ -624,6 +627,100 @@ def run_cp(args, w: synth.Workload):
         pg.destroy_process_group()
 
 
+def backward_flops_per_token(d: int, F: int, dtype: str) -> int:
+    """Flops of ipttt_backward per token.  fp32 (CUDA cores): the forward products it
+    recomputes (gate, up, target, each chunk's V^T Z: 6dF + 2d^2) and the gradient
+    products (gW0, gO W0, per chunk P, gV, gZ from the delta, gZ from the state,
+    the state's gradient: 14dF; gH and gWgate, gWup: 8dF; gU, gWtarget: 4d^2).
+    bf16 (tensor cores): the whole forward (10dF + 2d^2, its apply included) and
+    then gate and up pre-activations 4dF, gO W0 2dF, gW0 2dF, per chunk P and the
+    state gradient's deltas 4dF, Z G^T 2dF, Z P^T 2dF, three gZ terms 6dF, gH 4dF,
+    gWgate and gWup 4dF, gU and gWtarget 4d^2: 40dF + 6d^2."""
+    if dtype == "bf16":
+        return 40 * d * F + 6 * d * d
+    return 28 * d * F + 6 * d * d
+
+
+def run_backward(args, w: synth.Workload):
+    """The backward of one layer (ipttt_backward: fp32 gradients of <gO, O> +
+    <gS, S_final> with respect to H, X0 and the five weights) on the workload's
+    shapes.  bf16 workloads run it on the tensor cores (roofline: the bf16 peak),
+    fp32 ones on the CUDA cores (roofline: the fp32 FMA rate)."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    inp = synth.make_inputs(w, seed=rank)
+    cfg = ip.LayerConfig(B=w.B, T=w.T, d=w.d, F=w.F, C=w.C, eta=w.eta, clip=w.clip, dtype=w.dtype)
+    t = {k: inp[k].to(dev) for k in ("H", "X0") + WEIGHTS}
+    docs = inp["doc_starts"]
+    g = torch.Generator().manual_seed(11 + rank)
+    gO = torch.randn(w.B, w.T, w.d, generator=g).to(cfg.torch_dtype).to(dev)
+    gS = torch.randn(w.B, w.d, w.F, generator=g).to(dev)
+    del inp
+    ws = torch.empty(ip.backward_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return ip.backward(cfg, *(t[k] for k in ("H", "X0") + WEIGHTS), docs, gO, gS, workspace=ws)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if ip.get_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+    gpu_id = str(local)
+    try:
+        gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
+        if not gpu_id.startswith("GPU-"):
+            gpu_id = "GPU-" + gpu_id
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    launches0 = ip.kernel_launches()
+    sampler.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    launches = ip.kernel_launches() - launches0
+    ms = e0.elapsed_time(e1) / args.steps
+    status = ip.get_status()
+    tokens = w.B * w.T
+    flops = backward_flops_per_token(w.d, w.F, w.dtype) * tokens
+    ach = flops / (ms / 1000.0) / 1e12
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
+    peaks, peak_src = load_peaks()
+    if w.dtype == "bf16":
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        roof = {"kernel": "whole backward (tcgen05 GEMMs on bf16 operands, fp32 accumulators)", "bound": "tensor",
+                "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                "peak_note": f"sustained bf16 ({peak_src}); burst {peaks['bf16_tflops']}"}
+    else:
+        peak = fp32_fma_tflops(sms, mhz)
+        roof = {"kernel": "whole backward (fp32 CUDA-core GEMMs and elementwise kernels)", "bound": "alu",
+                "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                "peak_note": f"fp32 FMA rate: {sms} SMs x 128 lanes x 2 flops x {mhz:.0f} MHz"}
+    cfgd = config_dict(w, 1)
+    cfgd.update({"workload": f"backward_{w.name}", "gradients": "H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget (fp32)"})
+    out = {"metric": "In-Place TTT MLP layer backward tokens/s (fp32 gradients of O and S_final)",
+           "value": tokens / (ms / 1000.0), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+           "config": cfgd, "flops_per_token": backward_flops_per_token(w.d, w.F, w.dtype), "roofline": roof,
+           "clocks": clocks, "e2e": None, "gpu_launches": launches, "cpu_baseline": None,
+           "device_status": status}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -632,13 +729,16 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--chunk", type=int, default=None, help="override the chunk size C")
-    ap.add_argument("--mode", choices=("prefill", "decode", "cp"), default="prefill",
+    ap.add_argument("--mode", choices=("prefill", "decode", "cp", "backward"), default="prefill",
                     help="decode: token-by-token decoding of --decode-batch rows instead of the prefill step; "
-                         "cp: the sequence split along T over the GPUs (context parallelism)")
+                         "cp: the sequence split along T over the GPUs (context parallelism); "
+                         "backward: the layer's gradients (ipttt_backward)")
     ap.add_argument("--decode-batch", type=int, default=8)
     ap.add_argument("--cp-world", type=int, default=1,
                     help="with --mode cp on one GPU: run one rank's share of a split over this many ranks")
     ap.add_argument("--cp-rank", type=int, default=0, help="the rank that --cp-world runs")
+    ap.add_argument("--state-clip", action="store_true",
+                    help="the ablation that clips the accumulated state instead of each delta (fp32 workloads)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--piece-tokens", type=int, default=0,
                     help="e2e: tokens per pipelined piece of the host-buffer call (0: about T/8)")
@@ -659,6 +759,8 @@ def main(argv=None):
         run_decode(args, w)
     elif args.mode == "cp":
         run_cp(args, w)
+    elif args.mode == "backward":
+        run_backward(args, w)
     else:
         run_ours(args, w)
 

@@ -17,7 +17,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libipttt.so")
 BUILD_DIR = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "aux_kernels.cu", "tc_kernels.cu", "tgt_kernel.cu", "host_pipeline.cu", "decode.cu"]
+SOURCES = ["api.cu", "aux_kernels.cu", "tc_kernels.cu", "tgt_kernel.cu", "host_pipeline.cu", "decode.cu",
+           "backward.cu", "gemm.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", CSRC, "-I", INCLUDE]

@@ -114,7 +114,7 @@ struct PhaseScope {
   }
 };
 
-inline void counted(int n) { g_launches.fetch_add((uint64_t)n); }
+inline void counted(long long n) { g_launches.fetch_add((uint64_t)n); }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -125,6 +125,7 @@ struct Layout {
   bool grouped;
   size_t cp_docs, cp_plan;  // context-parallel calls: local document starts, per-row plan
   int group;  // bf16 path: chunks whose apply tiles share one launch (= snapshot ring slots)
+  bool keep_all;  // bf16 forward run for the backward: every chunk's state copy kept, U written
 };
 
 // Apply tiles of `group` consecutive chunks share one launch (and the snapshot
@@ -214,7 +215,9 @@ Shape shape_of(const ipttt_params& p) {
 // cp: the layout of the context-parallel calls, whose snapshot ring holds every
 // chunk's S_i (k + 1 slots: the apply runs after all the shard's updates) and
 // which keep the shard's document starts and per-row plan on the device.
-Layout layout_of(const ipttt_params& p, bool cp = false) {
+// keep_all: the forward run of the backward, which keeps S_i in slot i for every
+// chunk, scans chunk by chunk and writes U.
+Layout layout_of(const ipttt_params& p, bool cp = false, bool keep_all = false) {
   const Shape s = shape_of(p);
   const size_t B = s.B, T = s.T, d = s.d, F = s.F, k = s.k;
   Layout L{};
@@ -234,9 +237,10 @@ Layout layout_of(const ipttt_params& p, bool cp = false) {
     L.U = take(B * T * d * 2);
     L.V = take(B * T * d * 2);
     L.S = take(B * d * F * 4);
-    L.grouped = grouped_scan(p);
+    L.keep_all = keep_all;
+    L.grouped = !keep_all && grouped_scan(p);
     const size_t kg = (T + kGroupTokens - 1) / kGroupTokens;
-    L.group = cp ? (int)(L.grouped ? kg : s.k) + 1 : apply_group(L.grouped ? group_params(p) : p);
+    L.group = (cp || keep_all) ? (int)(L.grouped ? kg : s.k) + 1 : apply_group(L.grouped ? group_params(p) : p);
     L.snap = take((size_t)L.group * B * d * F * 2);
     L.raw = L.dpart = 0;
     L.gmeta = L.glo = L.P = L.E = 0;
@@ -272,7 +276,9 @@ ipttt_status check_params(const ipttt_params* p) {
   if (p->dtype != IPTTT_F32 && p->dtype != IPTTT_BF16) return IPTTT_ERR_DTYPE;
   if (p->B <= 0 || p->T <= 0 || p->d <= 0 || p->F <= 0 || p->C <= 0) return IPTTT_ERR_ARG;
   if (!isfinite(p->eta) || isnan(p->clip_thresh)) return IPTTT_ERR_ARG;
-  if ((p->flags & ~IPTTT_FLAG_RESIDUAL) != 0) return IPTTT_ERR_ARG;
+  if ((p->flags & ~(IPTTT_FLAG_RESIDUAL | IPTTT_FLAG_STATE_CLIP)) != 0) return IPTTT_ERR_ARG;
+  // the clip on the accumulated state runs on the fp32 path only
+  if ((p->flags & IPTTT_FLAG_STATE_CLIP) && p->dtype != IPTTT_F32) return IPTTT_ERR_UNSUPPORTED;
   const long long BT = (long long)p->B * p->T;
   if (BT > (1ll << 30) || (long long)p->d * p->F > (1ll << 31) || (long long)p->d * p->d > (1ll << 31) ||
       BT * (long long)p->F > (1ll << 40))
@@ -383,7 +389,7 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   // trip costs less than the producer's conv arithmetic recomputed for every
   // 512-column tile).
   const char* fe = getenv("IPTTT_FUSED_TARGET");
-  const bool fused_target = pair_gemm && fe && fe[0] == '1' && fused_target_supported(s.d) &&
+  const bool fused_target = pair_gemm && !L.keep_all && fe && fe[0] == '1' && fused_target_supported(s.d) &&
                             fused_target_workers(st) > 0;
   // the grouped scan's within-group products run on CTA pairs
   const bool grouped = scan_grouped(L, st);
@@ -573,9 +579,9 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   const bool need_final = t.Sfinal != nullptr || ss != nullptr;
   const int state_tiles = s.B * (s.d / 128) * ((s.F + 255) / 256);  // 128 x 256 tiles
   const int apply_tiles_per_chunk = s.B * (sq.C / arows) * (s.d / 128);
-  // State updates of chunks [c0, c1) in one launch: each block keeps its state
-  // tiles in TMEM through all of them and writes S_{c+1} snapshots into slot
-  // (c+1) % G.
+  // State updates of chunks [c0, c1) in one launch: each worker carries its state
+  // tiles' fp32 state in registers through all of them and writes S_{c+1}
+  // snapshots into slot (c+1) % G.
   auto update = [&](int c0, int c1) -> ipttt_status {
     if (c1 <= c0) return IPTTT_OK;
     PhaseScope ph(st, PH_UPDATE);
@@ -700,7 +706,10 @@ ipttt_status run_f32(const ipttt_params& p, const Tensors& t, uint8_t* ws, const
     r.mode = SM_RAW;
     r.out = raw; r.som = F; r.son = 1; r.sob = d * F;
     IP_CHECK(simt_gemm(r, s.B, st));
-    IP_CHECK(simt_update_state(S, raw, dpart, alpha, meta, s, i, p.eta, tau, st));
+    if (p.flags & IPTTT_FLAG_STATE_CLIP)
+      IP_CHECK(simt_update_state_clipped(S, raw, dpart, alpha, meta, s, i, p.eta, tau, st));
+    else
+      IP_CHECK(simt_update_state(S, raw, dpart, alpha, meta, s, i, p.eta, tau, st));
   }
   if (t.alpha) IP_CHECK(cudaMemcpyAsync(t.alpha, alpha, (size_t)s.B * s.k * 4, cudaMemcpyDeviceToDevice, st));
   if (t.Sfinal) IP_CHECK(state_export(false, S, t.Sfinal, s, st));
@@ -996,6 +1005,88 @@ const char* ipttt_strerror(ipttt_status s) {
 }
 
 const char* ipttt_version(void) { return "0.2.0"; }
+
+// The backward takes the forward's shape rules: any shape in fp32 (CUDA cores),
+// the tensor-core shapes in bf16.
+static ipttt_status backward_params(const ipttt_params* p) { return check_params(p); }
+
+// bf16 workspace: the forward's layout with every state copy kept, O of that
+// forward, then the backward's own buffers.
+struct BwdTcLayout {
+  Layout fwd;
+  size_t O, tc, total;
+};
+static BwdTcLayout bwd_tc_layout(const ipttt_params& p) {
+  BwdTcLayout L;
+  L.fwd = layout_of(p, false, true);
+  const Shape s = shape_of(p);
+  L.O = align256(L.fwd.total);
+  L.tc = L.O + align256((size_t)s.B * s.T * s.d * 2);
+  L.total = L.tc + bwd::tc_workspace_bytes(s);
+  return L;
+}
+
+size_t ipttt_backward_workspace_size(const ipttt_params* p) {
+  if (backward_params(p) != IPTTT_OK) return 0;
+  if (p->dtype == IPTTT_BF16) return bwd_tc_layout(*p).total;
+  return bwd::workspace_bytes(shape_of(*p));
+}
+
+ipttt_status ipttt_backward(const ipttt_params* p, const void* H, const void* X0, const void* Wgate, const void* Wup,
+                            const void* Wdown0, const void* conv_w, const void* Wtarget, const int32_t* doc_starts,
+                            int32_t n_doc_starts, const void* gO, const float* gS_final_opt, float* gH, float* gX0,
+                            float* gWgate, float* gWup, float* gWdown0, float* gconv_w, float* gWtarget,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  ipttt_status rc = backward_params(p);
+  if (rc != IPTTT_OK) return rc;
+  if (p->flags != 0) return IPTTT_ERR_ARG;
+  const void* must[] = {H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, gO, gH, gX0, gWgate, gWup, gWdown0, gconv_w,
+                        gWtarget};
+  for (const void* q : must)
+    if ((rc = check_tensor(q)) != IPTTT_OK) return rc;
+  if (gS_final_opt && !aligned(gS_final_opt, 16)) return IPTTT_ERR_ALIGN;
+  if (n_doc_starts < 0 || (n_doc_starts > 0 && !doc_starts)) return IPTTT_ERR_ARG;
+  const Shape s = shape_of(*p);
+  if (!workspace || workspace_bytes < ipttt_backward_workspace_size(p)) return IPTTT_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return IPTTT_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((rc = device_info(&di)) != IPTTT_OK) return rc;
+  const float tau = (p->clip_thresh > 0.0f && isfinite(p->clip_thresh)) ? p->clip_thresh : 0.0f;
+  g_err_detail[0] = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p->dtype == IPTTT_BF16) {
+    // the forward, every state copy kept, then the gradients on the tensor cores
+    const BwdTcLayout BL = bwd_tc_layout(*p);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    Tensors t{};
+    t.H = H; t.X0 = X0; t.Wg = Wgate; t.Wu = Wup; t.W0 = Wdown0; t.cw = conv_w; t.Wt = Wtarget;
+    t.doc = doc_starts;
+    t.n_doc = n_doc_starts;
+    t.O = ws + BL.O;
+    if ((rc = run_bf16(*p, t, ws, BL.fwd, nullptr, di, st)) != IPTTT_OK) return rc;
+    bwd::TcForward f;
+    f.Z = ws + BL.fwd.Z;
+    f.U = ws + BL.fwd.U;
+    f.V = ws + BL.fwd.V;
+    f.snap = ws + BL.fwd.snap;
+    f.alpha = reinterpret_cast<const float*>(ws + BL.fwd.alpha);
+    f.meta = reinterpret_cast<const ChunkMeta*>(ws + BL.fwd.meta);
+    f.flags = ws + BL.fwd.flags;
+    f.nslots = BL.fwd.group;
+    const cudaError_t e = bwd::run_tc(s, p->eta, tau, f, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, gO,
+                                      gS_final_opt, gH, gX0, gWgate, gWup, gWdown0, gconv_w, gWtarget, ws + BL.tc,
+                                      di->status, di->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail("backward", e);
+    counted(bwd::tc_launches());
+    return IPTTT_OK;
+  }
+  const cudaError_t e = bwd::run(s, p->dtype, p->eta, tau, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_starts,
+                                 n_doc_starts, gO, gS_final_opt, gH, gX0, gWgate, gWup, gWdown0, gconv_w, gWtarget,
+                                 static_cast<uint8_t*>(workspace), di->status, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail("backward", e);
+  counted(bwd::launches(s, p->dtype));
+  return IPTTT_OK;
+}
 
 const char* ipttt_last_error_detail(void) { return g_err_detail; }
 

@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(256) k_simt_gemm(SimtArgs a) {
     if (m >= a.M) continue;
     const int t = a.row0 + m;  // token index for the token-row modes
     bool keep_row = true;
-    if (a.mode == SM_V) {
+    if (a.mode == SM_V || a.mode == SM_ACC_L) {
       const int c = t / a.C;
       keep_row = t >= a.meta[(size_t)b * a.k + c].last_start;
     } else if (a.mode == SM_APPLY) {
@@ -437,6 +437,10 @@ __global__ void __launch_bounds__(256) k_simt_gemm(SimtArgs a) {
         case SM_Z: *o = silu_precise(acc0[i][jj]) * acc1[i][jj]; break;
         case SM_V: *o = keep_row ? acc0[i][jj] : 0.0f; break;
         case SM_RAW: *o = acc0[i][jj]; break;
+        case SM_ACC: *o += acc0[i][jj]; break;
+        case SM_ACC_L:
+          if (keep_row) *o += acc0[i][jj];
+          break;
         case SM_APPLY: {
           const float dv = keep_row ? acc1[i][jj] : 0.0f;
           *o = acc0[i][jj] + dv +
@@ -490,6 +494,39 @@ __global__ void k_state_update(float* S, const float* raw, size_t n, const float
   const float* rb = raw + b * n;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
     Sb[i] = fmaf(ae, rb[i], keep ? Sb[i] : 0.0f);
+}
+
+// The clip on the accumulated state (an ablation): per row b,
+//   S = c (keep S + eta raw),  c = tau / ||keep S + eta raw||_F when that norm exceeds tau, else 1,
+// with c stored in alpha[b][chunk].
+__global__ void k_state_accum(float* S, const float* raw, size_t n, const ChunkMeta* meta, int k, int chunk,
+                              float eta) {
+  const int b = blockIdx.y;
+  const bool keep = !meta[(size_t)b * k + chunk].has_start;
+  float* Sb = S + b * n;
+  const float* rb = raw + b * n;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    Sb[i] = fmaf(eta, rb[i], keep ? Sb[i] : 0.0f);
+}
+
+__global__ void k_state_scale(float* S, size_t n, const float* alpha, int k, int chunk) {
+  const int b = blockIdx.y;
+  const float c = alpha[(size_t)b * k + chunk];
+  if (c == 1.0f) return;
+  float* Sb = S + b * n;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    Sb[i] *= c;
+}
+
+cudaError_t simt_update_state_clipped(float* S, const float* raw, double* part, float* alpha, const ChunkMeta* meta,
+                                      const Shape& s, int chunk, float eta, float tau, cudaStream_t st) {
+  const size_t n = (size_t)s.d * s.F;
+  const int nblk = 64;
+  k_state_accum<<<dim3(256, s.B), 256, 0, st>>>(S, raw, n, meta, s.k, chunk, eta);
+  k_sumsq_partials<<<dim3(nblk, s.B), 256, 0, st>>>(S, n, part, nblk);
+  k_alpha_direct<<<(s.B + 63) / 64, 64, 0, st>>>(part, nblk, alpha, s.B, s.k, chunk, 1.0f, tau);
+  k_state_scale<<<dim3(256, s.B), 256, 0, st>>>(S, n, alpha, s.k, chunk);
+  return cudaGetLastError();
 }
 
 cudaError_t simt_update_state(float* S, const float* raw, double* part, float* alpha, const ChunkMeta* meta,

@@ -1,0 +1,61 @@
+// A general bf16 tensor-core GEMM (tcgen05, fp32 accumulators in TMEM) for the
+// backward of the layer, whose products come in three shapes:
+//
+//   GM_PLAIN       out[m][n]            = s * sum_k A(m, k) B(k, n)
+//   GM_CHUNK_ROWS  out[b][t0 + m][n]   (=, +=) s[b][i] * sum_k A(b, t0 + m, k) B_i(k, n)
+//                  for the tokens t0 + m of chunk i (rows outside the chosen
+//                  document segment of the chunk are left alone), B_i taken from
+//                  chunk i's slot of a stack of [d][F] matrices
+//   GM_CHUNK_K     out[i][b][m][n]      = sum over the tokens t of chunk i of A(b, t, m) B(b, t, n)
+//
+// Operands are bf16 tensor maps (3D {inner, rows, outer}, 128-byte swizzle) in
+// one of two orders: K-major (k is the inner, contiguous index) or MN-major (m,
+// resp. n, is).  Boxes: A K-major {64, 128}, A MN-major {64, 64}; B K-major
+// {64, 256}, B MN-major {64, 64}.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace ipttt {
+namespace gemm {
+
+enum Mode { GM_PLAIN = 0, GM_CHUNK_ROWS = 1, GM_CHUNK_K = 2 };
+// Rows of a chunk an GM_CHUNK_ROWS output keeps: all, the chunk's last document
+// segment, or its first segment when it continues the previous chunk's document.
+enum Rows { GR_ALL = 0, GR_LAST = 1, GR_FIRST = 2 };
+enum Out { GO_F32 = 0, GO_F32_ADD = 1, GO_BF16 = 2 };
+
+struct Args {
+  CUtensorMap amap, bmap;
+  int a_mn, b_mn;        // operand order (1: MN-major)
+  int mode;              // Mode
+  int M, N, K;           // PLAIN: all three; CHUNK_ROWS: N, K; CHUNK_K: M, N
+  int B, T, C, k;        // chunk modes: rows, tokens per row, chunk length, chunks per row
+  int chunk0, nchunks;   // chunk modes: chunks [chunk0, chunk0 + nchunks) of every row
+  int nslots;            // CHUNK_ROWS: B_i lies in slot i % nslots (outer index slot * B + b)
+  int out_kind;          // Out
+  void* out;             // fp32 or bf16, rows of ldo elements
+  long long ldo;         // elements between output rows
+  long long osz;         // elements between output matrices (per b, or per slot * B + b)
+  const float* scale;    // optional [B][k] scale (chunk modes) or [1] (PLAIN)
+  const ChunkMeta* meta; // CHUNK_ROWS with rows != GR_ALL: [B][k]
+  int rows;              // Rows
+  int* status;           // device status word (timeouts)
+};
+
+// Box sizes the maps must have for an operand of the given order.
+constexpr uint32_t kBoxInner = 64;
+inline uint32_t a_box_rows(bool mn) { return mn ? 64 : 128; }
+inline uint32_t b_box_rows(bool mn) { return mn ? 64 : 256; }
+
+// Launches the persistent kernel on up to num_sms CTAs.  cudaErrorInvalidValue
+// when N is not a multiple of 32 or a size is not positive.
+cudaError_t run(const Args& a, int num_sms, cudaStream_t st);
+
+}  // namespace gemm
+}  // namespace ipttt

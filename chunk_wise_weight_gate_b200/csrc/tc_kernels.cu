@@ -193,15 +193,19 @@ template <int ROWS>  // 0: p.tr rows per tile; 256: two 128-row halves
 __device__ __forceinline__ void decode_apply(const TcParams& p, int tile, Job& j) {
   const int rows = ROWS ? ROWS : p.tr;
   const int tiles_n = p.d / 128;
-  const int per_row = (p.C / rows) * tiles_n;
+  const int tiles_m = p.C / rows;
+  const int per_row = tiles_m * tiles_n;
   const int per_chunk = p.B * per_row;
   j.kind = K_APPLY;
   j.chunk = p.apply_chunk0 + tile / per_chunk;
   j.t0 = j.chunk * p.C;
   j.b = (tile % per_chunk) / per_row;
+  // Row blocks vary fastest: the tiles that read one 128-column slice of the
+  // chunk's snapshot (and of W0) are consecutive, so they run at the same time on
+  // neighbouring CTAs and the slice comes from DRAM once.
   const int r = tile % per_row;
-  j.m0 = (r / tiles_n) * rows;    // row offset inside the chunk
-  j.n0 = (r % tiles_n) * 128;     // output column (d index)
+  j.m0 = (r % tiles_m) * rows;    // row offset inside the chunk
+  j.n0 = (r / tiles_m) * 128;     // output column (d index)
   j.pair = 0;
   j.nseg = 1;
   j.acc_col[0] = 0;
@@ -326,9 +330,12 @@ __device__ __forceinline__ void issue_loads(const TcParams& p, const Job& j, int
   } else if constexpr (is_apply<FAM>()) {
     tma_load_3d(sa, &p.map[0], bar, kx, j.t0 + j.m0, j.b);        // Z rows of the chunk
     if (j.halves == 2) tma_load_3d(sa + A_BYTES, &p.map[0], bar, kx, j.t0 + j.m0 + 128, j.b);
-    tma_load_3d(sb, &p.map[1], bar, kx, j.n0, 0);                 // Wdown0 rows
+    // W0 (d F bf16, read by every tile of the launch) stays in L2; a snapshot slice
+    // is read by the chunk's row-block tiles at once, then never again
+    tma_load_3d_hint(sb, &p.map[1], bar, kx, j.n0, 0, l2_policy_evict_last());        // Wdown0 rows
     if (j.nsrc == 2)
-      tma_load_3d(sb + 128 * BK * 2, &p.map[2], bar, kx, j.n0, (j.chunk % p.nslots) * p.B + j.b);  // S_i rows
+      tma_load_3d_hint(sb + 128 * BK * 2, &p.map[2], bar, kx, j.n0, (j.chunk % p.nslots) * p.B + j.b,
+                       l2_policy_evict_first());                                     // S_i rows
   }
 }
 
@@ -943,8 +950,10 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&p.map[5], box, jb.n0 + 128 * half + 64 * hb, m0c + 32 * quarter,
-                       ((jb.chunk + 1) % p.nslots) * p.B + jb.b);
+          // the snapshots (2 d F bytes per chunk, read back only by a later launch)
+          // leave L2 first, so the chunk's V and Z, which every pair reads, stay there
+          tma_store_3d_hint(&p.map[5], box, jb.n0 + 128 * half + 64 * hb, m0c + 32 * quarter,
+                            ((jb.chunk + 1) % p.nslots) * p.B + jb.b, l2_policy_evict_first());
           bulk_commit();
         }
         ++stores;

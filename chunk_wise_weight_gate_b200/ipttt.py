@@ -27,7 +27,8 @@ EXPORTS = ("ipttt_workspace_size", "ipttt_forward", "ipttt_forward_ex", "ipttt_c
            "ipttt_kernel_launches", "ipttt_selftest_wait_timeout", "ipttt_forward_noalloc",
            "ipttt_forward_host_size", "ipttt_forward_host", "ipttt_decode_state_size", "ipttt_decode_host_size",
            "ipttt_decode_reset", "ipttt_decode_step", "ipttt_decode_export", "ipttt_cp_workspace_size",
-           "ipttt_cp_plan", "ipttt_cp_begin", "ipttt_cp_finish", "ipttt_last_error_detail")
+           "ipttt_cp_plan", "ipttt_cp_begin", "ipttt_cp_finish", "ipttt_last_error_detail",
+           "ipttt_backward_workspace_size", "ipttt_backward")
 PHASES = ("prep", "gate_up", "target", "gram", "apply", "update")
 DEBUG_OUTPUTS = ("D", "S_final", "alpha", "Z", "V")
 
@@ -39,6 +40,7 @@ class Params(ctypes.Structure):
 
 
 FLAG_RESIDUAL = 1
+FLAG_STATE_CLIP = 2  # the ablation: clip the accumulated state, not each delta (fp32 only)
 
 
 class IptttError(RuntimeError):
@@ -83,6 +85,10 @@ def lib() -> ctypes.CDLL:
         L.ipttt_version.restype = ctypes.c_char_p
         L.ipttt_last_error_detail.argtypes = []
         L.ipttt_last_error_detail.restype = ctypes.c_char_p
+        L.ipttt_backward_workspace_size.argtypes = [P]
+        L.ipttt_backward_workspace_size.restype = sz
+        L.ipttt_backward.argtypes = [P] + [vp] * 7 + [vp, i32, vp, vp] + [vp] * 7 + [vp, sz, vp]
+        L.ipttt_backward.restype = ctypes.c_int
         L.ipttt_profile_enable.argtypes = [ctypes.c_int]
         L.ipttt_profile_enable.restype = None
         L.ipttt_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64),
@@ -212,10 +218,12 @@ def _shape_check(cfg: LayerConfig, **tensors):
 
 
 def forward(cfg: LayerConfig, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_starts=None, *, O=None,
-            workspace=None, stream=None, debug=False, residual=False):
+            workspace=None, stream=None, debug=False, residual=False, state_clip=False):
     """One layer forward.  Returns O, or with debug=True (or a subset of
     DEBUG_OUTPUTS) a dict with O and the chosen internals D, S_final, alpha, Z, V,
-    produced by the same kernels as O.  residual=True writes H + output into O."""
+    produced by the same kernels as O.  residual=True writes H + output into O.
+    state_clip=True (fp32 only) clips the accumulated state instead of each delta;
+    alpha then holds the state's clip factor per chunk."""
     dt = cfg.torch_dtype
     _shape_check(cfg, H=H, X0=X0, Wgate=Wgate, Wup=Wup, Wdown0=Wdown0, conv_w=conv_w, Wtarget=Wtarget, O=O)
     dev = H.device
@@ -226,7 +234,7 @@ def forward(cfg: LayerConfig, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_st
     if residual and O.data_ptr() == H.data_ptr():
         raise ValueError("O must not alias H when residual=True")
     dp, nd, keep = _docs(doc_starts, dev)
-    p = cfg.params(FLAG_RESIDUAL if residual else 0)
+    p = cfg.params((FLAG_RESIDUAL if residual else 0) | (FLAG_STATE_CLIP if state_clip else 0))
     args = [_ptr(H, dt, "H"), _ptr(X0, dt, "X0"), _ptr(Wgate, dt, "Wgate"), _ptr(Wup, dt, "Wup"),
             _ptr(Wdown0, dt, "Wdown0"), _ptr(conv_w, dt, "conv_w"), _ptr(Wtarget, dt, "Wtarget"), dp, nd,
             _ptr(O, dt, "O")]
@@ -264,6 +272,46 @@ def core(cfg: LayerConfig, Z, V, Wdown0, doc_starts=None, *, workspace=None, str
                             nd, out["O"].data_ptr(), out["D"].data_ptr(), out["S_final"].data_ptr(),
                             out["alpha"].data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)),
            "ipttt_core")
+    return out
+
+
+def backward_workspace_size(cfg: LayerConfig) -> int:
+    """Bytes of device workspace ipttt_backward needs for this configuration."""
+    p = cfg.params()
+    n = lib().ipttt_backward_workspace_size(ctypes.byref(p))
+    if n == 0:
+        raise ValueError(f"invalid layer configuration {cfg}")
+    return n
+
+
+def backward(cfg: LayerConfig, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_starts, gO, gS_final=None, *,
+             workspace=None, stream=None):
+    """fp32 gradients of <gO, O> + <gS_final, S_final> with respect to the layer's
+    inputs (ipttt_backward); returns a dict keyed like the inputs."""
+    dt = cfg.torch_dtype
+    _shape_check(cfg, H=H, X0=X0, Wgate=Wgate, Wup=Wup, Wdown0=Wdown0, conv_w=conv_w, Wtarget=Wtarget, O=gO)
+    dev = H.device
+    p = cfg.params()
+    if workspace is None:
+        workspace = torch.empty(backward_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    f32 = torch.float32
+    out = {"H": torch.empty(cfg.B, cfg.T, cfg.d, dtype=f32, device=dev),
+           "X0": torch.empty(cfg.B, cfg.T, cfg.d, dtype=f32, device=dev),
+           "Wgate": torch.empty(cfg.F, cfg.d, dtype=f32, device=dev),
+           "Wup": torch.empty(cfg.F, cfg.d, dtype=f32, device=dev),
+           "Wdown0": torch.empty(cfg.d, cfg.F, dtype=f32, device=dev),
+           "conv_w": torch.empty(cfg.d, 5, dtype=f32, device=dev),
+           "Wtarget": torch.empty(cfg.d, cfg.d, dtype=f32, device=dev)}
+    if gS_final is not None and tuple(gS_final.shape) != (cfg.B, cfg.d, cfg.F):
+        raise ValueError(f"gS_final has shape {tuple(gS_final.shape)}, expected {(cfg.B, cfg.d, cfg.F)}")
+    dp, nd, keep = _docs(doc_starts, dev)
+    _check(lib().ipttt_backward(ctypes.byref(p), _ptr(H, dt, "H"), _ptr(X0, dt, "X0"), _ptr(Wgate, dt, "Wgate"),
+                                _ptr(Wup, dt, "Wup"), _ptr(Wdown0, dt, "Wdown0"), _ptr(conv_w, dt, "conv_w"),
+                                _ptr(Wtarget, dt, "Wtarget"), dp, nd, _ptr(gO, dt, "gO"),
+                                _ptr(gS_final, f32, "gS_final"),
+                                *(out[k].data_ptr() for k in ("H", "X0", "Wgate", "Wup", "Wdown0", "conv_w",
+                                                             "Wtarget")),
+                                workspace.data_ptr(), workspace.numel(), _stream(stream)), "ipttt_backward")
     return out
 
 

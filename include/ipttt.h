@@ -96,6 +96,14 @@ typedef struct {
  * to dtype.  O must not alias H. */
 #define IPTTT_FLAG_RESIDUAL 1
 
+/* The ablation that clips the accumulated fast weight instead of each chunk's
+ * delta (iplexlaw.co.kr review of arXiv 2604.06169, §6, leaves open which of the
+ * two the clip acts on): S_{i+1} = c_i (keep_i S_i + eta V_L^T Z_L) with
+ * c_i = tau / ||keep_i S_i + eta V_L^T Z_L||_F when that norm exceeds tau, else 1.
+ * dtype IPTTT_F32 only (IPTTT_ERR_UNSUPPORTED otherwise); the per-chunk factor
+ * returned in alpha_opt is c_i. */
+#define IPTTT_FLAG_STATE_CLIP 2
+
 /* Bytes of workspace that ipttt_forward / _ex / stream_forward need for *p.
  * Returns 0 when *p is invalid.  Pure host function. */
 IPTTT_API size_t ipttt_workspace_size(const ipttt_params* p);
@@ -331,6 +339,33 @@ IPTTT_API ipttt_status ipttt_decode_export(const ipttt_params* p, const void* st
 
 /* Library version, "major.minor.patch". */
 IPTTT_API const char* ipttt_version(void);
+
+/* Backward of the layer (ipttt_forward's inputs, params->flags must be 0).  Given
+ * gO = dL/dO ([B][T][d], the layer's dtype) and optionally gS_final = dL/dS_final
+ * (fp32 [B][d][F] row-major; NULL = 0), writes the fp32 gradients of
+ * L = <gO, O> + <gS_final, S_final> with respect to H and X0 ([B][T][d]), Wgate and
+ * Wup ([F][d]), Wdown0 ([d][F]), conv_w ([d][5]) and Wtarget ([d][d]), through the
+ * gated MLP, the chunk scan with its document resets, the per-chunk clip (the
+ * derivative of the branch the forward took; the clip has a kink at norm tau), and
+ * the masked conv target.  The pages give no backward: the layer is trained in
+ * place (cloud.tencent.com "榨干MLP的剩余价值", 验证模块一), and these are the chain
+ * rule through the forward defined above.  dtype IPTTT_F32 runs every product in
+ * fp32 on the CUDA cores (any shape).  dtype IPTTT_BF16 (the forward's tensor-core
+ * shapes) runs the forward first, keeping every chunk's bf16 state copy, then
+ * every product as a tcgen05 GEMM on bf16 operands with fp32 accumulators: the
+ * forward's Z and V, each chunk's raw delta V_L^T Z_L and the bf16 copies of the
+ * state gradients are operands, so the gradients carry bf16 operand rounding.
+ * Deterministic either way.  All pointers are device memory owned by the caller,
+ * 16-byte aligned; workspace (256-byte aligned) of ipttt_backward_workspace_size(p)
+ * bytes (fp32: k + 4 fp32 states [B][d][F]; bf16: about 2.5 k bf16 and k fp32
+ * states [B][d][F] besides the activations).  Errors as for ipttt_forward. */
+IPTTT_API size_t ipttt_backward_workspace_size(const ipttt_params* p);
+IPTTT_API ipttt_status ipttt_backward(const ipttt_params* p, const void* H, const void* X0, const void* Wgate,
+                                      const void* Wup, const void* Wdown0, const void* conv_w,
+                                      const void* Wtarget, const int32_t* doc_starts, int32_t n_doc_starts,
+                                      const void* gO, const float* gS_final_opt, float* gH, float* gX0,
+                                      float* gWgate, float* gWup, float* gWdown0, float* gconv_w,
+                                      float* gWtarget, void* workspace, size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 from oracle import ipttt_ablations as ab
-from tests.gpu_util import case, gpu, oracle, to_np
+from tests.gpu_util import case, gpu, maxrel, normrel, oracle, to_np
 from tests.test_gpu_parity import check_bf16
 
 pytestmark = pytest.mark.gpu
@@ -50,3 +50,45 @@ def test_target_without_both_parts_is_the_token_itself():
     mask = torch.from_numpy(ref["V"] != 0).any(dim=-1, keepdim=True)
     assert torch.equal(V, torch.where(mask, inp["X0"], torch.zeros_like(inp["X0"])))
     check_bf16(out, ref, cfg.clip)
+
+
+# The clip on the accumulated state (iplexlaw.co.kr review, §6, read the other way):
+# S_{i+1} = c_i (keep_i S_i + eta V_L^T Z_L).  fp32 path; held to the fp32 bars of
+# the forward (1e-5 on O and S_final) against oracle/ipttt_ablations.py.
+STATE_CLIP_CASES = {
+    # documents inside chunks and on a chunk boundary, a ragged last chunk; tau
+    # small enough that the state is clipped after most chunks
+    "docs_ragged": dict(B=2, T=100, C=12, d=24, F=40, eta=0.05, clip=0.05, docs=[13, 36, 41, 100 + 7, 100 + 70]),
+    # one document, several tiles of every product; the state first grows unclipped,
+    # then is clipped from the fourth chunk on
+    "tiles": dict(B=1, T=256, C=32, d=64, F=256, eta=0.01, clip=6.0, docs=[]),
+}
+
+
+def state_clip_oracle(cfg, inp):
+    a = {k: to_np(inp[k]) for k in ("H", "X0") + ("Wgate", "Wup", "Wdown0", "conv_w", "Wtarget")}
+    return ab.layer_forward_state_clip(a["H"], a["X0"], a["Wgate"], a["Wup"], a["Wdown0"], a["conv_w"],
+                                       a["Wtarget"], cfg.C, inp["doc_starts"].numpy(), cfg.eta, cfg.clip)
+
+
+@pytest.mark.parametrize("name", list(STATE_CLIP_CASES))
+def test_state_clip(name):
+    kw = dict(STATE_CLIP_CASES[name])
+    cfg, inp = case(dtype="f32", conv_std=0.3, wtarget="identity_noise", **kw)
+    out = gpu(cfg, inp, state_clip=True)
+    ref = state_clip_oracle(cfg, inp)
+    assert maxrel(to_np(out["O"]), ref["O"]) <= 1e-5
+    assert normrel(to_np(out["S_final"]), ref["S_final"]) <= 1e-5
+    assert maxrel(to_np(out["D"]), ref["D"]) <= 1e-4
+    assert np.max(np.abs(to_np(out["alpha"]) - ref["scale"])) <= 1e-5
+    # the case reaches the clip, and the accumulated-state reading differs from
+    # the per-delta one by far more than the tolerance
+    assert np.min(ref["scale"]) < 0.9
+    per_delta = oracle(cfg, inp)
+    assert maxrel(per_delta["D"], ref["D"]) > 1e-2
+
+
+def test_state_clip_is_fp32_only():
+    cfg, inp = case(**CASES["clip"])
+    with pytest.raises(Exception):
+        gpu(cfg, inp, state_clip=True)

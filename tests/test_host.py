@@ -64,6 +64,7 @@ def test_workspace_size_grows_with_tokens_and_is_zero_when_invalid():
     (dict(B=0), 1), (dict(T=-1), 1), (dict(C=0), 1), (dict(dtype=3), 4),
     (dict(eta=float("nan")), 1), (dict(clip_thresh=float("nan")), 1),
     (dict(d=200), 5), (dict(F=320), 5), (dict(C=96), 5), (dict(C=32), 5), (dict(C=8192), 5), (dict(flags=6), 1),
+    (dict(flags=2), 5),  # the accumulated-state clip runs on the fp32 path only
 ])
 def test_bad_params_are_rejected_before_launch(kw, code):
     assert call_forward(params(**kw)) == code
