@@ -463,46 +463,82 @@ __global__ void k_mask_first_bf16(const __nv_bfloat16* gO, __nv_bfloat16* gOF, c
   }
 }
 
-// G_{i+1} -> Gs[i] (bf16), G_i = keep_i G_{i+1} + R_i, for i = k-1 .. 0; G_k = gS (or 0).
-__global__ void k_reverse_scan(const float* R, const float* gS, __nv_bfloat16* Gs, const ChunkMeta* meta, int B,
-                               int k, size_t n) {
+// G_{i+1} -> Gs[i] (bf16), G_i = keep_i G_{i+1} + R_i, for i = k-1 .. 0; G_k = gS
+// (or 0).  8 consecutive elements per thread (n % 8 == 0), the next chunk's R
+// requested before the current one is added.
+__global__ void k_reverse_scan(const __nv_bfloat16* R, const float* gS, __nv_bfloat16* Gs, const ChunkMeta* meta,
+                               int B, int k, size_t n) {
   const size_t total = (size_t)B * n;
-  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+  for (size_t e = 8 * (blockIdx.x * (size_t)blockDim.x + threadIdx.x); e < total;
+       e += 8 * (size_t)gridDim.x * blockDim.x) {
     const int b = (int)(e / n);
-    float g = gS ? gS[e] : 0.0f;
+    float g[8];
+    if (gS) {
+      const float4 x = *reinterpret_cast<const float4*>(gS + e), y = *reinterpret_cast<const float4*>(gS + e + 4);
+      g[0] = x.x; g[1] = x.y; g[2] = x.z; g[3] = x.w; g[4] = y.x; g[5] = y.y; g[6] = y.z; g[7] = y.w;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) g[q] = 0.0f;
+    }
+    uint4 r = *reinterpret_cast<const uint4*>(R + (size_t)(k - 1) * total + e);
     for (int i = k - 1; i >= 0; --i) {
       const size_t o = (size_t)i * total + e;
-      Gs[o] = __float2bfloat16(g);
-      g = (meta[(size_t)b * k + i].has_start ? 0.0f : g) + R[o];
+      const uint4 cur = r;
+      if (i > 0) r = *reinterpret_cast<const uint4*>(R + o - total);
+      uint4 w;
+      uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(g[2 * q], g[2 * q + 1]);
+        wp[q] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      *reinterpret_cast<uint4*>(Gs + o) = w;
+      const bool keep = !meta[(size_t)b * k + i].has_start;
+      const uint32_t* cp = reinterpret_cast<const uint32_t*>(&cur);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&cp[q]);
+        g[2 * q] = (keep ? g[2 * q] : 0.0f) + __low2float(h);
+        g[2 * q + 1] = (keep ? g[2 * q + 1] : 0.0f) + __high2float(h);
+      }
     }
   }
 }
 
-// Per (row b, chunk i): c1 = alpha eta and c2 from <P_i, G_{i+1}> = sum over the
-// chunk's tokens of v_t . Y_t (V is zero outside the last segment).
-__global__ void k_clip_coeffs_tc(const __nv_bfloat16* V, const float* Y, const float* alpha, float* c1, float* c2,
-                                 int T, int d, int C, int k, float eta, float tau) {
+// <P_i, G_{i+1}> = sum over the tokens of chunk i of v_t . Y_t (V is zero outside
+// the last segment), as kDotParts fixed-order partial sums per (row, chunk) ...
+constexpr int kDotParts = 32;
+__global__ void k_vy_partials(const __nv_bfloat16* V, const float* Y, double* part, int T, int d, int C, int k) {
   __shared__ double sh[256];
-  const int i = blockIdx.x, b = blockIdx.y;
+  const int i = blockIdx.x, b = blockIdx.y, q = blockIdx.z;
   const int t0 = i * C, t1 = min(t0 + C, T);
   const size_t n = (size_t)(t1 - t0) * d;
+  const size_t lo = n * q / kDotParts, hi = n * (q + 1) / kDotParts;
   const __nv_bfloat16* v = V + ((size_t)b * T + t0) * d;
   const float* y = Y + ((size_t)b * T + t0) * d;
   double acc = 0.0;
-  for (size_t e = threadIdx.x; e < n; e += blockDim.x) acc += (double)__bfloat162float(v[e]) * (double)y[e];
+  for (size_t e = lo + threadIdx.x; e < hi; e += blockDim.x) acc += (double)__bfloat162float(v[e]) * (double)y[e];
   sh[threadIdx.x] = acc;
   __syncthreads();
   for (int o = 128; o > 0; o >>= 1) {
     if (threadIdx.x < o) sh[threadIdx.x] += sh[threadIdx.x + o];
     __syncthreads();
   }
-  if (threadIdx.x == 0) {
-    const float a = alpha[(size_t)b * k + i];
-    c1[(size_t)b * k + i] = a * eta;
-    const bool clipped = tau > 0.0f && a < 1.0f;
-    const double ae = (double)a * eta;
-    c2[(size_t)b * k + i] = clipped ? (float)(-ae * ae * ae * sh[0] / ((double)tau * tau)) : 0.0f;
-  }
+  if (threadIdx.x == 0) part[((size_t)b * k + i) * kDotParts + q] = sh[0];
+}
+
+// ... then per (row b, chunk i): c1 = alpha eta, and c2 for a clipped chunk.
+__global__ void k_clip_coeffs_tc(const double* part, const float* alpha, float* c1, float* c2, int n, float eta,
+                                 float tau) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;  // b k + i
+  if (j >= n) return;
+  double dot = 0.0;
+  for (int q = 0; q < kDotParts; ++q) dot += part[(size_t)j * kDotParts + q];
+  const float a = alpha[j];
+  c1[j] = a * eta;
+  const bool clipped = tau > 0.0f && a < 1.0f;
+  const double ae = (double)a * eta;
+  c2[j] = clipped ? (float)(-ae * ae * ae * dot / ((double)tau * tau)) : 0.0f;
 }
 
 // gV = c1 Y on the rows of each chunk's last segment, 0 elsewhere.
@@ -518,13 +554,42 @@ __global__ void k_gv_init(const float* Y, const float* c1, float* gV, const Chun
 }
 
 // gA = gZ Bu SiLU'(A), gBu = gZ SiLU(A), rounded to bf16 (the next products' operands).
-__global__ void k_gate_backward_bf16(const float* A, const float* Bu, const float* gZ, __nv_bfloat16* gA,
-                                     __nv_bfloat16* gBu, size_t n) {
+__global__ void k_gate_backward_bf16(const __nv_bfloat16* A, const __nv_bfloat16* Bu, const float* gZ,
+                                     __nv_bfloat16* gA, __nv_bfloat16* gBu, size_t n) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-    const float a = A[i], u = Bu[i], g = gZ[i];
+    const float a = __bfloat162float(A[i]), u = __bfloat162float(Bu[i]), g = gZ[i];
     const float s = 1.0f / (1.0f + expf(-a));
     gA[i] = __float2bfloat16(g * u * (s * (1.0f + a * (1.0f - s))));
     gBu[i] = __float2bfloat16(g * (a * s));
+  }
+}
+
+// gX0[s, c] = sum_o w[c, o] gU[s - o, c] over the taps o in use at token s - o,
+// 8 channels of one token per thread (d % 8 == 0): the taps in use are found
+// once for the 8, and gU comes in 32-byte rows.
+__global__ void k_conv_grad_input_v8(const float* gU, const float* cw, const uint8_t* flags, float* gX0, int B,
+                                     int T, int d, int C) {
+  const int g8 = d / 8;
+  const size_t n = (size_t)B * T * g8;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const int c0 = (int)(i % g8) * 8;
+    const size_t bt = i / g8;
+    const int s = (int)(bt % T), b = (int)(bt / T);
+    const uint8_t* f = flags + (size_t)b * T;
+    float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int o = 0; o < kTaps; ++o) {
+      const int t = s - o;
+      if (t < 0 || o >= taps_at(f, t, T, C)) continue;
+      const float4* u = reinterpret_cast<const float4*>(gU + ((size_t)b * T + t) * d + c0);
+      const float4 u0 = u[0], u1 = u[1];
+      const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = fmaf(cw[(c0 + q) * kTaps + o], uv[q], acc[q]);
+    }
+    float4* out = reinterpret_cast<float4*>(gX0 + bt * d + c0);
+    out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
 }
 
@@ -566,7 +631,7 @@ __global__ void k_f32_to_bf16(const float* x, __nv_bfloat16* y, size_t n) {
 }
 
 struct TcLayout {
-  size_t Af, Buf, gZ, gA, gBu, gOF, Y, gV, gVb, gU, P, R, Gs, c1, c2, cwf, cpart, total;
+  size_t Af, Buf, gZ, gA, gBu, gOF, Y, gV, gVb, gU, P, R, Gs, c1, c2, dpart, cwf, cpart, total;
 };
 
 TcLayout tc_layout(const Shape& s) {
@@ -578,8 +643,8 @@ TcLayout tc_layout(const Shape& s) {
     off += al256(bytes);
     return o;
   };
-  L.Af = take(B * T * F * 4);
-  L.Buf = take(B * T * F * 4);
+  L.Af = take(B * T * F * 2);
+  L.Buf = take(B * T * F * 2);
   L.gZ = take(B * T * F * 4);
   L.gA = take(B * T * F * 2);
   L.gBu = take(B * T * F * 2);
@@ -589,10 +654,11 @@ TcLayout tc_layout(const Shape& s) {
   L.gVb = take(B * T * d * 2);
   L.gU = take(B * T * d * 4);
   L.P = take(k * B * d * F * 2);
-  L.R = take(k * B * d * F * 4);
+  L.R = take(k * B * d * F * 2);
   L.Gs = take(k * B * d * F * 2);
   L.c1 = take(B * k * 4);
   L.c2 = take(B * k * 4);
+  L.dpart = take(B * k * kDotParts * sizeof(double));
   L.cwf = take(d * kTaps * 4);
   L.cpart = take((size_t)kConvParts * d * kTaps * 4);
   L.total = off;
@@ -608,8 +674,8 @@ bool gmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint6
 
 size_t tc_workspace_bytes(const Shape& s) { return tc_layout(s).total; }
 
-// Kernels run_tc launches: 18 GEMMs and 10 elementwise or reduction kernels.
-long long tc_launches() { return 28; }
+// Kernels run_tc launches: 18 GEMMs and 11 elementwise or reduction kernels.
+long long tc_launches() { return 29; }
 
 #define TC_MAP(m, ...) \
   do {                 \
@@ -627,9 +693,11 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
   const uint64_t BT = (uint64_t)(B * T);
   auto fp = [&](size_t o) { return reinterpret_cast<float*>(ws + o); };
   auto hp = [&](size_t o) { return reinterpret_cast<__nv_bfloat16*>(ws + o); };
-  float *Af = fp(L.Af), *Buf = fp(L.Buf), *gZ = fp(L.gZ), *Y = fp(L.Y), *gV = fp(L.gV), *gU = fp(L.gU),
-        *R = fp(L.R), *c1 = fp(L.c1), *c2 = fp(L.c2), *cwf = fp(L.cwf), *cpart = fp(L.cpart);
-  __nv_bfloat16 *gA = hp(L.gA), *gBu = hp(L.gBu), *gOF = hp(L.gOF), *gVb = hp(L.gVb), *P = hp(L.P), *Gs = hp(L.Gs);
+  float *gZ = fp(L.gZ), *Y = fp(L.Y), *gV = fp(L.gV), *gU = fp(L.gU), *c1 = fp(L.c1), *c2 = fp(L.c2),
+        *cwf = fp(L.cwf), *cpart = fp(L.cpart);
+  double* dpart = reinterpret_cast<double*>(ws + L.dpart);
+  __nv_bfloat16 *Af = hp(L.Af), *Buf = hp(L.Buf), *gA = hp(L.gA), *gBu = hp(L.gBu), *gOF = hp(L.gOF),
+                *gVb = hp(L.gVb), *P = hp(L.P), *R = hp(L.R), *Gs = hp(L.Gs);
   const __nv_bfloat16* Zb = static_cast<const __nv_bfloat16*>(f.Z);
   const __nv_bfloat16* Vb = static_cast<const __nv_bfloat16*>(f.V);
 
@@ -653,13 +721,13 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
     return gemm::run(g, num_sms, st);
   };
 
-  // 1. pre-activations A = H Wg^T, Bu = H Wu^T (fp32)
+  // 1. pre-activations A = H Wg^T, Bu = H Wu^T (bf16)
   TC_MAP(&g.amap, H, d, BT, 1, a_box_rows(false));
   TC_MAP(&g.bmap, Wg, d, F, 1, b_box_rows(false));
   g.a_mn = 0; g.b_mn = 0;
-  BW_CHECK(plain((int)BT, (int)F, (int)d, Af, F, GO_F32));
+  BW_CHECK(plain((int)BT, (int)F, (int)d, Af, F, GO_BF16));
   TC_MAP(&g.bmap, Wu, d, F, 1, b_box_rows(false));
-  BW_CHECK(plain((int)BT, (int)F, (int)d, Buf, F, GO_F32));
+  BW_CHECK(plain((int)BT, (int)F, (int)d, Buf, F, GO_BF16));
   // 2. gZ = gO W0 (W0 [d][F]: k = d rows, n = F contiguous)
   TC_MAP(&g.amap, gO, d, BT, 1, a_box_rows(false));
   TC_MAP(&g.bmap, W0, F, d, 1, b_box_rows(true));
@@ -670,22 +738,23 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
   TC_MAP(&g.bmap, Zb, F, BT, 1, b_box_rows(true));
   g.a_mn = 1; g.b_mn = 1;
   BW_CHECK(plain((int)d, (int)F, (int)BT, gW0, F, GO_F32));
-  // 4. P_i = V_L^T Z_L per chunk (bf16), and R_i = gO_F^T Z_F per chunk (fp32)
+  // 4. P_i = V_L^T Z_L and R_i = gO_F^T Z_F per chunk (bf16)
   TC_MAP(&g.amap, Vb, d, T, B, a_box_rows(true));
   TC_MAP(&g.bmap, Zb, F, T, B, b_box_rows(true));
   BW_CHECK(chunked(GM_CHUNK_K, (int)d, (int)F, 0, P, F, d * F, GO_BF16, nullptr, GR_ALL, 1));
   k_mask_first_bf16<<<grid_for(B * T * d), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(gO), gOF, f.meta, (int)B,
                                                           (int)T, (int)d, s.C, k);
   TC_MAP(&g.amap, gOF, d, T, B, a_box_rows(true));
-  BW_CHECK(chunked(GM_CHUNK_K, (int)d, (int)F, 0, R, F, d * F, GO_F32, nullptr, GR_ALL, 1));
+  BW_CHECK(chunked(GM_CHUNK_K, (int)d, (int)F, 0, R, F, d * F, GO_BF16, nullptr, GR_ALL, 1));
   // 5. reverse scan: bf16 G_{i+1} in slot i
-  k_reverse_scan<<<grid_for(B * d * F), 256, 0, st>>>(R, gS, Gs, f.meta, (int)B, k, (size_t)(d * F));
+  k_reverse_scan<<<grid_for(B * d * F / 8), 256, 0, st>>>(R, gS, Gs, f.meta, (int)B, k, (size_t)(d * F));
   // 6. Y = Z G_{i+1}^T on every chunk's tokens, then c1, c2 per chunk
   TC_MAP(&g.amap, Zb, F, T, B, a_box_rows(false));
   TC_MAP(&g.bmap, Gs, F, d, (uint64_t)k * B, b_box_rows(false));
   g.a_mn = 0; g.b_mn = 0;
   BW_CHECK(chunked(GM_CHUNK_ROWS, 0, (int)d, (int)F, Y, d, T * d, GO_F32, nullptr, GR_ALL, k));
-  k_clip_coeffs_tc<<<dim3(k, (unsigned)B), 256, 0, st>>>(Vb, Y, f.alpha, c1, c2, (int)T, (int)d, s.C, k, eta, tau);
+  k_vy_partials<<<dim3(k, (unsigned)B, kDotParts), 256, 0, st>>>(Vb, Y, dpart, (int)T, (int)d, s.C, k);
+  k_clip_coeffs_tc<<<(unsigned)((B * k + 127) / 128), 128, 0, st>>>(dpart, f.alpha, c1, c2, (int)(B * k), eta, tau);
   // 7. gV_L = c1 Y + c2 Z_L P_i^T
   k_gv_init<<<grid_for(B * T * d), 256, 0, st>>>(Y, c1, gV, f.meta, (int)B, (int)T, (int)d, s.C, k);
   TC_MAP(&g.bmap, P, F, d, (uint64_t)k * B, b_box_rows(false));
@@ -726,7 +795,7 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
   g.a_mn = 1; g.b_mn = 1;
   BW_CHECK(plain((int)d, (int)d, (int)BT, gWt, d, GO_F32));
   k_widen<<<grid_for(d * kTaps), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(cw), cwf, (size_t)(d * kTaps));
-  k_conv_grad_input<<<grid_for(BT * d), 256, 0, st>>>(gU, cwf, f.flags, gX0, (int)B, (int)T, (int)d, s.C);
+  k_conv_grad_input_v8<<<grid_for(BT * d / 8), 256, 0, st>>>(gU, cwf, f.flags, gX0, (int)B, (int)T, (int)d, s.C);
   k_conv_grad_weight_parts<<<dim3((unsigned)((d + 255) / 256), kConvParts), 256, 0, st>>>(
       gU, static_cast<const __nv_bfloat16*>(X0), f.flags, cpart, (int)B, (int)T, (int)d, s.C);
   k_conv_grad_weight_reduce<<<(unsigned)((d * kTaps + 255) / 256), 256, 0, st>>>(cpart, gcw, (int)d);
