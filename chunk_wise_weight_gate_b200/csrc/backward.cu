@@ -665,22 +665,14 @@ TcLayout tc_layout(const Shape& s) {
   return L;
 }
 
-// A bf16 tensor map for gemm.cu: {inner, rows, outer}, box {64, box_rows}.
-bool gmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer, uint32_t box_rows) {
-  return tck::make_map_bf16(m, base, inner, rows, outer, gemm::kBoxInner, box_rows);
-}
 
 }  // namespace
 
 size_t tc_workspace_bytes(const Shape& s) { return tc_layout(s).total; }
 
-// Kernels run_tc launches: 18 GEMMs and 11 elementwise or reduction kernels.
-long long tc_launches() { return 29; }
+// Kernels run_tc launches: 17 GEMMs and 11 elementwise or reduction kernels.
+long long tc_launches() { return 28; }
 
-#define TC_MAP(m, ...) \
-  do {                 \
-    if (!gmap(m, __VA_ARGS__)) return cudaErrorInvalidValue; \
-  } while (0)
 
 cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, const void* H, const void* X0,
                    const void* Wg, const void* Wu, const void* W0, const void* cw, const void* Wt, const void* gO,
@@ -722,76 +714,76 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
   };
 
   // 1. pre-activations A = H Wg^T, Bu = H Wu^T (bf16)
-  TC_MAP(&g.amap, H, d, BT, 1, a_box_rows(false));
-  TC_MAP(&g.bmap, Wg, d, F, 1, b_box_rows(false));
+  g.A = {H, (uint64_t)(d), (uint64_t)(BT), (uint64_t)(1)};
+  g.Bop = {Wg, (uint64_t)(d), (uint64_t)(F), (uint64_t)(1)};
   g.a_mn = 0; g.b_mn = 0;
   BW_CHECK(plain((int)BT, (int)F, (int)d, Af, F, GO_BF16));
-  TC_MAP(&g.bmap, Wu, d, F, 1, b_box_rows(false));
+  g.Bop = {Wu, (uint64_t)(d), (uint64_t)(F), (uint64_t)(1)};
   BW_CHECK(plain((int)BT, (int)F, (int)d, Buf, F, GO_BF16));
   // 2. gZ = gO W0 (W0 [d][F]: k = d rows, n = F contiguous)
-  TC_MAP(&g.amap, gO, d, BT, 1, a_box_rows(false));
-  TC_MAP(&g.bmap, W0, F, d, 1, b_box_rows(true));
+  g.A = {gO, (uint64_t)(d), (uint64_t)(BT), (uint64_t)(1)};
+  g.Bop = {W0, (uint64_t)(F), (uint64_t)(d), (uint64_t)(1)};
   g.a_mn = 0; g.b_mn = 1;
   BW_CHECK(plain((int)BT, (int)F, (int)d, gZ, F, GO_F32));
   // 3. gW0 = gO^T Z over every token
-  TC_MAP(&g.amap, gO, d, BT, 1, a_box_rows(true));
-  TC_MAP(&g.bmap, Zb, F, BT, 1, b_box_rows(true));
+  g.A = {gO, (uint64_t)(d), (uint64_t)(BT), (uint64_t)(1)};
+  g.Bop = {Zb, (uint64_t)(F), (uint64_t)(BT), (uint64_t)(1)};
   g.a_mn = 1; g.b_mn = 1;
   BW_CHECK(plain((int)d, (int)F, (int)BT, gW0, F, GO_F32));
   // 4. P_i = V_L^T Z_L and R_i = gO_F^T Z_F per chunk (bf16)
-  TC_MAP(&g.amap, Vb, d, T, B, a_box_rows(true));
-  TC_MAP(&g.bmap, Zb, F, T, B, b_box_rows(true));
+  g.A = {Vb, (uint64_t)(d), (uint64_t)(T), (uint64_t)(B)};
+  g.Bop = {Zb, (uint64_t)(F), (uint64_t)(T), (uint64_t)(B)};
   BW_CHECK(chunked(GM_CHUNK_K, (int)d, (int)F, 0, P, F, d * F, GO_BF16, nullptr, GR_ALL, 1));
   k_mask_first_bf16<<<grid_for(B * T * d), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(gO), gOF, f.meta, (int)B,
                                                           (int)T, (int)d, s.C, k);
-  TC_MAP(&g.amap, gOF, d, T, B, a_box_rows(true));
+  g.A = {gOF, (uint64_t)(d), (uint64_t)(T), (uint64_t)(B)};
   BW_CHECK(chunked(GM_CHUNK_K, (int)d, (int)F, 0, R, F, d * F, GO_BF16, nullptr, GR_ALL, 1));
   // 5. reverse scan: bf16 G_{i+1} in slot i
   k_reverse_scan<<<grid_for(B * d * F / 8), 256, 0, st>>>(R, gS, Gs, f.meta, (int)B, k, (size_t)(d * F));
   // 6. Y = Z G_{i+1}^T on every chunk's tokens, then c1, c2 per chunk
-  TC_MAP(&g.amap, Zb, F, T, B, a_box_rows(false));
-  TC_MAP(&g.bmap, Gs, F, d, (uint64_t)k * B, b_box_rows(false));
+  g.A = {Zb, (uint64_t)(F), (uint64_t)(T), (uint64_t)(B)};
+  g.Bop = {Gs, (uint64_t)(F), (uint64_t)(d), (uint64_t)((uint64_t)k * B)};
   g.a_mn = 0; g.b_mn = 0;
   BW_CHECK(chunked(GM_CHUNK_ROWS, 0, (int)d, (int)F, Y, d, T * d, GO_F32, nullptr, GR_ALL, k));
   k_vy_partials<<<dim3(k, (unsigned)B, kDotParts), 256, 0, st>>>(Vb, Y, dpart, (int)T, (int)d, s.C, k);
   k_clip_coeffs_tc<<<(unsigned)((B * k + 127) / 128), 128, 0, st>>>(dpart, f.alpha, c1, c2, (int)(B * k), eta, tau);
   // 7. gV_L = c1 Y + c2 Z_L P_i^T
   k_gv_init<<<grid_for(B * T * d), 256, 0, st>>>(Y, c1, gV, f.meta, (int)B, (int)T, (int)d, s.C, k);
-  TC_MAP(&g.bmap, P, F, d, (uint64_t)k * B, b_box_rows(false));
+  g.Bop = {P, (uint64_t)(F), (uint64_t)(d), (uint64_t)((uint64_t)k * B)};
   BW_CHECK(chunked(GM_CHUNK_ROWS, 0, (int)d, (int)F, gV, d, T * d, GO_F32_ADD, c2, GR_LAST, k));
   // 8. gZ += c1 V_L G_{i+1} + c2 V_L P_i + gO_F S_i (K = d; the [d][F] operands n-major)
-  TC_MAP(&g.amap, Vb, d, T, B, a_box_rows(false));
-  TC_MAP(&g.bmap, Gs, F, d, (uint64_t)k * B, b_box_rows(true));
+  g.A = {Vb, (uint64_t)(d), (uint64_t)(T), (uint64_t)(B)};
+  g.Bop = {Gs, (uint64_t)(F), (uint64_t)(d), (uint64_t)((uint64_t)k * B)};
   g.a_mn = 0; g.b_mn = 1;
   BW_CHECK(chunked(GM_CHUNK_ROWS, 0, (int)F, (int)d, gZ, F, T * F, GO_F32_ADD, c1, GR_LAST, k));
-  TC_MAP(&g.bmap, P, F, d, (uint64_t)k * B, b_box_rows(true));
+  g.Bop = {P, (uint64_t)(F), (uint64_t)(d), (uint64_t)((uint64_t)k * B)};
   BW_CHECK(chunked(GM_CHUNK_ROWS, 0, (int)F, (int)d, gZ, F, T * F, GO_F32_ADD, c2, GR_LAST, k));
-  TC_MAP(&g.amap, gO, d, T, B, a_box_rows(false));
-  TC_MAP(&g.bmap, f.snap, F, d, (uint64_t)f.nslots * B, b_box_rows(true));
+  g.A = {gO, (uint64_t)(d), (uint64_t)(T), (uint64_t)(B)};
+  g.Bop = {f.snap, (uint64_t)(F), (uint64_t)(d), (uint64_t)((uint64_t)f.nslots * B)};
   BW_CHECK(chunked(GM_CHUNK_ROWS, 0, (int)F, (int)d, gZ, F, T * F, GO_F32_ADD, nullptr, GR_FIRST, f.nslots));
   // 9. the gated activation; gH = gA Wg + gBu Wu; gWg = gA^T H, gWu = gBu^T H
   k_gate_backward_bf16<<<grid_for(BT * F), 256, 0, st>>>(Af, Buf, gZ, gA, gBu, (size_t)(BT * F));
-  TC_MAP(&g.amap, gA, F, BT, 1, a_box_rows(false));
-  TC_MAP(&g.bmap, Wg, d, F, 1, b_box_rows(true));
+  g.A = {gA, (uint64_t)(F), (uint64_t)(BT), (uint64_t)(1)};
+  g.Bop = {Wg, (uint64_t)(d), (uint64_t)(F), (uint64_t)(1)};
   g.a_mn = 0; g.b_mn = 1;
   BW_CHECK(plain((int)BT, (int)d, (int)F, gH, d, GO_F32));
-  TC_MAP(&g.amap, gBu, F, BT, 1, a_box_rows(false));
-  TC_MAP(&g.bmap, Wu, d, F, 1, b_box_rows(true));
+  g.A = {gBu, (uint64_t)(F), (uint64_t)(BT), (uint64_t)(1)};
+  g.Bop = {Wu, (uint64_t)(d), (uint64_t)(F), (uint64_t)(1)};
   BW_CHECK(plain((int)BT, (int)d, (int)F, gH, d, GO_F32_ADD));
-  TC_MAP(&g.amap, gA, F, BT, 1, a_box_rows(true));
-  TC_MAP(&g.bmap, H, d, BT, 1, b_box_rows(true));
+  g.A = {gA, (uint64_t)(F), (uint64_t)(BT), (uint64_t)(1)};
+  g.Bop = {H, (uint64_t)(d), (uint64_t)(BT), (uint64_t)(1)};
   g.a_mn = 1; g.b_mn = 1;
   BW_CHECK(plain((int)F, (int)d, (int)BT, gWg, d, GO_F32));
-  TC_MAP(&g.amap, gBu, F, BT, 1, a_box_rows(true));
+  g.A = {gBu, (uint64_t)(F), (uint64_t)(BT), (uint64_t)(1)};
   BW_CHECK(plain((int)F, (int)d, (int)BT, gWu, d, GO_F32));
   // 10. the target: gU = gV Wt^T, gWt = U^T gV, then the conv
   k_f32_to_bf16<<<grid_for(BT * d), 256, 0, st>>>(gV, gVb, (size_t)(BT * d));
-  TC_MAP(&g.amap, gVb, d, BT, 1, a_box_rows(false));
-  TC_MAP(&g.bmap, Wt, d, d, 1, b_box_rows(false));
+  g.A = {gVb, (uint64_t)(d), (uint64_t)(BT), (uint64_t)(1)};
+  g.Bop = {Wt, (uint64_t)(d), (uint64_t)(d), (uint64_t)(1)};
   g.a_mn = 0; g.b_mn = 0;
   BW_CHECK(plain((int)BT, (int)d, (int)d, gU, d, GO_F32));
-  TC_MAP(&g.amap, f.U, d, BT, 1, a_box_rows(true));
-  TC_MAP(&g.bmap, gVb, d, BT, 1, b_box_rows(true));
+  g.A = {f.U, (uint64_t)(d), (uint64_t)(BT), (uint64_t)(1)};
+  g.Bop = {gVb, (uint64_t)(d), (uint64_t)(BT), (uint64_t)(1)};
   g.a_mn = 1; g.b_mn = 1;
   BW_CHECK(plain((int)d, (int)d, (int)BT, gWt, d, GO_F32));
   k_widen<<<grid_for(d * kTaps), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(cw), cwf, (size_t)(d * kTaps));
@@ -802,7 +794,6 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
   return cudaGetLastError();
 }
 
-#undef TC_MAP
 
 }  // namespace bwd
 }  // namespace ipttt

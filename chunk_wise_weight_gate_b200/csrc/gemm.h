@@ -8,10 +8,9 @@
 //                  chunk i's slot of a stack of [d][F] matrices
 //   GM_CHUNK_K     out[i][b][m][n]      = sum over the tokens t of chunk i of A(b, t, m) B(b, t, n)
 //
-// Operands are bf16 tensor maps (3D {inner, rows, outer}, 128-byte swizzle) in
-// one of two orders: K-major (k is the inner, contiguous index) or MN-major (m,
-// resp. n, is).  Boxes: A K-major {64, 128}, A MN-major {64, 64}; B K-major
-// {64, 256}, B MN-major {64, 64}.
+// Operands are bf16 arrays {outer, rows, inner} read through 128-byte-swizzled
+// TMA boxes, in one of two orders: K-major (k is the inner, contiguous index) or
+// MN-major (m, resp. n, is).
 #pragma once
 
 #include <cuda.h>
@@ -30,9 +29,15 @@ enum Mode { GM_PLAIN = 0, GM_CHUNK_ROWS = 1, GM_CHUNK_K = 2 };
 enum Rows { GR_ALL = 0, GR_LAST = 1, GR_FIRST = 2 };
 enum Out { GO_F32 = 0, GO_F32_ADD = 1, GO_BF16 = 2 };
 
+// A bf16 operand: a row-major {outer, rows, inner} array (inner contiguous).
+struct Operand {
+  const void* base;
+  uint64_t inner, rows, outer;
+};
+
 struct Args {
-  CUtensorMap amap, bmap;
-  int a_mn, b_mn;        // operand order (1: MN-major)
+  Operand A, Bop;        // the tensor maps are made by run() for the form it picks
+  int a_mn, b_mn;        // operand order (1: MN-major); the per-chunk-K form takes both MN-major
   int mode;              // Mode
   int M, N, K;           // PLAIN: all three; CHUNK_ROWS: N, K; CHUNK_K: M, N
   int B, T, C, k;        // chunk modes: rows, tokens per row, chunk length, chunks per row
@@ -48,13 +53,10 @@ struct Args {
   int* status;           // device status word (timeouts)
 };
 
-// Box sizes the maps must have for an operand of the given order.
-constexpr uint32_t kBoxInner = 64;
-inline uint32_t a_box_rows(bool mn) { return mn ? 64 : 128; }
-inline uint32_t b_box_rows(bool mn) { return mn ? 64 : 256; }
-
-// Launches the persistent kernel on up to num_sms CTAs.  cudaErrorInvalidValue
-// when N is not a multiple of 32 or a size is not positive.
+// Launches the persistent kernel: on clusters of two CTAs (256-row tiles) when the
+// rows are at least 256 (and, per chunk rows, the chunk a multiple of 256), else
+// on up to num_sms single CTAs.  cudaErrorInvalidValue when N is not a multiple
+// of 32, a size is not positive or a tensor map cannot be made.
 cudaError_t run(const Args& a, int num_sms, cudaStream_t st);
 
 }  // namespace gemm

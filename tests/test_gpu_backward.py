@@ -40,6 +40,10 @@ CASES = {
     # (delta norms 10.6 .. 17.3: tau = 15 clips two of five, 7% and more from the kink)
     "bf16_tiles_ragged": dict(B=1, T=600, C=128, d=256, F=512, dtype="bf16", eta=0.01, clip=15.0,
                               docs=[70, 333], conv_std=0.3, wtarget="identity_noise", gS=True),
+    # 256-token chunks (the per-chunk-row products on CTA pairs), documents, a ragged
+    # last chunk (delta norms 18.9 .. 24.8: tau = 21.8 clips three of six, 2% and more from the kink)
+    "bf16_chunk256": dict(B=2, T=700, C=256, d=256, F=512, dtype="bf16", eta=0.01, clip=21.8,
+                          docs=[300, 700 + 100], conv_std=0.3, wtarget="identity_noise", gS=True),
     # no clip, no gS: the reverse scan starts from zero
     "bf16_noclip": dict(B=1, T=256, C=64, d=128, F=256, dtype="bf16", eta=0.05, clip=0.0, docs=[],
                         conv_std=0.3, wtarget="identity_noise", gS=False),
