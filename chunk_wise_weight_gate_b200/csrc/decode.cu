@@ -28,8 +28,7 @@ namespace ipttt {
 namespace {
 
 constexpr int kDecodeMaxRows = 16;  // rows per decode batch
-constexpr int kWarps = 8;           // warps per block; one output row (f or j) per warp
-constexpr int kFChunk = 2048;       // z columns staged in shared memory at a time
+constexpr int kWarps = 8;           // warps per block
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -54,100 +53,160 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// z[b][f] = bf16(SiLU(Wg[f] . h_b) * (Wu[f] . h_b)); one warp per f, h in shared memory.
-__global__ void __launch_bounds__(kWarps * 32) k_decode_gateup(const __nv_bfloat16* __restrict__ h,
-                                                             const __nv_bfloat16* __restrict__ Wg,
-                                                             const __nv_bfloat16* __restrict__ Wu,
-                                                             __nv_bfloat16* __restrict__ z, int B, int d, int F) {
+// z[b][f] = bf16(SiLU(Wg[f] . h_b) * (Wu[f] . h_b)).  A block holds four rows f,
+// two warps per row, each warp half of d (h in shared memory); the halves are
+// added in a fixed order.  Per batch of kApplyBatch 16-byte words a lane requests
+// the words of both weight rows before it uses any.  Block 0 also files this
+// token's h and x0 rows into the chunk buffers (row b at hbuf + b * rs).
+constexpr int kApplyBatch = 4;
+__global__ void __launch_bounds__(kWarps * 32, 2) k_decode_gateup(const __nv_bfloat16* __restrict__ h,
+                                                                const __nv_bfloat16* __restrict__ x0,
+                                                                const __nv_bfloat16* __restrict__ Wg,
+                                                                const __nv_bfloat16* __restrict__ Wu,
+                                                                __nv_bfloat16* __restrict__ z, __nv_bfloat16* hbuf,
+                                                                __nv_bfloat16* xbuf, long long rs, int B, int d,
+                                                                int F) {
   extern __shared__ uint4 hs[];  // [B][d / 8]
+  __shared__ float part[kWarps][2][kDecodeMaxRows];
   const int dv = d / 8;
-  for (int i = threadIdx.x; i < B * dv; i += blockDim.x) hs[i] = reinterpret_cast<const uint4*>(h)[i];
+  for (int i = threadIdx.x; i < B * dv; i += blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(h)[i];
+    hs[i] = v;
+    if (blockIdx.x == 0) {
+      const int b = i / dv, k = i % dv;
+      reinterpret_cast<uint4*>(hbuf + b * rs)[k] = v;
+      reinterpret_cast<uint4*>(xbuf + b * rs)[k] = reinterpret_cast<const uint4*>(x0)[i];
+    }
+  }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int f = blockIdx.x * kWarps + warp;
-  if (f >= F) return;
-  const uint4* wg = reinterpret_cast<const uint4*>(Wg + (size_t)f * d);
-  const uint4* wu = reinterpret_cast<const uint4*>(Wu + (size_t)f * d);
+  const int f = blockIdx.x * (kWarps / 2) + (warp >> 1);
+  const int half = warp & 1;
+  const int lo = half ? dv / 2 : 0, hi = half ? dv : dv / 2;
   float g[kDecodeMaxRows], u[kDecodeMaxRows];
 #pragma unroll
   for (int b = 0; b < kDecodeMaxRows; ++b) g[b] = u[b] = 0.0f;
-#pragma unroll 4
-  for (int k = lane; k < dv; k += 32) {
-    const uint4 a = wg[k], c = wu[k];
+  if (f < F) {
+    const uint4* wg = reinterpret_cast<const uint4*>(Wg + (size_t)f * d);
+    const uint4* wu = reinterpret_cast<const uint4*>(Wu + (size_t)f * d);
+    for (int k0 = lo + lane; k0 < hi; k0 += 32 * kApplyBatch) {
+      uint4 a[kApplyBatch], c[kApplyBatch];
 #pragma unroll
-    for (int b = 0; b < kDecodeMaxRows; ++b)
-      if (b < B) {
-        const uint4 x = hs[b * dv + k];
-        g[b] += dot8(a, x);
-        u[b] += dot8(c, x);
+      for (int q = 0; q < kApplyBatch; ++q) {
+        const int k = k0 + 32 * q;
+        if (k < hi) {
+          a[q] = wg[k];
+          c[q] = wu[k];
+        }
       }
+#pragma unroll
+      for (int q = 0; q < kApplyBatch; ++q) {
+        const int k = k0 + 32 * q;
+        if (k >= hi) break;
+#pragma unroll
+        for (int b = 0; b < kDecodeMaxRows; ++b) {
+          if (b >= B) break;
+          const uint4 x = hs[b * dv + k];
+          g[b] += dot8(a[q], x);
+          u[b] += dot8(c[q], x);
+        }
+      }
+    }
   }
 #pragma unroll
   for (int b = 0; b < kDecodeMaxRows; ++b)
     if (b < B) {
       const float gs = warp_sum(g[b]), us = warp_sum(u[b]);
-      if (lane == 0) z[(size_t)b * F + f] = __float2bfloat16_rn(silu_fast(gs) * us);
+      if (lane == 0) {
+        part[warp][0][b] = gs;
+        part[warp][1][b] = us;
+      }
     }
+  __syncthreads();
+  if (half == 0 && lane < B && f < F) {
+    const float gs = part[warp][0][lane] + part[warp + 1][0][lane];
+    const float us = part[warp][1][lane] + part[warp + 1][1][lane];
+    z[(size_t)lane * F + f] = __float2bfloat16_rn(silu_fast(gs) * us);
+  }
 }
 
-// o[b][j] = bf16(W0[j] . z_b + (m_b ? snap_b[j] . z_b : 0)).  A block holds kWarps/2
-// rows j, two warps per row, each summing half of every staged z chunk (kFChunk
-// columns at a time); the two halves are added in a fixed order at the end.
-__global__ void __launch_bounds__(kWarps * 32) k_decode_apply(const __nv_bfloat16* __restrict__ z,
-                                                            const __nv_bfloat16* __restrict__ W0,
-                                                            const __nv_bfloat16* __restrict__ snap,
-                                                            uint32_t mask, __nv_bfloat16* __restrict__ o, int B,
-                                                            int d, int F) {
-  extern __shared__ uint4 zs[];  // [B][kFChunk / 8], then the halves' partial sums
+// o[b][j] = bf16(W0[j] . z_b + (m_b ? snap_b[j] . z_b : 0)).  A block holds two
+// rows j, four warps per row, each warp a quarter of F; the quarters are added in
+// a fixed order.  Per batch of kApplyBatch 16-byte words a lane requests the W0
+// words first, then per row b the z_b words (small, L1/L2-resident) and the
+// snapshot words, so it keeps up to 3 kApplyBatch loads in flight without
+// block barriers in the loop.
+__global__ void __launch_bounds__(kWarps * 32, 2) k_decode_apply(const __nv_bfloat16* __restrict__ z,
+                                                               const __nv_bfloat16* __restrict__ W0,
+                                                               const __nv_bfloat16* __restrict__ snap,
+                                                               uint32_t mask, __nv_bfloat16* __restrict__ o, int B,
+                                                               int d, int F) {
+  __shared__ float part[kWarps][kDecodeMaxRows];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * (kWarps / 2) + (warp >> 1);
-  const int part = warp & 1;
+  const int j = blockIdx.x * (kWarps / 4) + (warp >> 2);
+  const int quarter = warp & 3;
+  const int fv = F / 8;
+  const int lo = fv * quarter / 4, hi = fv * (quarter + 1) / 4;
   float a0[kDecodeMaxRows], a1[kDecodeMaxRows];
 #pragma unroll
   for (int b = 0; b < kDecodeMaxRows; ++b) a0[b] = a1[b] = 0.0f;
-  for (int f0 = 0; f0 < F; f0 += kFChunk) {
-    const int fn = min(kFChunk, F - f0) / 8;
-    __syncthreads();
-    for (int i = threadIdx.x; i < B * fn; i += blockDim.x) {
-      const int b = i / fn, k = i % fn;
-      zs[b * (kFChunk / 8) + k] = reinterpret_cast<const uint4*>(z + (size_t)b * F + f0)[k];
-    }
-    __syncthreads();
-    if (j < d) {
-      const uint4* w = reinterpret_cast<const uint4*>(W0 + (size_t)j * F + f0);
-      const int k_lo = part * (fn / 2), k_hi = part ? fn : fn / 2;
-#pragma unroll 4
-      for (int k = k_lo + lane; k < k_hi; k += 32) {
-        const uint4 wv = w[k];
+  if (j < d) {
+    const uint4* w = reinterpret_cast<const uint4*>(W0 + (size_t)j * F);
+    for (int k0 = lo + lane; k0 < hi; k0 += 32 * kApplyBatch) {
+      uint4 wv[kApplyBatch];
 #pragma unroll
-        for (int b = 0; b < kDecodeMaxRows; ++b)
-          if (b < B) {
-            const uint4 x = zs[b * (kFChunk / 8) + k];
-            a0[b] += dot8(wv, x);
-            if (mask >> b & 1u) {
-              const uint4 sv = reinterpret_cast<const uint4*>(snap + ((size_t)b * d + j) * F + f0)[k];
-              a1[b] += dot8(sv, x);
-            }
+      for (int q = 0; q < kApplyBatch; ++q)
+        if (k0 + 32 * q < hi) wv[q] = w[k0 + 32 * q];
+#pragma unroll
+      for (int b = 0; b < kDecodeMaxRows; ++b) {
+        if (b >= B) break;
+        const uint4* zb = reinterpret_cast<const uint4*>(z + (size_t)b * F);
+        const uint4* sb = reinterpret_cast<const uint4*>(snap + ((size_t)b * d + j) * F);
+        const bool cont = (mask >> b) & 1u;
+        uint4 zv[kApplyBatch], sv[kApplyBatch];
+#pragma unroll
+        for (int q = 0; q < kApplyBatch; ++q) {
+          const int k = k0 + 32 * q;
+          if (k < hi) {
+            zv[q] = __ldg(zb + k);
+            if (cont) sv[q] = sb[k];
           }
+        }
+#pragma unroll
+        for (int q = 0; q < kApplyBatch; ++q) {
+          const int k = k0 + 32 * q;
+          if (k >= hi) break;
+          a0[b] += dot8(wv[q], zv[q]);
+          if (cont) a1[b] += dot8(sv[q], zv[q]);
+        }
       }
     }
   }
-  // halves: warp 2r+1 hands its sums to warp 2r through shared memory
-  __syncthreads();
-  float* red = reinterpret_cast<float*>(zs);  // [kWarps / 2][kDecodeMaxRows]
 #pragma unroll
   for (int b = 0; b < kDecodeMaxRows; ++b)
     if (b < B) {
       const float s = warp_sum(a0[b]) + warp_sum(a1[b]);
-      if (part == 1 && lane == 0) red[(warp >> 1) * kDecodeMaxRows + b] = s;
-      a0[b] = s;
+      if (lane == 0) part[warp][b] = s;
     }
   __syncthreads();
-  if (part == 0 && lane == 0 && j < d) {
-#pragma unroll
-    for (int b = 0; b < kDecodeMaxRows; ++b)
-      if (b < B) o[(size_t)b * d + j] = __float2bfloat16_rn(a0[b] + red[(warp >> 1) * kDecodeMaxRows + b]);
+  if (quarter == 0 && lane < B && j < d) {
+    const int w0 = warp;  // the row's first warp; its quarters follow
+    o[(size_t)lane * d + j] = __float2bfloat16_rn(((part[w0][lane] + part[w0 + 1][lane]) + part[w0 + 2][lane]) +
+                                                  part[w0 + 3][lane]);
   }
+}
+
+// Shared memory above the default 48 KB for the gate/up kernel's h rows (B d bf16),
+// raised once per device to the largest size asked for so far.
+bool decode_smem_ready(int smem) {
+  static int granted[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (smem <= granted[dev]) return true;
+  if (cudaFuncSetAttribute(k_decode_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return false;
+  granted[dev] = smem;
+  return true;
 }
 
 // Host bookkeeping of a decode state (lives in the caller's host buffer).
@@ -268,30 +327,20 @@ ipttt_status ipttt_decode_step(const ipttt_params* p, void* state, void* host_st
         hs->starts[hs->n_starts++] = b * C + hs->n;
       }
 
-  // keep this token's inputs for the chunk's update
-  if (cudaMemcpy2DAsync(base + L.H + hs->n * row, (size_t)C * row, h, row, row, B, cudaMemcpyDeviceToDevice, st) !=
-          cudaSuccess ||
-      cudaMemcpy2DAsync(base + L.X0 + hs->n * row, (size_t)C * row, x0, row, row, B, cudaMemcpyDeviceToDevice,
-                        st) != cudaSuccess)
-    return IPTTT_ERR_CUDA;
-
+  // the gate/up kernel also files this token's h and x0 rows for the chunk's update
   __nv_bfloat16* z = reinterpret_cast<__nv_bfloat16*>(base + L.z);
   {
     const int smem = B * d * 2;
-    if (cudaFuncSetAttribute(k_decode_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return IPTTT_ERR_CUDA;
-    k_decode_gateup<<<(F + kWarps - 1) / kWarps, kWarps * 32, smem, st>>>(
-        static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(Wgate),
-        static_cast<const __nv_bfloat16*>(Wup), z, B, d, F);
+    if (smem > 48 * 1024 && !decode_smem_ready(smem)) return IPTTT_ERR_CUDA;
+    k_decode_gateup<<<(F + kWarps / 2 - 1) / (kWarps / 2), kWarps * 32, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(x0),
+        static_cast<const __nv_bfloat16*>(Wgate), static_cast<const __nv_bfloat16*>(Wup), z,
+        reinterpret_cast<__nv_bfloat16*>(base + L.H + hs->n * row),
+        reinterpret_cast<__nv_bfloat16*>(base + L.X0 + hs->n * row), (long long)C * d, B, d, F);
   }
-  {
-    const int smem = B * kFChunk * 2;
-    if (cudaFuncSetAttribute(k_decode_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return IPTTT_ERR_CUDA;
-    k_decode_apply<<<(d + kWarps / 2 - 1) / (kWarps / 2), kWarps * 32, smem, st>>>(
-        z, static_cast<const __nv_bfloat16*>(Wdown0), reinterpret_cast<const __nv_bfloat16*>(base + L.snap),
-        hs->cont_mask, static_cast<__nv_bfloat16*>(o), B, d, F);
-  }
+  k_decode_apply<<<(d + kWarps / 4 - 1) / (kWarps / 4), kWarps * 32, 0, st>>>(
+      z, static_cast<const __nv_bfloat16*>(Wdown0), reinterpret_cast<const __nv_bfloat16*>(base + L.snap),
+      hs->cont_mask, static_cast<__nv_bfloat16*>(o), B, d, F);
   if (cudaGetLastError() != cudaSuccess) return IPTTT_ERR_CUDA;
 
   if (++hs->n < C) return IPTTT_OK;

@@ -532,22 +532,30 @@ class DecodeState:
 
     def step(self, h, x0, Wgate, Wup, Wdown0, conv_w, Wtarget, starts=None, *, o=None, stream=None):
         """One token of every row: h, x0 [B, d] on the device; starts: B flags (a
-        document begins at this token), or None.  Returns o [B, d]."""
+        document begins at this token), or None.  Returns o [B, d].  The weights
+        are checked once per set of tensors (by identity) and their pointers kept."""
         cfg = self.cfg
         dt = cfg.torch_dtype
         for name, t in (("h", h), ("x0", x0)):
             if tuple(t.shape) != (cfg.B, cfg.d):
                 raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {(cfg.B, cfg.d)}")
-        _shape_check(cfg, Wgate=Wgate, Wup=Wup, Wdown0=Wdown0, conv_w=conv_w, Wtarget=Wtarget)
+        ws = (Wgate, Wup, Wdown0, conv_w, Wtarget)
+        key = tuple(id(w) for w in ws)
+        if getattr(self, "_wkey", None) != key:
+            _shape_check(cfg, Wgate=Wgate, Wup=Wup, Wdown0=Wdown0, conv_w=conv_w, Wtarget=Wtarget)
+            self._wptr = [_ptr(w, dt, n) for w, n in zip(ws, ("Wgate", "Wup", "Wdown0", "conv_w", "Wtarget"))]
+            self._wref = ws  # keeps the tensors (and so their ids and pointers) alive
+            self._wkey = key
+        if getattr(self, "_p", None) is None:
+            self._p = cfg.params()
         if o is None:
             o = torch.empty(cfg.B, cfg.d, dtype=dt, device=h.device)
         flags = None
         if starts is not None:
             flags = (ctypes.c_int32 * cfg.B)(*[int(bool(x)) for x in starts])
-        _check(lib().ipttt_decode_step(ctypes.byref(cfg.params()), self.buf.data_ptr(), self.host,
-                                       _ptr(h, dt, "h"), _ptr(x0, dt, "x0"), flags, _ptr(Wgate, dt, "Wgate"),
-                                       _ptr(Wup, dt, "Wup"), _ptr(Wdown0, dt, "Wdown0"), _ptr(conv_w, dt, "conv_w"),
-                                       _ptr(Wtarget, dt, "Wtarget"), _ptr(o, dt, "o"), _stream(stream)),
+        _check(lib().ipttt_decode_step(ctypes.byref(self._p), self.buf.data_ptr(), self.host,
+                                       _ptr(h, dt, "h"), _ptr(x0, dt, "x0"), flags, *self._wptr, _ptr(o, dt, "o"),
+                                       _stream(stream)),
                "ipttt_decode_step")
         return o
 
