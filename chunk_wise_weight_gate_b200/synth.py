@@ -64,6 +64,8 @@ WORKLOADS = {
     "qwen3_4b_128k": Workload("qwen3_4b_128k", B=1, T=131072, C=1024, d=2560, F=9728),
     "packed_8x8k": Workload("packed_8x8k", B=8, T=8192, C=512, d=2560, F=9728, docs="packed"),
     "stack6_4x16k": Workload("stack6_4x16k", B=4, T=16384, C=512, d=2560, F=9728, layers=6),
+    # the Qwen3-4B layer on 4k tokens: a small case for profiler captures
+    "qwen3_4b_4k": Workload("qwen3_4b_4k", B=1, T=4096, C=512, d=2560, F=9728),
 }
 STACK_CHUNK_SIZES = (64, 128, 256, 512, 1024, 2048)
 
