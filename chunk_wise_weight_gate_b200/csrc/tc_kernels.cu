@@ -494,16 +494,26 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
         p.intra ? reinterpret_cast<const __nv_bfloat16*>(p.intra) + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
 #pragma unroll 1
     for (int c = c_begin; c < c_end; c += 32) {
+      // the row's E and H words are requested before the accumulator is read, so
+      // their latency overlaps the TMEM round trip
+      uint4 ev4[4], hv4[4];
+      if (erow && valid) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) ev4[q] = reinterpret_cast<const uint4*>(erow + c)[q];
+      }
+      if (hrow && valid) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) hv4[q] = reinterpret_cast<const uint4*>(hrow + c)[q];
+      }
       tmem_ld32(tacc + c, r0);
       if (j.nsrc == 2) tmem_ld32(tacc + 128 + c, r1);
       tmem_ld_wait();
       float e[32];
       if (erow && valid) {
         // the grouped scan's within-group term joins the fast-weight part
-        const uint4* e4 = reinterpret_cast<const uint4*>(erow + c);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const uint4 ev = e4[q];
+          const uint4 ev = ev4[q];
           const uint32_t ew4[4] = {ev.x, ev.y, ev.z, ev.w};
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
@@ -524,10 +534,9 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
       }
       if (valid) {
         if (hrow) {
-          const uint4* h4 = reinterpret_cast<const uint4*>(hrow + c);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const uint4 hv = h4[q];
+            const uint4 hv = hv4[q];
             const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -718,6 +727,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
       if (lane == 0) {
         if constexpr (PAIR) mbar_arrive_cluster(empty0 + 8u * buf);
         else mbar_arrive(&acc_empty[buf]);
+      }
+      if constexpr (is_apply<FAM>()) {
+        // while the next tile's MMAs run, bring this thread's rows of its
+        // within-group term and residual into L2
+        if (p.intra || p.resid) {
+          const int nt = seq_tile<FAM>(p, i + 1);
+          if (nt >= 0) {
+            Job jn;
+            decode<FAM>(p, nt, jn);
+            const int rin = FAM == FAM_APPLY256 ? half * 128 + row : row;
+            const int tn = jn.t0 + jn.m0 + rin;
+            if (tn < p.T && (FAM == FAM_APPLY256 || row < p.tr)) {
+              const size_t off = ((size_t)jn.b * p.T + tn) * p.d + jn.n0 + (FAM == FAM_APPLY256 ? 0 : half * 64);
+              const int bytes = FAM == FAM_APPLY256 ? 256 : 128;
+              for (int q = 0; q < bytes; q += 128) {
+                if (p.intra) prefetch_l2(reinterpret_cast<const uint8_t*>(p.intra) + off * 2 + q);
+                if (p.resid) prefetch_l2(reinterpret_cast<const uint8_t*>(p.resid) + off * 2 + q);
+              }
+            }
+          }
+        }
       }
     }
     if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
