@@ -193,6 +193,16 @@ bool grouped_scan(const ipttt_params& p) {
 
 int scan_unit_tokens(const ipttt_params& p) { return grouped_scan(p) ? kGroupTokens : p.C; }
 
+int device_sms() {
+  DeviceInfo* di = nullptr;
+  return device_info(&di) == IPTTT_OK ? di->num_sms : 0;
+}
+
+int* device_status() {
+  DeviceInfo* di = nullptr;
+  return device_info(&di) == IPTTT_OK ? di->status : nullptr;
+}
+
 namespace {
 
 ipttt_params group_params(const ipttt_params& p) {

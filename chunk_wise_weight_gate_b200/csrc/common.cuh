@@ -57,5 +57,8 @@ ipttt_status cuda_status(cudaError_t e);
 // 128 or 256 tokens in groups, else C.  Streaming pieces that are multiples of it give
 // one call's result bit for bit.
 int scan_unit_tokens(const ipttt_params& p);
+// The current device's SM count and the device status word (0 on failure).
+int device_sms();
+int* device_status();
 
 }  // namespace ipttt

@@ -16,6 +16,9 @@
 //
 // The two per-token kernels are batched matrix-vector products bound by HBM: each
 // reads Wgate, Wup, Wdown0 once for all rows and every row's bf16 state snapshot.
+// From kTensorRows rows on, the gate/up products run as two tcgen05 GEMMs
+// (Wgate, Wup as the M operand, the rows' h as an N = 32 operand), whose
+// multiply-adds the CUDA cores would otherwise bound.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -23,11 +26,15 @@
 
 #include "aux_kernels.h"
 #include "common.cuh"
+#include "gemm.h"
 
 namespace ipttt {
 namespace {
 
 constexpr int kDecodeMaxRows = 16;  // rows per decode batch
+constexpr int kTensorRows = 4;      // rows from which gate/up runs on the tensor cores
+constexpr int kGemmCols = 32;       // N of those GEMMs: the rows, padded
+constexpr int kW0Split = 7;         // K slices of the W0 GEMM (d / 256 pair tiles x 7 fill the SMs)
 constexpr int kWarps = 8;           // warps per block
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -139,8 +146,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_decode_gateup(const __nv_bfl
 __global__ void __launch_bounds__(kWarps * 32, 2) k_decode_apply(const __nv_bfloat16* __restrict__ z,
                                                                const __nv_bfloat16* __restrict__ W0,
                                                                const __nv_bfloat16* __restrict__ snap,
-                                                               uint32_t mask, __nv_bfloat16* __restrict__ o, int B,
-                                                               int d, int F) {
+                                                               uint32_t mask, const float* __restrict__ add,
+                                                               __nv_bfloat16* __restrict__ o, int B, int d,
+                                                               int F) {
   __shared__ float part[kWarps][kDecodeMaxRows];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * (kWarps / 4) + (warp >> 2);
@@ -191,8 +199,76 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_decode_apply(const __nv_bflo
   __syncthreads();
   if (quarter == 0 && lane < B && j < d) {
     const int w0 = warp;  // the row's first warp; its quarters follow
-    o[(size_t)lane * d + j] = __float2bfloat16_rn(((part[w0][lane] + part[w0 + 1][lane]) + part[w0 + 2][lane]) +
-                                                  part[w0 + 3][lane]);
+    const float sum = ((part[w0][lane] + part[w0 + 1][lane]) + part[w0 + 2][lane]) + part[w0 + 3][lane];
+    o[(size_t)lane * d + j] = __float2bfloat16_rn(add ? sum + add[(size_t)lane * d + j] : sum);
+  }
+}
+
+// t[b][j] = m_b ? snap_b[j] . z_b : 0 for many rows b: four warps per (b, j), each a
+// quarter of F, summed in a fixed order; each warp streams its own snapshot row, so
+// the B copies are read at the full width of the device rather than one W0 row's.
+__global__ void __launch_bounds__(kWarps * 32) k_decode_snap(const __nv_bfloat16* __restrict__ z,
+                                                           const __nv_bfloat16* __restrict__ snap, uint32_t mask,
+                                                           float* __restrict__ t, int B, int d, int F) {
+  __shared__ float part[kWarps];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long r = (long long)blockIdx.x * (kWarps / 4) + (warp >> 2);  // b d + j
+  const int quarter = warp & 3;
+  const int b = (int)(r / d), j = (int)(r % d);
+  float acc = 0.0f;
+  if (b < B && ((mask >> b) & 1u)) {
+    const int fv = F / 8;
+    const int lo = fv * quarter / 4, hi = fv * (quarter + 1) / 4;
+    const uint4* zb = reinterpret_cast<const uint4*>(z + (size_t)b * F);
+    const uint4* sb = reinterpret_cast<const uint4*>(snap + ((size_t)b * d + j) * F);
+    for (int k0 = lo + lane; k0 < hi; k0 += 32 * kApplyBatch) {
+      uint4 zv[kApplyBatch], sv[kApplyBatch];
+#pragma unroll
+      for (int q = 0; q < kApplyBatch; ++q)
+        if (k0 + 32 * q < hi) {
+          zv[q] = __ldg(zb + k0 + 32 * q);
+          sv[q] = sb[k0 + 32 * q];
+        }
+#pragma unroll
+      for (int q = 0; q < kApplyBatch; ++q)
+        if (k0 + 32 * q < hi) acc += dot8(sv[q], zv[q]);
+    }
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) part[warp] = acc;
+  __syncthreads();
+  if (quarter == 0 && lane == 0 && b < B) t[r] = ((part[warp] + part[warp + 1]) + part[warp + 2]) + part[warp + 3];
+}
+
+// This token's h and x0 rows into the chunk buffers (row b at hbuf + b * rs).
+__global__ void k_decode_file(const __nv_bfloat16* __restrict__ h, const __nv_bfloat16* __restrict__ x0,
+                              __nv_bfloat16* hbuf, __nv_bfloat16* xbuf, long long rs, int B, int d) {
+  const int dv = d / 8;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B * dv; i += gridDim.x * blockDim.x) {
+    const int b = i / dv, k = i % dv;
+    reinterpret_cast<uint4*>(hbuf + b * rs)[k] = reinterpret_cast<const uint4*>(h)[i];
+    reinterpret_cast<uint4*>(xbuf + b * rs)[k] = reinterpret_cast<const uint4*>(x0)[i];
+  }
+}
+
+// o[b][j] = bf16(sum over the K slices of part[q][j][b], in slice order, + t[b][j]).
+__global__ void k_decode_out(const float* __restrict__ part, const float* __restrict__ t,
+                             __nv_bfloat16* __restrict__ o, int B, int d, int slices) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B * d; i += gridDim.x * blockDim.x) {
+    const int b = i / d, j = i % d;
+    float s = 0.0f;
+    for (int q = 0; q < slices; ++q) s += part[((size_t)q * d + j) * kGemmCols + b];
+    o[i] = __float2bfloat16_rn(s + t[i]);
+  }
+}
+
+// z[b][f] = bf16(SiLU(g[f][b]) * u[f][b]) from the GEMMs' fp32 outputs [F][kGemmCols].
+__global__ void k_decode_gate_combine(const float* __restrict__ g, const float* __restrict__ u,
+                                      __nv_bfloat16* __restrict__ z, int B, int F) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B * F; i += gridDim.x * blockDim.x) {
+    const int b = i / F, f = i % F;
+    const size_t o = (size_t)f * kGemmCols + b;
+    z[i] = __float2bfloat16_rn(silu_fast(g[o]) * u[o]);
   }
 }
 
@@ -220,7 +296,7 @@ struct DecodeHost {
 };
 
 struct DecodeLayout {
-  size_t stream_state, H, X0, Oscr, snap, z, docs, ws, ws_bytes, total;
+  size_t stream_state, H, X0, Oscr, snap, z, gacc, uacc, tsnap, w0acc, docs, ws, ws_bytes, total;
 };
 
 ipttt_params chunk_params(const ipttt_params& p) {
@@ -241,6 +317,10 @@ bool decode_layout(const ipttt_params& p, DecodeLayout& L) {
   L.Oscr = off;         off += al256(rows);
   L.snap = off;         off += al256((size_t)p.B * p.d * p.F * 2);
   L.z = off;            off += al256((size_t)p.B * p.F * 2);
+  L.gacc = off;         off += al256((size_t)p.F * kGemmCols * 4);
+  L.uacc = off;         off += al256((size_t)p.F * kGemmCols * 4);
+  L.tsnap = off;        off += al256((size_t)p.B * p.d * 4);
+  L.w0acc = off;        off += al256((size_t)kW0Split * p.d * kGemmCols * 4);
   L.docs = off;         off += al256((size_t)p.B * p.C * 4);
   L.ws = off;           off += al256(ws);
   L.ws_bytes = ws;
@@ -327,20 +407,70 @@ ipttt_status ipttt_decode_step(const ipttt_params* p, void* state, void* host_st
         hs->starts[hs->n_starts++] = b * C + hs->n;
       }
 
-  // the gate/up kernel also files this token's h and x0 rows for the chunk's update
   __nv_bfloat16* z = reinterpret_cast<__nv_bfloat16*>(base + L.z);
-  {
+  __nv_bfloat16* hrow = reinterpret_cast<__nv_bfloat16*>(base + L.H + hs->n * row);
+  __nv_bfloat16* xrow = reinterpret_cast<__nv_bfloat16*>(base + L.X0 + hs->n * row);
+  if (B >= kTensorRows && d % 128 == 0 && F % 128 == 0) {
+    // g = Wgate h^T and u = Wup h^T as tcgen05 GEMMs (h rows past B read as zeros)
+    k_decode_file<<<(B * d / 8 + 255) / 256, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h),
+                                                            static_cast<const __nv_bfloat16*>(x0), hrow, xrow,
+                                                            (long long)C * d, B, d);
+    gemm::Args g{};
+    g.mode = gemm::GM_PLAIN;
+    g.M = F;
+    g.N = kGemmCols;
+    g.K = d;
+    g.Bop = {h, (uint64_t)d, (uint64_t)B, 1};
+    g.out_kind = gemm::GO_F32;
+    g.ldo = kGemmCols;
+    g.status = device_status();
+    const int sms = device_sms();
+    g.A = {Wgate, (uint64_t)d, (uint64_t)F, 1};
+    g.out = base + L.gacc;
+    if (gemm::run(g, sms, st) != cudaSuccess) return IPTTT_ERR_CUDA;
+    g.A = {Wup, (uint64_t)d, (uint64_t)F, 1};
+    g.out = base + L.uacc;
+    if (gemm::run(g, sms, st) != cudaSuccess) return IPTTT_ERR_CUDA;
+    k_decode_gate_combine<<<(B * F + 255) / 256, 256, 0, st>>>(reinterpret_cast<const float*>(base + L.gacc),
+                                                               reinterpret_cast<const float*>(base + L.uacc), z, B,
+                                                               F);
+  } else {
+    // the gate/up kernel also files this token's h and x0 rows for the chunk's update
     const int smem = B * d * 2;
     if (smem > 48 * 1024 && !decode_smem_ready(smem)) return IPTTT_ERR_CUDA;
     k_decode_gateup<<<(F + kWarps / 2 - 1) / (kWarps / 2), kWarps * 32, smem, st>>>(
         static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(x0),
-        static_cast<const __nv_bfloat16*>(Wgate), static_cast<const __nv_bfloat16*>(Wup), z,
-        reinterpret_cast<__nv_bfloat16*>(base + L.H + hs->n * row),
-        reinterpret_cast<__nv_bfloat16*>(base + L.X0 + hs->n * row), (long long)C * d, B, d, F);
+        static_cast<const __nv_bfloat16*>(Wgate), static_cast<const __nv_bfloat16*>(Wup), z, hrow, xrow,
+        (long long)C * d, B, d, F);
   }
-  k_decode_apply<<<(d + kWarps / 4 - 1) / (kWarps / 4), kWarps * 32, 0, st>>>(
-      z, static_cast<const __nv_bfloat16*>(Wdown0), reinterpret_cast<const __nv_bfloat16*>(base + L.snap),
-      hs->cont_mask, static_cast<__nv_bfloat16*>(o), B, d, F);
+  if (B >= kTensorRows) {
+    // the state copies row by row on their own, then W0 with their products added
+    float* tsnap = reinterpret_cast<float*>(base + L.tsnap);
+    k_decode_snap<<<(unsigned)(((long long)B * d + kWarps / 4 - 1) / (kWarps / 4)), kWarps * 32, 0, st>>>(
+        z, reinterpret_cast<const __nv_bfloat16*>(base + L.snap), hs->cont_mask, tsnap, B, d, F);
+    // W0 z_b for all rows as a tcgen05 GEMM (M = d, N = rows padded to 32), K split
+    // in kW0Split slices so that the tiles fill the SMs; the slices are added in order
+    gemm::Args g{};
+    g.mode = gemm::GM_PLAIN;
+    g.M = d;
+    g.N = kGemmCols;
+    g.K = F;
+    g.ksplit = F / 128 >= kW0Split ? kW0Split : 1;
+    g.A = {Wdown0, (uint64_t)F, (uint64_t)d, 1};
+    g.Bop = {z, (uint64_t)F, (uint64_t)B, 1};
+    g.out_kind = gemm::GO_F32;
+    g.out = base + L.w0acc;
+    g.ldo = kGemmCols;
+    g.osz = (long long)d * kGemmCols;
+    g.status = device_status();
+    if (gemm::run(g, device_sms(), st) != cudaSuccess) return IPTTT_ERR_CUDA;
+    k_decode_out<<<(B * d + 255) / 256, 256, 0, st>>>(reinterpret_cast<const float*>(base + L.w0acc), tsnap,
+                                                      static_cast<__nv_bfloat16*>(o), B, d, g.ksplit > 1 ? g.ksplit : 1);
+  } else {
+    k_decode_apply<<<(d + kWarps / 4 - 1) / (kWarps / 4), kWarps * 32, 0, st>>>(
+        z, static_cast<const __nv_bfloat16*>(Wdown0), reinterpret_cast<const __nv_bfloat16*>(base + L.snap),
+        hs->cont_mask, nullptr, static_cast<__nv_bfloat16*>(o), B, d, F);
+  }
   if (cudaGetLastError() != cudaSuccess) return IPTTT_ERR_CUDA;
 
   if (++hs->n < C) return IPTTT_OK;

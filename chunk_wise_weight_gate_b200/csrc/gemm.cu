@@ -65,7 +65,9 @@ struct Tile {
   int m0, n0;    // tile origin in the output's m and n
   int t0;        // chunk modes: first token of the chunk
   int mrows;     // rows of the output the tile may write (m < mrows)
-  int nk;        // K blocks of 64
+  int nk;        // K blocks of the tile
+  int kb0;       // its first K block
+  int slice;     // PLAIN with split K: the slice of K (output matrix)
   int z_b;       // outer coordinate of the B operand
 };
 
@@ -75,7 +77,7 @@ template <bool PAIR>
 __device__ __forceinline__ int num_tiles(const Args& a) {
   constexpr int TM = Cfg<PAIR>::TM;
   const int nt = cdiv(a.N, 256);
-  if (a.mode == GM_PLAIN) return cdiv(a.M, TM) * nt;
+  if (a.mode == GM_PLAIN) return cdiv(a.M, TM) * nt * max(1, a.ksplit);
   const int mt = a.mode == GM_CHUNK_ROWS ? cdiv(a.C, TM) : cdiv(a.M, TM);
   return a.nchunks * a.B * nt * mt;
 }
@@ -86,16 +88,24 @@ __device__ __forceinline__ void decode(const Args& a, int tile, Tile& t) {
   const int nt = cdiv(a.N, 256);
   if (a.mode == GM_PLAIN) {
     const int mt = cdiv(a.M, TM);
+    const int per_slice = mt * nt;
+    const int ks = max(1, a.ksplit);
+    const int nk_all = cdiv(a.K, Cfg<PAIR>::TK);
+    t.slice = tile / per_slice;
+    const int r = tile % per_slice;
     t.b = 0;
     t.chunk = 0;
-    t.m0 = (tile % mt) * TM;
-    t.n0 = (tile / mt) * 256;
+    t.m0 = (r % mt) * TM;
+    t.n0 = (r / mt) * 256;
     t.t0 = 0;
     t.mrows = a.M;
-    t.nk = cdiv(a.K, Cfg<PAIR>::TK);
+    t.kb0 = (int)((long long)nk_all * t.slice / ks);
+    t.nk = (int)((long long)nk_all * (t.slice + 1) / ks) - t.kb0;
     t.z_b = 0;
     return;
   }
+  t.slice = 0;
+  t.kb0 = 0;
   const int mt = a.mode == GM_CHUNK_ROWS ? cdiv(a.C, TM) : cdiv(a.M, TM);
   const int per_b = nt * mt;
   const int per_chunk = a.B * per_b;
@@ -137,7 +147,7 @@ __device__ __forceinline__ void load_stage(const KArgs& ka, const Tile& t, int k
   using Cf = Cfg<PAIR>;
   constexpr int TK = Cf::TK, BCOLS = Cf::BCOLS;
   const Args& a = ka.a;
-  const int k = kb * TK;
+  const int k = (t.kb0 + kb) * TK;
   const int m0 = t.m0 + 128 * r;       // this CTA's A rows
   const int n0 = t.n0 + BCOLS * r;     // this CTA's B columns
   if (a.mode == GM_CHUNK_K || a.a_mn) {
@@ -323,7 +333,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       const bool keep = keep_row(a, t, m);
       const float s = a.scale ? (a.mode == GM_PLAIN ? a.scale[0] : a.scale[(size_t)t.b * a.k + t.chunk]) : 1.0f;
       long long base;
-      if (a.mode == GM_PLAIN) base = (long long)m * a.ldo;
+      if (a.mode == GM_PLAIN) base = (long long)t.slice * a.osz + (long long)m * a.ldo;
       else if (a.mode == GM_CHUNK_ROWS) base = (long long)t.b * a.osz + (long long)(t.t0 + m) * a.ldo;
       else base = ((long long)t.chunk * a.B + t.b) * a.osz + (long long)m * a.ldo;
 #pragma unroll 1
@@ -422,7 +432,7 @@ int pair_workers(cudaStream_t st) {
 
 long long tiles_of(const Args& a, int tm) {
   const long long nt = (a.N + 255) / 256;
-  if (a.mode == GM_PLAIN) return (long long)((a.M + tm - 1) / tm) * nt;
+  if (a.mode == GM_PLAIN) return (long long)((a.M + tm - 1) / tm) * nt * std::max(1, a.ksplit);
   const long long mt = a.mode == GM_CHUNK_ROWS ? (a.C + tm - 1) / tm : (a.M + tm - 1) / tm;
   return (long long)a.nchunks * a.B * nt * mt;
 }
@@ -432,8 +442,10 @@ long long tiles_of(const Args& a, int tm) {
 cudaError_t run(const Args& a, int num_sms, cudaStream_t st) {
   if (a.N <= 0 || a.N % 32 != 0 || !a.out || !a.A.base || !a.Bop.base) return cudaErrorInvalidValue;
   if (a.mode == GM_PLAIN) {
-    if (a.M <= 0 || a.K <= 0) return cudaErrorInvalidValue;
+    // every slice holds at least one K block of either form (64 or 128 K)
+    if (a.M <= 0 || a.K <= 0 || a.ksplit < 0 || (a.ksplit > 1 && a.ksplit > a.K / 128)) return cudaErrorInvalidValue;
   } else {
+    if (a.ksplit > 1) return cudaErrorInvalidValue;
     if (a.B <= 0 || a.C <= 0 || a.C % 64 != 0 || a.nchunks <= 0 || a.chunk0 < 0 || a.chunk0 + a.nchunks > a.k)
       return cudaErrorInvalidValue;
     if (a.mode == GM_CHUNK_ROWS && (a.K <= 0 || a.nslots <= 0)) return cudaErrorInvalidValue;

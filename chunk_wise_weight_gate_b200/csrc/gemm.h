@@ -2,6 +2,8 @@
 // backward of the layer, whose products come in three shapes:
 //
 //   GM_PLAIN       out[m][n]            = s * sum_k A(m, k) B(k, n)
+//                  (with ksplit > 1: out[q][m][n] over the q-th of ksplit slices of K,
+//                  for a caller that adds them in a fixed order)
 //   GM_CHUNK_ROWS  out[b][t0 + m][n]   (=, +=) s[b][i] * sum_k A(b, t0 + m, k) B_i(k, n)
 //                  for the tokens t0 + m of chunk i (rows outside the chosen
 //                  document segment of the chunk are left alone), B_i taken from
@@ -50,6 +52,7 @@ struct Args {
   const float* scale;    // optional [B][k] scale (chunk modes) or [1] (PLAIN)
   const ChunkMeta* meta; // CHUNK_ROWS with rows != GR_ALL: [B][k]
   int rows;              // Rows
+  int ksplit;            // PLAIN: K in this many slices (0 or 1: one), slice s written at out + s * osz
   int* status;           // device status word (timeouts)
 };
 

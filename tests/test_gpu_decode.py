@@ -51,6 +51,23 @@ def test_decode_equals_forward_and_oracle():
     assert maxrel(orc["O"] - orc["D"], orc["O"]) > 5 * 2e-2
 
 
+def test_decode_batched_rows_on_the_tensor_cores():
+    # 8 rows: the gate/up products run as tcgen05 GEMMs (rows padded to 32); the
+    # outputs match the forward and the oracle as for 2 rows
+    B, T, C = 8, 300, 128
+    docs = [b * T + 37 * b for b in range(1, B)] + [60, T + 200]
+    cfg, inp = case(B, T, C, 256, 512, eta=2e-2, clip=0.0, docs=sorted(set(docs)))
+    dev = torch.device("cuda")
+    w = {k: inp[k].to(dev) for k in WEIGHTS}
+    _, out = decode_all(cfg, inp, T, w)
+    ref = ip.forward(cfg, inp["H"].to(dev), inp["X0"].to(dev), *(w[k] for k in WEIGHTS), inp["doc_starts"])
+    torch.cuda.synchronize()
+    assert maxrel(to_np(out), to_np(ref)) <= 1e-2
+    orc = oracle(cfg, inp)
+    assert maxrel(to_np(out), orc["O"]) <= 2e-2
+    assert maxrel(orc["O"] - orc["D"], orc["O"]) > 5 * 2e-2
+
+
 def test_decode_commits_the_prefill_state():
     # chunks of 512 tokens: a one-call forward then also scans chunk by chunk, as
     # the decode commits do (shorter chunks are scanned in groups of 512 tokens,
