@@ -1032,8 +1032,16 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
         bool ok = true;
         UpdJob jb;
         const uint32_t full0 = PAIR ? map_to_rank(smem_u32(full), 0) : 0u;  // the leader's full[0]
-        for (uint32_t i = 0; ok && upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
-          const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
+        // The next job's chunk metadata is requested one job ahead, so its round
+        // trip never stands between two chunks' loads.
+        bool have = upd_job<PAIR>(p, 0, wk, nwk, jb);
+        ChunkMeta m{};
+        if (have) m = p.meta[(size_t)jb.b * p.k + jb.chunk];
+        for (uint32_t i = 0; ok && have; ++i) {
+          UpdJob jn;
+          const bool hn = upd_job<PAIR>(p, i + 1, wk, nwk, jn);
+          ChunkMeta mn{};
+          if (hn) mn = p.meta[(size_t)jn.b * p.k + jn.chunk];
           const int t0 = jb.chunk * p.C;
           const int kb0 = (m.last_start - t0) / UPD_KB;
           const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
@@ -1061,6 +1069,9 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
                 tma_load_3d(sb + q * 64 * UPD_KB * 2, &p.map[4], &full[s], jb.n0 + 64 * q, ty, jb.b);
             }
           }
+          jb = jn;
+          m = mn;
+          have = hn;
         }
         if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
         counters[0] = it;
@@ -1071,14 +1082,20 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
         bool ok = true;
         UpdJob jb;
         const uint32_t idesc = idesc_bf16(PAIR ? 256 : 128, 256, true, true);
-        for (uint32_t i = 0; ok && upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
+        bool have = upd_job<PAIR>(p, 0, wk, nwk, jb);
+        ChunkMeta m{};
+        if (have) m = p.meta[(size_t)jb.b * p.k + jb.chunk];
+        for (uint32_t i = 0; ok && have; ++i) {
+          UpdJob jn;
+          const bool hn = upd_job<PAIR>(p, i + 1, wk, nwk, jn);
+          ChunkMeta mn{};
+          if (hn) mn = p.meta[(size_t)jn.b * p.k + jn.chunk];   // the next job's, one job ahead
           const int sl = (int)(i & 1);
           const uint32_t u = i >> 1;  // earlier uses of this slot
           const bool got =
               PAIR ? mbar_wait_cluster(&slot_free[sl], (u & 1) ^ 1) : mbar_wait(&slot_free[sl], (u & 1) ^ 1);
           if (!got || *abort_flag) { ok = false; break; }
           tc_fence_after();
-          const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
           const int t0 = jb.chunk * p.C;
           const int kb0 = (m.last_start - t0) / UPD_KB;
           const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
@@ -1103,6 +1120,9 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
           }
           if (!ok) break;
           if constexpr (PAIR) mma_commit_pair(&slot_full[sl], 3); else mma_commit(&slot_full[sl]);
+          jb = jn;
+          m = mn;
+          have = hn;
         }
         if (!ok) { *abort_flag = 1; set_status(p.status, IPTTT_ERR_TIMEOUT); }
         counters[1] = it;
