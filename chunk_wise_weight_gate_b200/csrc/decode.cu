@@ -32,7 +32,10 @@ namespace ipttt {
 namespace {
 
 constexpr int kDecodeMaxRows = 16;  // rows per decode batch
-constexpr int kTensorRows = 4;      // rows from which gate/up runs on the tensor cores
+// Rows from which the products run on the tensor cores.  Measured at d=2560, F=9728:
+// three rows decode at 35 k tokens/s on the CUDA-core kernels and four at 35 k on
+// the tensor cores, where the CUDA-core kernels built for up to 16 rows reach 26 k.
+constexpr int kTensorRows = 4;
 constexpr int kGemmCols = 32;       // N of those GEMMs: the rows, padded
 constexpr int kW0Split = 7;         // K slices of the W0 GEMM (d / 256 pair tiles x 7 fill the SMs)
 constexpr int kWarps = 8;           // warps per block
@@ -60,12 +63,20 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// z[b][f] = bf16(SiLU(Wg[f] . h_b) * (Wu[f] . h_b)).  A block holds four rows f,
-// two warps per row, each warp half of d (h in shared memory); the halves are
-// added in a fixed order.  Per batch of kApplyBatch 16-byte words a lane requests
-// the words of both weight rows before it uses any.  Block 0 also files this
-// token's h and x0 rows into the chunk buffers (row b at hbuf + b * rs).
-constexpr int kApplyBatch = 4;
+// Below kTensorRows rows both per-token kernels are persistent: two blocks per SM,
+// each warp taking its weight rows in a fixed stride, so the weights stream at
+// the full width of the device with no block launched per handful of rows.
+// NR: the most rows a build of the kernel takes (kTensorRows - 1).
+constexpr int kApplyBatch = 4;   // per operand, in the apply kernel
+// 16-byte words of both weight rows a lane requests at once
+template <int NR> constexpr int row_words() { return NR <= 3 ? 10 : 6; }
+
+// z[b][f] = bf16(SiLU(Wg[f] . h_b) * (Wu[f] . h_b)) for B <= NR rows.  Each
+// warp owns whole rows f (h in shared memory): a lane requests its kRowWords words
+// of both weight rows before it uses any, and the warp's sum is taken in a fixed
+// order.  Block 0 also files this token's h and x0 rows into the chunk buffers
+// (row b at hbuf + b * rs).
+template <int NR>
 __global__ void __launch_bounds__(kWarps * 32, 2) k_decode_gateup(const __nv_bfloat16* __restrict__ h,
                                                                 const __nv_bfloat16* __restrict__ x0,
                                                                 const __nv_bfloat16* __restrict__ Wg,
@@ -74,7 +85,6 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_decode_gateup(const __nv_bfl
                                                                 __nv_bfloat16* xbuf, long long rs, int B, int d,
                                                                 int F) {
   extern __shared__ uint4 hs[];  // [B][d / 8]
-  __shared__ float part[kWarps][2][kDecodeMaxRows];
   const int dv = d / 8;
   for (int i = threadIdx.x; i < B * dv; i += blockDim.x) {
     const uint4 v = reinterpret_cast<const uint4*>(h)[i];
@@ -87,31 +97,30 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_decode_gateup(const __nv_bfl
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int f = blockIdx.x * (kWarps / 2) + (warp >> 1);
-  const int half = warp & 1;
-  const int lo = half ? dv / 2 : 0, hi = half ? dv : dv / 2;
-  float g[kDecodeMaxRows], u[kDecodeMaxRows];
-#pragma unroll
-  for (int b = 0; b < kDecodeMaxRows; ++b) g[b] = u[b] = 0.0f;
-  if (f < F) {
+  const int nw = gridDim.x * kWarps;
+  for (int f = blockIdx.x * kWarps + warp; f < F; f += nw) {
     const uint4* wg = reinterpret_cast<const uint4*>(Wg + (size_t)f * d);
     const uint4* wu = reinterpret_cast<const uint4*>(Wu + (size_t)f * d);
-    for (int k0 = lo + lane; k0 < hi; k0 += 32 * kApplyBatch) {
-      uint4 a[kApplyBatch], c[kApplyBatch];
+    float g[NR], u[NR];
 #pragma unroll
-      for (int q = 0; q < kApplyBatch; ++q) {
+    for (int b = 0; b < NR; ++b) g[b] = u[b] = 0.0f;
+    for (int k0 = lane; k0 < dv; k0 += 32 * row_words<NR>()) {
+      constexpr int RW = row_words<NR>();
+      uint4 a[RW], c[RW];
+#pragma unroll
+      for (int q = 0; q < row_words<NR>(); ++q) {
         const int k = k0 + 32 * q;
-        if (k < hi) {
+        if (k < dv) {
           a[q] = wg[k];
           c[q] = wu[k];
         }
       }
 #pragma unroll
-      for (int q = 0; q < kApplyBatch; ++q) {
+      for (int q = 0; q < row_words<NR>(); ++q) {
         const int k = k0 + 32 * q;
-        if (k >= hi) break;
+        if (k >= dv) break;
 #pragma unroll
-        for (int b = 0; b < kDecodeMaxRows; ++b) {
+        for (int b = 0; b < NR; ++b) {
           if (b >= B) break;
           const uint4 x = hs[b * dv + k];
           g[b] += dot8(a[q], x);
@@ -119,46 +128,38 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_decode_gateup(const __nv_bfl
         }
       }
     }
-  }
 #pragma unroll
-  for (int b = 0; b < kDecodeMaxRows; ++b)
-    if (b < B) {
-      const float gs = warp_sum(g[b]), us = warp_sum(u[b]);
-      if (lane == 0) {
-        part[warp][0][b] = gs;
-        part[warp][1][b] = us;
+    for (int b = 0; b < NR; ++b)
+      if (b < B) {
+        const float gs = warp_sum(g[b]), us = warp_sum(u[b]);
+        if (lane == 0) z[(size_t)b * F + f] = __float2bfloat16_rn(silu_fast(gs) * us);
       }
-    }
-  __syncthreads();
-  if (half == 0 && lane < B && f < F) {
-    const float gs = part[warp][0][lane] + part[warp + 1][0][lane];
-    const float us = part[warp][1][lane] + part[warp + 1][1][lane];
-    z[(size_t)lane * F + f] = __float2bfloat16_rn(silu_fast(gs) * us);
   }
 }
 
-// o[b][j] = bf16(W0[j] . z_b + (m_b ? snap_b[j] . z_b : 0)).  A block holds two
-// rows j, four warps per row, each warp a quarter of F; the quarters are added in
-// a fixed order.  Per batch of kApplyBatch 16-byte words a lane requests the W0
-// words first, then per row b the z_b words (small, L1/L2-resident) and the
-// snapshot words, so it keeps up to 3 kApplyBatch loads in flight without
-// block barriers in the loop.
+// o[b][j] = bf16(W0[j] . z_b + (m_b ? snap_b[j] . z_b : 0)) for B <= NR rows.
+// A block holds two groups of four warps; a group takes one row j at a time, each
+// warp a quarter of F, and the quarters are added in a fixed order after a barrier
+// of the group's four warps alone.  Per batch of kApplyBatch 16-byte words a lane
+// requests the W0 words, then per row b the z_b words (small, L1/L2-resident) and
+// the snapshot words before it uses them.
+template <int NR>
 __global__ void __launch_bounds__(kWarps * 32, 2) k_decode_apply(const __nv_bfloat16* __restrict__ z,
                                                                const __nv_bfloat16* __restrict__ W0,
                                                                const __nv_bfloat16* __restrict__ snap,
-                                                               uint32_t mask, const float* __restrict__ add,
-                                                               __nv_bfloat16* __restrict__ o, int B, int d,
-                                                               int F) {
-  __shared__ float part[kWarps][kDecodeMaxRows];
+                                                               uint32_t mask, __nv_bfloat16* __restrict__ o, int B,
+                                                               int d, int F) {
+  __shared__ float part[2][kWarps][NR];  // by row parity: a group's next row never overwrites
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * (kWarps / 4) + (warp >> 2);
-  const int quarter = warp & 3;
+  const int grp = warp >> 2, quarter = warp & 3;
   const int fv = F / 8;
   const int lo = fv * quarter / 4, hi = fv * (quarter + 1) / 4;
-  float a0[kDecodeMaxRows], a1[kDecodeMaxRows];
+  const int ngrp = gridDim.x * 2;
+  int it = 0;
+  for (int j = blockIdx.x * 2 + grp; j < d; j += ngrp, ++it) {
+    float a0[NR], a1[NR];
 #pragma unroll
-  for (int b = 0; b < kDecodeMaxRows; ++b) a0[b] = a1[b] = 0.0f;
-  if (j < d) {
+    for (int b = 0; b < NR; ++b) a0[b] = a1[b] = 0.0f;
     const uint4* w = reinterpret_cast<const uint4*>(W0 + (size_t)j * F);
     for (int k0 = lo + lane; k0 < hi; k0 += 32 * kApplyBatch) {
       uint4 wv[kApplyBatch];
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_decode_apply(const __nv_bflo
       for (int q = 0; q < kApplyBatch; ++q)
         if (k0 + 32 * q < hi) wv[q] = w[k0 + 32 * q];
 #pragma unroll
-      for (int b = 0; b < kDecodeMaxRows; ++b) {
+      for (int b = 0; b < NR; ++b) {
         if (b >= B) break;
         const uint4* zb = reinterpret_cast<const uint4*>(z + (size_t)b * F);
         const uint4* sb = reinterpret_cast<const uint4*>(snap + ((size_t)b * d + j) * F);
@@ -189,18 +190,20 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_decode_apply(const __nv_bflo
         }
       }
     }
-  }
 #pragma unroll
-  for (int b = 0; b < kDecodeMaxRows; ++b)
-    if (b < B) {
-      const float s = warp_sum(a0[b]) + warp_sum(a1[b]);
-      if (lane == 0) part[warp][b] = s;
+    for (int b = 0; b < NR; ++b)
+      if (b < B) {
+        const float s = warp_sum(a0[b]) + warp_sum(a1[b]);
+        if (lane == 0) part[it & 1][warp][b] = s;
+      }
+    // the group's four warps only (barriers 1 and 2; 0 is the block's)
+    if (grp == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
+    else asm volatile("bar.sync 2, 128;" ::: "memory");
+    if (quarter == 0 && lane < B) {
+      const float* pp = &part[it & 1][warp][0];
+      const float sum = ((pp[lane] + pp[NR + lane]) + pp[2 * NR + lane]) + pp[3 * NR + lane];
+      o[(size_t)lane * d + j] = __float2bfloat16_rn(sum);
     }
-  __syncthreads();
-  if (quarter == 0 && lane < B && j < d) {
-    const int w0 = warp;  // the row's first warp; its quarters follow
-    const float sum = ((part[w0][lane] + part[w0 + 1][lane]) + part[w0 + 2][lane]) + part[w0 + 3][lane];
-    o[(size_t)lane * d + j] = __float2bfloat16_rn(add ? sum + add[(size_t)lane * d + j] : sum);
   }
 }
 
@@ -273,16 +276,36 @@ __global__ void k_decode_gate_combine(const float* __restrict__ g, const float* 
 }
 
 // Shared memory above the default 48 KB for the gate/up kernel's h rows (B d bf16),
-// raised once per device to the largest size asked for so far.
+// raised once per device and kernel build to the largest size asked for so far.
+template <int NR>
 bool decode_smem_ready(int smem) {
   static int granted[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (smem <= granted[dev]) return true;
-  if (cudaFuncSetAttribute(k_decode_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(k_decode_gateup<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return false;
   granted[dev] = smem;
   return true;
+}
+
+// The two per-token kernels on the CUDA cores, built for at most NR rows.
+template <int NR>
+bool decode_small(const void* h, const void* x0, const void* Wgate, const void* Wup, const void* Wdown0,
+                  __nv_bfloat16* z, __nv_bfloat16* hrow, __nv_bfloat16* xrow, const void* snap, uint32_t mask,
+                  void* o, long long rs, int B, int d, int F, cudaStream_t st) {
+  // the gate/up kernel also files this token's h and x0 rows for the chunk's update
+  const int smem = B * d * 2;
+  if (smem > 48 * 1024 && !decode_smem_ready<NR>(smem)) return false;
+  const int gblocks = std::max(1, std::min(2 * device_sms(), (F + kWarps - 1) / kWarps));
+  k_decode_gateup<NR><<<gblocks, kWarps * 32, smem, st>>>(
+      static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(x0),
+      static_cast<const __nv_bfloat16*>(Wgate), static_cast<const __nv_bfloat16*>(Wup), z, hrow, xrow, rs, B, d, F);
+  const int ablocks = std::max(1, std::min(2 * device_sms(), (d + 1) / 2));
+  k_decode_apply<NR><<<ablocks, kWarps * 32, 0, st>>>(z, static_cast<const __nv_bfloat16*>(Wdown0),
+                                                      static_cast<const __nv_bfloat16*>(snap), mask,
+                                                      static_cast<__nv_bfloat16*>(o), B, d, F);
+  return cudaGetLastError() == cudaSuccess;
 }
 
 // Host bookkeeping of a decode state (lives in the caller's host buffer).
@@ -410,7 +433,12 @@ ipttt_status ipttt_decode_step(const ipttt_params* p, void* state, void* host_st
   __nv_bfloat16* z = reinterpret_cast<__nv_bfloat16*>(base + L.z);
   __nv_bfloat16* hrow = reinterpret_cast<__nv_bfloat16*>(base + L.H + hs->n * row);
   __nv_bfloat16* xrow = reinterpret_cast<__nv_bfloat16*>(base + L.X0 + hs->n * row);
-  if (B >= kTensorRows && d % 128 == 0 && F % 128 == 0) {
+  // (the layout admits only the shapes the forward takes: d and F multiples of 128)
+  if (B < kTensorRows) {
+    if (!decode_small<kTensorRows - 1>(h, x0, Wgate, Wup, Wdown0, z, hrow, xrow, base + L.snap, hs->cont_mask, o,
+                                       (long long)C * d, B, d, F, st))
+      return IPTTT_ERR_CUDA;
+  } else {
     // g = Wgate h^T and u = Wup h^T as tcgen05 GEMMs (h rows past B read as zeros)
     k_decode_file<<<(B * d / 8 + 255) / 256, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h),
                                                             static_cast<const __nv_bfloat16*>(x0), hrow, xrow,
@@ -434,42 +462,29 @@ ipttt_status ipttt_decode_step(const ipttt_params* p, void* state, void* host_st
     k_decode_gate_combine<<<(B * F + 255) / 256, 256, 0, st>>>(reinterpret_cast<const float*>(base + L.gacc),
                                                                reinterpret_cast<const float*>(base + L.uacc), z, B,
                                                                F);
-  } else {
-    // the gate/up kernel also files this token's h and x0 rows for the chunk's update
-    const int smem = B * d * 2;
-    if (smem > 48 * 1024 && !decode_smem_ready(smem)) return IPTTT_ERR_CUDA;
-    k_decode_gateup<<<(F + kWarps / 2 - 1) / (kWarps / 2), kWarps * 32, smem, st>>>(
-        static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(x0),
-        static_cast<const __nv_bfloat16*>(Wgate), static_cast<const __nv_bfloat16*>(Wup), z, hrow, xrow,
-        (long long)C * d, B, d, F);
-  }
-  if (B >= kTensorRows) {
     // the state copies row by row on their own, then W0 with their products added
     float* tsnap = reinterpret_cast<float*>(base + L.tsnap);
     k_decode_snap<<<(unsigned)(((long long)B * d + kWarps / 4 - 1) / (kWarps / 4)), kWarps * 32, 0, st>>>(
         z, reinterpret_cast<const __nv_bfloat16*>(base + L.snap), hs->cont_mask, tsnap, B, d, F);
     // W0 z_b for all rows as a tcgen05 GEMM (M = d, N = rows padded to 32), K split
     // in kW0Split slices so that the tiles fill the SMs; the slices are added in order
-    gemm::Args g{};
-    g.mode = gemm::GM_PLAIN;
-    g.M = d;
-    g.N = kGemmCols;
-    g.K = F;
-    g.ksplit = F / 128 >= kW0Split ? kW0Split : 1;
-    g.A = {Wdown0, (uint64_t)F, (uint64_t)d, 1};
-    g.Bop = {z, (uint64_t)F, (uint64_t)B, 1};
-    g.out_kind = gemm::GO_F32;
-    g.out = base + L.w0acc;
-    g.ldo = kGemmCols;
-    g.osz = (long long)d * kGemmCols;
-    g.status = device_status();
-    if (gemm::run(g, device_sms(), st) != cudaSuccess) return IPTTT_ERR_CUDA;
+    gemm::Args w0{};
+    w0.mode = gemm::GM_PLAIN;
+    w0.M = d;
+    w0.N = kGemmCols;
+    w0.K = F;
+    w0.ksplit = F / 128 >= kW0Split ? kW0Split : 1;
+    w0.A = {Wdown0, (uint64_t)F, (uint64_t)d, 1};
+    w0.Bop = {z, (uint64_t)F, (uint64_t)B, 1};
+    w0.out_kind = gemm::GO_F32;
+    w0.out = base + L.w0acc;
+    w0.ldo = kGemmCols;
+    w0.osz = (long long)d * kGemmCols;
+    w0.status = device_status();
+    if (gemm::run(w0, sms, st) != cudaSuccess) return IPTTT_ERR_CUDA;
     k_decode_out<<<(B * d + 255) / 256, 256, 0, st>>>(reinterpret_cast<const float*>(base + L.w0acc), tsnap,
-                                                      static_cast<__nv_bfloat16*>(o), B, d, g.ksplit > 1 ? g.ksplit : 1);
-  } else {
-    k_decode_apply<<<(d + kWarps / 4 - 1) / (kWarps / 4), kWarps * 32, 0, st>>>(
-        z, static_cast<const __nv_bfloat16*>(Wdown0), reinterpret_cast<const __nv_bfloat16*>(base + L.snap),
-        hs->cont_mask, nullptr, static_cast<__nv_bfloat16*>(o), B, d, F);
+                                                      static_cast<__nv_bfloat16*>(o), B, d,
+                                                      w0.ksplit > 1 ? w0.ksplit : 1);
   }
   if (cudaGetLastError() != cudaSuccess) return IPTTT_ERR_CUDA;
 

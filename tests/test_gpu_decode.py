@@ -51,6 +51,23 @@ def test_decode_equals_forward_and_oracle():
     assert maxrel(orc["O"] - orc["D"], orc["O"]) > 5 * 2e-2
 
 
+@pytest.mark.parametrize("B", [1, 3])
+def test_decode_one_and_three_rows(B):
+    # the CUDA-core kernels below four rows, at their smallest and largest batch;
+    # a document starts inside the first chunk of the last row
+    T, C = 300, 128
+    cfg, inp = case(B, T, C, 256, 512, eta=2e-2, clip=0.0, docs=[(B - 1) * T + 90])
+    dev = torch.device("cuda")
+    w = {k: inp[k].to(dev) for k in WEIGHTS}
+    _, out = decode_all(cfg, inp, T, w)
+    ref = ip.forward(cfg, inp["H"].to(dev), inp["X0"].to(dev), *(w[k] for k in WEIGHTS), inp["doc_starts"])
+    torch.cuda.synchronize()
+    assert maxrel(to_np(out), to_np(ref)) <= 1e-2
+    orc = oracle(cfg, inp)
+    assert maxrel(to_np(out), orc["O"]) <= 2e-2
+    assert maxrel(orc["O"] - orc["D"], orc["O"]) > 5 * 2e-2
+
+
 def test_decode_batched_rows_on_the_tensor_cores():
     # 8 rows: the gate/up products run as tcgen05 GEMMs (rows padded to 32); the
     # outputs match the forward and the oracle as for 2 rows
