@@ -950,15 +950,15 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
       const int base = m.has_start ? 0 : (jb.c == 0 ? 2 : 1);
       const bool snap = jb.chunk + 1 < p.k;
       const float* sf = reinterpret_cast<const float*>(upd_state_block(p, jb.b, m0c, jb.n0, half));
-      // Folds 64 columns of the delta (two 32-column TMEM loads) into st[64 hb ..].
+      // Folds 64 columns of the delta (one 64-column TMEM load) into st[64 hb ..].
       // the chunk's clip factor times eta, when V was not pre-scaled by it
       const float sc = p.upd_scale ? p.alpha[(size_t)jb.b * p.k + jb.chunk] * p.eta : 1.0f;
-      auto fold = [&](const int hb, const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
+      auto fold = [&](const int hb, const uint32_t (&ra)[64]) {
 #pragma unroll
         for (int q = 0; q < 64; ++q) {
           const int c = 64 * hb + q;
           const float old = base == 2 ? sf[((c / 4) * 128 + row) * 4 + (c & 3)] : base == 1 ? st[c] : 0.0f;
-          st[c] = fmaf(sc, __uint_as_float(q < 32 ? ra[q & 31] : rb[q & 31]), old);
+          st[c] = fmaf(sc, __uint_as_float(ra[q]), old);
         }
       };
       // Snapshot box hb: 32 rows x 64 columns of bf16(S_{chunk+1}) (what the apply of
@@ -990,17 +990,15 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
       };
       if (!mbar_wait(&slot_full[sl], (i >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      // Two halves of the warp's 128 columns, one TMEM round trip each: the second
-      // half's loads are in flight while the first is folded and stored.
-      uint32_t x0[32], x1[32], y0[32], y1[32];
+      // Two halves of the warp's 128 columns, one 64-column TMEM load each: the
+      // second half's load is in flight while the first is folded and stored.
+      uint32_t x0[64], y0[64];
       const uint32_t tcol = tmem_base + sl * ACC_COLS + ((uint32_t)(quarter * 32) << 16) + 128 * half;
       if (cols) {
-        tmem_ld32(tcol, x0);
-        tmem_ld32(tcol + 32, x1);
+        tmem_ld64(tcol, x0);
         tmem_ld_wait();
-        fold(0, x0, x1);
-        tmem_ld32(tcol + 64, y0);
-        tmem_ld32(tcol + 96, y1);
+        fold(0, x0);
+        tmem_ld64(tcol + 64, y0);
         if (snap) store_box(0);
         tmem_ld_wait();
       }
@@ -1012,7 +1010,7 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
         else mbar_arrive(&slot_free[sl]);
       }
       if (!cols) continue;
-      fold(1, y0, y1);
+      fold(1, y0);
       if (snap) store_box(1);
       if (jb.c == p.dchunks - 1) {
         // the tile's last chunk of the launch: the fp32 state goes back to HBM
