@@ -580,6 +580,12 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
       !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, update_tokens_per_stage(s.C)) ||
       !make_map_bf16(&sc.map[5], snap, s.F, s.d, (uint64_t)G * s.B, 64, 32))
     return cuda_fail("tensor maps of the chunk scan", cudaErrorInvalidValue);
+  // the 256-row apply writes O through shared memory and TMA stores
+  if (apply_fam == FAM_APPLY256 && t.O) {
+    if (!make_map_bf16(&sc.map[6], t.O, s.d, s.T, s.B, 64, 32))
+      return cuda_fail("tensor map of O", cudaErrorInvalidValue);
+    sc.o_tma = 1;
+  }
   sc.out0 = t.O;
   sc.out1 = t.D;
   sc.resid = (p.flags & IPTTT_FLAG_RESIDUAL) ? t.H : nullptr;

@@ -70,9 +70,11 @@ template <> struct Cfg<FAM_APPLY> {
 // 256 token rows per apply tile: two M=128 MMAs share every B stage, so a byte
 // fetched from L2 feeds twice the flops; the two accumulators fill all of TMEM
 // (no double buffering; the epilogue is short next to the K = d_ff mainloop).
+// The epilogue stages O in one 32-row x 64-column box per warp and writes it with
+// TMA stores (the stores leave while the next tile's MMAs run).
 template <> struct Cfg<FAM_APPLY256> {
-  static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 64, B_OFF = 2 * A_BYTES, EPI_BYTES = 0,
-                       NBUF = 1;
+  static constexpr int STAGES = 3, STAGE_BYTES = 64 * 1024, KB = 64, B_OFF = 2 * A_BYTES,
+                       EPI_BYTES = NUM_EPI_WARPS * 4096, NBUF = 1;
 };
 // Pair gate/up and target: CTA r of the cluster holds A rows m0 + 128 r .. of the
 // 256-row tile and half of the N operand; 128 K per stage (two 64-wide boxes),
@@ -105,7 +107,7 @@ constexpr int smem_bytes() {
   return 1024 /*alignment slack*/ + Cfg<FAM>::STAGES * Cfg<FAM>::STAGE_BYTES + Cfg<FAM>::EPI_BYTES +
          256 /*barriers*/;
 }
-static_assert(smem_bytes<FAM_ZV>() <= 232448, "kernel exceeds shared memory");
+static_assert(smem_bytes<FAM_ZV>() <= 232448 && smem_bytes<FAM_APPLY256>() <= 232448, "kernel exceeds shared memory");
 
 struct Job {
   int kind;
@@ -366,7 +368,7 @@ __device__ __forceinline__ void epi_sync() {
 
 template <int FAM>
 __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, uint32_t tacc, int half, int row,
-                                              int lane, int ew, float* red) {
+                                              int lane, int ew, float* red, uint8_t* ebox, int& nst) {
   uint32_t r0[32], r1[32];
   float v[32];
   if constexpr (is_zv<FAM>()) {
@@ -486,6 +488,7 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
     const int t = j.t0 + j.m0 + row_in_tile;
     const bool valid = (two || row < p.tr) && t < p.T;
     const bool carry = j.nsrc == 2 && m.cont && t < m.first_end;
+    const bool tma_o = two && p.o_tma;
     __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out0) + ((size_t)j.b * p.T + t) * p.d + j.n0;
     const __nv_bfloat16* hrow =
         p.resid ? reinterpret_cast<const __nv_bfloat16*>(p.resid) + ((size_t)j.b * p.T + t) * p.d + j.n0 : nullptr;
@@ -546,13 +549,37 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const Job& j, u
             }
           }
         }
-        st_bf16x32(orow + c, v);
+        if (!tma_o) st_bf16x32(orow + c, v);
         if (drow) {
           float4* d4 = reinterpret_cast<float4*>(drow + c);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             d4[q] = make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
                                 __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3]));
+        }
+      }
+      if (tma_o) {
+        // 32 columns into the warp's box (128-byte swizzled rows); once the box holds
+        // 64 columns it goes out by TMA (rows past T are clipped by the tensor map)
+        if ((c & 63) == 0 && nst > 0) {
+          if (lane == 0) bulk_wait_read<0>();  // the box's previous store has read it
+          __syncwarp();
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int e = ((c & 63) >> 3) + q;
+          *reinterpret_cast<uint4*>(ebox + lane * 128 + ((e ^ (lane & 7)) << 4)) =
+              make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                         pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+        }
+        if ((c & 63) == 32) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&p.map[6], ebox, j.n0 + (c & ~63), j.t0 + j.m0 + half * 128 + (row - lane), j.b);
+            bulk_commit();
+          }
+          ++nst;
         }
       }
     }
@@ -601,6 +628,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
   if (warp == 0 && lane == 0) {
     const int nmaps = is_apply<FAM>() ? 3 : FAM == FAM_PZ ? 1 : (is_gram<FAM>() ? 2 : (p.kind == K_GATEUP ? 3 : 2));
     for (int i = 0; i < nmaps; ++i) prefetch_tmap(&p.map[i]);
+    if (FAM == FAM_APPLY256 && p.o_tma) prefetch_tmap(&p.map[6]);
   }
   if (warp == 1) {
     if constexpr (PAIR) {
@@ -707,6 +735,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
     const int row = quarter * 32 + lane;
     uint32_t tcount = 0;
     bool ok = true;
+    int nst = 0;  // O boxes this warp has stored (256-row apply)
     const uint32_t empty0 = PAIR ? map_to_rank(smem_u32(acc_empty), 0) : 0u;  // the leader's acc_empty[0]
     for (uint32_t i = 0;; ++i, ++tcount) {
       const int tile = seq_tile<FAM>(p, i);
@@ -721,7 +750,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_kernel(const __grid_constant__
       tc_fence_after();
       const uint32_t tacc = tmem_base + buf * ACC_COLS + ((uint32_t)(quarter * 32) << 16);
       if constexpr (PAIR) j.m0 += 128 * (int)rank;  // this CTA's rows of the pair tile
-      epilogue_tile<FAM>(p, j, tacc, half, row, lane, ew, red);
+      epilogue_tile<FAM>(p, j, tacc, half, row, lane, ew, red, epi + ew * 4096, nst);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
