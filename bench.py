@@ -231,7 +231,7 @@ def config_dict(w: synth.Workload, n: int) -> dict:
 # one step captured by ncu, keyed by (workload, chunk size, phase); the summaries in
 # profiles/ give the commands.  The roofline object carries a figure only for the
 # kernel and workload it was taken on.
-MEASURED_TRAFFIC = {("qwen3_4b_128k", 1024, "apply"): 2491883520.0}
+MEASURED_TRAFFIC = {("qwen3_4b_128k", 1024, "apply"): 2514658005.3}
 
 
 def sample_chunks(w: synth.Workload, tokens: int) -> int:
