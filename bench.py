@@ -287,7 +287,7 @@ def run_ours(args, w: synth.Workload):
     dev_w = [{k: l[k].to(dev) for k in WEIGHTS} for l in layers]
     docs = layers[0]["doc_starts"]
     cfg = ip.LayerConfig(B=w.B, T=w.T, d=w.d, F=w.F, C=w.C, eta=w.eta, clip=w.clip, dtype=w.dtype)
-    ws = ip.alloc_workspace(cfg, dev)
+    ws = ip.alloc_workspace(cfg, dev, state_clip=args.state_clip)
     O = torch.empty(w.B, w.T, w.d, dtype=cfg.torch_dtype, device=dev)
     Hbuf = [torch.empty_like(dev_in["H"]) for _ in range(2)] if w.layers > 1 else None
     docs_dev = docs.to(dev)

@@ -23,6 +23,7 @@
 #include "aux_kernels.h"
 #include "common.cuh"
 #include "tc_kernels.h"
+#include "gemm.h"
 
 namespace ipttt {
 
@@ -248,11 +249,17 @@ Layout layout_of(const ipttt_params& p, bool cp = false, bool keep_all = false) 
     L.V = take(B * T * d * 2);
     L.S = take(B * d * F * 4);
     L.keep_all = keep_all;
-    L.grouped = !keep_all && grouped_scan(p);
+    // the clip on the accumulated state scales the state chunk by chunk: no grouping
+    const bool state_clip = (p.flags & IPTTT_FLAG_STATE_CLIP) != 0;
+    L.grouped = !keep_all && !state_clip && grouped_scan(p);
     const size_t kg = (T + kGroupTokens - 1) / kGroupTokens;
     L.group = (cp || keep_all) ? (int)(L.grouped ? kg : s.k) + 1 : apply_group(L.grouped ? group_params(p) : p);
     L.snap = take((size_t)L.group * B * d * F * 2);
     L.raw = L.dpart = 0;
+    if (state_clip) {  // each chunk's raw delta in fp32, and the norm's partial sums
+      L.raw = take(B * d * F * 4);
+      L.dpart = take(B * 148 * 4 * sizeof(double));
+    }
     L.gmeta = L.glo = L.P = L.E = 0;
     if (L.grouped) {
       L.gmeta = take(B * kg * sizeof(ChunkMeta));
@@ -287,8 +294,6 @@ ipttt_status check_params(const ipttt_params* p) {
   if (p->B <= 0 || p->T <= 0 || p->d <= 0 || p->F <= 0 || p->C <= 0) return IPTTT_ERR_ARG;
   if (!isfinite(p->eta) || isnan(p->clip_thresh)) return IPTTT_ERR_ARG;
   if ((p->flags & ~(IPTTT_FLAG_RESIDUAL | IPTTT_FLAG_STATE_CLIP)) != 0) return IPTTT_ERR_ARG;
-  // the clip on the accumulated state runs on the fp32 path only
-  if ((p->flags & IPTTT_FLAG_STATE_CLIP) && p->dtype != IPTTT_F32) return IPTTT_ERR_UNSUPPORTED;
   const long long BT = (long long)p->B * p->T;
   if (BT > (1ll << 30) || (long long)p->d * p->F > (1ll << 31) || (long long)p->d * p->d > (1ll << 31) ||
       BT * (long long)p->F > (1ll << 40))
@@ -488,7 +493,10 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   if (t.Zout) IP_CHECK(cudaMemcpyAsync(t.Zout, Z, (size_t)s.B * s.T * s.F * 2, cudaMemcpyDeviceToDevice, st));
   if (t.Vout) IP_CHECK(cudaMemcpyAsync(t.Vout, V, (size_t)s.B * s.T * s.d * 2, cudaMemcpyDeviceToDevice, st));
 
-  if (!cp_finish) {
+  // The clip on the accumulated state takes its factors from the state itself, chunk
+  // by chunk in the scan, so it needs no Gram pass.
+  const bool state_clip = (p.flags & IPTTT_FLAG_STATE_CLIP) != 0;
+  if (!cp_finish && !state_clip) {
     PhaseScope ph(st, PH_GRAM);
     TcParams g = tp;
     // On CTA pairs: 256 x 256 token-block pairs, two partials (one per CTA) each.
@@ -540,7 +548,8 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
     IP_CHECK(launch_tc(FAM_ZV2, e, di->num_sms, st));
     counted(2);
   }
-  if (t.alpha) IP_CHECK(cudaMemcpyAsync(t.alpha, alpha, (size_t)s.B * s.k * 4, cudaMemcpyDeviceToDevice, st));
+  if (t.alpha && !state_clip)
+    IP_CHECK(cudaMemcpyAsync(t.alpha, alpha, (size_t)s.B * s.k * 4, cudaMemcpyDeviceToDevice, st));
 
   // A context-parallel shard starts from a zero state: S_0 (snapshot slot 0) and
   // the fp32 state are cleared; the incoming state is added in the finish.
@@ -601,6 +610,39 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   auto update = [&](int c0, int c1) -> ipttt_status {
     if (c1 <= c0) return IPTTT_OK;
     PhaseScope ph(st, PH_UPDATE);
+    if (state_clip) {
+      // Chunk by chunk: the raw delta V_L^T Z_L as a tcgen05 GEMM (fp32 out, V zero
+      // outside the last segment), then on the CUDA cores S = c (keep S + eta delta)
+      // with c = tau / ||keep S + eta delta||_F when that exceeds tau (fp32 state,
+      // row-major), and the bf16 copy of the new state for the apply.
+      float* raw = reinterpret_cast<float*>(ws + L.raw);
+      double* dpart = reinterpret_cast<double*>(ws + L.dpart);
+      for (int c = c0; c < c1; ++c) {
+        gemm::Args r{};
+        r.mode = gemm::GM_CHUNK_K;
+        r.A = {V, (uint64_t)s.d, (uint64_t)s.T, (uint64_t)s.B};
+        r.Bop = {Z, (uint64_t)s.F, (uint64_t)s.T, (uint64_t)s.B};
+        r.M = s.d;
+        r.N = s.F;
+        r.B = s.B;
+        r.T = s.T;
+        r.C = s.C;
+        r.k = s.k;
+        r.chunk0 = c;
+        r.nchunks = 1;
+        r.chunk_base = c;
+        r.out_kind = gemm::GO_F32;
+        r.out = raw;
+        r.ldo = s.F;
+        r.osz = (long long)s.d * s.F;
+        r.status = tp.status;
+        IP_CHECK(gemm::run(r, di->num_sms, st));
+        void* copy = c + 1 < s.k ? static_cast<uint8_t*>(snap) + (size_t)((c + 1) % G) * s.B * s.d * s.F * 2 : nullptr;
+        IP_CHECK(aux::state_clip_step(S, raw, dpart, alpha, meta, s, c, p.eta, tau, copy, st));
+        counted(4);
+      }
+      return IPTTT_OK;
+    }
     TcParams q = sc;
     q.chunk = c0;
     q.dchunks = c1 - c0;
@@ -647,9 +689,11 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   }
   if (need_final && (rc_ = update(sq.k - 1, sq.k)) != IPTTT_OK) return rc_;
   if (t.Sfinal) {
-    IP_CHECK(aux::state_export(true, S, t.Sfinal, s, st));
+    IP_CHECK(aux::state_export(!state_clip, S, t.Sfinal, s, st));
     counted(1);
   }
+  if (t.alpha && state_clip)
+    IP_CHECK(cudaMemcpyAsync(t.alpha, alpha, (size_t)s.B * s.k * 4, cudaMemcpyDeviceToDevice, st));
   if (ss) {
     IP_CHECK(aux::stream_advance(ss->pos, ss->cont, s.B, s.T, st));
     counted(1);
@@ -766,6 +810,8 @@ ipttt_status run(const ipttt_params* pp, const Tensors& t, void* workspace, size
   StreamState ss;
   StreamState* ssp = nullptr;
   if (state) {
+    // the bf16 state-clip reading keeps its state row-major, the stream state is blocked
+    if (is_bf16(p) && (p.flags & IPTTT_FLAG_STATE_CLIP)) return IPTTT_ERR_UNSUPPORTED;
     ss = state_of(p, state);
     ssp = &ss;
   }
@@ -910,6 +956,8 @@ ipttt_status cp_run(const ipttt_params* p, int32_t world, int32_t rank, const in
   ipttt_status rc = check_params(p);
   if (rc != IPTTT_OK) return rc;
   if (p->dtype != IPTTT_BF16) return IPTTT_ERR_UNSUPPORTED;
+  // the shards' aggregates add up only while the update is linear in the state
+  if (p->flags & IPTTT_FLAG_STATE_CLIP) return IPTTT_ERR_UNSUPPORTED;
   const Layout L = layout_of(*p, true);
   if (!workspace || workspace_bytes < L.total) return IPTTT_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return IPTTT_ERR_ALIGN;
@@ -1024,7 +1072,13 @@ const char* ipttt_version(void) { return "0.2.0"; }
 
 // The backward takes the forward's shape rules: any shape in fp32 (CUDA cores),
 // the tensor-core shapes in bf16.
-static ipttt_status backward_params(const ipttt_params* p) { return check_params(p); }
+// The gradients are those of the per-delta clip; the accumulated-state reading has
+// none here.
+static ipttt_status backward_params(const ipttt_params* p) {
+  const ipttt_status rc = check_params(p);
+  if (rc != IPTTT_OK) return rc;
+  return (p->flags & IPTTT_FLAG_STATE_CLIP) ? IPTTT_ERR_UNSUPPORTED : IPTTT_OK;
+}
 
 // bf16 workspace: the forward's layout with every state copy kept, O of that
 // forward, then the backward's own buffers.

@@ -529,6 +529,73 @@ cudaError_t simt_update_state_clipped(float* S, const float* raw, double* part, 
   return cudaGetLastError();
 }
 
+// The accumulated-state clip on the bf16 path, for states of d F = tens of millions
+// of values: one pass forms keep S + eta raw and its partial sums of squares (four
+// values per thread and step, fixed-order block sums), a second scales the state
+// by c and writes its bf16 copy for the apply.
+constexpr int kClipBlocks = 148 * 4;
+
+__global__ void __launch_bounds__(256) k_state_accum_sumsq(float* S, const float* raw, size_t n4,
+                                                           const ChunkMeta* meta, int k, int chunk, float eta,
+                                                           double* part) {
+  __shared__ double sh[256];
+  const int b = blockIdx.y;
+  const bool keep = !meta[(size_t)b * k + chunk].has_start;
+  float4* Sb = reinterpret_cast<float4*>(S) + b * n4;
+  const float4* rb = reinterpret_cast<const float4*>(raw) + b * n4;
+  double acc = 0.0;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+    const float4 r = rb[i];
+    float4 v = keep ? Sb[i] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    v.x = fmaf(eta, r.x, v.x);
+    v.y = fmaf(eta, r.y, v.y);
+    v.z = fmaf(eta, r.z, v.z);
+    v.w = fmaf(eta, r.w, v.w);
+    Sb[i] = v;
+    acc += ((double)v.x * v.x + (double)v.y * v.y) + ((double)v.z * v.z + (double)v.w * v.w);
+  }
+  sh[threadIdx.x] = acc;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) sh[threadIdx.x] += sh[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) part[(size_t)b * gridDim.x + blockIdx.x] = sh[0];
+}
+
+__global__ void __launch_bounds__(256) k_state_scale_copy(float* S, __nv_bfloat16* snap, size_t n4,
+                                                          const float* alpha, int k, int chunk) {
+  const int b = blockIdx.y;
+  const float c = alpha[(size_t)b * k + chunk];
+  float4* Sb = reinterpret_cast<float4*>(S) + b * n4;
+  uint2* out = snap ? reinterpret_cast<uint2*>(snap) + b * n4 : nullptr;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+    float4 v = Sb[i];
+    if (c != 1.0f) {
+      v.x *= c;
+      v.y *= c;
+      v.z *= c;
+      v.w *= c;
+      Sb[i] = v;
+    }
+    if (out) {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+      out[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+    }
+  }
+}
+
+cudaError_t state_clip_step(float* S, const float* raw, double* part, float* alpha, const ChunkMeta* meta,
+                            const Shape& s, int chunk, float eta, float tau, void* snap_bf16, cudaStream_t st) {
+  const size_t n = (size_t)s.d * s.F;
+  if (n % 4 != 0) return cudaErrorInvalidValue;
+  k_state_accum_sumsq<<<dim3(kClipBlocks, s.B), 256, 0, st>>>(S, raw, n / 4, meta, s.k, chunk, eta, part);
+  k_alpha_direct<<<(s.B + 63) / 64, 64, 0, st>>>(part, kClipBlocks, alpha, s.B, s.k, chunk, 1.0f, tau);
+  k_state_scale_copy<<<dim3(kClipBlocks, s.B), 256, 0, st>>>(S, static_cast<__nv_bfloat16*>(snap_bf16), n / 4,
+                                                               alpha, s.k, chunk);
+  return cudaGetLastError();
+}
+
 cudaError_t simt_update_state(float* S, const float* raw, double* part, float* alpha, const ChunkMeta* meta,
                               const Shape& s, int chunk, float eta, float tau, cudaStream_t st) {
   const size_t n = (size_t)s.d * s.F;

@@ -18,6 +18,12 @@ cudaError_t alpha_from_partials(const float* partials, float* alpha, int n, int 
                                 cudaStream_t st);
 cudaError_t state_export(bool blocked, const float* S, float* out, const Shape& s, cudaStream_t st);
 cudaError_t state_snapshot(const float* Sb, void* snap_bf16, const Shape& s, cudaStream_t st);
+// One chunk of the accumulated-state clip on the bf16 path (row-major fp32 state,
+// B x d F): S = c (keep S + eta raw), c = tau / ||keep S + eta raw||_F when that
+// exceeds tau (into alpha[b][chunk]); snap_bf16 (or null) receives bf16(S).  part
+// holds B x 592 partial sums.
+cudaError_t state_clip_step(float* S, const float* raw, double* part, float* alpha, const ChunkMeta* meta,
+                            const Shape& s, int chunk, float eta, float tau, void* snap_bf16, cudaStream_t st);
 
 // SM_ACC: out += sum; SM_ACC_L: the same on the rows of each chunk's last document segment.
 enum SimtMode { SM_Z = 0, SM_V = 1, SM_RAW = 2, SM_APPLY = 3, SM_ACC = 4, SM_ACC_L = 5 };

@@ -356,6 +356,8 @@ ipttt_status decode_check(const ipttt_params* p) {
   if (rc != IPTTT_OK) return rc;
   if (p->dtype != IPTTT_BF16 || p->B > kDecodeMaxRows || p->d % 8 != 0 || p->F % 8 != 0)
     return IPTTT_ERR_UNSUPPORTED;
+  // the chunk commits go through the streaming path, which takes the per-delta clip only
+  if (p->flags & IPTTT_FLAG_STATE_CLIP) return IPTTT_ERR_UNSUPPORTED;
   return IPTTT_OK;
 }
 

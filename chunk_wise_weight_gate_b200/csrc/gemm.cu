@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       long long base;
       if (a.mode == GM_PLAIN) base = (long long)t.slice * a.osz + (long long)m * a.ldo;
       else if (a.mode == GM_CHUNK_ROWS) base = (long long)t.b * a.osz + (long long)(t.t0 + m) * a.ldo;
-      else base = ((long long)t.chunk * a.B + t.b) * a.osz + (long long)m * a.ldo;
+      else base = ((long long)(t.chunk - a.chunk_base) * a.B + t.b) * a.osz + (long long)m * a.ldo;
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         uint32_t r[32];

@@ -54,6 +54,7 @@ struct Args {
   int rows;              // Rows
   int ksplit;            // PLAIN: K in this many slices (0 or 1: one), slice s written at out + s * osz
   int* status;           // device status word (timeouts)
+  int chunk_base;        // CHUNK_K: chunk i's matrices go to index i - chunk_base of out
 };
 
 // Launches the persistent kernel: on clusters of two CTAs (256-row tiles) when the

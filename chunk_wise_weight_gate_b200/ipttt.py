@@ -40,7 +40,7 @@ class Params(ctypes.Structure):
 
 
 FLAG_RESIDUAL = 1
-FLAG_STATE_CLIP = 2  # the ablation: clip the accumulated state, not each delta (fp32 only)
+FLAG_STATE_CLIP = 2  # the ablation: clip the accumulated state, not each delta
 
 
 class IptttError(RuntimeError):
@@ -197,15 +197,17 @@ def _docs(doc_starts, device) -> tuple[int | None, int, torch.Tensor | None]:
     return ds.data_ptr(), int(ds.numel()), ds
 
 
-def workspace_size(cfg: LayerConfig) -> int:
-    n = lib().ipttt_workspace_size(ctypes.byref(cfg.params()))
+def workspace_size(cfg: LayerConfig, state_clip: bool = False) -> int:
+    """Workspace bytes of a forward (state_clip: of the accumulated-state clip, which
+    keeps each chunk's raw delta in fp32 on the bf16 path too)."""
+    n = lib().ipttt_workspace_size(ctypes.byref(cfg.params(FLAG_STATE_CLIP if state_clip else 0)))
     if n == 0:
         raise ValueError(f"invalid layer configuration {cfg}")
     return int(n)
 
 
-def alloc_workspace(cfg: LayerConfig, device="cuda") -> torch.Tensor:
-    return torch.empty(workspace_size(cfg), dtype=torch.uint8, device=device)
+def alloc_workspace(cfg: LayerConfig, device="cuda", state_clip: bool = False) -> torch.Tensor:
+    return torch.empty(workspace_size(cfg, state_clip), dtype=torch.uint8, device=device)
 
 
 def _shape_check(cfg: LayerConfig, **tensors):
@@ -222,15 +224,15 @@ def forward(cfg: LayerConfig, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_st
     """One layer forward.  Returns O, or with debug=True (or a subset of
     DEBUG_OUTPUTS) a dict with O and the chosen internals D, S_final, alpha, Z, V,
     produced by the same kernels as O.  residual=True writes H + output into O.
-    state_clip=True (fp32 only) clips the accumulated state instead of each delta;
-    alpha then holds the state's clip factor per chunk."""
+    state_clip=True clips the accumulated state instead of each delta; alpha then
+    holds the state's clip factor per chunk."""
     dt = cfg.torch_dtype
     _shape_check(cfg, H=H, X0=X0, Wgate=Wgate, Wup=Wup, Wdown0=Wdown0, conv_w=conv_w, Wtarget=Wtarget, O=O)
     dev = H.device
     if O is None:
         O = torch.empty(cfg.B, cfg.T, cfg.d, dtype=dt, device=dev)
     if workspace is None:
-        workspace = alloc_workspace(cfg, dev)
+        workspace = alloc_workspace(cfg, dev, state_clip)
     if residual and O.data_ptr() == H.data_ptr():
         raise ValueError("O must not alias H when residual=True")
     dp, nd, keep = _docs(doc_starts, dev)

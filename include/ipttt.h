@@ -100,8 +100,11 @@ typedef struct {
  * delta (iplexlaw.co.kr review of arXiv 2604.06169, §6, leaves open which of the
  * two the clip acts on): S_{i+1} = c_i (keep_i S_i + eta V_L^T Z_L) with
  * c_i = tau / ||keep_i S_i + eta V_L^T Z_L||_F when that norm exceeds tau, else 1.
- * dtype IPTTT_F32 only (IPTTT_ERR_UNSUPPORTED otherwise); the per-chunk factor
- * returned in alpha_opt is c_i. */
+ * Both dtypes; the per-chunk factor returned in alpha_opt is c_i.  On the bf16 path
+ * each chunk's V_L^T Z_L is a tensor-core GEMM with an fp32 result and the state
+ * update, norm and scale run on the CUDA cores in fp32, chunk by chunk.  The
+ * context-parallel, decoding and backward entry points do not take it, nor does
+ * streaming on the bf16 path (IPTTT_ERR_UNSUPPORTED). */
 #define IPTTT_FLAG_STATE_CLIP 2
 
 /* Bytes of workspace that ipttt_forward / _ex / stream_forward need for *p.

@@ -88,7 +88,31 @@ def test_state_clip(name):
     assert maxrel(per_delta["D"], ref["D"]) > 1e-2
 
 
-def test_state_clip_is_fp32_only():
-    cfg, inp = case(**CASES["clip"])
-    with pytest.raises(Exception):
-        gpu(cfg, inp, state_clip=True)
+# The bf16 path: each chunk's V_L^T Z_L from a tcgen05 GEMM, the state kept, clipped
+# and copied to bf16 on the CUDA cores.  tau puts some chunks under the clip and
+# some over it; the fast-weight term is most of O here, so O sees the scan.
+STATE_CLIP_BF16_CASES = {
+    # documents inside chunks and at a row's chunk boundary; 128-token chunks, which
+    # the per-delta path would scan in groups of 512 tokens
+    "bf16_docs": dict(B=2, T=768, C=128, d=256, F=512, eta=2e-2, clip=30.0, docs=[100, 300, 768 + 500]),
+    # one document, 256-token chunks: the first unclipped, the rest clipped
+    "bf16_tiles": dict(B=1, T=1024, C=256, d=256, F=512, eta=1e-2, clip=30.0, docs=[]),
+}
+
+
+@pytest.mark.parametrize("name", list(STATE_CLIP_BF16_CASES))
+def test_state_clip_bf16(name):
+    kw = dict(STATE_CLIP_BF16_CASES[name])
+    cfg, inp = case(dtype="bf16", conv_std=0.3, wtarget="identity_noise", **kw)
+    out = gpu(cfg, inp, state_clip=True)
+    ref = state_clip_oracle(cfg, inp)
+    errs = (maxrel(to_np(out["O"]), ref["O"]), normrel(to_np(out["S_final"]), ref["S_final"]),
+            np.max(np.abs(to_np(out["alpha"]) - ref["scale"])))
+    print(name, "O", errs[0], "S_final", errs[1], "clip factors", errs[2])
+    assert errs[0] <= 2e-2
+    assert errs[1] <= 2e-2
+    assert normrel(to_np(out["D"]), ref["D"]) <= 2e-2
+    assert errs[2] <= 1e-2
+    assert np.min(ref["scale"]) < 0.9 and np.max(ref["scale"]) == 1.0
+    per_delta = oracle(cfg, inp)
+    assert maxrel(per_delta["O"], ref["O"]) > 5 * 2e-2

@@ -64,10 +64,28 @@ def test_workspace_size_grows_with_tokens_and_is_zero_when_invalid():
     (dict(B=0), 1), (dict(T=-1), 1), (dict(C=0), 1), (dict(dtype=3), 4),
     (dict(eta=float("nan")), 1), (dict(clip_thresh=float("nan")), 1),
     (dict(d=200), 5), (dict(F=320), 5), (dict(C=96), 5), (dict(C=32), 5), (dict(C=8192), 5), (dict(flags=6), 1),
-    (dict(flags=2), 5),  # the accumulated-state clip runs on the fp32 path only
 ])
 def test_bad_params_are_rejected_before_launch(kw, code):
     assert call_forward(params(**kw)) == code
+
+
+def test_state_clip_only_where_it_has_a_meaning():
+    # the forward takes the accumulated-state clip on both paths, with room for the
+    # raw delta; the backward (its gradients are those of the per-delta clip) and
+    # the context-parallel split (the clip is not linear in the state) do not
+    L = ip.lib()
+    for dt in (ip.BF16, ip.F32):
+        plain = L.ipttt_workspace_size(ctypes.byref(params(dtype=dt)))
+        clip = L.ipttt_workspace_size(ctypes.byref(params(dtype=dt, flags=2)))
+        assert clip >= plain > 0
+        assert L.ipttt_backward_workspace_size(ctypes.byref(params(dtype=dt, flags=2))) == 0
+        assert L.ipttt_backward_workspace_size(ctypes.byref(params(dtype=dt))) > 0
+    assert L.ipttt_decode_state_size(ctypes.byref(params(flags=2))) == 0
+    p = params(flags=2)
+    fake = [0x10000 + 256 * i for i in range(8)]
+    rc = L.ipttt_cp_begin(ctypes.byref(p), 2, 0, None, 0, *fake[:6], ctypes.c_void_p(fake[6]),
+                          ctypes.c_void_p(0x100000), ctypes.c_size_t(1 << 40), None)
+    assert rc == 5
 
 
 def test_null_misaligned_and_workspace_errors():
