@@ -312,6 +312,7 @@ struct Tensors {
   void* O;
   float *D, *Sfinal, *alpha;
   void *Zout, *Vout;
+  void* deltas;  // keep_all forward: every chunk's V_L^T Z_L, bf16 [k][B][d][F] (for the backward)
 };
 
 struct StreamState {
@@ -589,6 +590,13 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
       !make_map_bf16(&sc.map[4], Z, s.F, s.T, s.B, 64, update_tokens_per_stage(s.C)) ||
       !make_map_bf16(&sc.map[5], snap, s.F, s.d, (uint64_t)G * s.B, 64, 32))
     return cuda_fail("tensor maps of the chunk scan", cudaErrorInvalidValue);
+  // the forward of the backward also keeps each chunk's raw delta (the update's
+  // TMEM product before alpha eta), which the backward would otherwise recompute
+  if (L.keep_all && t.deltas && !grouped) {
+    if (!make_map_bf16(&sc.map[7], t.deltas, s.F, s.d, (uint64_t)s.k * s.B, 64, 32))
+      return cuda_fail("tensor map of the deltas", cudaErrorInvalidValue);
+    sc.delta_out = 1;
+  }
   // the 256-row apply writes O through shared memory and TMA stores
   if (apply_fam == FAM_APPLY256 && t.O) {
     if (!make_map_bf16(&sc.map[6], t.O, s.d, s.T, s.B, 64, 32))
@@ -601,7 +609,8 @@ ipttt_status run_bf16(const ipttt_params& p, const Tensors& t, uint8_t* ws, cons
   sc.S = S;
   sc.nslots = G;
   sc.dchunks = 1;
-  const bool need_final = t.Sfinal != nullptr || ss != nullptr;
+  // (the last chunk's update also writes its delta when the backward wants them)
+  const bool need_final = t.Sfinal != nullptr || ss != nullptr || sc.delta_out;
   const int state_tiles = s.B * (s.d / 128) * ((s.F + 255) / 256);  // 128 x 256 tiles
   const int apply_tiles_per_chunk = s.B * (sq.C / arows) * (s.d / 128);
   // State updates of chunks [c0, c1) in one launch: each worker carries its state
@@ -1133,8 +1142,10 @@ ipttt_status ipttt_backward(const ipttt_params* p, const void* H, const void* X0
     t.doc = doc_starts;
     t.n_doc = n_doc_starts;
     t.O = ws + BL.O;
+    t.deltas = bwd::tc_delta_buffer(ws + BL.tc, s);
     if ((rc = run_bf16(*p, t, ws, BL.fwd, nullptr, di, st)) != IPTTT_OK) return rc;
     bwd::TcForward f;
+    f.deltas_ready = !BL.fwd.grouped;
     f.Z = ws + BL.fwd.Z;
     f.U = ws + BL.fwd.U;
     f.V = ws + BL.fwd.V;
@@ -1147,7 +1158,7 @@ ipttt_status ipttt_backward(const ipttt_params* p, const void* H, const void* X0
                                       gS_final_opt, gH, gX0, gWgate, gWup, gWdown0, gconv_w, gWtarget, ws + BL.tc,
                                       di->status, di->num_sms, st);
     if (e != cudaSuccess) return cuda_fail("backward", e);
-    counted(bwd::tc_launches());
+    counted(bwd::tc_launches(f.deltas_ready));
     return IPTTT_OK;
   }
   const cudaError_t e = bwd::run(s, p->dtype, p->eta, tau, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_starts,

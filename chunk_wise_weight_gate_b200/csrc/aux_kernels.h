@@ -85,9 +85,12 @@ struct TcForward {
   const ChunkMeta* meta;
   const uint8_t* flags;
   int nslots;
+  bool deltas_ready;  // the forward's update wrote every chunk's V_L^T Z_L (bf16) into tc_delta_buffer
 };
 size_t tc_workspace_bytes(const Shape& s);
-long long tc_launches();
+// Where run_tc keeps the per-chunk deltas V_L^T Z_L ([k][B][d][F] bf16) in its workspace.
+void* tc_delta_buffer(uint8_t* ws, const Shape& s);
+long long tc_launches(bool deltas_ready);
 cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, const void* H, const void* X0,
                    const void* Wg, const void* Wu, const void* W0, const void* cw, const void* Wt, const void* gO,
                    const float* gS, float* gH, float* gX0, float* gWg, float* gWu, float* gW0, float* gcw,

@@ -670,8 +670,11 @@ TcLayout tc_layout(const Shape& s) {
 
 size_t tc_workspace_bytes(const Shape& s) { return tc_layout(s).total; }
 
-// Kernels run_tc launches: 17 GEMMs and 11 elementwise or reduction kernels.
-long long tc_launches() { return 28; }
+void* tc_delta_buffer(uint8_t* ws, const Shape& s) { return ws + tc_layout(s).P; }
+
+// Kernels run_tc launches: 17 GEMMs (16 when the forward wrote the deltas) and 11
+// elementwise or reduction kernels.
+long long tc_launches(bool deltas_ready) { return deltas_ready ? 27 : 28; }
 
 
 cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, const void* H, const void* X0,
@@ -730,10 +733,11 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
   g.Bop = {Zb, (uint64_t)(F), (uint64_t)(BT), (uint64_t)(1)};
   g.a_mn = 1; g.b_mn = 1;
   BW_CHECK(plain((int)d, (int)F, (int)BT, gW0, F, GO_F32));
-  // 4. P_i = V_L^T Z_L and R_i = gO_F^T Z_F per chunk (bf16)
+  // 4. P_i = V_L^T Z_L (unless the forward's state update wrote them) and
+  //    R_i = gO_F^T Z_F per chunk (bf16)
   g.A = {Vb, (uint64_t)(d), (uint64_t)(T), (uint64_t)(B)};
   g.Bop = {Zb, (uint64_t)(F), (uint64_t)(T), (uint64_t)(B)};
-  BW_CHECK(chunked(GM_CHUNK_K, (int)d, (int)F, 0, P, F, d * F, GO_BF16, nullptr, GR_ALL, 1));
+  if (!f.deltas_ready) BW_CHECK(chunked(GM_CHUNK_K, (int)d, (int)F, 0, P, F, d * F, GO_BF16, nullptr, GR_ALL, 1));
   k_mask_first_bf16<<<grid_for(B * T * d), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(gO), gOF, f.meta, (int)B,
                                                           (int)T, (int)d, s.C, k);
   g.A = {gOF, (uint64_t)(d), (uint64_t)(T), (uint64_t)(B)};

@@ -891,7 +891,9 @@ __device__ __forceinline__ float4* upd_state_block(const TcParams& p, int b, int
                                    ((size_t)(m0 / 128) * (p.F / 128) + n0 / 128 + h) * (128 * 128));
 }
 
-template <bool PAIR, int KB>
+// DELTA: also write each chunk's raw delta (the forward run for the backward); a
+// separate build, so the forward's own update carries none of that code.
+template <bool PAIR, int KB, bool DELTA>
 __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_constant__ TcParams p) {
   using Cf = UpdCfg<PAIR, KB>;
   constexpr int STAGES = Cf::STAGES;
@@ -936,6 +938,7 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
     prefetch_tmap(&p.map[3]);
     prefetch_tmap(&p.map[4]);
     prefetch_tmap(&p.map[5]);
+    if (DELTA) prefetch_tmap(&p.map[7]);
   }
   if (warp == UPD_WARP_MMA) {
     if constexpr (PAIR) {
@@ -993,7 +996,8 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
       // Snapshot box hb: 32 rows x 64 columns of bf16(S_{chunk+1}) (what the apply of
       // chunk+1 reads), 128-byte swizzled, stored by TMA.
       auto store_box = [&](const int hb) {
-        uint8_t* box = wboxes + (hb % UPD_BOXES) * UPD_BOX_BYTES;
+        // boxes in turn (with the deltas' boxes in between when DELTA)
+        uint8_t* box = wboxes + ((DELTA ? stores : hb) % UPD_BOXES) * UPD_BOX_BYTES;
         if (stores > 0) {
           // the store issued from this buffer UPD_BOXES boxes ago has read it
           if (lane == 0) bulk_wait_read<UPD_BOXES - 1>();
@@ -1017,6 +1021,29 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
         }
         ++stores;
       };
+      // For the backward: box hb of the chunk's raw delta V_L^T Z_L (the TMEM values
+      // before alpha eta), bf16, into the chunk's [d][F] matrix of map[7].
+      auto store_delta = [&](const int hb, const uint32_t (&ra)[64]) {
+        uint8_t* box = wboxes + (stores % UPD_BOXES) * UPD_BOX_BYTES;
+        if (stores > 0) {
+          if (lane == 0) bulk_wait_read<UPD_BOXES - 1>();
+          __syncwarp();
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          *reinterpret_cast<uint4*>(box + lane * 128 + ((e ^ (lane & 7)) << 4)) = make_uint4(
+              pack_bf16(__uint_as_float(ra[8 * e]), __uint_as_float(ra[8 * e + 1])),
+              pack_bf16(__uint_as_float(ra[8 * e + 2]), __uint_as_float(ra[8 * e + 3])),
+              pack_bf16(__uint_as_float(ra[8 * e + 4]), __uint_as_float(ra[8 * e + 5])),
+              pack_bf16(__uint_as_float(ra[8 * e + 6]), __uint_as_float(ra[8 * e + 7])));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&p.map[7], box, jb.n0 + 128 * half + 64 * hb, m0c + 32 * quarter, jb.chunk * p.B + jb.b);
+          bulk_commit();
+        }
+        ++stores;
+      };
       if (!mbar_wait(&slot_full[sl], (i >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
       // Two halves of the warp's 128 columns, one 64-column TMEM load each: the
@@ -1026,6 +1053,7 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
       if (cols) {
         tmem_ld64(tcol, x0);
         tmem_ld_wait();
+        if constexpr (DELTA) store_delta(0, x0);
         fold(0, x0);
         tmem_ld64(tcol + 64, y0);
         if (snap) store_box(0);
@@ -1039,6 +1067,7 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
         else mbar_arrive(&slot_free[sl]);
       }
       if (!cols) continue;
+      if constexpr (DELTA) store_delta(1, y0);
       fold(1, y0);
       if (snap) store_box(1);
       if (jb.c == p.dchunks - 1) {
@@ -1185,7 +1214,7 @@ static int max_pairs(cudaStream_t st) {
   if (have[dev]) return cached[dev];
   int n = 0;
   constexpr int smem = UpdCfg<true, KB>::SMEM;
-  if (cudaFuncSetAttribute(upd_kernel<true, KB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
+  if (cudaFuncSetAttribute(upd_kernel<true, KB, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
       cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -1199,7 +1228,7 @@ static int max_pairs(cudaStream_t st) {
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, upd_kernel<true, KB>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, upd_kernel<true, KB, false>, &cfg) != cudaSuccess) n = 0;
   }
   cudaGetLastError();
   cached[dev] = n;
@@ -1215,19 +1244,19 @@ static bool pair_update_enabled() {
 // The update kernel's register trade (setmaxnreg) balances only at the launch
 // register count it was written for; any other count could leave a warpgroup
 // waiting for registers, so such a build is refused.
-template <bool PAIR, int KB>
+template <bool PAIR, int KB, bool DELTA>
 static bool upd_regs_ok() {
   cudaFuncAttributes a;
-  if (cudaFuncGetAttributes(&a, upd_kernel<PAIR, KB>) != cudaSuccess) {
+  if (cudaFuncGetAttributes(&a, upd_kernel<PAIR, KB, DELTA>) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
   return a.numRegs == UPD_REGS_LAUNCH;
 }
 
-template <int KB>
+template <int KB, bool DELTA>
 static cudaError_t launch_update_kb(const TcParams& p, int num_sms, cudaStream_t st) {
-  if (!upd_regs_ok<true, KB>() || !upd_regs_ok<false, KB>()) return cudaErrorInvalidDeviceFunction;
+  if (!upd_regs_ok<true, KB, DELTA>() || !upd_regs_ok<false, KB, DELTA>()) return cudaErrorInvalidDeviceFunction;
   if (p.d % 256 == 0 && pair_update_enabled()) {
     const int np = max_pairs<KB>(st);
     if (np > 0) {
@@ -1246,14 +1275,17 @@ static cudaError_t launch_update_kb(const TcParams& p, int num_sms, cudaStream_t
       cfg.stream = st;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      return cudaLaunchKernelEx(&cfg, upd_kernel<true, KB>, q);
+      if (cudaFuncSetAttribute(upd_kernel<true, KB, DELTA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess)
+        return cudaErrorInvalidValue;
+      return cudaLaunchKernelEx(&cfg, upd_kernel<true, KB, DELTA>, q);
     }
   }
   constexpr int smem = UpdCfg<false, KB>::SMEM;
-  cudaError_t e = cudaFuncSetAttribute(upd_kernel<false, KB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(upd_kernel<false, KB, DELTA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(p.n_tiles, num_sms));
-  upd_kernel<false, KB><<<grid, UPD_THREADS, smem, st>>>(p);
+  upd_kernel<false, KB, DELTA><<<grid, UPD_THREADS, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -1262,7 +1294,9 @@ int update_tokens_per_stage(int C) { return C % 128 == 0 ? 128 : 64; }
 cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st) {
   if (p.n_tiles <= 0 || p.dchunks <= 0) return cudaSuccess;
   const int kb = p.upd_kb ? p.upd_kb : update_tokens_per_stage(p.C);
-  return kb == 128 ? launch_update_kb<128>(p, num_sms, st) : launch_update_kb<64>(p, num_sms, st);
+  if (p.delta_out)
+    return kb == 128 ? launch_update_kb<128, true>(p, num_sms, st) : launch_update_kb<64, true>(p, num_sms, st);
+  return kb == 128 ? launch_update_kb<128, false>(p, num_sms, st) : launch_update_kb<64, false>(p, num_sms, st);
 }
 
 // ------------------------------------------------------------------ failure-path self test

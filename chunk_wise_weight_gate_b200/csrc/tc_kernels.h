@@ -20,7 +20,8 @@ namespace tck {
 enum Family { FAM_ZV = 0, FAM_GRAM = 1, FAM_APPLY = 2, FAM_APPLY256 = 5, FAM_ZV2 = 6, FAM_GRAM2 = 8, FAM_PZ = 9 };
 
 struct TcParams {
-  CUtensorMap map[7];     // map[6]: the apply's O as 32-row x 64-column store boxes (o_tma)
+  CUtensorMap map[8];     // map[6]: the apply's O as 32-row x 64-column store boxes (o_tma);
+                          // map[7]: the update's raw deltas [k B][d][F] as the same boxes (delta_out)
   int kind;          // FAM_ZV: kind_gateup() or kind_vhat()
   int vn;            // FAM_ZV target GEMM: output columns per tile (128 or 256)
   int B, T, d, F, C, k;
@@ -51,6 +52,7 @@ struct TcParams {
   int upd_kb;             // update: tokens per stage (0: update_tokens_per_stage(C))
   int upd_scale;          // update: 1 = V is not pre-scaled; the delta is scaled by alpha[b][chunk] eta
   int o_tma;              // 256-row apply: O leaves through shared memory and TMA stores (map[6])
+  int delta_out;          // update: each chunk's raw delta V_L^T Z_L also goes out, bf16 (map[7])
 };
 
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
