@@ -632,12 +632,13 @@ def backward_flops_per_token(d: int, F: int, dtype: str) -> int:
     recomputes (gate, up, target, each chunk's V^T Z: 6dF + 2d^2) and the gradient
     products (gW0, gO W0, per chunk P, gV, gZ from the delta, gZ from the state,
     the state's gradient: 14dF; gH and gWgate, gWup: 8dF; gU, gWtarget: 4d^2).
-    bf16 (tensor cores): the whole forward (10dF + 2d^2, its apply included) and
-    then gate and up pre-activations 4dF, gO W0 2dF, gW0 2dF, per chunk P and the
-    state gradient's deltas 4dF, Z G^T 2dF, Z P^T 2dF, three gZ terms 6dF, gH 4dF,
-    gWgate and gWup 4dF, gU and gWtarget 4d^2: 40dF + 6d^2."""
+    bf16 (tensor cores): the whole forward (10dF + 2d^2, its apply included; its
+    state update's per-chunk P is kept for the gradients) and then gate and up
+    pre-activations 4dF, gO W0 2dF, gW0 2dF, the state gradient's deltas 2dF, Z G^T
+    2dF, Z P^T 2dF, three gZ terms 6dF, gH 4dF, gWgate and gWup 4dF, gU and
+    gWtarget 4d^2: 38dF + 6d^2."""
     if dtype == "bf16":
-        return 40 * d * F + 6 * d * d
+        return 38 * d * F + 6 * d * d
     return 28 * d * F + 6 * d * d
 
 
