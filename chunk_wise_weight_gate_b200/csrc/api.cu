@@ -1158,7 +1158,7 @@ ipttt_status ipttt_backward(const ipttt_params* p, const void* H, const void* X0
                                       gS_final_opt, gH, gX0, gWgate, gWup, gWdown0, gconv_w, gWtarget, ws + BL.tc,
                                       di->status, di->num_sms, st);
     if (e != cudaSuccess) return cuda_fail("backward", e);
-    counted(bwd::tc_launches(f.deltas_ready));
+    counted(bwd::tc_launches(f.deltas_ready, gS_final_opt != nullptr));
     return IPTTT_OK;
   }
   const cudaError_t e = bwd::run(s, p->dtype, p->eta, tau, H, X0, Wgate, Wup, Wdown0, conv_w, Wtarget, doc_starts,

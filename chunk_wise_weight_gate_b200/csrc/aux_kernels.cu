@@ -358,6 +358,23 @@ __global__ void k_blocked_to_bf16(const float* Sb, __nv_bfloat16* out, int B, in
   }
 }
 
+__global__ void k_rowmajor_to_blocked(const float* in, float* Sb, int B, int d, int F) {
+  const size_t total = (size_t)B * d * F;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int c = (int)(i % F);
+    const size_t br = i / F;
+    const int r = (int)(br % d);
+    const size_t b = br / d;
+    Sb[b * d * F + blocked_index(r, c, F)] = in[i];
+  }
+}
+
+cudaError_t state_import_blocked(const float* in, float* Sb, const Shape& s, cudaStream_t st) {
+  if (!in) return cudaMemsetAsync(Sb, 0, (size_t)s.B * s.d * s.F * sizeof(float), st);
+  k_rowmajor_to_blocked<<<148 * 8, 256, 0, st>>>(in, Sb, s.B, s.d, s.F);
+  return cudaGetLastError();
+}
+
 cudaError_t state_export(bool blocked, const float* S, float* out, const Shape& s, cudaStream_t st) {
   const size_t n = (size_t)s.B * s.d * s.F;
   if (!blocked) return cudaMemcpyAsync(out, S, n * sizeof(float), cudaMemcpyDeviceToDevice, st);

@@ -17,6 +17,8 @@ cudaError_t conv_target(int dtype, const void* X0, const void* cw, const uint8_t
 cudaError_t alpha_from_partials(const float* partials, float* alpha, int n, int npairs, float eta, float tau,
                                 cudaStream_t st);
 cudaError_t state_export(bool blocked, const float* S, float* out, const Shape& s, cudaStream_t st);
+// A row-major fp32 [B][d][F] state into the update kernel's blocked layout (null: zeros).
+cudaError_t state_import_blocked(const float* in, float* Sb, const Shape& s, cudaStream_t st);
 cudaError_t state_snapshot(const float* Sb, void* snap_bf16, const Shape& s, cudaStream_t st);
 // One chunk of the accumulated-state clip on the bf16 path (row-major fp32 state,
 // B x d F): S = c (keep S + eta raw), c = tau / ||keep S + eta raw||_F when that
@@ -90,7 +92,7 @@ struct TcForward {
 size_t tc_workspace_bytes(const Shape& s);
 // Where run_tc keeps the per-chunk deltas V_L^T Z_L ([k][B][d][F] bf16) in its workspace.
 void* tc_delta_buffer(uint8_t* ws, const Shape& s);
-long long tc_launches(bool deltas_ready);
+long long tc_launches(bool deltas_ready, bool has_gS);
 cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, const void* H, const void* X0,
                    const void* Wg, const void* Wu, const void* W0, const void* cw, const void* Wt, const void* gO,
                    const float* gS, float* gH, float* gX0, float* gWg, float* gWu, float* gW0, float* gcw,

@@ -27,6 +27,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
+#include <string.h>
 
 #include <algorithm>
 
@@ -463,48 +464,6 @@ __global__ void k_mask_first_bf16(const __nv_bfloat16* gO, __nv_bfloat16* gOF, c
   }
 }
 
-// G_{i+1} -> Gs[i] (bf16), G_i = keep_i G_{i+1} + R_i, for i = k-1 .. 0; G_k = gS
-// (or 0).  8 consecutive elements per thread (n % 8 == 0), the next chunk's R
-// requested before the current one is added.
-__global__ void k_reverse_scan(const __nv_bfloat16* R, const float* gS, __nv_bfloat16* Gs, const ChunkMeta* meta,
-                               int B, int k, size_t n) {
-  const size_t total = (size_t)B * n;
-  for (size_t e = 8 * (blockIdx.x * (size_t)blockDim.x + threadIdx.x); e < total;
-       e += 8 * (size_t)gridDim.x * blockDim.x) {
-    const int b = (int)(e / n);
-    float g[8];
-    if (gS) {
-      const float4 x = *reinterpret_cast<const float4*>(gS + e), y = *reinterpret_cast<const float4*>(gS + e + 4);
-      g[0] = x.x; g[1] = x.y; g[2] = x.z; g[3] = x.w; g[4] = y.x; g[5] = y.y; g[6] = y.z; g[7] = y.w;
-    } else {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) g[q] = 0.0f;
-    }
-    uint4 r = *reinterpret_cast<const uint4*>(R + (size_t)(k - 1) * total + e);
-    for (int i = k - 1; i >= 0; --i) {
-      const size_t o = (size_t)i * total + e;
-      const uint4 cur = r;
-      if (i > 0) r = *reinterpret_cast<const uint4*>(R + o - total);
-      uint4 w;
-      uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(g[2 * q], g[2 * q + 1]);
-        wp[q] = *reinterpret_cast<uint32_t*>(&h);
-      }
-      *reinterpret_cast<uint4*>(Gs + o) = w;
-      const bool keep = !meta[(size_t)b * k + i].has_start;
-      const uint32_t* cp = reinterpret_cast<const uint32_t*>(&cur);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&cp[q]);
-        g[2 * q] = (keep ? g[2 * q] : 0.0f) + __low2float(h);
-        g[2 * q + 1] = (keep ? g[2 * q + 1] : 0.0f) + __high2float(h);
-      }
-    }
-  }
-}
-
 // <P_i, G_{i+1}> = sum over the tokens of chunk i of v_t . Y_t (V is zero outside
 // the last segment), as kDotParts fixed-order partial sums per (row, chunk) ...
 constexpr int kDotParts = 32;
@@ -631,7 +590,7 @@ __global__ void k_f32_to_bf16(const float* x, __nv_bfloat16* y, size_t n) {
 }
 
 struct TcLayout {
-  size_t Af, Buf, gZ, gA, gBu, gOF, Y, gV, gVb, gU, P, R, Gs, c1, c2, dpart, cwf, cpart, total;
+  size_t Af, Buf, gZ, gA, gBu, gOF, Y, gV, gVb, gU, P, G, Gs, c1, c2, dpart, cwf, cpart, total;
 };
 
 TcLayout tc_layout(const Shape& s) {
@@ -654,7 +613,7 @@ TcLayout tc_layout(const Shape& s) {
   L.gVb = take(B * T * d * 2);
   L.gU = take(B * T * d * 4);
   L.P = take(k * B * d * F * 2);
-  L.R = take(k * B * d * F * 2);
+  L.G = take(B * d * F * 4);  // the reverse scan's fp32 state (blocked tiles)
   L.Gs = take(k * B * d * F * 2);
   L.c1 = take(B * k * 4);
   L.c2 = take(B * k * 4);
@@ -672,9 +631,13 @@ size_t tc_workspace_bytes(const Shape& s) { return tc_layout(s).total; }
 
 void* tc_delta_buffer(uint8_t* ws, const Shape& s) { return ws + tc_layout(s).P; }
 
-// Kernels run_tc launches: 17 GEMMs (16 when the forward wrote the deltas) and 11
-// elementwise or reduction kernels.
-long long tc_launches(bool deltas_ready) { return deltas_ready ? 27 : 28; }
+// Kernels run_tc launches: 16 GEMMs (15 when the forward wrote the deltas), the
+// reverse scan on the update kernel and 10 elementwise or reduction kernels, plus
+// the state layout kernel when a gradient of the final state is given (a memset
+// otherwise).
+long long tc_launches(bool deltas_ready, bool has_gS) {
+  return (deltas_ready ? 26 : 27) + (has_gS ? 1 : 0);
+}
 
 
 cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, const void* H, const void* X0,
@@ -692,7 +655,7 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
         *cwf = fp(L.cwf), *cpart = fp(L.cpart);
   double* dpart = reinterpret_cast<double*>(ws + L.dpart);
   __nv_bfloat16 *Af = hp(L.Af), *Buf = hp(L.Buf), *gA = hp(L.gA), *gBu = hp(L.gBu), *gOF = hp(L.gOF),
-                *gVb = hp(L.gVb), *P = hp(L.P), *R = hp(L.R), *Gs = hp(L.Gs);
+                *gVb = hp(L.gVb), *P = hp(L.P), *Gs = hp(L.Gs);
   const __nv_bfloat16* Zb = static_cast<const __nv_bfloat16*>(f.Z);
   const __nv_bfloat16* Vb = static_cast<const __nv_bfloat16*>(f.V);
 
@@ -733,17 +696,37 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
   g.Bop = {Zb, (uint64_t)(F), (uint64_t)(BT), (uint64_t)(1)};
   g.a_mn = 1; g.b_mn = 1;
   BW_CHECK(plain((int)d, (int)F, (int)BT, gW0, F, GO_F32));
-  // 4. P_i = V_L^T Z_L (unless the forward's state update wrote them) and
-  //    R_i = gO_F^T Z_F per chunk (bf16)
+  // 4. P_i = V_L^T Z_L (unless the forward's state update wrote them); gO_F, gO on
+  //    the continued first segment of each chunk
   g.A = {Vb, (uint64_t)(d), (uint64_t)(T), (uint64_t)(B)};
   g.Bop = {Zb, (uint64_t)(F), (uint64_t)(T), (uint64_t)(B)};
   if (!f.deltas_ready) BW_CHECK(chunked(GM_CHUNK_K, (int)d, (int)F, 0, P, F, d * F, GO_BF16, nullptr, GR_ALL, 1));
   k_mask_first_bf16<<<grid_for(B * T * d), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(gO), gOF, f.meta, (int)B,
                                                           (int)T, (int)d, s.C, k);
-  g.A = {gOF, (uint64_t)(d), (uint64_t)(T), (uint64_t)(B)};
-  BW_CHECK(chunked(GM_CHUNK_K, (int)d, (int)F, 0, R, F, d * F, GO_BF16, nullptr, GR_ALL, 1));
-  // 5. reverse scan: bf16 G_{i+1} in slot i
-  k_reverse_scan<<<grid_for(B * d * F / 8), 256, 0, st>>>(R, gS, Gs, f.meta, (int)B, k, (size_t)(d * F));
+  // 5. reverse scan on the state-update kernel: from G_k = gS, every chunk's
+  //    gO_F^T Z_F formed from zero in TMEM and added in fp32 (registers), bf16 G_{i+1}
+  //    into slot i of Gs before chunk i's term is added
+  float* G = fp(L.G);
+  BW_CHECK(aux::state_import_blocked(gS, G, s, st));
+  {
+    tck::TcParams q;
+    memset(&q, 0, sizeof(q));
+    q.B = (int)B; q.T = (int)T; q.d = (int)d; q.F = (int)F; q.C = s.C; q.k = k;
+    q.meta = f.meta;
+    q.S = G;
+    q.status = status;
+    q.nslots = k;
+    q.chunk = 0;
+    q.dchunks = k;
+    q.upd_kb = tck::update_tokens_per_stage(s.C);
+    q.n_tiles = (int)(B * (d / 128) * ((F + 255) / 256));
+    q.rev = 1;
+    if (!tck::make_map_bf16(&q.map[3], gOF, (uint64_t)d, (uint64_t)T, (uint64_t)B, 64, q.upd_kb) ||
+        !tck::make_map_bf16(&q.map[4], Zb, (uint64_t)F, (uint64_t)T, (uint64_t)B, 64, q.upd_kb) ||
+        !tck::make_map_bf16(&q.map[5], Gs, (uint64_t)F, (uint64_t)d, (uint64_t)k * B, 64, 32))
+      return cudaErrorInvalidValue;
+    BW_CHECK(tck::launch_update(q, num_sms, st));
+  }
   // 6. Y = Z G_{i+1}^T on every chunk's tokens, then c1, c2 per chunk
   g.A = {Zb, (uint64_t)(F), (uint64_t)(T), (uint64_t)(B)};
   g.Bop = {Gs, (uint64_t)(F), (uint64_t)(d), (uint64_t)((uint64_t)k * B)};

@@ -861,14 +861,14 @@ struct UpdJob {
 // Job i of worker w (a CTA, or a CTA pair) of nw, or false past the end.  The
 // worker's tiles are X_m = w + m nw; each is walked through every chunk of the
 // launch before the next.  The delta of job i goes to TMEM slot i % 2.
-template <bool PAIR>
+template <bool PAIR, bool REV = false>
 __device__ __forceinline__ bool upd_job(const TcParams& p, uint32_t i, int w, int nw, UpdJob& jb) {
   const uint32_t D = (uint32_t)p.dchunks;
   const long long X = (long long)w + (long long)(i / D) * nw;
   if (X >= p.n_tiles) return false;
   jb.X = (int)X;
   jb.c = (int)(i % D);
-  jb.chunk = p.chunk + jb.c;
+  jb.chunk = REV ? p.chunk + (int)D - 1 - jb.c : p.chunk + jb.c;  // REV: the chunks from the last
   // Row blocks vary fastest: the tiles in flight at one time (one per worker)
   // then cover few column blocks, so each chunk's Z columns come from DRAM about
   // once per launch (V, four times smaller, once per round of tiles).
@@ -882,6 +882,20 @@ __device__ __forceinline__ bool upd_job(const TcParams& p, uint32_t i, int w, in
   return true;
 }
 
+// K blocks of a chunk's delta: the forward's rows from the last segment's start;
+// the reverse scan's the continued first segment (gO_F is zero outside it; a chunk
+// without one still takes one block, of zeros, so its slot gets a delta).
+template <bool REV, int UKB>
+__device__ __forceinline__ void upd_kb_range(const TcParams& p, const ChunkMeta& m, int t0, int& kb0, int& kb1) {
+  if (REV) {
+    kb0 = 0;
+    kb1 = m.cont ? max(1, cdiv(min(m.first_end, p.T) - t0, UKB)) : 1;
+  } else {
+    kb0 = (m.last_start - t0) / UKB;
+    kb1 = cdiv(min(p.C, p.T - t0), UKB);
+  }
+}
+
 // fp32 state, 128 x 128 blocked tiles; tile column block h of the 128-row block
 // starting at d row m0 (a multiple of 128).  Inside a block, element (row, c) sits
 // at float4 index (c / 4) * 128 + row, so a warp holding 32 consecutive rows moves
@@ -893,7 +907,10 @@ __device__ __forceinline__ float4* upd_state_block(const TcParams& p, int b, int
 
 // DELTA: also write each chunk's raw delta (the forward run for the backward); a
 // separate build, so the forward's own update carries none of that code.
-template <bool PAIR, int KB, bool DELTA>
+// REV: the reverse scan of the backward, G_i = keep_i G_{i+1} + gO_F^T Z_F from the
+// last chunk down (A operand gO_F in place of V, rows of the continued first
+// segment); each chunk's slot i receives bf16(G_{i+1}), the state before the chunk.
+template <bool PAIR, int KB, bool DELTA, bool REV>
 __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_constant__ TcParams p) {
   using Cf = UpdCfg<PAIR, KB>;
   constexpr int STAGES = Cf::STAGES;
@@ -971,7 +988,7 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
     for (int e = 0; e < 128; ++e) st[e] = 0.0f;
 
     UpdJob jb;
-    for (uint32_t i = 0; upd_job<PAIR>(p, i, wk, nwk, jb); ++i) {
+    for (uint32_t i = 0; upd_job<PAIR, REV>(p, i, wk, nwk, jb); ++i) {
       const int sl = (int)(i & 1);
       const ChunkMeta m = p.meta[(size_t)jb.b * p.k + jb.chunk];
       const int m0c = jb.m0 + rofs;
@@ -979,9 +996,17 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
       // what the delta is added to: nothing (a document starts in the chunk: the
       // carried state is dropped), the state in registers, or (the tile's first
       // chunk of the launch) the state as the previous launch or the caller left it
-      const int base = m.has_start ? 0 : (jb.c == 0 ? 2 : 1);
-      const bool snap = jb.chunk + 1 < p.k;
       const float* sf = reinterpret_cast<const float*>(upd_state_block(p, jb.b, m0c, jb.n0, half));
+      if constexpr (REV) {
+        // the reverse scan stores the state before the chunk: bring in the start state first
+        if (jb.c == 0 && jb.n0 + 128 * half < p.F) {
+#pragma unroll
+          for (int q = 0; q < 128; ++q) st[q] = sf[((q / 4) * 128 + row) * 4 + (q & 3)];
+        }
+      }
+      const int base = m.has_start ? 0 : ((!REV && jb.c == 0) ? 2 : 1);
+      const bool snap = REV || jb.chunk + 1 < p.k;
+      const int slot = REV ? jb.chunk % p.nslots : (jb.chunk + 1) % p.nslots;
       // Folds 64 columns of the delta (one 64-column TMEM load) into st[64 hb ..].
       // the chunk's clip factor times eta, when V was not pre-scaled by it
       const float sc = p.upd_scale ? p.alpha[(size_t)jb.b * p.k + jb.chunk] * p.eta : 1.0f;
@@ -1016,7 +1041,7 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
           // the snapshots (2 d F bytes per chunk, read back only by a later launch)
           // leave L2 first, so the chunk's V and Z, which every pair reads, stay there
           tma_store_3d_hint(&p.map[5], box, jb.n0 + 128 * half + 64 * hb, m0c + 32 * quarter,
-                            ((jb.chunk + 1) % p.nslots) * p.B + jb.b, l2_policy_evict_first());
+                            slot * p.B + jb.b, l2_policy_evict_first());
           bulk_commit();
         }
         ++stores;
@@ -1054,9 +1079,10 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
         tmem_ld64(tcol, x0);
         tmem_ld_wait();
         if constexpr (DELTA) store_delta(0, x0);
+        if (REV && snap) store_box(0);
         fold(0, x0);
         tmem_ld64(tcol + 64, y0);
-        if (snap) store_box(0);
+        if (!REV && snap) store_box(0);
         tmem_ld_wait();
       }
       // the slot's delta is in registers: the MMAs may overwrite it
@@ -1068,8 +1094,9 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
       }
       if (!cols) continue;
       if constexpr (DELTA) store_delta(1, y0);
+      if (REV && snap) store_box(1);
       fold(1, y0);
-      if (snap) store_box(1);
+      if (!REV && snap) store_box(1);
       if (jb.c == p.dchunks - 1) {
         // the tile's last chunk of the launch: the fp32 state goes back to HBM
         float4* dst = upd_state_block(p, jb.b, m0c, jb.n0, half);
@@ -1090,17 +1117,17 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
         const uint32_t full0 = PAIR ? map_to_rank(smem_u32(full), 0) : 0u;  // the leader's full[0]
         // The next job's chunk metadata is requested one job ahead, so its round
         // trip never stands between two chunks' loads.
-        bool have = upd_job<PAIR>(p, 0, wk, nwk, jb);
+        bool have = upd_job<PAIR, REV>(p, 0, wk, nwk, jb);
         ChunkMeta m{};
         if (have) m = p.meta[(size_t)jb.b * p.k + jb.chunk];
         for (uint32_t i = 0; ok && have; ++i) {
           UpdJob jn;
-          const bool hn = upd_job<PAIR>(p, i + 1, wk, nwk, jn);
+          const bool hn = upd_job<PAIR, REV>(p, i + 1, wk, nwk, jn);
           ChunkMeta mn{};
           if (hn) mn = p.meta[(size_t)jn.b * p.k + jn.chunk];
           const int t0 = jb.chunk * p.C;
-          const int kb0 = (m.last_start - t0) / UPD_KB;
-          const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
+          int kb0, kb1;
+          upd_kb_range<REV, UPD_KB>(p, m, t0, kb0, kb1);
           for (int kb = kb0; kb < kb1; ++kb, ++it) {
             const int s = it % STAGES;
             const uint32_t ph = (it / STAGES) & 1;
@@ -1138,12 +1165,12 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
         bool ok = true;
         UpdJob jb;
         const uint32_t idesc = idesc_bf16(PAIR ? 256 : 128, 256, true, true);
-        bool have = upd_job<PAIR>(p, 0, wk, nwk, jb);
+        bool have = upd_job<PAIR, REV>(p, 0, wk, nwk, jb);
         ChunkMeta m{};
         if (have) m = p.meta[(size_t)jb.b * p.k + jb.chunk];
         for (uint32_t i = 0; ok && have; ++i) {
           UpdJob jn;
-          const bool hn = upd_job<PAIR>(p, i + 1, wk, nwk, jn);
+          const bool hn = upd_job<PAIR, REV>(p, i + 1, wk, nwk, jn);
           ChunkMeta mn{};
           if (hn) mn = p.meta[(size_t)jn.b * p.k + jn.chunk];   // the next job's, one job ahead
           const int sl = (int)(i & 1);
@@ -1153,8 +1180,8 @@ __global__ void __launch_bounds__(UPD_THREADS, 1) upd_kernel(const __grid_consta
           if (!got || *abort_flag) { ok = false; break; }
           tc_fence_after();
           const int t0 = jb.chunk * p.C;
-          const int kb0 = (m.last_start - t0) / UPD_KB;
-          const int kb1 = cdiv(min(p.C, p.T - t0), UPD_KB);
+          int kb0, kb1;
+          upd_kb_range<REV, UPD_KB>(p, m, t0, kb0, kb1);
           const uint32_t tacc = tmem_base + sl * ACC_COLS;
           for (int kb = kb0; kb < kb1; ++kb, ++it) {
             const int s = it % STAGES;
@@ -1214,7 +1241,7 @@ static int max_pairs(cudaStream_t st) {
   if (have[dev]) return cached[dev];
   int n = 0;
   constexpr int smem = UpdCfg<true, KB>::SMEM;
-  if (cudaFuncSetAttribute(upd_kernel<true, KB, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
+  if (cudaFuncSetAttribute(upd_kernel<true, KB, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
       cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -1228,7 +1255,7 @@ static int max_pairs(cudaStream_t st) {
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, upd_kernel<true, KB, false>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, upd_kernel<true, KB, false, false>, &cfg) != cudaSuccess) n = 0;
   }
   cudaGetLastError();
   cached[dev] = n;
@@ -1244,19 +1271,20 @@ static bool pair_update_enabled() {
 // The update kernel's register trade (setmaxnreg) balances only at the launch
 // register count it was written for; any other count could leave a warpgroup
 // waiting for registers, so such a build is refused.
-template <bool PAIR, int KB, bool DELTA>
+template <bool PAIR, int KB, bool DELTA, bool REV>
 static bool upd_regs_ok() {
   cudaFuncAttributes a;
-  if (cudaFuncGetAttributes(&a, upd_kernel<PAIR, KB, DELTA>) != cudaSuccess) {
+  if (cudaFuncGetAttributes(&a, upd_kernel<PAIR, KB, DELTA, REV>) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
   return a.numRegs == UPD_REGS_LAUNCH;
 }
 
-template <int KB, bool DELTA>
+template <int KB, bool DELTA, bool REV>
 static cudaError_t launch_update_kb(const TcParams& p, int num_sms, cudaStream_t st) {
-  if (!upd_regs_ok<true, KB, DELTA>() || !upd_regs_ok<false, KB, DELTA>()) return cudaErrorInvalidDeviceFunction;
+  if (!upd_regs_ok<true, KB, DELTA, REV>() || !upd_regs_ok<false, KB, DELTA, REV>())
+    return cudaErrorInvalidDeviceFunction;
   if (p.d % 256 == 0 && pair_update_enabled()) {
     const int np = max_pairs<KB>(st);
     if (np > 0) {
@@ -1275,17 +1303,17 @@ static cudaError_t launch_update_kb(const TcParams& p, int num_sms, cudaStream_t
       cfg.stream = st;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      if (cudaFuncSetAttribute(upd_kernel<true, KB, DELTA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      if (cudaFuncSetAttribute(upd_kernel<true, KB, DELTA, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
           cudaSuccess)
         return cudaErrorInvalidValue;
-      return cudaLaunchKernelEx(&cfg, upd_kernel<true, KB, DELTA>, q);
+      return cudaLaunchKernelEx(&cfg, upd_kernel<true, KB, DELTA, REV>, q);
     }
   }
   constexpr int smem = UpdCfg<false, KB>::SMEM;
-  cudaError_t e = cudaFuncSetAttribute(upd_kernel<false, KB, DELTA>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(upd_kernel<false, KB, DELTA, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(p.n_tiles, num_sms));
-  upd_kernel<false, KB, DELTA><<<grid, UPD_THREADS, smem, st>>>(p);
+  upd_kernel<false, KB, DELTA, REV><<<grid, UPD_THREADS, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -1294,9 +1322,14 @@ int update_tokens_per_stage(int C) { return C % 128 == 0 ? 128 : 64; }
 cudaError_t launch_update(const TcParams& p, int num_sms, cudaStream_t st) {
   if (p.n_tiles <= 0 || p.dchunks <= 0) return cudaSuccess;
   const int kb = p.upd_kb ? p.upd_kb : update_tokens_per_stage(p.C);
+  if (p.rev)
+    return kb == 128 ? launch_update_kb<128, false, true>(p, num_sms, st)
+                     : launch_update_kb<64, false, true>(p, num_sms, st);
   if (p.delta_out)
-    return kb == 128 ? launch_update_kb<128, true>(p, num_sms, st) : launch_update_kb<64, true>(p, num_sms, st);
-  return kb == 128 ? launch_update_kb<128, false>(p, num_sms, st) : launch_update_kb<64, false>(p, num_sms, st);
+    return kb == 128 ? launch_update_kb<128, true, false>(p, num_sms, st)
+                     : launch_update_kb<64, true, false>(p, num_sms, st);
+  return kb == 128 ? launch_update_kb<128, false, false>(p, num_sms, st)
+                   : launch_update_kb<64, false, false>(p, num_sms, st);
 }
 
 // ------------------------------------------------------------------ failure-path self test

@@ -53,6 +53,8 @@ struct TcParams {
   int upd_scale;          // update: 1 = V is not pre-scaled; the delta is scaled by alpha[b][chunk] eta
   int o_tma;              // 256-row apply: O leaves through shared memory and TMA stores (map[6])
   int delta_out;          // update: each chunk's raw delta V_L^T Z_L also goes out, bf16 (map[7])
+  int rev;                // update: the backward's reverse scan (map[3] = gO_F, S = the start state G_k;
+                          // slot i of map[5] receives bf16(G_{i+1}))
 };
 
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
