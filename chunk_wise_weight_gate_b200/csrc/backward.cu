@@ -191,6 +191,14 @@ __global__ void k_conv_grad_weight(const float* gU, const float* X0, const uint8
 }
 
 unsigned grid_for(size_t n) { return (unsigned)std::min<size_t>((n + 255) / 256, 148 * 16); }
+// Kernels with one token per block iteration and threads over w channel groups:
+// blocks of w threads rounded up to a warp (at most 1024), as many as fit on the
+// SMs at once (at most one per token).
+unsigned token_block(long long w) { return (unsigned)std::min<long long>(1024, (w + 31) / 32 * 32); }
+unsigned token_grid(long long tokens, long long w) {
+  const long long per_sm = std::max<long long>(1, 2048 / token_block(w));
+  return (unsigned)std::max<long long>(1, std::min<long long>(tokens, 148 * per_sm));
+}
 
 }  // namespace
 
@@ -453,14 +461,18 @@ cudaError_t run(const Shape& s, int dtype, float eta, float tau, const void* H_,
 //   then the gated activation, gH, gWgate, gWup, the target GEMM and the conv as on the fp32 path.
 namespace {
 
+// gO on the continued first segment of each chunk, zero elsewhere; 8 channels of
+// one token per thread (d % 8 == 0, 16-byte rows).
 __global__ void k_mask_first_bf16(const __nv_bfloat16* gO, __nv_bfloat16* gOF, const ChunkMeta* meta, int B, int T,
                                   int d, int C, int k) {
-  const size_t n = (size_t)B * T * d;
+  const int g8 = d / 8;
+  const size_t n = (size_t)B * T * g8;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-    const size_t bt = i / d;
+    const size_t bt = i / g8;
     const int t = (int)(bt % T), b = (int)(bt / T);
     const ChunkMeta m = meta[(size_t)b * k + t / C];
-    gOF[i] = (m.cont && t < m.first_end) ? gO[i] : __float2bfloat16(0.0f);
+    const bool keep = m.cont && t < m.first_end;
+    reinterpret_cast<uint4*>(gOF)[i] = keep ? reinterpret_cast<const uint4*>(gO)[i] : make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -503,52 +515,89 @@ __global__ void k_clip_coeffs_tc(const double* part, const float* alpha, float* 
 // gV = c1 Y on the rows of each chunk's last segment, 0 elsewhere.
 __global__ void k_gv_init(const float* Y, const float* c1, float* gV, const ChunkMeta* meta, int B, int T, int d,
                           int C, int k) {
-  const size_t n = (size_t)B * T * d;
-  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
-    const size_t bt = e / d;
-    const int t = (int)(bt % T), b = (int)(bt / T);
-    const int i = t / C;
-    gV[e] = t >= meta[(size_t)b * k + i].last_start ? c1[(size_t)b * k + i] * Y[e] : 0.0f;
+  // one token per block iteration (its chunk's row start and c1 read once), 4 channels per thread
+  const int g4 = d / 4;
+  const long long BT = (long long)B * T;
+  for (long long bt = blockIdx.x; bt < BT; bt += gridDim.x) {
+    const int t = (int)(bt % T);
+    const size_t bi = (size_t)(bt / T) * k + t / C;
+    const bool in_last = t >= meta[bi].last_start;
+    const float sc = in_last ? c1[bi] : 0.0f;
+    const float4* y = reinterpret_cast<const float4*>(Y + bt * d);
+    float4* o = reinterpret_cast<float4*>(gV + bt * d);
+    for (int c = threadIdx.x; c < g4; c += blockDim.x) {
+      if (in_last) {
+        const float4 v = y[c];
+        o[c] = make_float4(sc * v.x, sc * v.y, sc * v.z, sc * v.w);
+      } else {
+        o[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      }
+    }
   }
 }
 
-// gA = gZ Bu SiLU'(A), gBu = gZ SiLU(A), rounded to bf16 (the next products' operands).
+// gA = gZ Bu SiLU'(A), gBu = gZ SiLU(A), rounded to bf16 (the next products' operands);
+// 8 elements per thread (n % 8 == 0).
 __global__ void k_gate_backward_bf16(const __nv_bfloat16* A, const __nv_bfloat16* Bu, const float* gZ,
                                      __nv_bfloat16* gA, __nv_bfloat16* gBu, size_t n) {
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-    const float a = __bfloat162float(A[i]), u = __bfloat162float(Bu[i]), g = gZ[i];
-    const float s = 1.0f / (1.0f + expf(-a));
-    gA[i] = __float2bfloat16(g * u * (s * (1.0f + a * (1.0f - s))));
-    gBu[i] = __float2bfloat16(g * (a * s));
+  const size_t n8 = n / 8;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
+    const uint4 av = reinterpret_cast<const uint4*>(A)[i], uv = reinterpret_cast<const uint4*>(Bu)[i];
+    const float4 g0 = reinterpret_cast<const float4*>(gZ)[2 * i], g1 = reinterpret_cast<const float4*>(gZ)[2 * i + 1];
+    const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    const __nv_bfloat162* ap = reinterpret_cast<const __nv_bfloat162*>(&av);
+    const __nv_bfloat162* up = reinterpret_cast<const __nv_bfloat162*>(&uv);
+    uint4 oa, ob;
+    __nv_bfloat162* pa = reinterpret_cast<__nv_bfloat162*>(&oa);
+    __nv_bfloat162* pb = reinterpret_cast<__nv_bfloat162*>(&ob);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float a0 = __low2float(ap[q]), a1 = __high2float(ap[q]);
+      const float u0 = __low2float(up[q]), u1 = __high2float(up[q]);
+      const float s0 = 1.0f / (1.0f + expf(-a0)), s1 = 1.0f / (1.0f + expf(-a1));
+      pa[q] = __floats2bfloat162_rn(g[2 * q] * u0 * (s0 * (1.0f + a0 * (1.0f - s0))),
+                                    g[2 * q + 1] * u1 * (s1 * (1.0f + a1 * (1.0f - s1))));
+      pb[q] = __floats2bfloat162_rn(g[2 * q] * (a0 * s0), g[2 * q + 1] * (a1 * s1));
+    }
+    reinterpret_cast<uint4*>(gA)[i] = oa;
+    reinterpret_cast<uint4*>(gBu)[i] = ob;
   }
 }
 
-// gX0[s, c] = sum_o w[c, o] gU[s - o, c] over the taps o in use at token s - o,
-// 8 channels of one token per thread (d % 8 == 0): the taps in use are found
-// once for the 8, and gU comes in 32-byte rows.
+// gX0[s, c] = sum_o w[c, o] gU[s - o, c] over the taps o in use at token s - o.
+// Threads over groups of 8 channels (d % 8 == 0), each holding its 8 x kTaps
+// weights; blocks over tokens, the taps in use found once per token.
 __global__ void k_conv_grad_input_v8(const float* gU, const float* cw, const uint8_t* flags, float* gX0, int B,
                                      int T, int d, int C) {
   const int g8 = d / 8;
-  const size_t n = (size_t)B * T * g8;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-    const int c0 = (int)(i % g8) * 8;
-    const size_t bt = i / g8;
-    const int s = (int)(bt % T), b = (int)(bt / T);
-    const uint8_t* f = flags + (size_t)b * T;
-    float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+  const long long BT = (long long)B * T;
+  for (int c8 = threadIdx.x; c8 < g8; c8 += blockDim.x) {
+    const int c0 = c8 * 8;
+    float w[8 * kTaps];  // w[q * kTaps + o] = cw[c0 + q][o]: 40 consecutive floats, 16-byte aligned
+    const float4* wv = reinterpret_cast<const float4*>(cw + (size_t)c0 * kTaps);
 #pragma unroll
-    for (int o = 0; o < kTaps; ++o) {
-      const int t = s - o;
-      if (t < 0 || o >= taps_at(f, t, T, C)) continue;
-      const float4* u = reinterpret_cast<const float4*>(gU + ((size_t)b * T + t) * d + c0);
-      const float4 u0 = u[0], u1 = u[1];
-      const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = fmaf(cw[(c0 + q) * kTaps + o], uv[q], acc[q]);
+    for (int j = 0; j < 2 * kTaps; ++j) {
+      const float4 x = wv[j];
+      w[4 * j] = x.x; w[4 * j + 1] = x.y; w[4 * j + 2] = x.z; w[4 * j + 3] = x.w;
     }
-    float4* out = reinterpret_cast<float4*>(gX0 + bt * d + c0);
-    out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    for (long long bt = blockIdx.x; bt < BT; bt += gridDim.x) {
+      const int s = (int)(bt % T);
+      const uint8_t* f = flags + (bt - s);
+      float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int o = 0; o < kTaps; ++o) {
+        const int t = s - o;
+        if (t < 0 || o >= taps_at(f, t, T, C)) continue;
+        const float4* u = reinterpret_cast<const float4*>(gU + (bt - o) * d + c0);
+        const float4 u0 = u[0], u1 = u[1];
+        const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = fmaf(w[q * kTaps + o], uv[q], acc[q]);
+      }
+      float4* out = reinterpret_cast<float4*>(gX0 + bt * d + c0);
+      out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
   }
 }
 
@@ -556,7 +605,7 @@ __global__ void k_conv_grad_input_v8(const float* gU, const float* cw, const uin
 // use, in two fixed-order steps: block (channel block, part) sums a contiguous
 // range of tokens for 256 channels (threads over channels, so loads are
 // coalesced), then the parts are added in order.
-constexpr int kConvParts = 64;
+constexpr int kConvParts = 256;
 __global__ void k_conv_grad_weight_parts(const float* gU, const __nv_bfloat16* X0, const uint8_t* flags,
                                          float* part, int B, int T, int d, int C) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
@@ -564,6 +613,7 @@ __global__ void k_conv_grad_weight_parts(const float* gU, const __nv_bfloat16* X
   const long long BT = (long long)B * T;
   const long long lo = BT * blockIdx.y / kConvParts, hi = BT * (blockIdx.y + 1) / kConvParts;
   float acc[kTaps] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 4
   for (long long bt = lo; bt < hi; ++bt) {
     const int t = (int)(bt % T), b = (int)(bt / T);
     const float g = gU[bt * d + c];
@@ -701,7 +751,7 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
   g.A = {Vb, (uint64_t)(d), (uint64_t)(T), (uint64_t)(B)};
   g.Bop = {Zb, (uint64_t)(F), (uint64_t)(T), (uint64_t)(B)};
   if (!f.deltas_ready) BW_CHECK(chunked(GM_CHUNK_K, (int)d, (int)F, 0, P, F, d * F, GO_BF16, nullptr, GR_ALL, 1));
-  k_mask_first_bf16<<<grid_for(B * T * d), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(gO), gOF, f.meta, (int)B,
+  k_mask_first_bf16<<<grid_for(B * T * d / 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(gO), gOF, f.meta, (int)B,
                                                           (int)T, (int)d, s.C, k);
   // 5. reverse scan on the state-update kernel: from G_k = gS, every chunk's
   //    gO_F^T Z_F formed from zero in TMEM and added in fp32 (registers), bf16 G_{i+1}
@@ -735,7 +785,7 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
   k_vy_partials<<<dim3(k, (unsigned)B, kDotParts), 256, 0, st>>>(Vb, Y, dpart, (int)T, (int)d, s.C, k);
   k_clip_coeffs_tc<<<(unsigned)((B * k + 127) / 128), 128, 0, st>>>(dpart, f.alpha, c1, c2, (int)(B * k), eta, tau);
   // 7. gV_L = c1 Y + c2 Z_L P_i^T
-  k_gv_init<<<grid_for(B * T * d), 256, 0, st>>>(Y, c1, gV, f.meta, (int)B, (int)T, (int)d, s.C, k);
+  k_gv_init<<<token_grid(BT, d / 4), token_block(d / 4), 0, st>>>(Y, c1, gV, f.meta, (int)B, (int)T, (int)d, s.C, k);
   g.Bop = {P, (uint64_t)(F), (uint64_t)(d), (uint64_t)((uint64_t)k * B)};
   BW_CHECK(chunked(GM_CHUNK_ROWS, 0, (int)d, (int)F, gV, d, T * d, GO_F32_ADD, c2, GR_LAST, k));
   // 8. gZ += c1 V_L G_{i+1} + c2 V_L P_i + gO_F S_i (K = d; the [d][F] operands n-major)
@@ -749,7 +799,7 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
   g.Bop = {f.snap, (uint64_t)(F), (uint64_t)(d), (uint64_t)((uint64_t)f.nslots * B)};
   BW_CHECK(chunked(GM_CHUNK_ROWS, 0, (int)F, (int)d, gZ, F, T * F, GO_F32_ADD, nullptr, GR_FIRST, f.nslots));
   // 9. the gated activation; gH = gA Wg + gBu Wu; gWg = gA^T H, gWu = gBu^T H
-  k_gate_backward_bf16<<<grid_for(BT * F), 256, 0, st>>>(Af, Buf, gZ, gA, gBu, (size_t)(BT * F));
+  k_gate_backward_bf16<<<grid_for(BT * F / 8), 256, 0, st>>>(Af, Buf, gZ, gA, gBu, (size_t)(BT * F));
   g.A = {gA, (uint64_t)(F), (uint64_t)(BT), (uint64_t)(1)};
   g.Bop = {Wg, (uint64_t)(d), (uint64_t)(F), (uint64_t)(1)};
   g.a_mn = 0; g.b_mn = 1;
@@ -774,7 +824,8 @@ cudaError_t run_tc(const Shape& s, float eta, float tau, const TcForward& f, con
   g.a_mn = 1; g.b_mn = 1;
   BW_CHECK(plain((int)d, (int)d, (int)BT, gWt, d, GO_F32));
   k_widen<<<grid_for(d * kTaps), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(cw), cwf, (size_t)(d * kTaps));
-  k_conv_grad_input_v8<<<grid_for(BT * d / 8), 256, 0, st>>>(gU, cwf, f.flags, gX0, (int)B, (int)T, (int)d, s.C);
+  k_conv_grad_input_v8<<<token_grid(BT, d / 8), token_block(d / 8), 0, st>>>(gU, cwf, f.flags, gX0, (int)B, (int)T,
+                                                                           (int)d, s.C);
   k_conv_grad_weight_parts<<<dim3((unsigned)((d + 255) / 256), kConvParts), 256, 0, st>>>(
       gU, static_cast<const __nv_bfloat16*>(X0), f.flags, cpart, (int)B, (int)T, (int)d, s.C);
   k_conv_grad_weight_reduce<<<(unsigned)((d * kTaps + 255) / 256), 256, 0, st>>>(cpart, gcw, (int)d);
