@@ -358,14 +358,17 @@ __global__ void k_blocked_to_bf16(const float* Sb, __nv_bfloat16* out, int B, in
   }
 }
 
+// Four consecutive columns (c % 4 == 0) stay consecutive in the blocked layout, so
+// each thread moves one float4 (F % 128 == 0).
 __global__ void k_rowmajor_to_blocked(const float* in, float* Sb, int B, int d, int F) {
-  const size_t total = (size_t)B * d * F;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-    const int c = (int)(i % F);
-    const size_t br = i / F;
+  const size_t total4 = (size_t)B * d * F / 4;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total4; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t e = 4 * i;
+    const int c = (int)(e % F);
+    const size_t br = e / F;
     const int r = (int)(br % d);
     const size_t b = br / d;
-    Sb[b * d * F + blocked_index(r, c, F)] = in[i];
+    *reinterpret_cast<float4*>(Sb + b * d * F + blocked_index(r, c, F)) = reinterpret_cast<const float4*>(in)[i];
   }
 }
 

@@ -613,14 +613,19 @@ __global__ void k_conv_grad_weight_parts(const float* gU, const __nv_bfloat16* X
   const long long BT = (long long)B * T;
   const long long lo = BT * blockIdx.y / kConvParts, hi = BT * (blockIdx.y + 1) / kConvParts;
   float acc[kTaps] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+  int t = (int)(lo % T);            // token and row of bt, advanced with it
+  const uint8_t* f = flags + (lo - t);
 #pragma unroll 4
   for (long long bt = lo; bt < hi; ++bt) {
-    const int t = (int)(bt % T), b = (int)(bt / T);
     const float g = gU[bt * d + c];
-    const int n = taps_at(flags + (size_t)b * T, t, T, C);
+    const int n = taps_at(f, t, T, C);
 #pragma unroll
     for (int o = 0; o < kTaps; ++o)
       if (o < n) acc[o] = fmaf(__bfloat162float(X0[(bt + o) * d + c]), g, acc[o]);
+    if (++t == T) {
+      t = 0;
+      f += T;
+    }
   }
 #pragma unroll
   for (int o = 0; o < kTaps; ++o) part[((size_t)blockIdx.y * d + c) * kTaps + o] = acc[o];
