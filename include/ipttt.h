@@ -360,8 +360,10 @@ IPTTT_API const char* ipttt_version(void);
  * state gradients are operands, so the gradients carry bf16 operand rounding.
  * Deterministic either way.  All pointers are device memory owned by the caller,
  * 16-byte aligned; workspace (256-byte aligned) of ipttt_backward_workspace_size(p)
- * bytes (fp32: k + 4 fp32 states [B][d][F]; bf16: about 2.5 k bf16 and k fp32
- * states [B][d][F] besides the activations).  Errors as for ipttt_forward. */
+ * bytes (fp32: k + 4 fp32 states [B][d][F]; bf16: three bf16 states [B][d][F]
+ * per chunk (the forward's state copies, the raw deltas, the state-gradient copies),
+ * one fp32 state, and about 20 F bytes per token of activations and their
+ * gradients).  Errors as for ipttt_forward. */
 IPTTT_API size_t ipttt_backward_workspace_size(const ipttt_params* p);
 IPTTT_API ipttt_status ipttt_backward(const ipttt_params* p, const void* H, const void* X0, const void* Wgate,
                                       const void* Wup, const void* Wdown0, const void* conv_w,
